@@ -1,0 +1,364 @@
+"""huffman_decode_02_b200 -- DFloat11 (DF11) lossless BF16 weight codec for
+B200 (sm_100a): host encoder + GPU decoder behind the C ABI of libdf11.so.
+
+This module is a thin binding: it marshals arguments (numpy / torch buffers,
+CUDA streams) into the C calls declared in ``include/df11.h`` and does no
+part of the codec itself.  PyTorch is used for device memory and streams
+only.  There is no fallback: if ``libdf11.so`` is missing or fails to load,
+importing this package raises.
+
+Typical use::
+
+    import huffman_decode_02_b200 as df11
+    t = df11.encode(w_bf16_bits)          # host: numpy uint16 / torch bf16 (CPU)
+    d = t.to("cuda")                      # device copy of the compressed arrays
+    w = df11.decode(d)                    # torch.bfloat16 on the GPU, bit-exact
+
+    blk = df11.encode_multi([q, k, v, o, gate, up, down, n1, n2])
+    dblk = blk.to("cuda")
+    scratch = df11.decode_block(dblk)     # one launch; dblk.views(scratch) -> matrices
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Iterable, Sequence
+
+import numpy as np
+
+from . import build as _build
+
+__all__ = [
+    "DF11Error", "CorruptStreamError", "Params", "DF11Tensor", "encode", "encode_multi",
+    "decode", "decode_block", "read_error", "exponent_histogram", "lib_path", "sm_count",
+    "KERR_COUNT_MISMATCH", "KERR_BAD_CODE", "KERR_BAD_BLOCK", "KERR_OVERRUN", "KERR_TIMEOUT",
+]
+
+KERR_COUNT_MISMATCH = 0x1
+KERR_BAD_CODE = 0x2
+KERR_BAD_BLOCK = 0x4
+KERR_OVERRUN = 0x8
+KERR_TIMEOUT = 0x10
+
+_STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported parameter", 3: "tensor too large",
+           4: "corrupt compressed data", 5: "CUDA error", 6: "out of host memory"}
+
+
+class DF11Error(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what}: {_STATUS.get(status, status)} (status {status})")
+        self.status = status
+
+
+class CorruptStreamError(DF11Error):
+    pass
+
+
+# --------------------------------------------------------------- ctypes ABI
+class _Params(ctypes.Structure):
+    _fields_ = [("max_code_len", ctypes.c_uint32), ("bytes_per_thread", ctypes.c_uint32),
+                ("threads_per_block", ctypes.c_uint32), ("reserved", ctypes.c_uint32)]
+
+
+class _Tensor(ctypes.Structure):
+    _fields_ = [("n_elems", ctypes.c_uint64), ("total_bits", ctypes.c_uint64),
+                ("n_threads", ctypes.c_uint64), ("n_blocks", ctypes.c_uint64),
+                ("params", _Params), ("code_len", ctypes.c_uint8 * 256),
+                ("enc_bytes", ctypes.c_uint64), ("sm_bytes", ctypes.c_uint64),
+                ("gaps_bytes", ctypes.c_uint64), ("block_start_bytes", ctypes.c_uint64),
+                ("lut_bytes", ctypes.c_uint64),
+                ("enc", ctypes.c_void_p), ("sm", ctypes.c_void_p), ("gaps", ctypes.c_void_p),
+                ("block_start", ctypes.c_void_p), ("lut", ctypes.c_void_p)]
+
+
+_ARRAYS = ("enc", "sm", "gaps", "block_start", "lut")
+_LIB = None
+
+
+def lib_path() -> str:
+    return _build.LIB_PATH
+
+
+def _lib():
+    global _LIB
+    if _LIB is not None:
+        return _LIB
+    path = _build.LIB_PATH
+    if not os.path.exists(path):
+        raise ImportError(f"libdf11.so is not built ({path}); run __graft_entry__.build() or "
+                          "python -m huffman_decode_02_b200.build")
+    lib = ctypes.CDLL(path)
+    P, T, u64, u32, vp = ctypes.POINTER, _Tensor, ctypes.c_uint64, ctypes.c_uint32, ctypes.c_void_p
+    u16pp = P(P(ctypes.c_uint16))
+    lib.df11_abi_version.restype = u32
+    lib.df11_sizeof_tensor.restype = ctypes.c_size_t
+    lib.df11_default_params.argtypes = [P(_Params)]
+    lib.df11_default_params.restype = None
+    lib.df11_status_str.restype = ctypes.c_char_p
+    lib.df11_exponent_histogram.argtypes = [u16pp, P(u64), u32, P(u64)]
+    lib.df11_encode_size.argtypes = [P(ctypes.c_uint16), u64, P(_Params), P(T)]
+    lib.df11_encode.argtypes = [P(ctypes.c_uint16), u64, P(T)]
+    lib.df11_encode_multi_size.argtypes = [u16pp, P(u64), u32, P(_Params), P(T)]
+    lib.df11_encode_multi.argtypes = [u16pp, P(u64), u32, P(T)]
+    lib.df11_validate.argtypes = [P(T)]
+    lib.df11_decode.argtypes = [P(T), vp, vp, vp]
+    lib.df11_decode_block.argtypes = [P(T), P(u64), u32, vp, vp, vp]
+    lib.df11_read_error.argtypes = [vp, vp, P(u32)]
+    lib.df11_device_sm_count.argtypes = [P(ctypes.c_int)]
+    if lib.df11_abi_version() != 1 or lib.df11_sizeof_tensor() != ctypes.sizeof(_Tensor):
+        raise ImportError("libdf11.so ABI does not match this binding")
+    _LIB = lib
+    return lib
+
+
+def _check(status: int, what: str) -> None:
+    if status != 0:
+        cls = CorruptStreamError if status == 4 else DF11Error
+        raise cls(status, what)
+
+
+class Params:
+    """Encoder parameters (see df11_params in include/df11.h)."""
+
+    def __init__(self, max_code_len: int = 32, bytes_per_thread: int = 8, threads_per_block: int = 256):
+        self.max_code_len = max_code_len
+        self.bytes_per_thread = bytes_per_thread
+        self.threads_per_block = threads_per_block
+
+    def _c(self) -> _Params:
+        return _Params(self.max_code_len, self.bytes_per_thread, self.threads_per_block, 0)
+
+
+# ---------------------------------------------------------------- helpers
+def _as_u16(w) -> np.ndarray:
+    """BF16 bits as a contiguous numpy uint16 view (no copy when possible)."""
+    try:
+        import torch
+        if isinstance(w, torch.Tensor):
+            if w.device.type != "cpu":
+                raise ValueError("encode() runs on the host: pass a CPU tensor")
+            if w.dtype not in (torch.bfloat16, torch.int16, torch.uint16):
+                raise TypeError(f"expected BF16 bits, got {w.dtype}")
+            w = w.contiguous().view(torch.int16).numpy()
+    except ImportError:  # pragma: no cover
+        pass
+    a = np.asarray(w)
+    if a.dtype.itemsize != 2:
+        raise TypeError(f"expected 16-bit BF16 bit patterns, got {a.dtype}")
+    return np.ascontiguousarray(a).reshape(-1).view(np.uint16)
+
+
+def _u16_ptr(a: np.ndarray):
+    if a.size == 0:
+        return ctypes.cast(ctypes.c_void_p(0), ctypes.POINTER(ctypes.c_uint16))
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_uint16))
+
+
+def _stream_handle(stream) -> ctypes.c_void_p:
+    if stream is None:
+        import torch
+        return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, int):
+        return ctypes.c_void_p(stream)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+class DF11Tensor:
+    """A compressed tensor: the df11_tensor descriptor plus its five arrays,
+    either on the host (numpy uint8 / uint32 arrays, or pinned torch tensors)
+    or on a CUDA device (torch tensors).  ``shapes`` records the original
+    matrix shapes for block tensors (element offsets in ``offsets``)."""
+
+    def __init__(self, desc: _Tensor, arrays: dict, device: str, shapes, offsets):
+        self.desc = desc
+        self.arrays = arrays
+        self.device = device
+        self.shapes = list(shapes)
+        self.offsets = list(offsets)
+
+    # scalar fields
+    n_elems = property(lambda self: int(self.desc.n_elems))
+    total_bits = property(lambda self: int(self.desc.total_bits))
+    n_threads = property(lambda self: int(self.desc.n_threads))
+    n_blocks = property(lambda self: int(self.desc.n_blocks))
+
+    @property
+    def code_len(self) -> np.ndarray:
+        return np.frombuffer(bytes(self.desc.code_len), dtype=np.uint8).copy()
+
+    def nbytes(self, which: str) -> int:
+        return int(getattr(self.desc, which + "_bytes"))
+
+    def compressed_bytes(self) -> int:
+        """Bytes the stored format needs: exponent stream, sign/mantissa,
+        gaps, block starts and the 256-byte code-length table."""
+        return ((self.total_bits + 7) // 8 + self.n_elems + (5 * self.n_threads + 7) // 8
+                + 4 * (self.n_blocks + 1) + 256)
+
+    def bits_per_weight(self) -> float:
+        return 8.0 * self.compressed_bytes() / max(1, self.n_elems)
+
+    def host_array(self, which: str) -> np.ndarray:
+        a = self.arrays[which]
+        if self.device != "cpu":
+            a = a.cpu()
+        if not isinstance(a, np.ndarray):
+            a = a.numpy()
+        return a.view(np.uint32) if which == "block_start" else a.view(np.uint8)
+
+    def _bind(self) -> _Tensor:
+        d = _Tensor.from_buffer_copy(self.desc)
+        for name in _ARRAYS:
+            a = self.arrays[name]
+            ptr = a.ctypes.data if isinstance(a, np.ndarray) else a.data_ptr()
+            setattr(d, name, ptr)
+        return d
+
+    def to(self, device, non_blocking: bool = False) -> "DF11Tensor":
+        """Copies the five arrays to a device (torch tensors, 16-byte aligned)."""
+        import torch
+        dev = torch.device(device)
+        arrays = {}
+        for name in _ARRAYS:
+            a = self.arrays[name]
+            if isinstance(a, np.ndarray):
+                a = torch.from_numpy(a.view(np.uint8))
+            b = torch.empty(a.numel() * a.element_size(), dtype=torch.uint8, device=dev)
+            b.copy_(a.view(torch.uint8).reshape(-1), non_blocking=non_blocking)
+            arrays[name] = b
+        return DF11Tensor(_Tensor.from_buffer_copy(self.desc), arrays, str(dev), self.shapes, self.offsets)
+
+    def views(self, decoded):
+        """Splits a decoded block buffer into the original matrices."""
+        out = []
+        for shape, lo, hi in zip(self.shapes, self.offsets[:-1], self.offsets[1:]):
+            out.append(decoded[lo:hi].view(*shape) if shape else decoded[lo:hi])
+        return out
+
+
+def _alloc_host(nbytes: int, pinned: bool):
+    if pinned:
+        import torch
+        return torch.empty(max(nbytes, 16), dtype=torch.uint8, pin_memory=True)
+    # 64-byte aligned numpy buffer
+    raw = np.empty(max(nbytes, 16) + 64, dtype=np.uint8)
+    off = (-raw.ctypes.data) % 64
+    return raw[off: off + max(nbytes, 16)]
+
+
+def _encode_impl(mats: list[np.ndarray], shapes, params: Params | None, pinned: bool) -> DF11Tensor:
+    lib = _lib()
+    k = len(mats)
+    ptrs = (ctypes.POINTER(ctypes.c_uint16) * max(1, k))(*[_u16_ptr(m) for m in mats])
+    sizes = (ctypes.c_uint64 * max(1, k))(*[m.size for m in mats])
+    desc = _Tensor()
+    pc = (params or Params())._c()
+    _check(lib.df11_encode_multi_size(ptrs, sizes, k, ctypes.byref(pc), ctypes.byref(desc)), "encode (size)")
+    arrays = {name: _alloc_host(int(getattr(desc, name + "_bytes")), pinned) for name in _ARRAYS}
+    for name in _ARRAYS:
+        a = arrays[name]
+        setattr(desc, name, a.ctypes.data if isinstance(a, np.ndarray) else a.data_ptr())
+    _check(lib.df11_encode_multi(ptrs, sizes, k, ctypes.byref(desc)), "encode")
+    for name in _ARRAYS:
+        setattr(desc, name, None)
+    offsets = [0]
+    for m in mats:
+        offsets.append(offsets[-1] + m.size)
+    return DF11Tensor(desc, arrays, "cpu", shapes, offsets)
+
+
+def encode(w, params: Params | None = None, pinned: bool = False) -> DF11Tensor:
+    """Host encoder for one BF16 matrix (numpy uint16 bits or a CPU torch
+    tensor): histogram, length-limited canonical Huffman code, packing, aux."""
+    shape = tuple(getattr(w, "shape", ()))
+    return _encode_impl([_as_u16(w)], [shape], params, pinned)
+
+
+def encode_multi(mats: Sequence, params: Params | None = None, pinned: bool = False) -> DF11Tensor:
+    """Encodes several matrices (a transformer block) as one stream with one
+    shared table; ``DF11Tensor.offsets`` gives each matrix's element offset."""
+    arrs = [_as_u16(m) for m in mats]
+    shapes = [tuple(getattr(m, "shape", ())) for m in mats]
+    return _encode_impl(arrs, shapes, params, pinned)
+
+
+def exponent_histogram(mats: Iterable) -> np.ndarray:
+    arrs = [_as_u16(m) for m in mats]
+    k = len(arrs)
+    ptrs = (ctypes.POINTER(ctypes.c_uint16) * max(1, k))(*[_u16_ptr(m) for m in arrs])
+    sizes = (ctypes.c_uint64 * max(1, k))(*[m.size for m in arrs])
+    out = np.zeros(256, dtype=np.uint64)
+    _check(_lib().df11_exponent_histogram(ptrs, sizes, k, out.ctypes.data_as(ctypes.POINTER(ctypes.c_uint64))),
+           "exponent_histogram")
+    return out
+
+
+def _check_device(t: DF11Tensor):
+    if t.device == "cpu":
+        raise ValueError("decode needs the compressed arrays on a CUDA device: call .to('cuda') first")
+
+
+def _new_err(device):
+    import torch
+    return torch.zeros(1, dtype=torch.int32, device=device)
+
+
+def decode(t: DF11Tensor, out=None, err=None, stream=None):
+    """Decodes a device-resident DF11Tensor into a BF16 tensor (one launch).
+    ``err`` (int32[1] device tensor) collects kernel error bits; when it is
+    not given, a fresh one is allocated and checked after the launch (which
+    synchronises the stream)."""
+    import torch
+    _check_device(t)
+    if out is None:
+        out = torch.empty(t.n_elems, dtype=torch.bfloat16, device=t.device)
+    own_err = err is None
+    if own_err:
+        err = _new_err(t.device)
+    d = t._bind()
+    _check(_lib().df11_decode(ctypes.byref(d), ctypes.c_void_p(out.data_ptr()),
+                              ctypes.c_void_p(err.data_ptr()), _stream_handle(stream)), "decode")
+    if own_err:
+        read_error(err, stream)
+    return out
+
+
+def decode_block(t: DF11Tensor, scratch=None, err=None, stream=None):
+    """Decodes every matrix of a block tensor (from encode_multi) in one
+    launch into ``scratch`` (BF16, >= n_elems); ``t.views(scratch)`` returns
+    the matrices."""
+    import torch
+    _check_device(t)
+    if scratch is None:
+        scratch = torch.empty(t.n_elems, dtype=torch.bfloat16, device=t.device)
+    if scratch.numel() < t.n_elems:
+        raise ValueError("scratch buffer smaller than the block")
+    own_err = err is None
+    if own_err:
+        err = _new_err(t.device)
+    offs = (ctypes.c_uint64 * len(t.offsets))(*t.offsets)
+    d = t._bind()
+    _check(_lib().df11_decode_block(ctypes.byref(d), offs, len(t.offsets) - 1,
+                                    ctypes.c_void_p(scratch.data_ptr()),
+                                    ctypes.c_void_p(err.data_ptr()), _stream_handle(stream)),
+           "decode_block")
+    if own_err:
+        read_error(err, stream)
+    return scratch
+
+
+def read_error(err, stream=None) -> int:
+    """Reads the kernel error word (synchronises the stream); raises
+    CorruptStreamError if any bit is set."""
+    v = ctypes.c_uint32(0)
+    st = _lib().df11_read_error(ctypes.c_void_p(err.data_ptr()), _stream_handle(stream), ctypes.byref(v))
+    if st == 4:
+        raise CorruptStreamError(4, f"decode kernel reported error bits 0x{v.value:x}")
+    _check(st, "read_error")
+    return int(v.value)
+
+
+def sm_count() -> int:
+    v = ctypes.c_int(0)
+    _check(_lib().df11_device_sm_count(ctypes.byref(v)), "sm_count")
+    return int(v.value)

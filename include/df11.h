@@ -1,0 +1,196 @@
+/*
+ * df11.h -- C ABI of the DFloat11 (DF11) codec library, libdf11.so.
+ *
+ * DF11 stores a BF16 weight as a Huffman code of its 8-bit exponent plus one
+ * raw byte holding its sign and 7-bit mantissa, about 11 bits per weight, and
+ * rebuilds the exact BF16 bits on the GPU right before the weight is used.
+ *
+ * Sources (web pages on DFloat11; cited by title and section):
+ *  - "DFloat11 : compression sans perte pour l'inference GPU qui reduit les
+ *    LLM a 70 % de leur taille" (fr.news.hada.io).  Sections used:
+ *      << La marge de compression restante dans l'exposant BFloat16 >>
+ *      << Le format DFloat11 >>
+ *      << Decodage fonde sur des LUT hierarchiques >>
+ *      << Noyau GPU en deux etapes et metadonnees auxiliaires >>
+ *      << Decompression par bloc transformer >>
+ *  - "70% Size, 100% Accuracy: Lossless LLM Compression for Efficient GPU
+ *    Inference via Dynamic-Length Float" (chatpaper.ai), abstract.
+ *
+ * Conventions for every call:
+ *  - Plain C types only.  Streams are passed as `void *` holding a
+ *    cudaStream_t (NULL = the legacy default stream).
+ *  - The caller owns every buffer.  The library never allocates device
+ *    memory; host encoding uses a size-then-fill pattern.
+ *  - Errors are returned as df11_status; nothing is thrown across the ABI.
+ *  - Device calls are asynchronous on the given stream and return launch /
+ *    argument errors immediately.  Data corruption found by a kernel is
+ *    reported by OR-ing bits into a caller-owned device word (err_word).
+ *  - Thread safety: calls share no mutable global state.
+ */
+#ifndef DF11_H
+#define DF11_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum df11_status {
+    DF11_OK = 0,
+    DF11_ERR_INVALID_ARG = 1, /* NULL pointer, bad size, bad alignment, bad params */
+    DF11_ERR_UNSUPPORTED = 2, /* a parameter value this build does not implement */
+    DF11_ERR_TOO_LARGE = 3,   /* more than 2^32 - 1 elements in one stream */
+    DF11_ERR_CORRUPT = 4,     /* inconsistent stream / aux data (host checks) */
+    DF11_ERR_CUDA = 5,        /* a CUDA runtime call failed */
+    DF11_ERR_NOMEM = 6        /* host allocation failed */
+} df11_status;
+
+/* Bits a decode kernel ORs into err_word when the data is inconsistent. */
+#define DF11_KERR_COUNT_MISMATCH 0x1u /* codes in a thread block != its span  */
+#define DF11_KERR_BAD_CODE 0x2u       /* a bit pattern that is no code        */
+#define DF11_KERR_BAD_BLOCK 0x4u      /* block_start not monotone / too big   */
+#define DF11_KERR_OVERRUN 0x8u        /* a thread's codes run past its end    */
+
+/* Encoder parameters.
+ *  max_code_len      -- length cap L_MAX for the exponent code, 1..32.  The
+ *                       pages give 32 as the bound implied by 5-bit gaps
+ *                       and observe 24..32 in LLMs ("Decodage fonde sur des
+ *                       LUT hierarchiques", "Noyau GPU en deux etapes...").
+ *  bytes_per_thread  -- n, bytes of the exponent stream owned by one decode
+ *                       thread.  The pages use n = 8; this build supports 8.
+ *  threads_per_block -- T, threads that share one stored output position.
+ *                       The pages do not give T; this build supports 256. */
+typedef struct df11_params {
+    uint32_t max_code_len;
+    uint32_t bytes_per_thread;
+    uint32_t threads_per_block;
+    uint32_t reserved; /* must be 0 */
+} df11_params;
+
+/* A compressed tensor (or a whole transformer block encoded with one shared
+ * table).  Plain data: the struct never owns the arrays it points to.
+ *
+ * Format ("Le format DFloat11", "Noyau GPU en deux etapes et metadonnees
+ * auxiliaires"), with the readings this library takes where the pages are
+ * silent:
+ *  enc         EncodedExponent: canonical Huffman codes of the exponents in
+ *              element order, packed MSB-first; zero-padded to enc_bytes
+ *              = n_blocks * T * n + 16.
+ *  sm          PackedSignMantissa: byte i = (sign_i << 7) | mantissa_i;
+ *              zero-padded to sm_bytes = round_up(n_elems, 16) + 16.
+ *  gaps        Gaps: one 5-bit field per thread (MSB-first, thread order):
+ *              bit offset, from the thread's first byte, of the first code
+ *              that starts in its n bytes (the end of the stream counts as
+ *              a start).  n_blocks * T fields, zero-padded to gaps_bytes.
+ *  block_start u32 per thread block: index of the first element decoded by
+ *              that block, plus a final entry equal to n_elems.
+ *  lut         decode tables derived from code_len (layout private to the
+ *              library, lut_bytes long): a multi-code LUT on the first W
+ *              bits of a window, a code-count LUT, and canonical limits for
+ *              codes longer than W bits.
+ *  code_len    the table: code length of every exponent value (0 = absent).
+ *              Codes are canonical: ordered by (length, exponent value).
+ *
+ * For the encode calls the pointers are HOST arrays the caller allocated
+ * with the *_bytes sizes returned by the size call.  For the decode calls
+ * they are DEVICE arrays holding the same bytes, each 16-byte aligned. */
+typedef struct df11_tensor {
+    uint64_t n_elems;
+    uint64_t total_bits; /* bits of code in enc (padding excluded) */
+    uint64_t n_threads;  /* ceil(total_bits / (8 * n)) */
+    uint64_t n_blocks;   /* ceil(n_threads / T) */
+    df11_params params;
+    uint8_t code_len[256];
+    uint64_t enc_bytes;
+    uint64_t sm_bytes;
+    uint64_t gaps_bytes;
+    uint64_t block_start_bytes;
+    uint64_t lut_bytes;
+    uint8_t *enc;
+    uint8_t *sm;
+    uint8_t *gaps;
+    uint32_t *block_start;
+    uint8_t *lut;
+} df11_tensor;
+
+/* ------------------------------------------------------------------ host */
+
+/* ABI version of this header (bumped on any layout change) and
+ * sizeof(df11_tensor) as compiled into the library, so that bindings can
+ * check their mirror of the struct. */
+#define DF11_ABI_VERSION 1u
+uint32_t df11_abi_version(void);
+size_t df11_sizeof_tensor(void);
+
+/* Default parameters: max_code_len 32, bytes_per_thread 8, T 256. */
+void df11_default_params(df11_params *p);
+
+/* Human-readable name of a status code (static string). */
+const char *df11_status_str(df11_status s);
+
+/* Exponent histogram of k matrices taken as one sequence ("Le format
+ * DFloat11": the tree is built from the exponent distribution).
+ * mats[i] points to sizes[i] BF16 values (as uint16 bits).  count[256] out. */
+df11_status df11_exponent_histogram(const uint16_t *const *mats, const uint64_t *sizes,
+                                    uint32_t k, uint64_t count[256]);
+
+/* Size pass of the encoder for one matrix of n BF16 values: computes the
+ * histogram, the length-limited optimal code lengths (canonical code), the
+ * stream size, the aux sizes and every *_bytes field of *t.  The pointer
+ * fields of *t are left untouched.  params may be NULL (defaults). */
+df11_status df11_encode_size(const uint16_t *bf16, uint64_t n, const df11_params *params,
+                             df11_tensor *t);
+
+/* Fill pass: writes enc, sm, gaps, block_start and lut into the caller's
+ * host arrays *t points to (sizes from df11_encode_size on the same data).
+ * Arrays are fully written, padding included. */
+df11_status df11_encode(const uint16_t *bf16, uint64_t n, df11_tensor *t);
+
+/* Same two passes for k matrices encoded as ONE stream with ONE shared table
+ * ("Decompression par bloc transformer": every matrix of a transformer block
+ * is decompressed in one batch).  Element i of matrix j sits at element
+ * offset (sizes[0] + ... + sizes[j-1]) + i of the decoded block. */
+df11_status df11_encode_multi_size(const uint16_t *const *mats, const uint64_t *sizes, uint32_t k,
+                                   const df11_params *params, df11_tensor *t);
+df11_status df11_encode_multi(const uint16_t *const *mats, const uint64_t *sizes, uint32_t k,
+                              df11_tensor *t);
+
+/* Host-side consistency check of a tensor's scalar fields and sizes
+ * (no array contents are read). */
+df11_status df11_validate(const df11_tensor *t);
+
+/* ---------------------------------------------------------------- device */
+
+/* Decodes one compressed tensor into out (n_elems BF16 values, as uint16,
+ * 16-byte aligned device memory).  One kernel launch on `stream`; the whole
+ * decode (table staging, per-thread decode, block scan, sign/mantissa merge,
+ * stores) runs on the GPU.  err_word: caller-owned device uint32 that the
+ * kernel ORs DF11_KERR_* bits into (it is not cleared here); may be NULL,
+ * in which case corruption is not reported.  n_elems == 0 is a no-op. */
+df11_status df11_decode(const df11_tensor *t, uint16_t *out, uint32_t *err_word, void *stream);
+
+/* Decodes every matrix of a transformer block, encoded with
+ * df11_encode_multi, in ONE launch into a reusable BF16 scratch buffer of at
+ * least t->n_elems elements ("Decompression par bloc transformer").
+ * mat_offsets[0..k] are the element offsets of the k matrices in the
+ * scratch (mat_offsets[0] == 0, mat_offsets[k] == n_elems, non-decreasing);
+ * they are validated and matrix j is then the view
+ * scratch[mat_offsets[j] .. mat_offsets[j+1]).  err_word as in df11_decode. */
+df11_status df11_decode_block(const df11_tensor *blk, const uint64_t *mat_offsets, uint32_t k,
+                              uint16_t *scratch, uint32_t *err_word, void *stream);
+
+/* Copies *err_word to the host after the stream's work so far completes
+ * (synchronises the stream) and returns DF11_ERR_CORRUPT if any bit is set. */
+df11_status df11_read_error(const uint32_t *err_word, void *stream, uint32_t *host_value);
+
+/* Number of SMs the decode kernel sizes its persistent grid to on the
+ * current device (for reporting). */
+df11_status df11_device_sm_count(int *sm_count);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DF11_H */

@@ -1,0 +1,196 @@
+"""GPU parity: the sm_100a decode through the C ABI against the oracle,
+element by element, bit-exact (compared as uint16 bit patterns so that -0.0,
+subnormals and NaN payloads count)."""
+import ctypes
+
+import numpy as np
+import pytest
+
+import oracle
+import workloads
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+import huffman_decode_02_b200 as df11  # noqa: E402
+
+
+def _dev():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    return torch.device("cuda:0")
+
+
+def _bits(x: torch.Tensor) -> np.ndarray:
+    return x.view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+def _oracle_decode(t: df11.DF11Tensor) -> np.ndarray:
+    """The oracle's bit-serial decode of the product's stream."""
+    enc = t.host_array("enc")
+    sm = t.host_array("sm")
+    return oracle.decode(enc, t.total_bits, sm, t.n_elems, t.code_len)
+
+
+def _gpu_roundtrip(w, params=None, check_oracle=True):
+    dev = _dev()
+    w = np.ascontiguousarray(w).reshape(-1).view(np.uint16)
+    t = df11.encode(w, params)
+    d = t.to(dev)
+    out = df11.decode(d)
+    torch.cuda.synchronize()
+    got = _bits(out)
+    if check_oracle:
+        ref = _oracle_decode(t)
+        assert np.array_equal(ref, w)  # the oracle reproduces the input
+        np.testing.assert_array_equal(got, ref)
+    else:
+        np.testing.assert_array_equal(got, w)
+    return t, d, got
+
+
+@pytest.mark.parametrize("name", workloads.ADVERSARIAL_NAMES)
+def test_adversarial_bit_exact(name):
+    _gpu_roundtrip(workloads.adversarial(name))
+
+
+@pytest.mark.parametrize("cap", [8, 12, 16, 24])
+def test_length_cap_bit_exact(cap):
+    _gpu_roundtrip(workloads.adversarial("fibonacci_exponents"), df11.Params(max_code_len=cap))
+
+
+def test_long_codes_bit_exact():
+    rng = np.random.default_rng(21)
+    e = np.minimum(rng.geometric(0.42, size=3_000_001), 31) + 100
+    w = ((e << 7) | rng.integers(0, 128, e.size) | (rng.integers(0, 2, e.size) << 15)).astype(np.uint16)
+    t, _, _ = _gpu_roundtrip(w)
+    assert t.code_len.max() > 20
+
+
+def test_config1_1024x1024_seed0():
+    w = workloads.normal_matrix(1024, 1024, 0.02, seed=0)
+    t, _, _ = _gpu_roundtrip(w)
+    assert t.n_blocks > 4 * 148 // 8  # several tiles per CTA group
+
+
+def test_config2_4096x4096_seed1():
+    _gpu_roundtrip(workloads.normal_matrix(4096, 4096, 0.02, seed=1))
+
+
+@pytest.mark.parametrize("n", [1, 7, 15, 16, 17, 255, 4096 + 3, 131_071, 2_000_003])
+def test_ragged_sizes(n):
+    w = workloads.adversarial("ragged_normal")
+    w = np.concatenate([w, w])[:n] if n > w.size else w[:n]
+    _gpu_roundtrip(w)
+
+
+def test_block_decode_small_and_views():
+    dev = _dev()
+    mats = [workloads.normal_matrix(r, c, s, seed=i) for i, (r, c, s) in
+            enumerate([(256, 128, 0.02), (64, 128, 0.03), (3, 7, 0.5), (128, 256, 0.01)])]
+    blk = df11.encode_multi(mats)
+    d = blk.to(dev)
+    scratch = torch.full((blk.n_elems + 100,), float("nan"), dtype=torch.bfloat16, device=dev)
+    df11.decode_block(d, scratch)
+    for m, v in zip(mats, d.views(scratch)):
+        assert tuple(v.shape) == m.shape
+        np.testing.assert_array_equal(_bits(v).reshape(-1), m.reshape(-1))
+    # reuse of the same scratch for a second block
+    mats2 = [workloads.normal_matrix(300, 100, 0.02, seed=77)]
+    blk2 = df11.encode_multi(mats2).to(dev)
+    df11.decode_block(blk2, scratch)
+    np.testing.assert_array_equal(_bits(scratch[: blk2.n_elems]), mats2[0].reshape(-1))
+
+
+def test_decode_on_side_stream_and_repeat():
+    dev = _dev()
+    w = workloads.normal_matrix(2048, 1024, 0.02, seed=5)
+    d = df11.encode(w).to(dev)
+    s = torch.cuda.Stream(device=dev)
+    out = torch.empty(w.size, dtype=torch.bfloat16, device=dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    with torch.cuda.stream(s):
+        for _ in range(3):
+            df11.decode(d, out, err, stream=s)
+    s.synchronize()
+    assert df11.read_error(err, s) == 0
+    np.testing.assert_array_equal(_bits(out), w.reshape(-1))
+
+
+def test_corrupt_block_start_is_reported():
+    dev = _dev()
+    w = workloads.normal_matrix(512, 512, 0.02, seed=6)
+    d = df11.encode(w).to(dev)
+    bs = d.arrays["block_start"].view(torch.int32)
+    bs[3] += 5  # block 2 claims 5 more elements, block 3 5 fewer
+    with pytest.raises(df11.CorruptStreamError):
+        df11.decode(d)
+
+
+def test_corrupt_stream_bits_are_reported():
+    dev = _dev()
+    w = workloads.normal_matrix(512, 512, 0.02, seed=8)
+    d = df11.encode(w).to(dev)
+    enc = d.arrays["enc"]
+    enc[1000:1100] ^= 0x5A  # scramble 100 bytes of codes
+    with pytest.raises(df11.CorruptStreamError):
+        df11.decode(d)
+
+
+def test_sign_mantissa_flip_changes_only_that_weight():
+    dev = _dev()
+    w = workloads.normal_matrix(256, 256, 0.02, seed=9).reshape(-1)
+    d = df11.encode(w).to(dev)
+    d.arrays["sm"][12345] ^= 0x81
+    got = _bits(df11.decode(d))
+    exp = w.copy()
+    exp[12345] ^= 0x8001  # sign bit and mantissa bit 0
+    np.testing.assert_array_equal(got, exp)
+
+
+def test_bad_arguments_rejected():
+    dev = _dev()
+    w = workloads.normal_matrix(64, 64, 0.02, seed=1)
+    d = df11.encode(w).to(dev)
+    out = torch.empty(w.size + 8, dtype=torch.bfloat16, device=dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    with pytest.raises(df11.DF11Error):
+        df11.decode(d, out[1:], err)  # not 16-byte aligned
+    bad = df11.DF11Tensor(df11._Tensor.from_buffer_copy(d.desc), d.arrays, d.device, d.shapes, d.offsets)
+    bad.desc.n_threads += 1
+    with pytest.raises(df11.DF11Error):
+        df11.decode(bad, out, err)
+    offs = (ctypes.c_uint64 * 2)(0, w.size - 1)
+    st = df11._lib().df11_decode_block(ctypes.byref(d._bind()), offs, 1, ctypes.c_void_p(out.data_ptr()),
+                                       ctypes.c_void_p(err.data_ptr()), ctypes.c_void_p(0))
+    assert st == 1
+
+
+@pytest.mark.slow
+def test_config3_llama8b_block_full_size():
+    """The benchmark's workload, in the benchmark's launch configuration:
+    every element compared with the oracle's decode of the same stream."""
+    dev = _dev()
+    mats = workloads.llama8b_block(seed=0)
+    blk = df11.encode_multi(mats)
+    assert blk.n_elems == 218_112_000
+    d = blk.to(dev)
+    scratch = torch.empty(blk.n_elems, dtype=torch.bfloat16, device=dev)
+    df11.decode_block(d, scratch)
+    got = _bits(scratch)
+    ref = _oracle_decode(blk)
+    np.testing.assert_array_equal(got, ref)
+    np.testing.assert_array_equal(ref, np.concatenate([m.reshape(-1) for m in mats]))
+
+
+@pytest.mark.slow
+def test_config4_heavy_tail_full_size():
+    dev = _dev()
+    w = workloads.heavy_tail_matrix(seed=4)
+    t = df11.encode(w)
+    assert t.code_len.max() >= 20
+    d = t.to(dev)
+    got = _bits(df11.decode(d))
+    ref = _oracle_decode(t)
+    np.testing.assert_array_equal(got, ref)
+    np.testing.assert_array_equal(ref, w.reshape(-1))

@@ -1,0 +1,238 @@
+"""Host-side checks of libdf11 (no GPU): the C ABI loads and exports every
+declared call; the product encoder's output is checked against the oracle
+(optimal cost, byte-exact stream for the product's own code, aux recomputed
+from the stream); the decode tables are exercised by a CPU walk that mirrors
+the kernel's lookup rule."""
+import ctypes
+import os
+import re
+import struct
+
+import numpy as np
+import pytest
+
+import huffman_decode_02_b200 as df11
+import oracle
+import workloads
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _header_functions():
+    src = open(os.path.join(ROOT, "include", "df11.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(df11_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(df11.lib_path())
+    names = _header_functions()
+    assert len(names) >= 14
+    for name in names:
+        assert hasattr(lib, name), name
+    assert df11._lib().df11_abi_version() == 1
+
+
+def test_status_strings():
+    lib = df11._lib()
+    assert lib.df11_status_str(0) == b"ok"
+    assert b"corrupt" in lib.df11_status_str(4)
+
+
+def _cost(count, lengths):
+    return int(np.dot(np.asarray(count, dtype=np.int64), np.asarray(lengths, dtype=np.int64)))
+
+
+def _unpack_gaps(packed: np.ndarray, n: int) -> np.ndarray:
+    bits = np.unpackbits(packed)[: 5 * n].reshape(n, 5)
+    return (bits * np.array([16, 8, 4, 2, 1], dtype=np.uint8)).sum(axis=1).astype(np.uint8)
+
+
+CASES = ["all_bf16_patterns", "all_zero", "all_equal", "two_values", "random_u16",
+         "neg_zero_and_nan", "single", "empty", "subnormals", "ragged_normal",
+         "uniform_exponents", "fibonacci_exponents"]
+
+
+def check_against_oracle(w, t, cap=32):
+    w = np.ascontiguousarray(w).reshape(-1).view(np.uint16)
+    count = oracle.histogram(w)
+    assert np.array_equal(df11.exponent_histogram([w]), count)
+    lengths = t.code_len
+    k = int(np.count_nonzero(count))
+    # only exponents that occur get a code; cost is optimal under the cap
+    assert np.array_equal(lengths > 0, count > 0)
+    assert lengths.max(initial=0) <= cap
+    if k:
+        assert _cost(count, lengths) == _cost(count, oracle.package_merge_lengths(count, cap))
+        assert oracle.is_prefix_free(lengths)
+        assert oracle.kraft_sum_2p32(lengths) == (1 << 32 if k >= 2 else 1 << 31)
+    assert t.total_bits == _cost(count, lengths)
+    # the stream is exactly the oracle's encoding with the product's lengths
+    enc_o, sm_o, bits_o = oracle.encode(w, lengths)
+    enc = t.host_array("enc")
+    assert bits_o == t.total_bits
+    assert np.array_equal(enc[: enc_o.size], enc_o)
+    assert not enc[enc_o.size:].any()
+    sm = t.host_array("sm")
+    assert np.array_equal(sm[: w.size], sm_o[: w.size])
+    assert not sm[w.size:].any()
+    # aux recomputed from the stream by the oracle's bit-serial walk
+    a = oracle.aux(enc_o, bits_o, w.size, lengths, 8, 256)
+    assert a["n_threads"] == t.n_threads and a["n_blocks"] == t.n_blocks
+    assert np.array_equal(t.host_array("block_start")[: t.n_blocks + 1], a["block_start"])
+    packed = t.host_array("gaps")
+    n_fields = t.n_blocks * 256
+    assert np.array_equal(_unpack_gaps(packed, n_fields), a["gaps"])
+    assert np.array_equal(packed[: (5 * n_fields + 7) // 8], oracle.pack_gaps(a["gaps"]))
+    # and the oracle decodes the product's stream back to the input
+    out = oracle.decode(enc_o, bits_o, sm_o, w.size, lengths)
+    assert np.array_equal(out, w)
+
+
+@pytest.mark.parametrize("name", CASES)
+def test_encoder_matches_oracle_adversarial(name):
+    w = workloads.adversarial(name)
+    t = df11.encode(w)
+    check_against_oracle(w, t)
+
+
+@pytest.mark.parametrize("cap", [8, 12, 20])
+def test_encoder_length_cap(cap):
+    w = workloads.adversarial("fibonacci_exponents")
+    t = df11.encode(w, df11.Params(max_code_len=cap))
+    check_against_oracle(w, t, cap)
+    assert t.code_len.max() == cap
+
+
+def test_encoder_normal_matrix_small():
+    w = workloads.normal_matrix(512, 384, 0.02, seed=0)
+    t = df11.encode(w)
+    check_against_oracle(w, t)
+    assert 9.5 < t.bits_per_weight() < 11.5
+
+
+def test_encoder_multichunk_boundaries():
+    """Longer than the host chunk (2^20 elements), so chunk seams are hit."""
+    w = workloads.adversarial("ragged_normal")
+    w = np.concatenate([w, w[:1_000_001]])
+    t = df11.encode(w)
+    check_against_oracle(w, t)
+
+
+def test_encode_multi_equals_concatenation():
+    mats = [workloads.normal_matrix(r, c, s, seed=i) for i, (r, c, s) in
+            enumerate([(64, 96, 0.02), (3, 5, 0.05), (128, 64, 0.01), (1, 1, 1.0)])]
+    blk = df11.encode_multi(mats)
+    cat = df11.encode(np.concatenate([m.reshape(-1) for m in mats]))
+    for name in ("enc", "sm", "gaps", "block_start", "lut"):
+        assert np.array_equal(blk.host_array(name), cat.host_array(name)), name
+    assert blk.offsets == [0, 64 * 96, 64 * 96 + 15, 64 * 96 + 15 + 128 * 64, 64 * 96 + 15 + 128 * 64 + 1]
+
+
+def test_invalid_params_rejected():
+    w = workloads.normal_matrix(8, 8, 0.02, seed=0)
+    with pytest.raises(df11.DF11Error):
+        df11.encode(w, df11.Params(bytes_per_thread=4))
+    with pytest.raises(df11.DF11Error):
+        df11.encode(w, df11.Params(max_code_len=0))
+    full = workloads.adversarial("uniform_exponents")  # 256 symbols need >= 8 bits
+    with pytest.raises(df11.DF11Error):
+        df11.encode(full, df11.Params(max_code_len=7))
+
+
+# ------------------------------------------------ decode-table walk on CPU
+
+def _lut_fields(lut: np.ndarray):
+    hdr = struct.unpack_from("<6I", lut.tobytes(), 0)
+    magic, w1, w2, max_len, min_len, n_syms = hdr
+    lim = np.frombuffer(lut.tobytes(), dtype=np.uint64, count=33, offset=64)
+    offs = np.frombuffer(lut.tobytes(), dtype=np.uint32, count=33, offset=336)
+    symrot = lut[480:736]
+    clut = lut[768:768 + (1 << 14)]
+    slut = np.frombuffer(lut.tobytes(), dtype=np.uint32, count=1 << 12, offset=768 + (1 << 14))
+    return dict(magic=magic, w1=w1, w2=w2, max_len=max_len, lim=lim, offs=offs, symrot=symrot,
+                clut=clut, slut=slut)
+
+
+def _unrotate(r):
+    return ((r << 1) | (r >> 7)) & 0xFF
+
+
+def _walk(t):
+    """Decodes every thread's range with the product's tables, using the
+    kernel's rule: bits at/after the thread's end are ones; stop when the
+    remaining count reaches zero; zero entries fall back to the limits.
+    Returns (exponents in element order, per-thread counts)."""
+    f = _lut_fields(t.host_array("lut"))
+    assert f["magic"] == 0x31314644
+    enc = t.host_array("enc")
+    bits_all = np.unpackbits(enc)
+    gaps = _unpack_gaps(t.host_array("gaps"), t.n_blocks * 256 + 1) if t.n_blocks else np.zeros(1, np.uint8)
+    out = []
+    counts = []
+    for th in range(t.n_threads):
+        gap = int(gaps[th])
+        end = t.total_bits - 64 * th if th == t.n_threads - 1 else 64 + int(gaps[th + 1])
+        window = np.ones(96 + 64, dtype=np.uint8)
+        seg = bits_all[64 * th: 64 * th + 96]
+        window[: min(96, seg.size)] = seg
+        window[end:] = 1
+        pos, n1 = gap, 0
+        # pass 1 (count table)
+        while pos < end:
+            v = int("".join(map(str, window[pos:pos + f["w1"]])), 2)
+            e = int(f["clut"][v])
+            if e == 0:
+                x = int("".join(map(str, window[pos:pos + 32])), 2)
+                l = next(l for l in range(f["w1"] + 1, f["max_len"] + 1) if x < int(f["lim"][l]))
+                pos += l
+                n1 += 1
+            else:
+                pos += e & 15
+                n1 += e >> 4
+        assert pos == end
+        # pass 2 (symbol table)
+        pos, syms = gap, []
+        while pos < end:
+            v = int("".join(map(str, window[pos:pos + f["w2"]])), 2)
+            e = int(f["slut"][v])
+            if e == 0:
+                x = int("".join(map(str, window[pos:pos + 32])), 2)
+                l = next(l for l in range(f["w2"] + 1, f["max_len"] + 1) if x < int(f["lim"][l]))
+                syms.append(int(f["symrot"][((x >> (32 - l)) + int(f["offs"][l])) & 0xFFFFFFFF & 255]))
+                pos += l
+            else:
+                nc = (e >> 29) & 3
+                syms.extend([(e >> (8 * j)) & 0xFF for j in range(nc)])
+                pos += (e >> 24) & 31
+        assert pos == end and len(syms) == n1
+        out.extend(_unrotate(np.array(syms, dtype=np.uint32)).tolist())
+        counts.append(n1)
+    return np.array(out, dtype=np.uint32), np.array(counts)
+
+
+@pytest.mark.parametrize("name", ["neg_zero_and_nan", "two_values", "all_equal", "fibonacci_small",
+                                  "normal_small", "uniform_small", "long_codes"])
+def test_table_walk_reproduces_exponents(name):
+    rng = np.random.default_rng(9)
+    if name == "fibonacci_small":
+        w = workloads.adversarial("fibonacci_exponents")[:30_000]
+    elif name == "normal_small":
+        w = workloads.normal_matrix(100, 211, 0.02, seed=4).reshape(-1)
+    elif name == "uniform_small":
+        w = workloads.adversarial("uniform_exponents")[:6000]
+    elif name == "long_codes":
+        # exponents with geometric frequencies: long codes (> 14 bits) occur
+        e = np.minimum(rng.geometric(0.45, size=40_000), 30) + 90
+        w = ((e << 7) | rng.integers(0, 128, e.size)).astype(np.uint16)
+    else:
+        w = workloads.adversarial(name)[:20_000]
+    t = df11.encode(w)
+    expo, counts = _walk(t)
+    assert np.array_equal(expo, (w.reshape(-1) >> 7) & 0xFF)
+    bs = t.host_array("block_start")
+    per_block = np.add.reduceat(np.concatenate([counts, np.zeros(t.n_blocks * 256 - counts.size, int)]),
+                                np.arange(0, t.n_blocks * 256, 256)) if t.n_blocks else []
+    assert np.array_equal(np.diff(bs[: t.n_blocks + 1]), per_block)
+    if name == "long_codes":
+        assert t.code_len.max() > 14
