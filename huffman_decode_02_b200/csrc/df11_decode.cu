@@ -16,20 +16,29 @@
 //     decoded in one launch.
 //
 // B200 design (what differs from the pages' own kernel):
-//  * Persistent CTAs, one per SM (1024 threads = 4 groups of 256).  Each
-//    group decodes one format block (256 threads x 8 bytes) at a time and
-//    strides over the blocks; the decode tables are staged into shared
-//    memory once per CTA with one TMA bulk copy (cp.async.bulk, no
+//  * Persistent CTAs, one per SM (1024 threads = 8 groups of 128).  Each
+//    group decodes one format block (256 format threads x 8 bytes) at a
+//    time and strides over the blocks; the decode tables are staged into
+//    shared memory once per CTA with one TMA bulk copy (cp.async.bulk, no
 //    multicast).
-//  * Each thread holds its 8 bytes plus the next thread's first 4 bytes in
-//    a 96-bit shift register (three funnel shifts per step).  Bits at and
+//  * Every CUDA thread runs two format threads side by side (two
+//    independent decode chains in one loop): each lookup is a dependent
+//    shift -> index -> shared load chain, and two chains per thread hide
+//    its latency twice over.
+//  * Each chain holds its 8 bytes plus the next chain's first 4 bytes in a
+//    96-bit shift register (three funnel shifts per step).  Bits at and
 //    after the thread's last code end (known exactly from the next thread's
 //    gap) are set to 1: a run of ones shorter than the longest code is never
 //    a whole code of a canonical code, so a table lookup can never take a
 //    code that belongs to the next thread.
 //  * Pass 1 counts with a 14-bit count table (several codes per lookup);
-//    pass 2 decodes with a 12-bit table holding up to three symbols per
-//    entry.  Codes longer than the window fall back to canonical limits.
+//    one add per lookup updates both the code count and the bits taken,
+//    the entry's low bits are the shift amount, and a code longer than the
+//    window leaves the loop through its condition (flag bit), so the loop
+//    body is a lookup, an add, three funnel shifts and a compare.
+//  * Pass 2 decodes with a 12-bit table of up to four symbols per entry and
+//    stops on the code count pass 1 found.  Codes longer than the window
+//    fall back to canonical limits.
 //  * Warp shuffle scan + one cross-warp step (named barrier per group).
 //  * Exponents are kept rotated by one bit, so the merge with the
 //    sign/mantissa bytes is two bit-selects and two byte-permutes per four
@@ -55,6 +64,7 @@ constexpr uint32_t kSmemBytes = kLutBytes + kGroupsPerCta * kGroupBytes + 16u;  
 constexpr uint32_t kFull = 0xFFFFFFFFu;
 constexpr uint32_t kKernErrTimeout = 0x10u;  // table staging did not complete
 static_assert(kGroupBytes % 16 == 0, "group stride keeps 16-byte alignment");
+static_assert(kLutBytes % 16 == 0, "bulk copy size");
 static_assert(kSmemBytes <= 227u * 1024u, "fits one CTA's shared memory");
 
 struct DecodeArgs {
@@ -72,11 +82,6 @@ struct DecodeArgs {
 };
 
 // ----------------------------------------------------------------- PTX
-__device__ __forceinline__ uint2 ld_stream_u2(const void *p) {
-    uint2 r;
-    asm("ld.global.nc.L1::no_allocate.v2.u32 {%0, %1}, [%2];" : "=r"(r.x), "=r"(r.y) : "l"(p));
-    return r;
-}
 __device__ __forceinline__ uint4 ld_stream_u4(const void *p) {
     uint4 r;
     asm("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
@@ -88,8 +93,44 @@ __device__ __forceinline__ void st_u4(void *p, uint32_t a, uint32_t b, uint32_t 
     asm volatile("st.global.v4.b32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(a), "r"(b), "r"(c), "r"(d)
                  : "memory");
 }
+// Shared memory through 32-bit shared-window addresses.  Volatile keeps them
+// ordered with the barriers (also volatile asm).
+__device__ __forceinline__ uint32_t lds_u32(uint32_t a) {
+    uint32_t v;
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ uint32_t lds_u8(uint32_t a) {
+    uint32_t v;
+    asm volatile("ld.shared.u8 %0, [%1];" : "=r"(v) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ uint64_t lds_u64(uint32_t a) {
+    uint64_t v;
+    asm volatile("ld.shared.u64 %0, [%1];" : "=l"(v) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ uint2 lds_u2(uint32_t a) {
+    uint2 v;
+    asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ uint4 lds_u4(uint32_t a) {
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ void sts_u32(uint32_t a, uint32_t v) {
+    asm volatile("st.shared.u32 [%0], %1;" ::"r"(a), "r"(v) : "memory");
+}
+__device__ __forceinline__ void sts_zero16(uint32_t a) {
+    asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(a), "r"(0u) : "memory");
+}
+__device__ __forceinline__ void red_or(uint32_t a, uint32_t v) {
+    asm volatile("red.shared.or.b32 [%0], %1;" ::"r"(a), "r"(v) : "memory");
+}
 __device__ __forceinline__ void group_barrier(uint32_t group) {
-    asm volatile("bar.sync %0, %1;" ::"r"(group + 1u), "r"((uint32_t)kThreadsPerBlockFmt) : "memory");
+    asm volatile("bar.sync %0, %1;" ::"r"(group + 1u), "r"((uint32_t)kGroupThreads) : "memory");
 }
 __device__ __forceinline__ uint32_t bswap32(uint32_t x) { return __byte_perm(x, 0u, 0x0123u); }
 __device__ __forceinline__ uint32_t smem_addr(const void *p) {
@@ -114,9 +155,7 @@ __device__ __forceinline__ bool wait_tables(uint32_t bar) {
 
 // Bulk copy of the decode tables into shared memory (TMA engine, one
 // thread), completion tracked by an mbarrier that every thread waits on.
-__device__ __forceinline__ bool stage_tables(uint8_t *dst, const uint8_t *src, uint32_t bytes,
-                                             uint64_t *mbar) {
-    const uint32_t bar = smem_addr(mbar);
+__device__ __forceinline__ bool stage_tables(uint32_t dst, const uint8_t *src, uint32_t bytes, uint32_t bar) {
     if (threadIdx.x == 0) {
         asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar) : "memory");
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -126,57 +165,164 @@ __device__ __forceinline__ bool stage_tables(uint8_t *dst, const uint8_t *src, u
         asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
                      : "memory");
         asm volatile(
-            "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-                smem_addr(dst)),
+            "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
             "l"(src), "r"(bytes), "r"(bar)
             : "memory");
     }
     return wait_tables(bar);
 }
 
-// Length of a code longer than the table window, from the canonical limits:
-// the smallest l with window < lim[l].  0 if no code matches.
-__device__ __forceinline__ uint32_t long_code_length(uint32_t x, const uint64_t *lim, uint32_t from,
-                                                     uint32_t max_len) {
-    for (uint32_t l = from; l <= max_len; ++l)
-        if ((uint64_t)x < lim[l]) return l;
+// Length of a code longer than the table window, from the canonical limits
+// in shared memory: the smallest l with window < lim[l].  0 if none.
+__device__ __noinline__ uint32_t long_code_length(uint32_t x, uint32_t lim_addr, uint32_t from, uint32_t max_len) {
+    for (uint32_t l = from; l <= max_len; ++l) {
+        const uint64_t lim = lds_u64(lim_addr + 8u * l);
+        if ((uint64_t)x < lim) return l;
+    }
     return 0u;
 }
 
+// Shifts the 96-bit window left by n bits (n <= 32), filling with ones.
+__device__ __forceinline__ void shift_window_clamped(uint32_t &hi, uint32_t &lo, uint32_t &fl, uint32_t n) {
+    hi = __funnelshift_lc(lo, hi, n);
+    lo = __funnelshift_lc(fl, lo, n);
+    fl = __funnelshift_lc(kFull, fl, n);
+}
+
 struct BlockInputs {
-    uint32_t w0, w1, w2;   // this thread's 8 bytes and the next 4 (big-endian words)
-    uint32_t g_hi, g_lo;   // the two 32-bit gap words holding bits [5t, 5t + 10)
-    uint32_t s, e;         // block_start[b], block_start[b + 1]
+    uint4 v;              // 16 stream bytes: chain A's 8, then chain B's 8
+    uint32_t wn;          // lane 31 only: the next thread's first 4 bytes
+    uint32_t g_hi, g_lo;  // the two 32-bit gap words holding bits [5tA, 5tA + 15)
+    uint32_t s, e;        // block_start[b], block_start[b + 1]
 };
 
-__device__ __forceinline__ void load_block_inputs(const DecodeArgs &a, uint64_t blk, uint32_t gt,
+__device__ __forceinline__ void load_block_inputs(const DecodeArgs &a, uint64_t blk, uint32_t lt,
                                                   uint32_t lane, BlockInputs &in) {
-    const uint64_t t = blk * (uint64_t)kThreadsPerBlockFmt + gt;
-    const uint2 v = ld_stream_u2(a.enc + 8ull * t);
-    in.w0 = v.x;
-    in.w1 = v.y;
-    // the next thread's first word: from the neighbour lane, or a load for lane 31
-    in.w2 = (lane == 31u) ? __ldg(reinterpret_cast<const uint32_t *>(a.enc + 8ull * t + 8ull)) : 0u;
-    const uint64_t bit = 5ull * t;
-    const uint64_t word = bit >> 5;
+    const uint64_t tA = blk * (uint64_t)kThreadsPerBlockFmt + 2u * lt;
+    in.v = ld_stream_u4(a.enc + 8ull * tA);  // 16-byte aligned: tA is even
+    in.wn = (lane == 31u) ? __ldg(reinterpret_cast<const uint32_t *>(a.enc + 8ull * tA + 16ull)) : 0u;
+    const uint64_t word = (5ull * tA) >> 5;
     in.g_hi = __ldg(a.gaps32 + word);
     in.g_lo = __ldg(a.gaps32 + word + 1);
     in.s = __ldg(a.bstart + blk);
     in.e = __ldg(a.bstart + blk + 1);
 }
 
+// Merges 16 rotated exponents with their 16 sign/mantissa bytes into 16
+// BF16 words (8 u32): per 4 weights two bit-selects and two byte-permutes.
+__device__ __forceinline__ void merge16(const uint4 smv, const uint4 ex, uint32_t o[8]) {
+    const uint32_t S[4] = {smv.x, smv.y, smv.z, smv.w};
+    const uint32_t R[4] = {ex.x, ex.y, ex.z, ex.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const uint32_t hi8 = (S[q] & 0x80808080u) | (R[q] & 0x7F7F7F7Fu);
+        const uint32_t lo8 = (R[q] & 0x80808080u) | (S[q] & 0x7F7F7F7Fu);
+        o[2 * q] = __byte_perm(lo8, hi8, 0x5140u);
+        o[2 * q + 1] = __byte_perm(lo8, hi8, 0x7362u);
+    }
+}
+
+// The chunks holding the block's first and last elements, by one warp:
+// lanes 0..15 take the first chunk, lanes 16..31 the last one, one element
+// each (only elements inside [s, e) are written).
+__device__ __forceinline__ void merge_edges(const uint8_t *sm, uint16_t *out, uint32_t sb, uint32_t base,
+                                            uint32_t c_full, uint32_t span, uint32_t s, uint32_t e,
+                                            uint32_t lane) {
+    const bool head = s != base;
+    const bool tail = (span & 15u) != 0u && !(head && c_full == 0u);
+    const uint32_t c = (lane < 16u) ? 0u : c_full;
+    const bool mine = (lane < 16u) ? head : tail;
+    const uint32_t g = base + 16u * c + (lane & 15u);
+    if (mine && g >= s && g < e) {
+        const uint32_t sm8 = __ldg(sm + g);
+        const uint32_t r = lds_u8(sb + (g - base));
+        // r = rotated exponent: high byte (s & 0x80) | (r & 0x7F), low byte (r & 0x80) | (s & 0x7F)
+        const uint32_t hi8 = (sm8 & 0x80u) | (r & 0x7Fu);
+        const uint32_t lo8 = (r & 0x80u) | (sm8 & 0x7Fu);
+        out[g] = (uint16_t)(lo8 | (hi8 << 8));
+    }
+}
+
+// One decode chain: the 96-bit window (hi, lo, fl) of a format thread, the
+// bits it must consume (rem0), and a running accumulator.
+struct Chain {
+    uint32_t hi, lo, fl;
+    int32_t rem0;
+};
+
+// Builds a chain from its three big-endian stream words, its first code's
+// bit offset and the end of its last code; bits at/after the end become 1.
+__device__ __forceinline__ Chain make_chain(uint32_t x0, uint32_t x1, uint32_t x2, uint32_t gap, int32_t end,
+                                            uint32_t &err) {
+    Chain c;
+    int32_t rem0 = end - (int32_t)gap;
+    if (rem0 < 0) {
+        err |= DF11_KERR_OVERRUN;
+        rem0 = 0;
+        end = (int32_t)gap;
+    }
+    x0 |= __funnelshift_rc(kFull, 0u, (uint32_t)max(end, 0));
+    x1 |= __funnelshift_rc(kFull, 0u, (uint32_t)max(end - 32, 0));
+    x2 |= __funnelshift_rc(kFull, 0u, (uint32_t)max(end - 64, 0));
+    c.hi = __funnelshift_lc(x1, x0, gap);
+    c.lo = __funnelshift_lc(x2, x1, gap);
+    c.fl = __funnelshift_lc(kFull, x2, gap);
+    c.rem0 = rem0;
+    return c;
+}
+
+// Long-code step of the count pass for one chain whose accumulator carries
+// the escape flag.  Returns true if the chain still has bits to consume.
+__device__ __forceinline__ bool count_long_code(uint32_t &acc, uint32_t lim, uint32_t &hi, uint32_t &lo,
+                                                uint32_t &fl, uint32_t s_lim, uint32_t from, uint32_t max_len,
+                                                uint32_t &err) {
+    acc -= kEscape;
+    const uint32_t l = long_code_length(hi, s_lim, from, max_len);
+    if (l == 0u) {
+        err |= DF11_KERR_BAD_CODE;
+        acc = lim;  // stop this chain
+        return false;
+    }
+    acc += (l << 24) | (1u << 8);
+    shift_window_clamped(hi, lo, fl, l);
+    return acc < lim;
+}
+
+// Long-code step of the decoding pass: writes the symbol, advances.
+__device__ __forceinline__ bool decode_long_code(uint32_t &pacc, uint32_t pend, uint32_t &hi, uint32_t &lo,
+                                                 uint32_t &fl, uint32_t sb, uint32_t s_lim, uint32_t s_offs,
+                                                 uint32_t s_symrot, uint32_t from, uint32_t max_len) {
+    pacc -= kEscape;
+    const uint32_t l = long_code_length(hi, s_lim, from, max_len);
+    if (l == 0u) {  // reported by the count pass
+        pacc = pend;
+        return false;
+    }
+    const uint32_t idx = (hi >> (32u - l)) + lds_u32(s_offs + 4u * l);
+    const uint32_t p = pacc >> 8;
+    red_or(sb + (p & ~3u), lds_u8(s_symrot + (idx & 255u)) << (8u * (p & 3u)));
+    pacc += 1u << 8;
+    shift_window_clamped(hi, lo, fl, l);
+    return pacc < pend;
+}
+
 __global__ void __launch_bounds__(kCtaThreads, 1) df11_decode_kernel(const DecodeArgs a) {
     extern __shared__ __align__(128) uint8_t smem[];
-    uint8_t *s_lut = smem;
-    uint64_t *s_mbar = reinterpret_cast<uint64_t *>(smem + kLutBytes + kGroupsPerCta * kGroupBytes);
+    const uint32_t s_base = smem_addr(smem);
+    const uint32_t s_lim = s_base + kOffLim;
+    const uint32_t s_offs = s_base + kOffOffs;
+    const uint32_t s_symrot = s_base + kOffSymRot;
+    const uint32_t s_clut = s_base + kOffCountLut;
+    const uint32_t s_slut = s_base + kOffSymLut;
+    const uint32_t s_mbar = s_base + kLutBytes + kGroupsPerCta * kGroupBytes;
 
     const uint32_t tid = threadIdx.x;
-    const uint32_t group = tid / kThreadsPerBlockFmt;
-    const uint32_t gt = tid % kThreadsPerBlockFmt;  // thread within the format block
+    const uint32_t group = tid / kGroupThreads;
+    const uint32_t lt = tid % kGroupThreads;  // thread within the group
     const uint32_t lane = tid & 31u;
-    const uint32_t warp = gt >> 5;                   // warp within the group
-    uint8_t *sbuf = smem + kLutBytes + group * kGroupBytes;
-    uint32_t *wtot = reinterpret_cast<uint32_t *>(sbuf + kSbufBytes);
+    const uint32_t warp = lt >> 5;            // warp within the group
+    const uint32_t sb = s_base + kLutBytes + group * kGroupBytes;  // this group's exponent buffer
+    const uint32_t wtot = sb + kSbufBytes;                          // per-warp totals
     uint32_t my_err = 0;
 
     const uint64_t stride = (uint64_t)gridDim.x * kGroupsPerCta;
@@ -184,46 +330,42 @@ __global__ void __launch_bounds__(kCtaThreads, 1) df11_decode_kernel(const Decod
 
     // Prefetch the first block's inputs while the tables stream in.
     BlockInputs cur{};
-    if (blk < a.n_blocks) load_block_inputs(a, blk, gt, lane, cur);
+    if (blk < a.n_blocks) load_block_inputs(a, blk, lt, lane, cur);
 
-    const bool staged = stage_tables(s_lut, a.lut, kLutBytes, s_mbar);
+    const bool staged = stage_tables(s_base, a.lut, kLutBytes, s_mbar);
     if (__syncthreads_or(!staged)) {
         // Uniform over the CTA.  One more bounded wait so no copy is left in
         // flight into this CTA's shared memory, then report and stop.
         if (tid == 0) {
-            wait_tables(smem_addr(s_mbar));
+            wait_tables(s_mbar);
             if (a.err) atomicOr(a.err, kKernErrTimeout);
         }
         __syncthreads();
         return;
     }
 
-    const LutHeader *hdr = reinterpret_cast<const LutHeader *>(s_lut + kOffHeader);
-    const uint64_t *s_lim = reinterpret_cast<const uint64_t *>(s_lut + kOffLim);
-    const uint32_t *s_offs = reinterpret_cast<const uint32_t *>(s_lut + kOffOffs);
-    const uint8_t *s_symrot = s_lut + kOffSymRot;
-    const uint8_t *s_clut = s_lut + kOffCountLut;
-    const uint32_t *s_slut = reinterpret_cast<const uint32_t *>(s_lut + kOffSymLut);
+    const LutHeader *hdr = reinterpret_cast<const LutHeader *>(smem + kOffHeader);
     const uint32_t w1 = hdr->w1, w2 = hdr->w2, max_len = hdr->max_len;
     if (hdr->magic != kMagic || w1 < 1u || w1 > (uint32_t)kW1Max || w2 < 1u || w2 > (uint32_t)kW2Max ||
         max_len > 32u) {
         if (tid == 0 && a.err) atomicOr(a.err, DF11_KERR_BAD_CODE);
         return;  // uniform over the CTA: nothing was written yet
     }
-    // Every non-zero table entry must take at least one bit and stay inside
-    // its window, so each decode step makes progress: the per-thread loops
-    // then end after at most 95 steps whatever the stream holds.
+    // Every table entry must be the escape flag or take 1..W bits for
+    // 1..(bits) codes, so each lookup makes progress: the decode loops then
+    // end after at most 95 lookups plus 95 long codes whatever the stream.
     {
         bool bad = false;
         for (uint32_t i = tid; i < (1u << w1); i += kCtaThreads) {
-            const uint32_t ent = s_clut[i];
-            bad |= ent != 0u && (count_entry_bits(ent) == 0u || count_entry_bits(ent) > w1 ||
-                                 count_entry_codes(ent) == 0u);
+            const uint32_t ent = lds_u32(s_clut + 4u * i);
+            const uint32_t nb = count_entry_bits(ent), nc = count_entry_codes(ent);
+            bad |= ent != kEscape && (ent != count_entry(nb, nc) || nb == 0u || nb > w1 || nc == 0u || nc > nb);
         }
         for (uint32_t i = tid; i < (1u << w2); i += kCtaThreads) {
-            const uint32_t ent = s_slut[i];
-            bad |= ent != 0u && (sym_entry_bits(ent) == 0u || sym_entry_bits(ent) > w2 ||
-                                 sym_entry_codes(ent) == 0u);
+            const uint2 ent = lds_u2(s_slut + 8u * i);
+            const uint32_t nb = sym_entry_bits(ent.y), nc = sym_entry_codes(ent.y);
+            bad |= ent.y != kEscape && (ent.y != sym_entry_meta(nb, nc) || nb == 0u || nb > w2 || nc == 0u ||
+                                        nc > (uint32_t)kSymsPerEntry || nc > nb);
         }
         if (__syncthreads_or(bad)) {
             if (tid == 0 && a.err) atomicOr(a.err, DF11_KERR_BAD_CODE);
@@ -235,156 +377,163 @@ __global__ void __launch_bounds__(kCtaThreads, 1) df11_decode_kernel(const Decod
     for (; blk < a.n_blocks; blk += stride) {
         const BlockInputs in = cur;
         const uint64_t nxt = blk + stride;
-        if (nxt < a.n_blocks) load_block_inputs(a, nxt, gt, lane, cur);
+        if (nxt < a.n_blocks) load_block_inputs(a, nxt, lt, lane, cur);
 
-        const uint64_t t = blk * (uint64_t)kThreadsPerBlockFmt + gt;
+        const uint64_t tA = blk * (uint64_t)kThreadsPerBlockFmt + 2u * lt;
         const uint32_t s = in.s, e = in.e;
         const uint32_t base = s & ~15u;  // first 16-element chunk of the block's output
         const bool range_ok = (e >= s) && ((uint64_t)e <= a.n_elems) && (e - s <= (uint32_t)kMaxCodesPerBlock);
-        const uint32_t n_chunks = range_ok ? (e - base + 15u) >> 4 : 0u;
+        // chunks [c_lo, c_full) lie wholly inside [s, e)
+        const uint32_t span = range_ok ? e - base : 0u;
+        const uint32_t c_lo = (s != base) ? 1u : 0u;
+        const uint32_t c_full = span >> 4;
+        const uint32_t c0 = c_lo + lt;
+        uint4 smv0 = make_uint4(0, 0, 0, 0);
+        if (c0 < c_full) smv0 = ld_stream_u4(a.sm + (uint64_t)base + 16ull * c0);
 
-        // First two sign/mantissa vectors this thread will merge.
-        uint4 smv0 = make_uint4(0, 0, 0, 0), smv1 = make_uint4(0, 0, 0, 0);
-        if (gt < n_chunks) smv0 = ld_stream_u4(a.sm + (uint64_t)base + 16ull * gt);
-        if (gt + kThreadsPerBlockFmt < n_chunks)
-            smv1 = ld_stream_u4(a.sm + (uint64_t)base + 16ull * (gt + kThreadsPerBlockFmt));
+        // ---- the two chains: format threads tA and tA + 1
+        // gaps are an MSB-first bit string: bits [5tA, 5tA + 15) hold the
+        // gaps of tA, tA + 1 and tA + 2
+        const uint32_t gb = __funnelshift_l(bswap32(in.g_lo), bswap32(in.g_hi), (uint32_t)((5ull * tA) & 31u));
+        uint32_t gapA = gb >> 27, gapB = (gb >> 22) & 31u;
+        const uint32_t gapC = (gb >> 17) & 31u;
+        int32_t endA, endB;
+        if (tA >= a.n_threads) { gapA = 0; endA = 0; }
+        else if (tA + 1 == a.n_threads) endA = (int32_t)(a.total_bits - 64ull * tA);
+        else endA = 64 + (int32_t)gapB;
+        if (tA + 1 >= a.n_threads) { gapB = 0; endB = 0; }
+        else if (tA + 2 == a.n_threads) endB = (int32_t)(a.total_bits - 64ull * (tA + 1));
+        else endB = 64 + (int32_t)gapC;
+        uint32_t nextw = __shfl_down_sync(kFull, in.v.x, 1);
+        if (lane == 31u) nextw = in.wn;
+        const Chain A = make_chain(bswap32(in.v.x), bswap32(in.v.y), bswap32(in.v.z), gapA, endA, my_err);
+        const Chain B = make_chain(bswap32(in.v.z), bswap32(in.v.w), bswap32(nextw), gapB, endB, my_err);
 
-        // ---- this thread's bits: [gap, end) of its 96-bit window
-        uint32_t w0 = bswap32(in.w0), w1v = bswap32(in.w1);
-        uint32_t w2v = __shfl_down_sync(kFull, in.w0, 1);
-        if (lane == 31u) w2v = in.w2;
-        w2v = bswap32(w2v);
-        // gaps are an MSB-first bit string: bits [5t, 5t + 10) hold this
-        // thread's gap and the next thread's
-        const uint32_t gb = __funnelshift_l(bswap32(in.g_lo), bswap32(in.g_hi), (uint32_t)((5ull * t) & 31u));
-        uint32_t gap = gb >> 27;
-        const uint32_t gap_next = (gb >> 22) & 31u;
-        int32_t end;
-        if (t >= a.n_threads) { gap = 0; end = 0; }
-        else if (t + 1 == a.n_threads) end = (int32_t)(a.total_bits - 64ull * t);
-        else end = 64 + (int32_t)gap_next;
-        int32_t rem0 = end - (int32_t)gap;
-        if (rem0 < 0) { my_err |= DF11_KERR_OVERRUN; rem0 = 0; }
-        // set every bit at or after `end` to 1
+        // ---- pass 1: count the codes of both chains
+        uint32_t cA, cB;
         {
-            const int32_t v0 = min(max(end, 0), 32), v1 = min(max(end - 32, 0), 32),
-                          v2 = min(max(end - 64, 0), 32);
-            w0 |= (v0 >= 32) ? 0u : (kFull >> v0);
-            w1v |= (v1 >= 32) ? 0u : (kFull >> v1);
-            w2v |= (v2 >= 32) ? 0u : (kFull >> v2);
-        }
-        // 96-bit window starting at the first code
-        const uint32_t r_hi = __funnelshift_lc(w1v, w0, gap);
-        const uint32_t r_lo = __funnelshift_lc(w2v, w1v, gap);
-        const uint32_t r_fl = __funnelshift_lc(kFull, w2v, gap);
-
-        // ---- pass 1: count the codes
-        uint32_t cnt = 0;
-        {
-            uint32_t hi = r_hi, lo = r_lo, fl = r_fl;
-            int32_t rem = rem0;
-            while (rem > 0) {
-                const uint32_t ent = s_clut[hi >> sh1];
-                uint32_t nb = count_entry_bits(ent);
-                uint32_t nc = count_entry_codes(ent);
-                if (ent == 0u) {
-                    nb = long_code_length(hi, s_lim, w1 + 1u, max_len);
-                    nc = 1u;
-                    if (nb == 0u) { my_err |= DF11_KERR_BAD_CODE; break; }
+            uint32_t hA = A.hi, lA = A.lo, fA = A.fl, hB = B.hi, lB = B.lo, fB = B.fl;
+            uint32_t aA = 0, aB = 0;
+            const uint32_t limA = (uint32_t)A.rem0 << 24, limB = (uint32_t)B.rem0 << 24;
+            for (;;) {
+                while ((aA < limA) | (aB < limB)) {
+                    uint32_t eA = lds_u32(s_clut + ((hA >> sh1) << 2));
+                    uint32_t eB = lds_u32(s_clut + ((hB >> sh1) << 2));
+                    eA = (aA < limA) ? eA : 0u;
+                    eB = (aB < limB) ? eB : 0u;
+                    aA += eA;
+                    aB += eB;
+                    hA = __funnelshift_l(lA, hA, eA);
+                    lA = __funnelshift_l(fA, lA, eA);
+                    fA = __funnelshift_l(kFull, fA, eA);
+                    hB = __funnelshift_l(lB, hB, eB);
+                    lB = __funnelshift_l(fB, lB, eB);
+                    fB = __funnelshift_l(kFull, fB, eB);
                 }
-                cnt += nc;
-                rem -= (int32_t)nb;
-                hi = __funnelshift_lc(lo, hi, nb);
-                lo = __funnelshift_lc(fl, lo, nb);
-                fl = __funnelshift_lc(kFull, fl, nb);
+                bool more = false;
+                if (aA >= kEscape) more |= count_long_code(aA, limA, hA, lA, fA, s_lim, w1 + 1u, max_len, my_err);
+                if (aB >= kEscape) more |= count_long_code(aB, limB, hB, lB, fB, s_lim, w1 + 1u, max_len, my_err);
+                if (!more) break;
             }
-            if (rem < 0) my_err |= DF11_KERR_OVERRUN;
+            cA = (aA >> 8) & 0xFFFFu;
+            cB = (aB >> 8) & 0xFFFFu;
+            if ((aA >> 24) != (uint32_t)A.rem0 || (aB >> 24) != (uint32_t)B.rem0) my_err |= DF11_KERR_OVERRUN;
         }
 
-        // ---- block scan: warp inclusive scan, then across the 8 warps
+        // ---- clear the exponent buffer span this block uses (the decoding
+        // pass ORs symbols into it); the scan barrier orders this before it
+        for (uint32_t c = lt; c < ((span + 15u) >> 4) + 1u; c += kGroupThreads) sts_zero16(sb + 16u * c);
+
+        // ---- block scan: warp inclusive scan, then across the group's warps
+        const uint32_t cnt = cA + cB;
         uint32_t incl = cnt;
 #pragma unroll
         for (uint32_t d = 1; d < 32; d <<= 1) {
             const uint32_t v = __shfl_up_sync(kFull, incl, d);
             if (lane >= d) incl += v;
         }
-        if (lane == 31u) wtot[warp] = incl;
+        constexpr uint32_t kWarps = kGroupThreads / 32;
+        if (lane == 31u) sts_u32(wtot + 4u * warp, incl);
         group_barrier(group);
-        uint32_t wpre = 0, total = 0;
-        {
-            const uint4 ta = *reinterpret_cast<const uint4 *>(wtot);
-            const uint4 tb = *reinterpret_cast<const uint4 *>(wtot + 4);
-            const uint32_t tw[8] = {ta.x, ta.y, ta.z, ta.w, tb.x, tb.y, tb.z, tb.w};
+        uint32_t wsum = (lane < kWarps) ? lds_u32(wtot + 4u * lane) : 0u;
 #pragma unroll
-            for (uint32_t w = 0; w < 8; ++w) {
-                wpre += (w < warp) ? tw[w] : 0u;
-                total += tw[w];
-            }
+        for (uint32_t d = 1; d < kWarps; d <<= 1) {
+            const uint32_t v = __shfl_up_sync(kFull, wsum, d);
+            if (lane >= d) wsum += v;
         }
+        const uint32_t total = __shfl_sync(kFull, wsum, kWarps - 1u);
+        const uint32_t wpre = __shfl_sync(kFull, wsum, (warp + kWarps - 1u) % kWarps) * (warp != 0u ? 1u : 0u);
         const bool ok = range_ok && (total == e - s);
-        if (!ok && gt == 0) my_err |= range_ok ? DF11_KERR_COUNT_MISMATCH : DF11_KERR_BAD_BLOCK;
+        if (!ok && lt == 0) my_err |= range_ok ? DF11_KERR_COUNT_MISMATCH : DF11_KERR_BAD_BLOCK;
 
-        // ---- pass 2: decode again, write rotated exponents to the buffer
+        // ---- pass 2: decode both chains again into the exponent buffer
         if (ok) {
-            uint32_t hi = r_hi, lo = r_lo, fl = r_fl;
-            int32_t rem = rem0;
-            uint32_t p = (s - base) + wpre + incl - cnt;  // buffer index of this thread's first code
-            while (rem > 0) {
-                p = min(p, kSbufBytes - 3u);  // keeps a corrupt table inside this group's buffer
-                const uint32_t ent = s_slut[hi >> sh2];
-                uint32_t nb, nc;
-                if (ent != 0u) {
-                    nb = sym_entry_bits(ent);
-                    nc = sym_entry_codes(ent);
-                    sbuf[p] = (uint8_t)ent;
-                    if (nc > 1u) sbuf[p + 1] = (uint8_t)(ent >> 8);
-                    if (nc > 2u) sbuf[p + 2] = (uint8_t)(ent >> 16);
-                } else {
-                    nb = long_code_length(hi, s_lim, w2 + 1u, max_len);
-                    if (nb == 0u) break;  // reported by pass 1
-                    nc = 1u;
-                    sbuf[p] = s_symrot[((hi >> (32u - nb)) + s_offs[nb]) & 255u];
+            uint32_t hA = A.hi, lA = A.lo, fA = A.fl, hB = B.hi, lB = B.lo, fB = B.fl;
+            const uint32_t startA = (s - base) + wpre + incl - cnt;  // buffer index of A's first code
+            const uint32_t startB = startA + cA;
+            uint32_t pA = startA << 8, pB = startB << 8;
+            const uint32_t endPA = (startA + cA) << 8, endPB = (startB + cB) << 8;
+            for (;;) {
+                while ((pA < endPA) | (pB < endPB)) {
+                    const uint2 eA = lds_u2(s_slut + ((hA >> sh2) << 3));
+                    const uint2 eB = lds_u2(s_slut + ((hB >> sh2) << 3));
+                    const bool actA = pA < endPA, actB = pB < endPB;
+                    const int32_t mA = actA ? (int32_t)eA.y : 0;
+                    const int32_t mB = actB ? (int32_t)eB.y : 0;
+                    // up to four symbol bytes land in the word holding byte p
+                    // and the next one; unused symbol bytes are zero
+                    const uint32_t bA = pA >> 8, bB = pB >> 8;
+                    const uint32_t shA = (bA & 3u) << 3, shB = (bB & 3u) << 3;
+                    const uint32_t wA = sb + (bA & ~3u), wB = sb + (bB & ~3u);
+                    if (actA) {
+                        red_or(wA, eA.x << shA);
+                        if (shA) red_or(wA + 4u, __funnelshift_l(eA.x, 0u, shA));
+                    }
+                    if (actB) {
+                        red_or(wB, eB.x << shB);
+                        if (shB) red_or(wB + 4u, __funnelshift_l(eB.x, 0u, shB));
+                    }
+                    pA += (uint32_t)mA;
+                    pB += (uint32_t)mB;
+                    hA = __funnelshift_l(lA, hA, (uint32_t)mA);
+                    lA = __funnelshift_l(fA, lA, (uint32_t)mA);
+                    fA = __funnelshift_l(kFull, fA, (uint32_t)mA);
+                    hB = __funnelshift_l(lB, hB, (uint32_t)mB);
+                    lB = __funnelshift_l(fB, lB, (uint32_t)mB);
+                    fB = __funnelshift_l(kFull, fB, (uint32_t)mB);
                 }
-                p += nc;
-                rem -= (int32_t)nb;
-                hi = __funnelshift_lc(lo, hi, nb);
-                lo = __funnelshift_lc(fl, lo, nb);
-                fl = __funnelshift_lc(kFull, fl, nb);
+                bool more = false;
+                if (pA >= kEscape)
+                    more |= decode_long_code(pA, endPA, hA, lA, fA, sb, s_lim, s_offs, s_symrot, w2 + 1u, max_len);
+                if (pB >= kEscape)
+                    more |= decode_long_code(pB, endPB, hB, lB, fB, sb, s_lim, s_offs, s_symrot, w2 + 1u, max_len);
+                if (!more) break;
             }
         }
         group_barrier(group);
 
         // ---- merge with sign/mantissa and store, 16 weights per step
         if (ok) {
-            for (uint32_t c = gt; c < n_chunks; c += kThreadsPerBlockFmt) {
-                uint4 smv;
-                if (c == gt) smv = smv0;
-                else if (c == gt + kThreadsPerBlockFmt) smv = smv1;
-                else smv = ld_stream_u4(a.sm + (uint64_t)base + 16ull * c);
-                const uint4 ex = *reinterpret_cast<const uint4 *>(sbuf + 16u * c);
-                const uint32_t S[4] = {smv.x, smv.y, smv.z, smv.w};
-                const uint32_t R[4] = {ex.x, ex.y, ex.z, ex.w};
-                uint32_t o[8];
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const uint32_t hi8 = (S[q] & 0x80808080u) | (R[q] & 0x7F7F7F7Fu);
-                    const uint32_t lo8 = (R[q] & 0x80808080u) | (S[q] & 0x7F7F7F7Fu);
-                    o[2 * q] = __byte_perm(lo8, hi8, 0x5140u);
-                    o[2 * q + 1] = __byte_perm(lo8, hi8, 0x7362u);
-                }
-                const uint32_t g0 = base + 16u * c;
-                uint16_t *dst = a.out + g0;
-                if (g0 >= s && g0 + 16u <= e) {
+            if (c0 < c_full) {
+                const uint8_t *smp = a.sm + (uint64_t)base + 16ull * c0;
+                uint16_t *dst = a.out + (uint64_t)base + 16ull * c0;
+                uint32_t ex_addr = sb + 16u * c0;
+                uint4 smv = smv0;
+                for (uint32_t c = c0;;) {
+                    const uint4 ex = lds_u4(ex_addr);
+                    uint32_t o[8];
+                    merge16(smv, ex, o);
                     st_u4(dst, o[0], o[1], o[2], o[3]);
                     st_u4(dst + 8, o[4], o[5], o[6], o[7]);
-                } else {
-#pragma unroll
-                    for (uint32_t j = 0; j < 16; ++j) {
-                        const uint32_t g = g0 + j;
-                        if (g >= s && g < e) dst[j] = (uint16_t)(o[j >> 1] >> (16u * (j & 1u)));
-                    }
+                    c += kGroupThreads;
+                    if (c >= c_full) break;
+                    smp += 16u * kGroupThreads;
+                    dst += 16u * kGroupThreads;
+                    ex_addr += 16u * kGroupThreads;
+                    smv = ld_stream_u4(smp);
                 }
             }
+            if (warp == 0) merge_edges(a.sm, a.out, sb, base, c_full, span, s, e, lane);
         }
         group_barrier(group);
     }
@@ -418,11 +567,11 @@ df11_status prepare_device(int *sm_count) {
 bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
 
 df11_status launch_decode(const df11_tensor *t, uint16_t *out, uint32_t *err_word, void *stream) {
-    if (!t || !out) return DF11_ERR_INVALID_ARG;
+    if (!t) return DF11_ERR_INVALID_ARG;
     df11_status st = df11_validate(t);
     if (st != DF11_OK) return st;
-    if (t->n_elems == 0) return DF11_OK;
-    if (!t->enc || !t->sm || !t->gaps || !t->block_start || !t->lut) return DF11_ERR_INVALID_ARG;
+    if (t->n_elems == 0) return DF11_OK;  // nothing to write; out may be NULL
+    if (!out || !t->enc || !t->sm || !t->gaps || !t->block_start || !t->lut) return DF11_ERR_INVALID_ARG;
     if (!aligned16(t->enc) || !aligned16(t->sm) || !aligned16(t->gaps) || !aligned16(t->lut) ||
         !aligned16(t->block_start) || !aligned16(out))
         return DF11_ERR_INVALID_ARG;

@@ -282,7 +282,7 @@ void build_luts(const uint8_t len[256], uint8_t *lut) {
         return sym_rot[i & 255];
     };
     // count LUT
-    uint8_t *clut = lut + df11::kOffCountLut;
+    uint32_t *clut = reinterpret_cast<uint32_t *>(lut + df11::kOffCountLut);
     for (uint32_t v = 0; v < (1u << h.w1); ++v) {
         const uint32_t x = v << (32 - h.w1);
         uint32_t pos = 0, n = 0;
@@ -292,7 +292,7 @@ void build_luts(const uint8_t len[256], uint8_t *lut) {
             pos += (uint32_t)l;
             ++n;
         }
-        clut[v] = (uint8_t)(n ? (pos | (n << 4)) : 0);
+        clut[v] = n ? df11::count_entry(pos, n) : df11::kEscape;
     }
     // symbol LUT
     uint32_t *slut = reinterpret_cast<uint32_t *>(lut + df11::kOffSymLut);
@@ -306,7 +306,8 @@ void build_luts(const uint8_t len[256], uint8_t *lut) {
             pos += (uint32_t)l;
             ++n;
         }
-        slut[v] = n ? (syms | (pos << 24) | (n << 29)) : 0u;
+        slut[2 * v] = n ? syms : 0u;
+        slut[2 * v + 1] = n ? df11::sym_entry_meta(pos, n) : df11::kEscape;
     }
 }
 

@@ -143,13 +143,13 @@ def test_invalid_params_rejected():
 # ------------------------------------------------ decode-table walk on CPU
 
 def _lut_fields(lut: np.ndarray):
-    hdr = struct.unpack_from("<6I", lut.tobytes(), 0)
-    magic, w1, w2, max_len, min_len, n_syms = hdr
-    lim = np.frombuffer(lut.tobytes(), dtype=np.uint64, count=33, offset=64)
-    offs = np.frombuffer(lut.tobytes(), dtype=np.uint32, count=33, offset=336)
+    b = lut.tobytes()
+    magic, w1, w2, max_len, min_len, n_syms = struct.unpack_from("<6I", b, 0)
+    lim = np.frombuffer(b, dtype=np.uint64, count=33, offset=64)
+    offs = np.frombuffer(b, dtype=np.uint32, count=33, offset=336)
     symrot = lut[480:736]
-    clut = lut[768:768 + (1 << 14)]
-    slut = np.frombuffer(lut.tobytes(), dtype=np.uint32, count=1 << 12, offset=768 + (1 << 14))
+    clut = np.frombuffer(b, dtype=np.uint32, count=1 << 13, offset=768)
+    slut = np.frombuffer(b, dtype=np.uint32, count=2 << 12, offset=768 + 4 * (1 << 13)).reshape(-1, 2)
     return dict(magic=magic, w1=w1, w2=w2, max_len=max_len, lim=lim, offs=offs, symrot=symrot,
                 clut=clut, slut=slut)
 
@@ -158,18 +158,29 @@ def _unrotate(r):
     return ((r << 1) | (r >> 7)) & 0xFF
 
 
+ESC = 0x80000000
+
+
 def _walk(t):
     """Decodes every thread's range with the product's tables, using the
-    kernel's rule: bits at/after the thread's end are ones; stop when the
-    remaining count reaches zero; zero entries fall back to the limits.
+    kernel's rules: bits at/after the thread's end are ones; the count pass
+    adds whole entries into one accumulator (bits taken in the top byte,
+    codes in bits 8..23) and leaves its loop on the escape flag or once the
+    bits reach the thread's span; the decode pass stops on the code count.
     Returns (exponents in element order, per-thread counts)."""
     f = _lut_fields(t.host_array("lut"))
-    assert f["magic"] == 0x31314644
+    assert f["magic"] == 0x32314644
     enc = t.host_array("enc")
     bits_all = np.unpackbits(enc)
     gaps = _unpack_gaps(t.host_array("gaps"), t.n_blocks * 256 + 1) if t.n_blocks else np.zeros(1, np.uint8)
-    out = []
-    counts = []
+
+    def win(window, pos, n):
+        return int("".join(map(str, window[pos:pos + n])), 2)
+
+    def long_len(x, lo):
+        return next(l for l in range(lo, f["max_len"] + 1) if x < int(f["lim"][l]))
+
+    out, counts = [], []
     for th in range(t.n_threads):
         gap = int(gaps[th])
         end = t.total_bits - 64 * th if th == t.n_threads - 1 else 64 + int(gaps[th + 1])
@@ -177,34 +188,36 @@ def _walk(t):
         seg = bits_all[64 * th: 64 * th + 96]
         window[: min(96, seg.size)] = seg
         window[end:] = 1
-        pos, n1 = gap, 0
+        rem0 = end - gap
         # pass 1 (count table)
-        while pos < end:
-            v = int("".join(map(str, window[pos:pos + f["w1"]])), 2)
-            e = int(f["clut"][v])
-            if e == 0:
-                x = int("".join(map(str, window[pos:pos + 32])), 2)
-                l = next(l for l in range(f["w1"] + 1, f["max_len"] + 1) if x < int(f["lim"][l]))
-                pos += l
-                n1 += 1
-            else:
-                pos += e & 15
-                n1 += e >> 4
-        assert pos == end
-        # pass 2 (symbol table)
+        pos, acc, lim = gap, 0, rem0 << 24
+        while True:
+            while acc < lim:
+                e = int(f["clut"][win(window, pos, f["w1"])])
+                acc += e
+                pos += e & 31
+            if acc < ESC:
+                break
+            acc -= ESC
+            l = long_len(win(window, pos, 32), f["w1"] + 1)
+            acc += (l << 24) | (1 << 8)
+            pos += l
+        n1 = (acc >> 8) & 0xFFFF
+        assert pos == end and (acc >> 24) == rem0
+        # pass 2 (symbol table), stops after n1 codes
         pos, syms = gap, []
-        while pos < end:
-            v = int("".join(map(str, window[pos:pos + f["w2"]])), 2)
-            e = int(f["slut"][v])
-            if e == 0:
-                x = int("".join(map(str, window[pos:pos + 32])), 2)
-                l = next(l for l in range(f["w2"] + 1, f["max_len"] + 1) if x < int(f["lim"][l]))
+        while len(syms) < n1:
+            s_, m = (int(x) for x in f["slut"][win(window, pos, f["w2"])])
+            if m == ESC:
+                x = win(window, pos, 32)
+                l = long_len(x, f["w2"] + 1)
                 syms.append(int(f["symrot"][((x >> (32 - l)) + int(f["offs"][l])) & 0xFFFFFFFF & 255]))
                 pos += l
             else:
-                nc = (e >> 29) & 3
-                syms.extend([(e >> (8 * j)) & 0xFF for j in range(nc)])
-                pos += (e >> 24) & 31
+                nc = (m >> 8) & 0xFF
+                assert 1 <= nc <= 4
+                syms.extend([(s_ >> (8 * j)) & 0xFF for j in range(nc)])
+                pos += m & 31
         assert pos == end and len(syms) == n1
         out.extend(_unrotate(np.array(syms, dtype=np.uint32)).tolist())
         counts.append(n1)
