@@ -63,7 +63,8 @@ class _Params(ctypes.Structure):
 class _Tensor(ctypes.Structure):
     _fields_ = [("n_elems", ctypes.c_uint64), ("total_bits", ctypes.c_uint64),
                 ("n_threads", ctypes.c_uint64), ("n_blocks", ctypes.c_uint64),
-                ("params", _Params), ("code_len", ctypes.c_uint8 * 256),
+                ("params", _Params), ("max_block_codes", ctypes.c_uint32),
+                ("reserved2", ctypes.c_uint32), ("code_len", ctypes.c_uint8 * 256),
                 ("enc_bytes", ctypes.c_uint64), ("sm_bytes", ctypes.c_uint64),
                 ("gaps_bytes", ctypes.c_uint64), ("block_start_bytes", ctypes.c_uint64),
                 ("lut_bytes", ctypes.c_uint64),
@@ -105,7 +106,7 @@ def _lib():
     lib.df11_decode_block.argtypes = [P(T), P(u64), u32, vp, vp, vp]
     lib.df11_read_error.argtypes = [vp, vp, P(u32)]
     lib.df11_device_sm_count.argtypes = [P(ctypes.c_int)]
-    if lib.df11_abi_version() != 1 or lib.df11_sizeof_tensor() != ctypes.sizeof(_Tensor):
+    if lib.df11_abi_version() != 2 or lib.df11_sizeof_tensor() != ctypes.sizeof(_Tensor):
         raise ImportError("libdf11.so ABI does not match this binding")
     _LIB = lib
     return lib

@@ -18,9 +18,16 @@
 // B200 design (what differs from the pages' own kernel):
 //  * Persistent CTAs, one per SM (1024 threads = 8 groups of 128).  Each
 //    group decodes one format block (256 format threads x 8 bytes) at a
-//    time and strides over the blocks; the decode tables are staged into
-//    shared memory once per CTA with one TMA bulk copy (cp.async.bulk, no
-//    multicast).
+//    time and strides over the blocks.  The compact decode tables arrive by
+//    one TMA bulk copy (cp.async.bulk, no multicast) and are replicated in
+//    shared memory so that each lane reads its own copy (near
+//    conflict-free random lookups).  Each group's next-block inputs (stream
+//    bytes, gaps, block starts) and first sign/mantissa vectors are fetched
+//    by bulk copies on per-group mbarriers, so no register holds prefetched
+//    data across the decode loops.
+//  * The exponent buffer holds 8192 symbols per group; tensors whose blocks
+//    hold more codes (average code under 2 bits) use a second instance with
+//    4 groups of 16 KB buffers.
 //  * Every CUDA thread runs two format threads side by side (two
 //    independent decode chains in one loop): each lookup is a dependent
 //    shift -> index -> shared load chain, and two chains per thread hide
@@ -58,19 +65,79 @@ namespace {
 
 using namespace df11;
 
-constexpr uint32_t kSbufBytes = (uint32_t)kMaxCodesPerBlock + 64u;  // + head offset (<16) + slack
-constexpr uint32_t kGroupBytes = kSbufBytes + 32u;                    // + 8 warp totals
-constexpr uint32_t kSmemBytes = kLutBytes + kGroupsPerCta * kGroupBytes + 16u;  // + mbarrier
+// Shared memory layout of one CTA:
+//   [0, 768)                 table header, canonical limits, symbol list
+//   kOffCountRep             count table, kCountCopies copies interleaved:
+//                            entry i of copy c at word (i * kCountCopies + c)
+//   kOffSymRep               symbol table, kSymCopies copies interleaved:
+//                            entry i of copy c at u64 (i * kSymCopies + c)
+//   kOffGroups               per group: exponent buffer, warp totals, staged
+//                            inputs of the next block, the first
+//                            sign/mantissa vectors of this one, 2 mbarriers
+//   table mbarrier
+// Lane l reads copy (l mod copies), so the 32 random lookups of a warp fall
+// in different banks: a lookup costs one or two shared-memory wavefronts
+// instead of the 3..8 of a single table.
+#ifndef DF11_COUNT_COPIES
+#define DF11_COUNT_COPIES 4
+#endif
+#ifndef DF11_SYM_COPIES
+#define DF11_SYM_COPIES 2
+#endif
+constexpr uint32_t kCountCopies = DF11_COUNT_COPIES;
+constexpr uint32_t kSymCopies = DF11_SYM_COPIES;
+constexpr uint32_t log2u(uint32_t x) { return x <= 1u ? 0u : 1u + log2u(x >> 1); }
+constexpr uint32_t kCountShift = log2u(4u * kCountCopies);  // byte stride of one replicated entry
+constexpr uint32_t kSymShift = log2u(8u * kSymCopies);
+static_assert((1u << kCountShift) == 4u * kCountCopies && (1u << kSymShift) == 8u * kSymCopies, "power of two");
+constexpr uint32_t kOffCountRep = 768;
+constexpr uint32_t kOffSymRep = kOffCountRep + 4u * kCountCopies * (1u << kW1Max);
+constexpr uint32_t kOffGroups = kOffSymRep + 8u * kSymCopies * (1u << kW2Max);
+constexpr uint32_t kEncStage = kThreadsPerBlockFmt * kBytesPerThread + 16u;  // + next block's first 16
+constexpr uint32_t kGapStage = kThreadsPerBlockFmt * 5u / 8u + 16u;          // + next block's first gaps
+constexpr uint32_t kSmStage = 16u * kGroupThreads;                           // one vector per thread
 constexpr uint32_t kFull = 0xFFFFFFFFu;
-constexpr uint32_t kKernErrTimeout = 0x10u;  // table staging did not complete
-static_assert(kGroupBytes % 16 == 0, "group stride keeps 16-byte alignment");
+#ifndef DF11_LOOP_CAP
+#define DF11_LOOP_CAP 128
+#endif
+constexpr uint32_t kLoopCap = DF11_LOOP_CAP;  // lookups per decode loop (95 suffice)
+constexpr uint32_t kKernErrTimeout = 0x10u;  // an asynchronous copy did not complete in time
+static_assert(kGroupThreads == 128, "group scan assumes four warps");
 static_assert(kLutBytes % 16 == 0, "bulk copy size");
-static_assert(kSmemBytes <= 227u * 1024u, "fits one CTA's shared memory");
+
+// Per-instance layout: G groups per CTA, buffers of S symbols (+ 16: the
+// 16-element chunk alignment of the block start is at most 15).
+template <int G, int S>
+struct Cfg {
+    static constexpr uint32_t kGroups = G;
+    static constexpr uint32_t kBufSyms = S;
+    static constexpr uint32_t kCtaThreads = G * kGroupThreads;
+    static constexpr uint32_t kSbufBytes = S + 16u;  // + the word after the last one
+    static constexpr uint32_t kGrpWtot = kSbufBytes;
+    static constexpr uint32_t kGrpEnc = kGrpWtot + 16u;
+    static constexpr uint32_t kGrpGap = kGrpEnc + kEncStage;
+    static constexpr uint32_t kGrpBs = kGrpGap + kGapStage;
+    static constexpr uint32_t kGrpSm = kGrpBs + 32u;
+    // the first sign/mantissa vectors are staged when shared memory allows
+    static constexpr bool kStageSm = kOffGroups + G * (kGrpSm + kSmStage + 16u) + 16u <= 227u * 1024u;
+    static constexpr uint32_t kGrpMbar = kGrpSm + (kStageSm ? kSmStage : 0u);
+    static constexpr uint32_t kGroupBytes = kGrpMbar + 16u;
+    static constexpr uint32_t kSmemBytes = kOffGroups + G * kGroupBytes + 16u;
+    static_assert(S % 16 == 0, "whole chunks");
+    static_assert(((S + 19u) >> 4) * 16u <= kSbufBytes, "zeroing stays inside the buffer");
+    static_assert(kGroupBytes % 16 == 0 && kGrpEnc % 16 == 0 && kGrpGap % 16 == 0 && kGrpBs % 16 == 0 &&
+                      kGrpSm % 16 == 0,
+                  "bulk copy destinations are 16-byte aligned");
+    static_assert(kLutBytes <= G * kGroupBytes, "tables stage in the group area");
+    static_assert(kSmemBytes <= 227u * 1024u, "fits one CTA's shared memory");
+};
+using CfgWide = Cfg<8, 8192>;    // blocks of up to 8192 - 15 codes (any LLM-like data)
+using CfgDense = Cfg<4, 16400>;  // any block (1-bit codes: 16384 per block)
 
 struct DecodeArgs {
     const uint8_t *enc;
     const uint8_t *sm;
-    const uint32_t *gaps32;
+    const uint8_t *gaps;
     const uint32_t *bstart;
     const uint8_t *lut;
     uint16_t *out;
@@ -123,9 +190,10 @@ __device__ __forceinline__ uint4 lds_u4(uint32_t a) {
 __device__ __forceinline__ void sts_u32(uint32_t a, uint32_t v) {
     asm volatile("st.shared.u32 [%0], %1;" ::"r"(a), "r"(v) : "memory");
 }
-__device__ __forceinline__ void sts_zero16(uint32_t a) {
-    asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(a), "r"(0u) : "memory");
+__device__ __forceinline__ void sts_u4(uint32_t a, uint32_t x, uint32_t y, uint32_t z, uint32_t w) {
+    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(x), "r"(y), "r"(z), "r"(w) : "memory");
 }
+__device__ __forceinline__ void sts_zero16(uint32_t a) { sts_u4(a, 0u, 0u, 0u, 0u); }
 __device__ __forceinline__ void red_or(uint32_t a, uint32_t v) {
     asm volatile("red.shared.or.b32 [%0], %1;" ::"r"(a), "r"(v) : "memory");
 }
@@ -137,75 +205,54 @@ __device__ __forceinline__ uint32_t smem_addr(const void *p) {
     return (uint32_t)__cvta_generic_to_shared(p);
 }
 
-// Bounded wait for phase 0 of the table mbarrier.  Returns false if the
-// copy did not complete within the iteration limit.
-__device__ __forceinline__ bool wait_tables(uint32_t bar) {
+// Bounded wait for the given phase of an mbarrier.  Returns false if the
+// phase did not complete within the iteration limit.
+__device__ __forceinline__ bool wait_phase(uint32_t bar, uint32_t phase) {
     uint32_t done = 0;
     for (uint32_t it = 0; it < (1u << 22) && !done; ++it) {
         asm volatile(
             "{\n\t.reg .pred p;\n\t"
-            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], 0;\n\t"
+            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
             "selp.u32 %0, 1, 0, p;\n\t}"
             : "=r"(done)
-            : "r"(bar)
+            : "r"(bar), "r"(phase)
             : "memory");
     }
     return done != 0;
 }
-
-// Bulk copy of the decode tables into shared memory (TMA engine, one
-// thread), completion tracked by an mbarrier that every thread waits on.
-__device__ __forceinline__ bool stage_tables(uint32_t dst, const uint8_t *src, uint32_t bytes, uint32_t bar) {
-    if (threadIdx.x == 0) {
-        asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar) : "memory");
-        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    }
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
-                     : "memory");
-        asm volatile(
-            "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
-            "l"(src), "r"(bytes), "r"(bar)
-            : "memory");
-    }
-    return wait_tables(bar);
+__device__ __forceinline__ void mbar_init(uint32_t bar) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void mbar_expect(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+// One-dimensional bulk copy global -> shared (TMA engine), completion counted
+// on the mbarrier.  Addresses 16-byte aligned, size a multiple of 16.
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+                 "l"(src), "r"(bytes), "r"(bar)
+                 : "memory");
 }
 
 // Length of a code longer than the table window, from the canonical limits
-// in shared memory: the smallest l with window < lim[l].  0 if none.
-__device__ __noinline__ uint32_t long_code_length(uint32_t x, uint32_t lim_addr, uint32_t from, uint32_t max_len) {
-    for (uint32_t l = from; l <= max_len; ++l) {
-        const uint64_t lim = lds_u64(lim_addr + 8u * l);
-        if ((uint64_t)x < lim) return l;
+// in shared memory (non-decreasing in l): the smallest l in [from, max_len]
+// with window < lim[l], by binary search.  0 if none.
+__device__ __forceinline__ uint32_t long_code_length(uint32_t x, uint32_t lim_addr, uint32_t from, uint32_t max_len) {
+    if (from > max_len || (uint64_t)x >= lds_u64(lim_addr + 8u * max_len)) return 0u;
+    uint32_t lo = from, hi = max_len;  // answer in [lo, hi]
+    while (lo < hi) {
+        const uint32_t mid = (lo + hi) >> 1;
+        if ((uint64_t)x < lds_u64(lim_addr + 8u * mid)) hi = mid;
+        else lo = mid + 1u;
     }
-    return 0u;
+    return lo;
 }
 
-// Shifts the 96-bit window left by n bits (n <= 32), filling with ones.
+// Shifts a 96-bit window left by n bits (n <= 32), filling with ones.
 __device__ __forceinline__ void shift_window_clamped(uint32_t &hi, uint32_t &lo, uint32_t &fl, uint32_t n) {
     hi = __funnelshift_lc(lo, hi, n);
     lo = __funnelshift_lc(fl, lo, n);
     fl = __funnelshift_lc(kFull, fl, n);
-}
-
-struct BlockInputs {
-    uint4 v;              // 16 stream bytes: chain A's 8, then chain B's 8
-    uint32_t wn;          // lane 31 only: the next thread's first 4 bytes
-    uint32_t g_hi, g_lo;  // the two 32-bit gap words holding bits [5tA, 5tA + 15)
-    uint32_t s, e;        // block_start[b], block_start[b + 1]
-};
-
-__device__ __forceinline__ void load_block_inputs(const DecodeArgs &a, uint64_t blk, uint32_t lt,
-                                                  uint32_t lane, BlockInputs &in) {
-    const uint64_t tA = blk * (uint64_t)kThreadsPerBlockFmt + 2u * lt;
-    in.v = ld_stream_u4(a.enc + 8ull * tA);  // 16-byte aligned: tA is even
-    in.wn = (lane == 31u) ? __ldg(reinterpret_cast<const uint32_t *>(a.enc + 8ull * tA + 16ull)) : 0u;
-    const uint64_t word = (5ull * tA) >> 5;
-    in.g_hi = __ldg(a.gaps32 + word);
-    in.g_lo = __ldg(a.gaps32 + word + 1);
-    in.s = __ldg(a.bstart + blk);
-    in.e = __ldg(a.bstart + blk + 1);
 }
 
 // Merges 16 rotated exponents with their 16 sign/mantissa bytes into 16
@@ -226,8 +273,7 @@ __device__ __forceinline__ void merge16(const uint4 smv, const uint4 ex, uint32_
 // lanes 0..15 take the first chunk, lanes 16..31 the last one, one element
 // each (only elements inside [s, e) are written).
 __device__ __forceinline__ void merge_edges(const uint8_t *sm, uint16_t *out, uint32_t sb, uint32_t base,
-                                            uint32_t c_full, uint32_t span, uint32_t s, uint32_t e,
-                                            uint32_t lane) {
+                                            uint32_t c_full, uint32_t span, uint32_t s, uint32_t e, uint32_t lane) {
     const bool head = s != base;
     const bool tail = (span & 15u) != 0u && !(head && c_full == 0u);
     const uint32_t c = (lane < 16u) ? 0u : c_full;
@@ -243,8 +289,8 @@ __device__ __forceinline__ void merge_edges(const uint8_t *sm, uint16_t *out, ui
     }
 }
 
-// One decode chain: the 96-bit window (hi, lo, fl) of a format thread, the
-// bits it must consume (rem0), and a running accumulator.
+// One decode chain: the 96-bit window (hi, lo, fl) of a format thread and
+// the bits it must consume.
 struct Chain {
     uint32_t hi, lo, fl;
     int32_t rem0;
@@ -271,130 +317,291 @@ __device__ __forceinline__ Chain make_chain(uint32_t x0, uint32_t x1, uint32_t x
     return c;
 }
 
-// Long-code step of the count pass for one chain whose accumulator carries
-// the escape flag.  Returns true if the chain still has bits to consume.
-__device__ __forceinline__ bool count_long_code(uint32_t &acc, uint32_t lim, uint32_t &hi, uint32_t &lo,
-                                                uint32_t &fl, uint32_t s_lim, uint32_t from, uint32_t max_len,
-                                                uint32_t &err) {
-    acc -= kEscape;
+// Long code at the top of a chain's window (its table entry was the escape):
+// shifts the window past it and returns the count-table style entry that
+// accounts for it (1 code, l bits) with a zero shift amount.  An invalid
+// pattern stops the chain: the entry then brings the accumulator to `lim`.
+__device__ __forceinline__ uint32_t count_long_code(uint32_t acc, uint32_t lim, uint32_t &hi, uint32_t &lo,
+                                                    uint32_t &fl, uint32_t s_lim, uint32_t from, uint32_t max_len,
+                                                    uint32_t &err) {
     const uint32_t l = long_code_length(hi, s_lim, from, max_len);
     if (l == 0u) {
         err |= DF11_KERR_BAD_CODE;
-        acc = lim;  // stop this chain
-        return false;
+        return (lim - acc + 31u) & ~31u;  // reaches lim; low bits clear: no window shift
     }
-    acc += (l << 24) | (1u << 8);
     shift_window_clamped(hi, lo, fl, l);
-    return acc < lim;
+    return (1u << 8) | (l << 24);
 }
 
-// Long-code step of the decoding pass: writes the symbol, advances.
-__device__ __forceinline__ bool decode_long_code(uint32_t &pacc, uint32_t pend, uint32_t &hi, uint32_t &lo,
-                                                 uint32_t &fl, uint32_t sb, uint32_t s_lim, uint32_t s_offs,
-                                                 uint32_t s_symrot, uint32_t from, uint32_t max_len) {
-    pacc -= kEscape;
+// Same for the decoding pass: ORs the long code's symbol into the buffer at
+// index p, shifts the window and returns the meta word of 1 code with a
+// zero shift amount; an invalid pattern stops the chain at pend.
+__device__ __forceinline__ uint32_t decode_long_code(uint32_t pacc, uint32_t pend, uint32_t &hi, uint32_t &lo,
+                                                     uint32_t &fl, uint32_t sb, uint32_t s_lim, uint32_t s_offs,
+                                                     uint32_t s_symrot, uint32_t from, uint32_t max_len) {
     const uint32_t l = long_code_length(hi, s_lim, from, max_len);
-    if (l == 0u) {  // reported by the count pass
-        pacc = pend;
-        return false;
-    }
+    if (l == 0u) return (pend - pacc + 31u) & ~31u;  // reported by the count pass
     const uint32_t idx = (hi >> (32u - l)) + lds_u32(s_offs + 4u * l);
     const uint32_t p = pacc >> 8;
     red_or(sb + (p & ~3u), lds_u8(s_symrot + (idx & 255u)) << (8u * (p & 3u)));
-    pacc += 1u << 8;
     shift_window_clamped(hi, lo, fl, l);
-    return pacc < pend;
+    return 1u << 8;
 }
 
-__global__ void __launch_bounds__(kCtaThreads, 1) df11_decode_kernel(const DecodeArgs a) {
+// Count pass for both chains of a thread (count table, fused accumulator).
+// Long codes are resolved in place (a short divergent branch), so all lanes
+// keep looping together.
+__device__ __forceinline__ void count_pass(const Chain &A, const Chain &B, uint32_t cnt_lane, uint32_t sh1,
+                                           uint32_t s_lim, uint32_t from, uint32_t max_len, uint32_t &cA,
+                                           uint32_t &cB, uint32_t &err) {
+    uint32_t hA = A.hi, lA = A.lo, fA = A.fl, hB = B.hi, lB = B.lo, fB = B.fl;
+    uint32_t aA = 0, aB = 0;
+    const uint32_t limA = (uint32_t)A.rem0 << 24, limB = (uint32_t)B.rem0 << 24;
+    // A valid chain needs at most 95 lookups; the cap only guards against a
+    // malformed table or stream (reported as an overrun below).
+    uint32_t guard = kLoopCap;
+    while (((aA < limA) | (aB < limB)) && guard != 0u) {
+        --guard;
+        uint32_t eA = lds_u32(cnt_lane + ((hA >> sh1) << kCountShift));
+        uint32_t eB = lds_u32(cnt_lane + ((hB >> sh1) << kCountShift));
+        eA = (aA < limA) ? eA : 0u;
+        eB = (aB < limB) ? eB : 0u;
+        if ((eA | eB) >= kEscape) {
+            if (eA == kEscape) eA = count_long_code(aA, limA, hA, lA, fA, s_lim, from, max_len, err);
+            if (eB == kEscape) eB = count_long_code(aB, limB, hB, lB, fB, s_lim, from, max_len, err);
+        }
+        aA += eA;
+        aB += eB;
+        hA = __funnelshift_l(lA, hA, eA);
+        lA = __funnelshift_l(fA, lA, eA);
+        fA = __funnelshift_l(kFull, fA, eA);
+        hB = __funnelshift_l(lB, hB, eB);
+        lB = __funnelshift_l(fB, lB, eB);
+        fB = __funnelshift_l(kFull, fB, eB);
+    }
+    cA = (aA >> 8) & 0xFFFFu;
+    cB = (aB >> 8) & 0xFFFFu;
+    if ((aA >> 24) != (uint32_t)A.rem0 || (aB >> 24) != (uint32_t)B.rem0) err |= DF11_KERR_OVERRUN;
+}
+
+// Decoding pass for both chains of a thread: writes each code's rotated
+// exponent into the group buffer.  Symbol bytes are OR-ed into the (zeroed)
+// buffer, one or two aligned words per lookup; unused symbol bytes of a
+// table entry are zero.  Stops on the code counts of the count pass.
+__device__ __forceinline__ void decode_pass(const Chain &A, const Chain &B, uint32_t startA, uint32_t cA,
+                                            uint32_t startB, uint32_t cB, uint32_t sb, uint32_t sym_lane,
+                                            uint32_t sh2, uint32_t s_lim, uint32_t s_offs, uint32_t s_symrot,
+                                            uint32_t from, uint32_t max_len) {
+    uint32_t hA = A.hi, lA = A.lo, fA = A.fl, hB = B.hi, lB = B.lo, fB = B.fl;
+    uint32_t pA = startA << 8, pB = startB << 8;
+    const uint32_t endPA = (startA + cA) << 8, endPB = (startB + cB) << 8;
+    uint32_t guard = kLoopCap;  // as in the count pass
+    while (((pA < endPA) | (pB < endPB)) && guard != 0u) {
+        --guard;
+        const uint2 eA = lds_u2(sym_lane + ((hA >> sh2) << kSymShift));
+        const uint2 eB = lds_u2(sym_lane + ((hB >> sh2) << kSymShift));
+        const bool actA = pA < endPA, actB = pB < endPB;
+        uint32_t mA = actA ? eA.y : 0u;
+        uint32_t mB = actB ? eB.y : 0u;
+        if ((mA | mB) >= kEscape) {
+            if (mA == kEscape)
+                mA = decode_long_code(pA, endPA, hA, lA, fA, sb, s_lim, s_offs, s_symrot, from, max_len);
+            if (mB == kEscape)
+                mB = decode_long_code(pB, endPB, hB, lB, fB, sb, s_lim, s_offs, s_symrot, from, max_len);
+        }
+        const uint32_t bA = pA >> 8, bB = pB >> 8;
+        const uint32_t shA = (bA & 3u) << 3, shB = (bB & 3u) << 3;
+        const uint32_t wA = sb + (bA & ~3u), wB = sb + (bB & ~3u);
+        if (actA) {  // (an escape entry has no symbol bytes: these OR zero)
+            red_or(wA, eA.x << shA);
+            if (shA) red_or(wA + 4u, __funnelshift_l(eA.x, 0u, shA));
+        }
+        if (actB) {
+            red_or(wB, eB.x << shB);
+            if (shB) red_or(wB + 4u, __funnelshift_l(eB.x, 0u, shB));
+        }
+        pA += mA;
+        pB += mB;
+        hA = __funnelshift_l(lA, hA, mA);
+        lA = __funnelshift_l(fA, lA, mA);
+        fA = __funnelshift_l(kFull, fA, mA);
+        hB = __funnelshift_l(lB, hB, mB);
+        lB = __funnelshift_l(fB, lB, mB);
+        fB = __funnelshift_l(kFull, fB, mB);
+    }
+}
+
+// Merges chunks c_first, c_first + 128, ... < c_end (chunk c covers output
+// elements base + 16c .. +16, at buffer offset 16c) with sign/mantissa.
+__device__ __forceinline__ void merge_chunks(const uint8_t *sm, uint16_t *out, uint32_t sb, uint32_t base,
+                                             uint32_t c_first, uint32_t c_end, uint4 smv) {
+    if (c_first >= c_end) return;
+    const uint8_t *smp = sm + (uint64_t)base + 16ull * c_first;
+    uint16_t *dst = out + (uint64_t)base + 16ull * c_first;
+    uint32_t ex_addr = sb + 16u * c_first;
+    for (uint32_t c = c_first;;) {
+        const uint4 ex = lds_u4(ex_addr);
+        uint32_t o[8];
+        merge16(smv, ex, o);
+        st_u4(dst, o[0], o[1], o[2], o[3]);
+        st_u4(dst + 8, o[4], o[5], o[6], o[7]);
+        c += kGroupThreads;
+        if (c >= c_end) break;
+        smp += 16u * kGroupThreads;
+        dst += 16u * kGroupThreads;
+        ex_addr += 16u * kGroupThreads;
+        smv = ld_stream_u4(smp);
+    }
+}
+
+// Issues the bulk copies of block `blk`'s inputs into the group's staging
+// area: its 2048 stream bytes plus the next block's first 16 (the last
+// thread's look-ahead), its 160 gap bytes (+16: the next block's first
+// gaps), and the 32-byte aligned window holding block_start[blk], [blk + 1].
+template <class C>
+__device__ __forceinline__ void issue_inputs(const DecodeArgs &a, uint64_t blk, uint32_t grp, uint32_t mbar) {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    mbar_expect(mbar, kEncStage + kGapStage + 32u);
+    bulk_g2s(grp + C::kGrpEnc, a.enc + blk * (uint64_t)(kThreadsPerBlockFmt * kBytesPerThread), kEncStage, mbar);
+    bulk_g2s(grp + C::kGrpGap, a.gaps + blk * (uint64_t)(kThreadsPerBlockFmt * 5u / 8u), kGapStage, mbar);
+    bulk_g2s(grp + C::kGrpBs, reinterpret_cast<const uint8_t *>(a.bstart) + ((4ull * blk) & ~15ull), 32u, mbar);
+}
+
+template <class C>
+__global__ void __launch_bounds__(C::kCtaThreads, 1) df11_decode_kernel(const DecodeArgs a) {
     extern __shared__ __align__(128) uint8_t smem[];
     const uint32_t s_base = smem_addr(smem);
     const uint32_t s_lim = s_base + kOffLim;
     const uint32_t s_offs = s_base + kOffOffs;
     const uint32_t s_symrot = s_base + kOffSymRot;
-    const uint32_t s_clut = s_base + kOffCountLut;
-    const uint32_t s_slut = s_base + kOffSymLut;
-    const uint32_t s_mbar = s_base + kLutBytes + kGroupsPerCta * kGroupBytes;
+    const uint32_t s_tmbar = s_base + kOffGroups + C::kGroups * C::kGroupBytes;
+    const uint32_t s_stage = s_base + kOffGroups;  // compact tables land here first
 
     const uint32_t tid = threadIdx.x;
     const uint32_t group = tid / kGroupThreads;
     const uint32_t lt = tid % kGroupThreads;  // thread within the group
     const uint32_t lane = tid & 31u;
     const uint32_t warp = lt >> 5;            // warp within the group
-    const uint32_t sb = s_base + kLutBytes + group * kGroupBytes;  // this group's exponent buffer
-    const uint32_t wtot = sb + kSbufBytes;                          // per-warp totals
+    const uint32_t grp = s_base + kOffGroups + group * C::kGroupBytes;
+    const uint32_t sb = grp;                  // exponent buffer
+    const uint32_t wtot = grp + C::kGrpWtot;  // 4 warp totals
+    const uint32_t mb_in = grp + C::kGrpMbar, mb_sm = grp + C::kGrpMbar + 8u;
+    const uint32_t cnt_lane = s_base + kOffCountRep + 4u * (lane % kCountCopies);
+    const uint32_t sym_lane = s_base + kOffSymRep + 8u * (lane % kSymCopies);
     uint32_t my_err = 0;
 
-    const uint64_t stride = (uint64_t)gridDim.x * kGroupsPerCta;
-    uint64_t blk = (uint64_t)blockIdx.x * kGroupsPerCta + group;
+    const uint64_t stride = (uint64_t)gridDim.x * C::kGroups;
+    uint64_t blk = (uint64_t)blockIdx.x * C::kGroups + group;
 
-    // Prefetch the first block's inputs while the tables stream in.
-    BlockInputs cur{};
-    if (blk < a.n_blocks) load_block_inputs(a, blk, lt, lane, cur);
-
-    const bool staged = stage_tables(s_base, a.lut, kLutBytes, s_mbar);
+    // ---- decode tables: one bulk copy, then validate and replicate
+    if (tid == 0) {
+        mbar_init(s_tmbar);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+    if (tid == 0) {
+        mbar_expect(s_tmbar, kLutBytes);
+        bulk_g2s(s_stage, a.lut, kLutBytes, s_tmbar);
+    }
+    const bool staged = wait_phase(s_tmbar, 0u);
     if (__syncthreads_or(!staged)) {
         // Uniform over the CTA.  One more bounded wait so no copy is left in
         // flight into this CTA's shared memory, then report and stop.
         if (tid == 0) {
-            wait_tables(s_mbar);
+            wait_phase(s_tmbar, 0u);
             if (a.err) atomicOr(a.err, kKernErrTimeout);
         }
         __syncthreads();
         return;
     }
-
-    const LutHeader *hdr = reinterpret_cast<const LutHeader *>(smem + kOffHeader);
+    const LutHeader *hdr = reinterpret_cast<const LutHeader *>(smem + kOffGroups + kOffHeader);
     const uint32_t w1 = hdr->w1, w2 = hdr->w2, max_len = hdr->max_len;
-    if (hdr->magic != kMagic || w1 < 1u || w1 > (uint32_t)kW1Max || w2 < 1u || w2 > (uint32_t)kW2Max ||
-        max_len > 32u) {
-        if (tid == 0 && a.err) atomicOr(a.err, DF11_KERR_BAD_CODE);
-        return;  // uniform over the CTA: nothing was written yet
-    }
-    // Every table entry must be the escape flag or take 1..W bits for
-    // 1..(bits) codes, so each lookup makes progress: the decode loops then
-    // end after at most 95 lookups plus 95 long codes whatever the stream.
     {
-        bool bad = false;
-        for (uint32_t i = tid; i < (1u << w1); i += kCtaThreads) {
-            const uint32_t ent = lds_u32(s_clut + 4u * i);
+        bool bad = !(hdr->magic == kMagic && w1 >= 1u && w1 <= (uint32_t)kW1Max && w2 >= 1u &&
+                     w2 <= (uint32_t)kW2Max && max_len <= 32u);
+        // header, limits and symbol list go to the front
+        for (uint32_t i = tid; i < kOffCountLut / 16u; i += C::kCtaThreads) {
+            const uint4 v = lds_u4(s_stage + 16u * i);
+            sts_u4(s_base + 16u * i, v.x, v.y, v.z, v.w);
+        }
+        // each store writes kCW copies of a count entry / kSW of a symbol
+        // entry; the loops cover every (entry, copy), so every copy a lane can
+        // read is written and validated here
+        constexpr uint32_t kCW = kCountCopies < 4u ? kCountCopies : 4u;
+        constexpr uint32_t kSW = kSymCopies < 2u ? kSymCopies : 2u;
+        static_assert(kCountCopies % kCW == 0u && kSymCopies % kSW == 0u, "copies fill whole stores");
+        for (uint32_t i = tid; i < (1u << kW1Max) * (kCountCopies / kCW); i += C::kCtaThreads) {
+            const uint32_t ent = lds_u32(s_stage + kOffCountLut + 4u * (i / (kCountCopies / kCW)));
             const uint32_t nb = count_entry_bits(ent), nc = count_entry_codes(ent);
             bad |= ent != kEscape && (ent != count_entry(nb, nc) || nb == 0u || nb > w1 || nc == 0u || nc > nb);
+            const uint32_t dst = s_base + kOffCountRep + 4u * kCW * i;
+            if (kCW == 4u) sts_u4(dst, ent, ent, ent, ent);
+            else if (kCW == 2u) asm volatile("st.shared.v2.u32 [%0], {%1, %1};" ::"r"(dst), "r"(ent) : "memory");
+            else sts_u32(dst, ent);
         }
-        for (uint32_t i = tid; i < (1u << w2); i += kCtaThreads) {
-            const uint2 ent = lds_u2(s_slut + 8u * i);
+        for (uint32_t i = tid; i < (1u << kW2Max) * (kSymCopies / kSW); i += C::kCtaThreads) {
+            const uint2 ent = lds_u2(s_stage + kOffSymLut + 8u * (i / (kSymCopies / kSW)));
             const uint32_t nb = sym_entry_bits(ent.y), nc = sym_entry_codes(ent.y);
             bad |= ent.y != kEscape && (ent.y != sym_entry_meta(nb, nc) || nb == 0u || nb > w2 || nc == 0u ||
                                         nc > (uint32_t)kSymsPerEntry || nc > nb);
+            const uint32_t dst = s_base + kOffSymRep + 8u * kSW * i;
+            if (kSW == 2u) sts_u4(dst, ent.x, ent.y, ent.x, ent.y);
+            else asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(dst), "r"(ent.x), "r"(ent.y) : "memory");
         }
+        // Every entry is the escape flag or takes 1..W bits for 1..(bits)
+        // codes, so each lookup makes progress: the decode loops then end
+        // after at most 95 lookups plus 95 long codes whatever the stream.
         if (__syncthreads_or(bad)) {
             if (tid == 0 && a.err) atomicOr(a.err, DF11_KERR_BAD_CODE);
-            return;
+            return;  // uniform over the CTA: nothing was written to global memory
         }
     }
     const uint32_t sh1 = 32u - w1, sh2 = 32u - w2;
 
-    for (; blk < a.n_blocks; blk += stride) {
-        const BlockInputs in = cur;
-        const uint64_t nxt = blk + stride;
-        if (nxt < a.n_blocks) load_block_inputs(a, nxt, lt, lane, cur);
+    // ---- the group's mbarriers (inputs of the next block; first
+    // sign/mantissa vectors of this one) and its first block's inputs
+    if (lt == 0) {
+        mbar_init(mb_in);
+        mbar_init(mb_sm);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        if (blk < a.n_blocks) issue_inputs<C>(a, blk, grp, mb_in);
+    }
+    group_barrier(group);
+    uint32_t ph_in = 0, ph_sm = 0;
 
+    for (; blk < a.n_blocks; blk += stride) {
+        if (!wait_phase(mb_in, ph_in)) my_err |= kKernErrTimeout;
+        ph_in ^= 1u;
         const uint64_t tA = blk * (uint64_t)kThreadsPerBlockFmt + 2u * lt;
-        const uint32_t s = in.s, e = in.e;
+        const uint32_t bs_off = (uint32_t)((4ull * blk) & 15ull);
+        const uint32_t s = lds_u32(grp + C::kGrpBs + bs_off), e = lds_u32(grp + C::kGrpBs + bs_off + 4u);
         const uint32_t base = s & ~15u;  // first 16-element chunk of the block's output
-        const bool range_ok = (e >= s) && ((uint64_t)e <= a.n_elems) && (e - s <= (uint32_t)kMaxCodesPerBlock);
-        // chunks [c_lo, c_full) lie wholly inside [s, e)
+        // buffer index of output element g is g - base (< span)
+        const bool range_ok = (e >= s) && ((uint64_t)e <= a.n_elems) && (e - base <= C::kBufSyms);
         const uint32_t span = range_ok ? e - base : 0u;
         const uint32_t c_lo = (s != base) ? 1u : 0u;
-        const uint32_t c_full = span >> 4;
+        const uint32_t c_full = span >> 4;  // chunks [c_lo, c_full) lie wholly inside [s, e)
         const uint32_t c0 = c_lo + lt;
-        uint4 smv0 = make_uint4(0, 0, 0, 0);
-        if (c0 < c_full) smv0 = ld_stream_u4(a.sm + (uint64_t)base + 16ull * c0);
+        if (C::kStageSm && lt == 0) {
+            // this block's first sign/mantissa vectors (one per thread), up to
+            // the end of the block's last chunk; always at least 16 bytes
+            const uint32_t from = range_ok ? base + 16u * c_lo : 0u;
+            const uint32_t upto = range_ok ? ((e + 15u) & ~15u) : 16u;
+            const uint32_t bytes = upto > from ? min(kSmStage, upto - from) : 16u;
+            const uint32_t src = upto > from ? from : (range_ok ? base : 0u);
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            mbar_expect(mb_sm, bytes);
+            bulk_g2s(grp + C::kGrpSm, a.sm + src, bytes, mb_sm);
+        }
 
         // ---- the two chains: format threads tA and tA + 1
-        // gaps are an MSB-first bit string: bits [5tA, 5tA + 15) hold the
-        // gaps of tA, tA + 1 and tA + 2
-        const uint32_t gb = __funnelshift_l(bswap32(in.g_lo), bswap32(in.g_hi), (uint32_t)((5ull * tA) & 31u));
+        const uint4 v = lds_u4(grp + C::kGrpEnc + 16u * lt);
+        const uint32_t nextw = lds_u32(grp + C::kGrpEnc + 16u * lt + 16u);
+        // gaps are an MSB-first bit string: bits [10 lt, 10 lt + 15) of the
+        // block's gap bytes hold the gaps of tA, tA + 1 and tA + 2
+        const uint32_t gq = (10u * lt) >> 5;
+        const uint32_t g_hi = lds_u32(grp + C::kGrpGap + 4u * gq), g_lo = lds_u32(grp + C::kGrpGap + 4u * gq + 4u);
+        const uint32_t gb = __funnelshift_l(bswap32(g_lo), bswap32(g_hi), (10u * lt) & 31u);
         uint32_t gapA = gb >> 27, gapB = (gb >> 22) & 31u;
         const uint32_t gapC = (gb >> 17) & 31u;
         int32_t endA, endB;
@@ -404,135 +611,62 @@ __global__ void __launch_bounds__(kCtaThreads, 1) df11_decode_kernel(const Decod
         if (tA + 1 >= a.n_threads) { gapB = 0; endB = 0; }
         else if (tA + 2 == a.n_threads) endB = (int32_t)(a.total_bits - 64ull * (tA + 1));
         else endB = 64 + (int32_t)gapC;
-        uint32_t nextw = __shfl_down_sync(kFull, in.v.x, 1);
-        if (lane == 31u) nextw = in.wn;
-        const Chain A = make_chain(bswap32(in.v.x), bswap32(in.v.y), bswap32(in.v.z), gapA, endA, my_err);
-        const Chain B = make_chain(bswap32(in.v.z), bswap32(in.v.w), bswap32(nextw), gapB, endB, my_err);
+        const Chain A = make_chain(bswap32(v.x), bswap32(v.y), bswap32(v.z), gapA, endA, my_err);
+        const Chain B = make_chain(bswap32(v.z), bswap32(v.w), bswap32(nextw), gapB, endB, my_err);
 
         // ---- pass 1: count the codes of both chains
         uint32_t cA, cB;
-        {
-            uint32_t hA = A.hi, lA = A.lo, fA = A.fl, hB = B.hi, lB = B.lo, fB = B.fl;
-            uint32_t aA = 0, aB = 0;
-            const uint32_t limA = (uint32_t)A.rem0 << 24, limB = (uint32_t)B.rem0 << 24;
-            for (;;) {
-                while ((aA < limA) | (aB < limB)) {
-                    uint32_t eA = lds_u32(s_clut + ((hA >> sh1) << 2));
-                    uint32_t eB = lds_u32(s_clut + ((hB >> sh1) << 2));
-                    eA = (aA < limA) ? eA : 0u;
-                    eB = (aB < limB) ? eB : 0u;
-                    aA += eA;
-                    aB += eB;
-                    hA = __funnelshift_l(lA, hA, eA);
-                    lA = __funnelshift_l(fA, lA, eA);
-                    fA = __funnelshift_l(kFull, fA, eA);
-                    hB = __funnelshift_l(lB, hB, eB);
-                    lB = __funnelshift_l(fB, lB, eB);
-                    fB = __funnelshift_l(kFull, fB, eB);
-                }
-                bool more = false;
-                if (aA >= kEscape) more |= count_long_code(aA, limA, hA, lA, fA, s_lim, w1 + 1u, max_len, my_err);
-                if (aB >= kEscape) more |= count_long_code(aB, limB, hB, lB, fB, s_lim, w1 + 1u, max_len, my_err);
-                if (!more) break;
-            }
-            cA = (aA >> 8) & 0xFFFFu;
-            cB = (aB >> 8) & 0xFFFFu;
-            if ((aA >> 24) != (uint32_t)A.rem0 || (aB >> 24) != (uint32_t)B.rem0) my_err |= DF11_KERR_OVERRUN;
-        }
+        count_pass(A, B, cnt_lane, sh1, s_lim, w1 + 1u, max_len, cA, cB, my_err);
 
-        // ---- clear the exponent buffer span this block uses (the decoding
-        // pass ORs symbols into it); the scan barrier orders this before it
-        for (uint32_t c = lt; c < ((span + 15u) >> 4) + 1u; c += kGroupThreads) sts_zero16(sb + 16u * c);
+        // ---- clear the buffer span (the decoding pass ORs into it); the scan
+        // barrier orders this before any write of the decoding pass
+        // (OR-stores reach buffer index span + 2 at most: bytes [0, span + 4))
+        for (uint32_t c = lt; c < (span + 19u) >> 4; c += kGroupThreads) sts_zero16(sb + 16u * c);
 
         // ---- block scan: warp inclusive scan, then across the group's warps
         const uint32_t cnt = cA + cB;
         uint32_t incl = cnt;
 #pragma unroll
         for (uint32_t d = 1; d < 32; d <<= 1) {
-            const uint32_t v = __shfl_up_sync(kFull, incl, d);
-            if (lane >= d) incl += v;
+            const uint32_t x = __shfl_up_sync(kFull, incl, d);
+            if (lane >= d) incl += x;
         }
         constexpr uint32_t kWarps = kGroupThreads / 32;
         if (lane == 31u) sts_u32(wtot + 4u * warp, incl);
         group_barrier(group);
+        // every thread has read this block's staged inputs: fetch the next
+        const uint64_t nxt = blk + stride;
+        if (lt == 0 && nxt < a.n_blocks) issue_inputs<C>(a, nxt, grp, mb_in);
         uint32_t wsum = (lane < kWarps) ? lds_u32(wtot + 4u * lane) : 0u;
 #pragma unroll
         for (uint32_t d = 1; d < kWarps; d <<= 1) {
-            const uint32_t v = __shfl_up_sync(kFull, wsum, d);
-            if (lane >= d) wsum += v;
+            const uint32_t x = __shfl_up_sync(kFull, wsum, d);
+            if (lane >= d) wsum += x;
         }
         const uint32_t total = __shfl_sync(kFull, wsum, kWarps - 1u);
         const uint32_t wpre = __shfl_sync(kFull, wsum, (warp + kWarps - 1u) % kWarps) * (warp != 0u ? 1u : 0u);
         const bool ok = range_ok && (total == e - s);
         if (!ok && lt == 0) my_err |= range_ok ? DF11_KERR_COUNT_MISMATCH : DF11_KERR_BAD_BLOCK;
 
-        // ---- pass 2: decode both chains again into the exponent buffer
+        // ---- pass 2: decode both chains again into the buffer
         if (ok) {
-            uint32_t hA = A.hi, lA = A.lo, fA = A.fl, hB = B.hi, lB = B.lo, fB = B.fl;
             const uint32_t startA = (s - base) + wpre + incl - cnt;  // buffer index of A's first code
-            const uint32_t startB = startA + cA;
-            uint32_t pA = startA << 8, pB = startB << 8;
-            const uint32_t endPA = (startA + cA) << 8, endPB = (startB + cB) << 8;
-            for (;;) {
-                while ((pA < endPA) | (pB < endPB)) {
-                    const uint2 eA = lds_u2(s_slut + ((hA >> sh2) << 3));
-                    const uint2 eB = lds_u2(s_slut + ((hB >> sh2) << 3));
-                    const bool actA = pA < endPA, actB = pB < endPB;
-                    const int32_t mA = actA ? (int32_t)eA.y : 0;
-                    const int32_t mB = actB ? (int32_t)eB.y : 0;
-                    // up to four symbol bytes land in the word holding byte p
-                    // and the next one; unused symbol bytes are zero
-                    const uint32_t bA = pA >> 8, bB = pB >> 8;
-                    const uint32_t shA = (bA & 3u) << 3, shB = (bB & 3u) << 3;
-                    const uint32_t wA = sb + (bA & ~3u), wB = sb + (bB & ~3u);
-                    if (actA) {
-                        red_or(wA, eA.x << shA);
-                        if (shA) red_or(wA + 4u, __funnelshift_l(eA.x, 0u, shA));
-                    }
-                    if (actB) {
-                        red_or(wB, eB.x << shB);
-                        if (shB) red_or(wB + 4u, __funnelshift_l(eB.x, 0u, shB));
-                    }
-                    pA += (uint32_t)mA;
-                    pB += (uint32_t)mB;
-                    hA = __funnelshift_l(lA, hA, (uint32_t)mA);
-                    lA = __funnelshift_l(fA, lA, (uint32_t)mA);
-                    fA = __funnelshift_l(kFull, fA, (uint32_t)mA);
-                    hB = __funnelshift_l(lB, hB, (uint32_t)mB);
-                    lB = __funnelshift_l(fB, lB, (uint32_t)mB);
-                    fB = __funnelshift_l(kFull, fB, (uint32_t)mB);
-                }
-                bool more = false;
-                if (pA >= kEscape)
-                    more |= decode_long_code(pA, endPA, hA, lA, fA, sb, s_lim, s_offs, s_symrot, w2 + 1u, max_len);
-                if (pB >= kEscape)
-                    more |= decode_long_code(pB, endPB, hB, lB, fB, sb, s_lim, s_offs, s_symrot, w2 + 1u, max_len);
-                if (!more) break;
-            }
+            decode_pass(A, B, startA, cA, startA + cA, cB, sb, sym_lane, sh2, s_lim, s_offs, s_symrot, w2 + 1u,
+                        max_len);
         }
         group_barrier(group);
 
         // ---- merge with sign/mantissa and store, 16 weights per step
+        if (C::kStageSm) {
+            if (!wait_phase(mb_sm, ph_sm)) my_err |= kKernErrTimeout;
+            ph_sm ^= 1u;
+        }
         if (ok) {
-            if (c0 < c_full) {
-                const uint8_t *smp = a.sm + (uint64_t)base + 16ull * c0;
-                uint16_t *dst = a.out + (uint64_t)base + 16ull * c0;
-                uint32_t ex_addr = sb + 16u * c0;
-                uint4 smv = smv0;
-                for (uint32_t c = c0;;) {
-                    const uint4 ex = lds_u4(ex_addr);
-                    uint32_t o[8];
-                    merge16(smv, ex, o);
-                    st_u4(dst, o[0], o[1], o[2], o[3]);
-                    st_u4(dst + 8, o[4], o[5], o[6], o[7]);
-                    c += kGroupThreads;
-                    if (c >= c_full) break;
-                    smp += 16u * kGroupThreads;
-                    dst += 16u * kGroupThreads;
-                    ex_addr += 16u * kGroupThreads;
-                    smv = ld_stream_u4(smp);
-                }
-            }
+            uint4 smv0 = make_uint4(0, 0, 0, 0);
+            if (c0 < c_full)
+                smv0 = C::kStageSm ? lds_u4(grp + C::kGrpSm + 16u * lt)
+                                   : ld_stream_u4(a.sm + (uint64_t)base + 16ull * c0);
+            merge_chunks(a.sm, a.out, sb, base, c0, c_full, smv0);
             if (warp == 0) merge_edges(a.sm, a.out, sb, base, c_full, span, s, e, lane);
         }
         group_barrier(group);
@@ -543,6 +677,12 @@ __global__ void __launch_bounds__(kCtaThreads, 1) df11_decode_kernel(const Decod
 // ----------------------------------------------------------------- host
 std::atomic<int> g_sm_count[64];
 std::atomic<int> g_attr_set[64];
+
+template <class C>
+cudaError_t set_smem_attr() {
+    return cudaFuncSetAttribute(df11_decode_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)C::kSmemBytes);
+}
 
 df11_status prepare_device(int *sm_count) {
     int dev = 0;
@@ -555,8 +695,7 @@ df11_status prepare_device(int *sm_count) {
         g_sm_count[dev].store(sms, std::memory_order_relaxed);
     }
     if (!g_attr_set[dev].load(std::memory_order_acquire)) {
-        if (cudaFuncSetAttribute(df11_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)kSmemBytes) != cudaSuccess)
+        if (set_smem_attr<CfgWide>() != cudaSuccess || set_smem_attr<CfgDense>() != cudaSuccess)
             return DF11_ERR_CUDA;
         g_attr_set[dev].store(1, std::memory_order_release);
     }
@@ -565,6 +704,13 @@ df11_status prepare_device(int *sm_count) {
 }
 
 bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
+
+template <class C>
+void launch(const DecodeArgs &a, uint64_t n_blocks, int sms, cudaStream_t stream) {
+    const uint64_t ctas_needed = (n_blocks + C::kGroups - 1) / C::kGroups;
+    const unsigned grid = (unsigned)(ctas_needed < (uint64_t)sms ? ctas_needed : (uint64_t)sms);
+    df11_decode_kernel<C><<<grid, C::kCtaThreads, C::kSmemBytes, stream>>>(a);
+}
 
 df11_status launch_decode(const df11_tensor *t, uint16_t *out, uint32_t *err_word, void *stream) {
     if (!t) return DF11_ERR_INVALID_ARG;
@@ -581,7 +727,7 @@ df11_status launch_decode(const df11_tensor *t, uint16_t *out, uint32_t *err_wor
     DecodeArgs a;
     a.enc = t->enc;
     a.sm = t->sm;
-    a.gaps32 = reinterpret_cast<const uint32_t *>(t->gaps);
+    a.gaps = t->gaps;
     a.bstart = t->block_start;
     a.lut = t->lut;
     a.out = out;
@@ -590,9 +736,10 @@ df11_status launch_decode(const df11_tensor *t, uint16_t *out, uint32_t *err_wor
     a.total_bits = t->total_bits;
     a.n_threads = t->n_threads;
     a.n_blocks = t->n_blocks;
-    const uint64_t ctas_needed = (t->n_blocks + kGroupsPerCta - 1) / kGroupsPerCta;
-    const unsigned grid = (unsigned)(ctas_needed < (uint64_t)sms ? ctas_needed : (uint64_t)sms);
-    df11_decode_kernel<<<grid, kCtaThreads, kSmemBytes, reinterpret_cast<cudaStream_t>(stream)>>>(a);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    // a block's buffer span is at most its code count + 15
+    if (t->max_block_codes + 15u <= CfgWide::kBufSyms) launch<CfgWide>(a, t->n_blocks, sms, s);
+    else launch<CfgDense>(a, t->n_blocks, sms, s);
     if (cudaGetLastError() != cudaSuccess) return DF11_ERR_CUDA;
     return DF11_OK;
 }

@@ -258,6 +258,8 @@ void build_luts(const uint8_t len[256], uint8_t *lut) {
     h.max_len = (uint32_t)max_len;
     h.min_len = (uint32_t)min_len;
     h.n_syms = (uint32_t)n_syms;
+    h.w1_max = (uint32_t)df11::kW1Max;
+    h.w2_max = (uint32_t)df11::kW2Max;
     std::memcpy(lut + df11::kOffHeader, &h, sizeof(h));
 
     uint64_t lim[33] = {};
@@ -281,8 +283,9 @@ void build_luts(const uint8_t len[256], uint8_t *lut) {
         uint32_t i = (x >> (32 - l)) + offs[l];
         return sym_rot[i & 255];
     };
-    // count LUT
+    // count LUT (entries past 2^w1 are never indexed; they hold the escape)
     uint32_t *clut = reinterpret_cast<uint32_t *>(lut + df11::kOffCountLut);
+    for (uint32_t v = 0; v < (1u << df11::kW1Max); ++v) clut[v] = df11::kEscape;
     for (uint32_t v = 0; v < (1u << h.w1); ++v) {
         const uint32_t x = v << (32 - h.w1);
         uint32_t pos = 0, n = 0;
@@ -294,8 +297,12 @@ void build_luts(const uint8_t len[256], uint8_t *lut) {
         }
         clut[v] = n ? df11::count_entry(pos, n) : df11::kEscape;
     }
-    // symbol LUT
+    // symbol LUT (same for entries past 2^w2)
     uint32_t *slut = reinterpret_cast<uint32_t *>(lut + df11::kOffSymLut);
+    for (uint32_t v = 0; v < (1u << df11::kW2Max); ++v) {
+        slut[2 * v] = 0u;
+        slut[2 * v + 1] = df11::kEscape;
+    }
     for (uint32_t v = 0; v < (1u << h.w2); ++v) {
         const uint32_t x = v << (32 - h.w2);
         uint32_t pos = 0, n = 0, syms = 0;
@@ -343,7 +350,7 @@ df11_status fill_sizes(const Sequence &seq, const df11_params *params, df11_tens
     t->enc_bytes = padded_threads * kBytesPerThread + 16;
     t->sm_bytes = ((seq.n + 15) / 16) * 16 + 16;
     t->gaps_bytes = ((padded_threads * 5 + 7) / 8 + 15) / 16 * 16 + 16;
-    t->block_start_bytes = (t->n_blocks + 1) * 4;
+    t->block_start_bytes = ((t->n_blocks + 1) * 4 + 15) / 16 * 16 + 16;
     t->lut_bytes = df11::kLutBytes;
     return DF11_OK;
 }
@@ -446,7 +453,10 @@ df11_status fill_arrays(const Sequence &seq, df11_tensor *t) {
     std::memset(enc + used, 0, (size_t)(t->enc_bytes - used));
     std::memset(sm + n, 0, (size_t)(t->sm_bytes - n));
     bstart[n_blocks] = (uint32_t)n;
-    if (n_blocks == 0) bstart[0] = 0;
+    uint32_t most = 0;
+    for (uint64_t b = 0; b < n_blocks; ++b) most = std::max(most, bstart[b + 1] - bstart[b]);
+    t->max_block_codes = most;
+    std::memset(bstart + n_blocks + 1, 0, (size_t)(t->block_start_bytes - 4 * (n_blocks + 1)));
 
     // gaps: eight 5-bit fields = five bytes, MSB-first
     uint8_t *pg = t->gaps;
@@ -563,8 +573,9 @@ df11_status df11_validate(const df11_tensor *t) {
     if (t->enc_bytes < padded * kBytesPerThread + 16) return DF11_ERR_INVALID_ARG;
     if (t->sm_bytes < ((t->n_elems + 15) / 16) * 16 + 16) return DF11_ERR_INVALID_ARG;
     if (t->gaps_bytes < (padded * 5 + 7) / 8 + 16) return DF11_ERR_INVALID_ARG;
-    if (t->block_start_bytes < (t->n_blocks + 1) * 4) return DF11_ERR_INVALID_ARG;
+    if (t->block_start_bytes < ((t->n_blocks + 1) * 4 + 15) / 16 * 16 + 16) return DF11_ERR_INVALID_ARG;
     if (t->lut_bytes < df11::kLutBytes) return DF11_ERR_INVALID_ARG;
+    if (t->max_block_codes > (uint32_t)df11::kMaxCodesPerBlock || t->reserved2 != 0) return DF11_ERR_CORRUPT;
     // Kraft: sum 2^-len <= 1 and lengths within the cap
     uint64_t kraft = 0;
     int k = 0;

@@ -32,12 +32,19 @@
 
 namespace df11 {
 
-constexpr uint32_t kMagic = 0x32314644u;  // "DF12": table layout version 2
-constexpr int kW1Max = 13;                // count LUT window (bits)
-constexpr int kW2Max = 12;                // symbol LUT window (bits)
+constexpr uint32_t kMagic = 0x33314644u;  // "DF13": table layout version 3
+#ifndef DF11_COUNT_WINDOW
+#define DF11_COUNT_WINDOW 12
+#endif
+#ifndef DF11_SYM_WINDOW
+#define DF11_SYM_WINDOW 12
+#endif
+constexpr int kW1Max = DF11_COUNT_WINDOW;  // count LUT window (bits)
+constexpr int kW2Max = DF11_SYM_WINDOW;    // symbol LUT window (bits)
 constexpr int kSymsPerEntry = 4;          // codes per symbol-LUT entry
 
-// Byte offsets inside the lut array.
+// Byte offsets inside the lut array (the compact tables; the decode kernel
+// replicates them in shared memory, see df11_decode.cu).
 constexpr uint32_t kOffHeader = 0;
 constexpr uint32_t kOffLim = 64;                     // uint64_t[33]
 constexpr uint32_t kOffOffs = kOffLim + 33 * 8 + 8;  // uint32_t[33] (336)
@@ -52,7 +59,9 @@ struct LutHeader {
     uint32_t max_len;  // longest code length
     uint32_t min_len;  // shortest code length
     uint32_t n_syms;   // exponent values with a code
-    uint32_t pad[10];
+    uint32_t w1_max;   // entries in the count LUT: 2^w1_max
+    uint32_t w2_max;   // entries in the symbol LUT: 2^w2_max
+    uint32_t pad[8];
 };
 static_assert(sizeof(LutHeader) == 64, "header is 64 bytes");
 

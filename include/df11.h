@@ -85,13 +85,17 @@ typedef struct df11_params {
  *              that starts in its n bytes (the end of the stream counts as
  *              a start).  n_blocks * T fields, zero-padded to gaps_bytes.
  *  block_start u32 per thread block: index of the first element decoded by
- *              that block, plus a final entry equal to n_elems.
+ *              that block, plus a final entry equal to n_elems; zero-padded
+ *              to block_start_bytes = round_up(4 * (n_blocks + 1), 16) + 16.
  *  lut         decode tables derived from code_len (layout private to the
  *              library, lut_bytes long): a multi-code LUT on the first W
  *              bits of a window, a code-count LUT, and canonical limits for
  *              codes longer than W bits.
  *  code_len    the table: code length of every exponent value (0 = absent).
  *              Codes are canonical: ordered by (length, exponent value).
+ *  max_block_codes  the largest block_start[b + 1] - block_start[b]; the
+ *              decoder picks its on-chip buffer size from it (a block whose
+ *              span exceeds the buffer is reported as DF11_KERR_BAD_BLOCK).
  *
  * For the encode calls the pointers are HOST arrays the caller allocated
  * with the *_bytes sizes returned by the size call.  For the decode calls
@@ -102,6 +106,8 @@ typedef struct df11_tensor {
     uint64_t n_threads;  /* ceil(total_bits / (8 * n)) */
     uint64_t n_blocks;   /* ceil(n_threads / T) */
     df11_params params;
+    uint32_t max_block_codes; /* most codes in one thread block (set by the encoder) */
+    uint32_t reserved2;       /* 0 */
     uint8_t code_len[256];
     uint64_t enc_bytes;
     uint64_t sm_bytes;
@@ -120,7 +126,7 @@ typedef struct df11_tensor {
 /* ABI version of this header (bumped on any layout change) and
  * sizeof(df11_tensor) as compiled into the library, so that bindings can
  * check their mirror of the struct. */
-#define DF11_ABI_VERSION 1u
+#define DF11_ABI_VERSION 2u
 uint32_t df11_abi_version(void);
 size_t df11_sizeof_tensor(void);
 

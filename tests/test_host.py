@@ -30,7 +30,7 @@ def test_library_exports_every_declared_symbol():
     assert len(names) >= 14
     for name in names:
         assert hasattr(lib, name), name
-    assert df11._lib().df11_abi_version() == 1
+    assert df11._lib().df11_abi_version() == 2
 
 
 def test_status_strings():
@@ -80,6 +80,7 @@ def check_against_oracle(w, t, cap=32):
     a = oracle.aux(enc_o, bits_o, w.size, lengths, 8, 256)
     assert a["n_threads"] == t.n_threads and a["n_blocks"] == t.n_blocks
     assert np.array_equal(t.host_array("block_start")[: t.n_blocks + 1], a["block_start"])
+    assert t.desc.max_block_codes == (int(np.diff(a["block_start"]).max()) if t.n_blocks else 0)
     packed = t.host_array("gaps")
     n_fields = t.n_blocks * 256
     assert np.array_equal(_unpack_gaps(packed, n_fields), a["gaps"])
@@ -144,12 +145,13 @@ def test_invalid_params_rejected():
 
 def _lut_fields(lut: np.ndarray):
     b = lut.tobytes()
-    magic, w1, w2, max_len, min_len, n_syms = struct.unpack_from("<6I", b, 0)
+    magic, w1, w2, max_len, min_len, n_syms, w1_max, w2_max = struct.unpack_from("<8I", b, 0)
     lim = np.frombuffer(b, dtype=np.uint64, count=33, offset=64)
     offs = np.frombuffer(b, dtype=np.uint32, count=33, offset=336)
     symrot = lut[480:736]
-    clut = np.frombuffer(b, dtype=np.uint32, count=1 << 13, offset=768)
-    slut = np.frombuffer(b, dtype=np.uint32, count=2 << 12, offset=768 + 4 * (1 << 13)).reshape(-1, 2)
+    assert len(b) == 768 + 4 * (1 << w1_max) + 8 * (1 << w2_max)
+    clut = np.frombuffer(b, dtype=np.uint32, count=1 << w1_max, offset=768)
+    slut = np.frombuffer(b, dtype=np.uint32, count=2 << w2_max, offset=768 + 4 * (1 << w1_max)).reshape(-1, 2)
     return dict(magic=magic, w1=w1, w2=w2, max_len=max_len, lim=lim, offs=offs, symrot=symrot,
                 clut=clut, slut=slut)
 
@@ -169,7 +171,7 @@ def _walk(t):
     bits reach the thread's span; the decode pass stops on the code count.
     Returns (exponents in element order, per-thread counts)."""
     f = _lut_fields(t.host_array("lut"))
-    assert f["magic"] == 0x32314644
+    assert f["magic"] == 0x33314644
     enc = t.host_array("enc")
     bits_all = np.unpackbits(enc)
     gaps = _unpack_gaps(t.host_array("gaps"), t.n_blocks * 256 + 1) if t.n_blocks else np.zeros(1, np.uint8)
