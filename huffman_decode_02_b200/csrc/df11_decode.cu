@@ -350,8 +350,10 @@ __device__ __forceinline__ uint32_t decode_long_code(uint32_t pacc, uint32_t pen
 
 // Count pass for both chains of a thread (count table, fused accumulator).
 // Long codes are resolved in place (a short divergent branch), so all lanes
-// keep looping together.
-__device__ __forceinline__ void count_pass(const Chain &A, const Chain &B, uint32_t cnt_lane, uint32_t sh1,
+// keep looping together.  Table reads are plain C++ shared-memory loads so
+// the compiler may schedule and predicate freely; `cnt` points at this
+// lane's copy of the count table (entry i at cnt[i * kCountCopies]).
+__device__ __forceinline__ void count_pass(const Chain &A, const Chain &B, const uint32_t *cnt, uint32_t sh1,
                                            uint32_t s_lim, uint32_t from, uint32_t max_len, uint32_t &cA,
                                            uint32_t &cB, uint32_t &err) {
     uint32_t hA = A.hi, lA = A.lo, fA = A.fl, hB = B.hi, lB = B.lo, fB = B.fl;
@@ -362,11 +364,11 @@ __device__ __forceinline__ void count_pass(const Chain &A, const Chain &B, uint3
     uint32_t guard = kLoopCap;
     while (((aA < limA) | (aB < limB)) && guard != 0u) {
         --guard;
-        uint32_t eA = lds_u32(cnt_lane + ((hA >> sh1) << kCountShift));
-        uint32_t eB = lds_u32(cnt_lane + ((hB >> sh1) << kCountShift));
+        uint32_t eA = cnt[(hA >> sh1) * kCountCopies];
+        uint32_t eB = cnt[(hB >> sh1) * kCountCopies];
         eA = (aA < limA) ? eA : 0u;
         eB = (aB < limB) ? eB : 0u;
-        if ((eA | eB) >= kEscape) {
+        if ((eA | eB) >= kEscape) {  // rare: a long code
             if (eA == kEscape) eA = count_long_code(aA, limA, hA, lA, fA, s_lim, from, max_len, err);
             if (eB == kEscape) eB = count_long_code(aB, limB, hB, lB, fB, s_lim, from, max_len, err);
         }
@@ -385,25 +387,27 @@ __device__ __forceinline__ void count_pass(const Chain &A, const Chain &B, uint3
 }
 
 // Decoding pass for both chains of a thread: writes each code's rotated
-// exponent into the group buffer.  Symbol bytes are OR-ed into the (zeroed)
-// buffer, one or two aligned words per lookup; unused symbol bytes of a
-// table entry are zero.  Stops on the code counts of the count pass.
+// exponent into the group buffer `buf` (word-addressed).  Symbol bytes are
+// OR-ed into the (zeroed) buffer, one or two aligned words per lookup;
+// unused symbol bytes of a table entry are zero.  Stops on the code counts
+// of the count pass.  `sym` points at this lane's copy of the symbol table
+// (entry i at sym[i * kSymCopies]).
 __device__ __forceinline__ void decode_pass(const Chain &A, const Chain &B, uint32_t startA, uint32_t cA,
-                                            uint32_t startB, uint32_t cB, uint32_t sb, uint32_t sym_lane,
-                                            uint32_t sh2, uint32_t s_lim, uint32_t s_offs, uint32_t s_symrot,
-                                            uint32_t from, uint32_t max_len) {
+                                            uint32_t startB, uint32_t cB, uint32_t *buf, uint32_t sb,
+                                            const uint2 *sym, uint32_t sh2, uint32_t s_lim, uint32_t s_offs,
+                                            uint32_t s_symrot, uint32_t from, uint32_t max_len) {
     uint32_t hA = A.hi, lA = A.lo, fA = A.fl, hB = B.hi, lB = B.lo, fB = B.fl;
     uint32_t pA = startA << 8, pB = startB << 8;
     const uint32_t endPA = (startA + cA) << 8, endPB = (startB + cB) << 8;
     uint32_t guard = kLoopCap;  // as in the count pass
     while (((pA < endPA) | (pB < endPB)) && guard != 0u) {
         --guard;
-        const uint2 eA = lds_u2(sym_lane + ((hA >> sh2) << kSymShift));
-        const uint2 eB = lds_u2(sym_lane + ((hB >> sh2) << kSymShift));
+        const uint2 eA = sym[(hA >> sh2) * kSymCopies];
+        const uint2 eB = sym[(hB >> sh2) * kSymCopies];
         const bool actA = pA < endPA, actB = pB < endPB;
         uint32_t mA = actA ? eA.y : 0u;
         uint32_t mB = actB ? eB.y : 0u;
-        if ((mA | mB) >= kEscape) {
+        if ((mA | mB) >= kEscape) {  // rare: a long code
             if (mA == kEscape)
                 mA = decode_long_code(pA, endPA, hA, lA, fA, sb, s_lim, s_offs, s_symrot, from, max_len);
             if (mB == kEscape)
@@ -411,14 +415,15 @@ __device__ __forceinline__ void decode_pass(const Chain &A, const Chain &B, uint
         }
         const uint32_t bA = pA >> 8, bB = pB >> 8;
         const uint32_t shA = (bA & 3u) << 3, shB = (bB & 3u) << 3;
-        const uint32_t wA = sb + (bA & ~3u), wB = sb + (bB & ~3u);
-        if (actA) {  // (an escape entry has no symbol bytes: these OR zero)
-            red_or(wA, eA.x << shA);
-            if (shA) red_or(wA + 4u, __funnelshift_l(eA.x, 0u, shA));
+        uint32_t *wA = buf + (bA >> 2), *wB = buf + (bB >> 2);
+        // (an escape entry has no symbol bytes: its stores OR zero)
+        if (actA) {
+            atomicOr(wA, eA.x << shA);
+            if (shA) atomicOr(wA + 1, __funnelshift_l(eA.x, 0u, shA));
         }
         if (actB) {
-            red_or(wB, eB.x << shB);
-            if (shB) red_or(wB + 4u, __funnelshift_l(eB.x, 0u, shB));
+            atomicOr(wB, eB.x << shB);
+            if (shB) atomicOr(wB + 1, __funnelshift_l(eB.x, 0u, shB));
         }
         pA += mA;
         pB += mB;
@@ -486,8 +491,9 @@ __global__ void __launch_bounds__(C::kCtaThreads, 1) df11_decode_kernel(const De
     const uint32_t sb = grp;                  // exponent buffer
     const uint32_t wtot = grp + C::kGrpWtot;  // 4 warp totals
     const uint32_t mb_in = grp + C::kGrpMbar, mb_sm = grp + C::kGrpMbar + 8u;
-    const uint32_t cnt_lane = s_base + kOffCountRep + 4u * (lane % kCountCopies);
-    const uint32_t sym_lane = s_base + kOffSymRep + 8u * (lane % kSymCopies);
+    const uint32_t *cnt_lane = reinterpret_cast<const uint32_t *>(smem + kOffCountRep) + (lane % kCountCopies);
+    const uint2 *sym_lane = reinterpret_cast<const uint2 *>(smem + kOffSymRep) + (lane % kSymCopies);
+    uint32_t *buf = reinterpret_cast<uint32_t *>(smem + kOffGroups + group * C::kGroupBytes);
     uint32_t my_err = 0;
 
     const uint64_t stride = (uint64_t)gridDim.x * C::kGroups;
@@ -651,8 +657,8 @@ __global__ void __launch_bounds__(C::kCtaThreads, 1) df11_decode_kernel(const De
         // ---- pass 2: decode both chains again into the buffer
         if (ok) {
             const uint32_t startA = (s - base) + wpre + incl - cnt;  // buffer index of A's first code
-            decode_pass(A, B, startA, cA, startA + cA, cB, sb, sym_lane, sh2, s_lim, s_offs, s_symrot, w2 + 1u,
-                        max_len);
+            decode_pass(A, B, startA, cA, startA + cA, cB, buf, sb, sym_lane, sh2, s_lim, s_offs, s_symrot,
+                        w2 + 1u, max_len);
         }
         group_barrier(group);
 
