@@ -181,6 +181,7 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="llama8b-block")
+    ap.add_argument("--max-code-len", type=int, default=12, help="length cap of the exponent code")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -205,7 +206,7 @@ def main():
     # ---- workload: this rank's block, encoded on the host, uploaded once
     desc, gen = WORKLOADS[args.workload]
     mats = gen(rank)
-    blk = df11.encode_multi(mats, pinned=True)
+    blk = df11.encode_multi(mats, df11.Params(max_code_len=args.max_code_len), pinned=True)
     d = blk.to(dev)
     n = blk.n_elems
     scratch = torch.empty(n, dtype=torch.bfloat16, device=dev)
@@ -311,6 +312,7 @@ def main():
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "u32", "data": "synthetic",
             "config": {"workload": desc, "n_elems_per_rank": n, "bits_per_weight": round(blk.bits_per_weight(), 3),
+                       "max_code_len": int(blk.code_len.max()), "code_len_cap": args.max_code_len,
                        "parallelism": f"independent blocks x{world} (no collective on the data path)",
                        "l2": (f"inputs larger than L2 ({alg / 1e6:.0f} MB moved per step), no flush"
                               if alg > 2 * 126e6 else "L2-resident working set (small config; not a roofline claim)"),

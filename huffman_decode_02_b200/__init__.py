@@ -121,7 +121,7 @@ def _check(status: int, what: str) -> None:
 class Params:
     """Encoder parameters (see df11_params in include/df11.h)."""
 
-    def __init__(self, max_code_len: int = 32, bytes_per_thread: int = 8, threads_per_block: int = 256):
+    def __init__(self, max_code_len: int = 12, bytes_per_thread: int = 8, threads_per_block: int = 256):
         self.max_code_len = max_code_len
         self.bytes_per_thread = bytes_per_thread
         self.threads_per_block = threads_per_block

@@ -353,6 +353,7 @@ __device__ __forceinline__ uint32_t decode_long_code(uint32_t pacc, uint32_t pen
 // keep looping together.  Table reads are plain C++ shared-memory loads so
 // the compiler may schedule and predicate freely; `cnt` points at this
 // lane's copy of the count table (entry i at cnt[i * kCountCopies]).
+template <bool kLong>
 __device__ __forceinline__ void count_pass(const Chain &A, const Chain &B, const uint32_t *cnt, uint32_t sh1,
                                            uint32_t s_lim, uint32_t from, uint32_t max_len, uint32_t &cA,
                                            uint32_t &cB, uint32_t &err) {
@@ -368,7 +369,10 @@ __device__ __forceinline__ void count_pass(const Chain &A, const Chain &B, const
         uint32_t eB = cnt[(hB >> sh1) * kCountCopies];
         eA = (aA < limA) ? eA : 0u;
         eB = (aB < limB) ? eB : 0u;
-        if ((eA | eB) >= kEscape) {  // rare: a long code
+        // Long codes exist only when the code is longer than the window; an
+        // escape entry reaching the short-code instance (a corrupt table)
+        // sets bit 31 of the accumulator and stops that chain.
+        if (kLong && (eA | eB) >= kEscape) {  // rare: a long code
             if (eA == kEscape) eA = count_long_code(aA, limA, hA, lA, fA, s_lim, from, max_len, err);
             if (eB == kEscape) eB = count_long_code(aB, limB, hB, lB, fB, s_lim, from, max_len, err);
         }
@@ -392,6 +396,7 @@ __device__ __forceinline__ void count_pass(const Chain &A, const Chain &B, const
 // unused symbol bytes of a table entry are zero.  Stops on the code counts
 // of the count pass.  `sym` points at this lane's copy of the symbol table
 // (entry i at sym[i * kSymCopies]).
+template <bool kLong>
 __device__ __forceinline__ void decode_pass(const Chain &A, const Chain &B, uint32_t startA, uint32_t cA,
                                             uint32_t startB, uint32_t cB, uint32_t *buf, uint32_t sb,
                                             const uint2 *sym, uint32_t sh2, uint32_t s_lim, uint32_t s_offs,
@@ -407,7 +412,7 @@ __device__ __forceinline__ void decode_pass(const Chain &A, const Chain &B, uint
         const bool actA = pA < endPA, actB = pB < endPB;
         uint32_t mA = actA ? eA.y : 0u;
         uint32_t mB = actB ? eB.y : 0u;
-        if ((mA | mB) >= kEscape) {  // rare: a long code
+        if (kLong && (mA | mB) >= kEscape) {  // rare: a long code
             if (mA == kEscape)
                 mA = decode_long_code(pA, endPA, hA, lA, fA, sb, s_lim, s_offs, s_symrot, from, max_len);
             if (mB == kEscape)
@@ -472,7 +477,9 @@ __device__ __forceinline__ void issue_inputs(const DecodeArgs &a, uint64_t blk, 
     bulk_g2s(grp + C::kGrpBs, reinterpret_cast<const uint8_t *>(a.bstart) + ((4ull * blk) & ~15ull), 32u, mbar);
 }
 
-template <class C>
+// kLong: compiled with the long-code path (codes longer than the table
+// windows); without it the loops carry no escape handling at all.
+template <class C, bool kLong>
 __global__ void __launch_bounds__(C::kCtaThreads, 1) df11_decode_kernel(const DecodeArgs a) {
     extern __shared__ __align__(128) uint8_t smem[];
     const uint32_t s_base = smem_addr(smem);
@@ -622,7 +629,7 @@ __global__ void __launch_bounds__(C::kCtaThreads, 1) df11_decode_kernel(const De
 
         // ---- pass 1: count the codes of both chains
         uint32_t cA, cB;
-        count_pass(A, B, cnt_lane, sh1, s_lim, w1 + 1u, max_len, cA, cB, my_err);
+        count_pass<kLong>(A, B, cnt_lane, sh1, s_lim, w1 + 1u, max_len, cA, cB, my_err);
 
         // ---- clear the buffer span (the decoding pass ORs into it); the scan
         // barrier orders this before any write of the decoding pass
@@ -657,7 +664,7 @@ __global__ void __launch_bounds__(C::kCtaThreads, 1) df11_decode_kernel(const De
         // ---- pass 2: decode both chains again into the buffer
         if (ok) {
             const uint32_t startA = (s - base) + wpre + incl - cnt;  // buffer index of A's first code
-            decode_pass(A, B, startA, cA, startA + cA, cB, buf, sb, sym_lane, sh2, s_lim, s_offs, s_symrot,
+            decode_pass<kLong>(A, B, startA, cA, startA + cA, cB, buf, sb, sym_lane, sh2, s_lim, s_offs, s_symrot,
                         w2 + 1u, max_len);
         }
         group_barrier(group);
@@ -684,9 +691,9 @@ __global__ void __launch_bounds__(C::kCtaThreads, 1) df11_decode_kernel(const De
 std::atomic<int> g_sm_count[64];
 std::atomic<int> g_attr_set[64];
 
-template <class C>
+template <class C, bool kLong>
 cudaError_t set_smem_attr() {
-    return cudaFuncSetAttribute(df11_decode_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    return cudaFuncSetAttribute(df11_decode_kernel<C, kLong>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 (int)C::kSmemBytes);
 }
 
@@ -701,7 +708,8 @@ df11_status prepare_device(int *sm_count) {
         g_sm_count[dev].store(sms, std::memory_order_relaxed);
     }
     if (!g_attr_set[dev].load(std::memory_order_acquire)) {
-        if (set_smem_attr<CfgWide>() != cudaSuccess || set_smem_attr<CfgDense>() != cudaSuccess)
+        if (set_smem_attr<CfgWide, false>() != cudaSuccess || set_smem_attr<CfgWide, true>() != cudaSuccess ||
+            set_smem_attr<CfgDense, false>() != cudaSuccess || set_smem_attr<CfgDense, true>() != cudaSuccess)
             return DF11_ERR_CUDA;
         g_attr_set[dev].store(1, std::memory_order_release);
     }
@@ -711,11 +719,11 @@ df11_status prepare_device(int *sm_count) {
 
 bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
 
-template <class C>
+template <class C, bool kLong>
 void launch(const DecodeArgs &a, uint64_t n_blocks, int sms, cudaStream_t stream) {
     const uint64_t ctas_needed = (n_blocks + C::kGroups - 1) / C::kGroups;
     const unsigned grid = (unsigned)(ctas_needed < (uint64_t)sms ? ctas_needed : (uint64_t)sms);
-    df11_decode_kernel<C><<<grid, C::kCtaThreads, C::kSmemBytes, stream>>>(a);
+    df11_decode_kernel<C, kLong><<<grid, C::kCtaThreads, C::kSmemBytes, stream>>>(a);
 }
 
 df11_status launch_decode(const df11_tensor *t, uint16_t *out, uint32_t *err_word, void *stream) {
@@ -743,9 +751,16 @@ df11_status launch_decode(const df11_tensor *t, uint16_t *out, uint32_t *err_wor
     a.n_threads = t->n_threads;
     a.n_blocks = t->n_blocks;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    // a block's buffer span is at most its code count + 15
-    if (t->max_block_codes + 15u <= CfgWide::kBufSyms) launch<CfgWide>(a, t->n_blocks, sms, s);
-    else launch<CfgDense>(a, t->n_blocks, sms, s);
+    // a block's buffer span is at most its code count + 15; codes no longer
+    // than both table windows never take the long-code path
+    uint32_t max_len = 0;
+    for (int k = 0; k < 256; ++k) max_len = t->code_len[k] > max_len ? t->code_len[k] : max_len;
+    const bool lng = max_len > (uint32_t)(kW1Max < kW2Max ? kW1Max : kW2Max);
+    const bool wide = t->max_block_codes + 15u <= CfgWide::kBufSyms;
+    if (wide && !lng) launch<CfgWide, false>(a, t->n_blocks, sms, s);
+    else if (wide) launch<CfgWide, true>(a, t->n_blocks, sms, s);
+    else if (!lng) launch<CfgDense, false>(a, t->n_blocks, sms, s);
+    else launch<CfgDense, true>(a, t->n_blocks, sms, s);
     if (cudaGetLastError() != cudaSuccess) return DF11_ERR_CUDA;
     return DF11_OK;
 }

@@ -485,7 +485,7 @@ size_t df11_sizeof_tensor(void) { return sizeof(df11_tensor); }
 
 void df11_default_params(df11_params *p) {
     if (!p) return;
-    p->max_code_len = 32;
+    p->max_code_len = 12;
     p->bytes_per_thread = (uint32_t)kBytesPerThread;
     p->threads_per_block = (uint32_t)kThreadsPerBlockFmt;
     p->reserved = 0;

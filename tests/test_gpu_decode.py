@@ -54,7 +54,7 @@ def test_adversarial_bit_exact(name):
     _gpu_roundtrip(workloads.adversarial(name))
 
 
-@pytest.mark.parametrize("cap", [8, 12, 16, 24])
+@pytest.mark.parametrize("cap", [8, 12, 16, 24, 32])
 def test_length_cap_bit_exact(cap):
     _gpu_roundtrip(workloads.adversarial("fibonacci_exponents"), df11.Params(max_code_len=cap))
 
@@ -63,8 +63,10 @@ def test_long_codes_bit_exact():
     rng = np.random.default_rng(21)
     e = np.minimum(rng.geometric(0.42, size=3_000_001), 31) + 100
     w = ((e << 7) | rng.integers(0, 128, e.size) | (rng.integers(0, 2, e.size) << 15)).astype(np.uint16)
+    t, _, _ = _gpu_roundtrip(w, df11.Params(max_code_len=32))
+    assert t.code_len.max() > 20  # the long-code instance
     t, _, _ = _gpu_roundtrip(w)
-    assert t.code_len.max() > 20
+    assert t.code_len.max() == 12  # default cap: the short-code instance
 
 
 def test_config1_1024x1024_seed0():
@@ -75,6 +77,7 @@ def test_config1_1024x1024_seed0():
 
 def test_config2_4096x4096_seed1():
     _gpu_roundtrip(workloads.normal_matrix(4096, 4096, 0.02, seed=1))
+    _gpu_roundtrip(workloads.normal_matrix(4096, 4096, 0.02, seed=1), df11.Params(max_code_len=32))
 
 
 @pytest.mark.parametrize("n", [1, 7, 15, 16, 17, 255, 4096 + 3, 131_071, 2_000_003])
@@ -167,12 +170,14 @@ def test_bad_arguments_rejected():
 
 
 @pytest.mark.slow
-def test_config3_llama8b_block_full_size():
-    """The benchmark's workload, in the benchmark's launch configuration:
+@pytest.mark.parametrize("cap", [12, 32])
+def test_config3_llama8b_block_full_size(cap):
+    """The benchmark's workload, in the benchmark's launch configuration
+    (cap 12, the default), and with uncapped codes (cap 32, long-code path):
     every element compared with the oracle's decode of the same stream."""
     dev = _dev()
     mats = workloads.llama8b_block(seed=0)
-    blk = df11.encode_multi(mats)
+    blk = df11.encode_multi(mats, df11.Params(max_code_len=cap))
     assert blk.n_elems == 218_112_000
     d = blk.to(dev)
     scratch = torch.empty(blk.n_elems, dtype=torch.bfloat16, device=dev)
@@ -184,11 +189,14 @@ def test_config3_llama8b_block_full_size():
 
 
 @pytest.mark.slow
-def test_config4_heavy_tail_full_size():
+@pytest.mark.parametrize("cap", [32, 12])
+def test_config4_heavy_tail_full_size(cap):
+    """Long codes (cap 32: up to 27 bits, through the long-code path) and the
+    default 12-bit cap."""
     dev = _dev()
     w = workloads.heavy_tail_matrix(seed=4)
-    t = df11.encode(w)
-    assert t.code_len.max() >= 20
+    t = df11.encode(w, df11.Params(max_code_len=cap))
+    assert t.code_len.max() >= (20 if cap == 32 else 12)
     d = t.to(dev)
     got = _bits(df11.decode(d))
     ref = _oracle_decode(t)

@@ -53,7 +53,7 @@ CASES = ["all_bf16_patterns", "all_zero", "all_equal", "two_values", "random_u16
          "uniform_exponents", "fibonacci_exponents"]
 
 
-def check_against_oracle(w, t, cap=32):
+def check_against_oracle(w, t, cap=12):
     w = np.ascontiguousarray(w).reshape(-1).view(np.uint16)
     count = oracle.histogram(w)
     assert np.array_equal(df11.exponent_histogram([w]), count)
@@ -110,6 +110,10 @@ def test_encoder_normal_matrix_small():
     t = df11.encode(w)
     check_against_oracle(w, t)
     assert 9.5 < t.bits_per_weight() < 11.5
+    t32 = df11.encode(w, df11.Params(max_code_len=32))
+    check_against_oracle(w, t32, cap=32)
+    # the default 12-bit cap costs almost nothing on weight-like data
+    assert t.total_bits - t32.total_bits < 0.002 * t32.total_bits
 
 
 def test_encoder_multichunk_boundaries():
@@ -242,7 +246,7 @@ def test_table_walk_reproduces_exponents(name):
         w = ((e << 7) | rng.integers(0, 128, e.size)).astype(np.uint16)
     else:
         w = workloads.adversarial(name)[:20_000]
-    t = df11.encode(w)
+    t = df11.encode(w, df11.Params(max_code_len=32))
     expo, counts = _walk(t)
     assert np.array_equal(expo, (w.reshape(-1) >> 7) & 0xFF)
     bs = t.host_array("block_start")
