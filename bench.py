@@ -112,6 +112,24 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(rows)}
 
 
+def rank_seed(rank: int) -> int:
+    """Each rank decodes its own block (weak scaling): seed = rank."""
+    return rank
+
+
+def max_over_ranks(value: float, dist, device) -> float:
+    """The slowest rank's time (all ranks call this in the same order)."""
+    import torch
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_rate(bytes_per_rank: float, world: int, seconds_max: float) -> float:
+    """Whole-job decoded GB/s: every rank's bytes over the slowest rank's time."""
+    return bytes_per_rank * world / seconds_max / 1e9
+
+
 def algorithmic_bytes(t) -> int:
     """Bytes one decode launch must move: exponent stream, sign/mantissa,
     gaps, block starts and decode tables read once, BF16 written once."""
@@ -205,7 +223,7 @@ def main():
 
     # ---- workload: this rank's block, encoded on the host, uploaded once
     desc, gen = WORKLOADS[args.workload]
-    mats = gen(rank)
+    mats = gen(rank_seed(rank))
     blk = df11.encode_multi(mats, df11.Params(max_code_len=args.max_code_len), pinned=True)
     d = blk.to(dev)
     n = blk.n_elems
@@ -249,12 +267,10 @@ def main():
     clocks = sampler.stop()
     ms_total = e0.elapsed_time(e1)
     if world > 1:
-        tt = torch.tensor([ms_total], dtype=torch.float64, device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms_total = float(tt.item())
+        ms_total = max_over_ranks(ms_total, dist, dev)
     assert df11.read_error(err, stream) == 0
     ms_step = ms_total / args.steps
-    value = 2.0 * n * world / (ms_step * 1e-3) / 1e9  # decoded BF16 GB/s, all ranks
+    value = aggregate_rate(2.0 * n, world, ms_step * 1e-3)  # decoded BF16 GB/s, all ranks
 
     peak, peak_kind = _peaks()
     alg = algorithmic_bytes(blk)
@@ -284,9 +300,7 @@ def main():
     torch.cuda.synchronize(dev)
     e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
     if world > 1:
-        tt = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e2e_ms = float(tt.item())
+        e2e_ms = max_over_ranks(e2e_ms, dist, dev)
     e2e_ok = bool(np.array_equal(host_out.view(torch.int16).numpy().view(np.uint16)[:1_000_000],
                                  mats[0].reshape(-1)[:1_000_000]))
 
@@ -323,7 +337,7 @@ def main():
                          "peak_kind": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs, copy burst)"
                          if peak_kind == "measured" else "fallback 6650 GB/s",
                          "algorithmic_bytes_per_launch": alg},
-            "e2e": {"value": 2.0 * n * world / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+            "e2e": {"value": aggregate_rate(2.0 * n, world, e2e_ms * 1e-3), "unit": "GB/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": 2 * n, "ms_per_step": e2e_ms,
                     "bit_exact_sample": e2e_ok},
             "gpu_launches": args.steps,
