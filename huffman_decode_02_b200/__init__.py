@@ -30,7 +30,7 @@ from . import build as _build
 
 __all__ = [
     "DF11Error", "CorruptStreamError", "Params", "DF11Tensor", "encode", "encode_multi",
-    "decode", "decode_block", "read_error", "exponent_histogram", "lib_path", "sm_count",
+    "decode", "decode_block", "gemm", "read_error", "exponent_histogram", "lib_path", "sm_count",
     "KERR_COUNT_MISMATCH", "KERR_BAD_CODE", "KERR_BAD_BLOCK", "KERR_OVERRUN", "KERR_TIMEOUT",
 ]
 
@@ -106,6 +106,7 @@ def _lib():
     lib.df11_decode_block.argtypes = [P(T), P(u64), u32, vp, vp, vp]
     lib.df11_read_error.argtypes = [vp, vp, P(u32)]
     lib.df11_device_sm_count.argtypes = [P(ctypes.c_int)]
+    lib.df11_gemm_bf16.argtypes = [vp, vp, vp, u32, u32, u32, vp, vp]
     if lib.df11_abi_version() != 2 or lib.df11_sizeof_tensor() != ctypes.sizeof(_Tensor):
         raise ImportError("libdf11.so ABI does not match this binding")
     _LIB = lib
@@ -346,6 +347,31 @@ def decode_block(t: DF11Tensor, scratch=None, err=None, stream=None):
     if own_err:
         read_error(err, stream)
     return scratch
+
+
+def gemm(x, w, out=None, err=None, stream=None):
+    """Y = X @ W^T on the tensor cores: x [T, in] and w [out, in] BF16 CUDA
+    tensors (w may be a view of a decoded block), FP32 result [T, out]."""
+    import torch
+    if x.dtype != torch.bfloat16 or w.dtype != torch.bfloat16 or x.dim() != 2 or w.dim() != 2:
+        raise TypeError("gemm expects 2-D bfloat16 tensors")
+    if not x.is_contiguous() or not w.is_contiguous():
+        raise ValueError("gemm expects contiguous tensors")
+    T, k = x.shape
+    n, k2 = w.shape
+    if k != k2:
+        raise ValueError("inner dimensions differ")
+    if out is None:
+        out = torch.empty(T, n, dtype=torch.float32, device=x.device)
+    own_err = err is None
+    if own_err:
+        err = _new_err(x.device)
+    _check(_lib().df11_gemm_bf16(ctypes.c_void_p(x.data_ptr()), ctypes.c_void_p(w.data_ptr()),
+                                 ctypes.c_void_p(out.data_ptr()), T, n, k, ctypes.c_void_p(err.data_ptr()),
+                                 _stream_handle(stream)), "gemm")
+    if own_err:
+        read_error(err, stream)
+    return out
 
 
 def read_error(err, stream=None) -> int:

@@ -1,0 +1,308 @@
+// df11_gemm.cu -- the consumer of the decoded weights: Y = X * W^T in BF16
+// with FP32 accumulation on the 5th-generation tensor cores (tcgen05),
+// reading W straight from the decode scratch buffer.
+//
+// Sources: "DFloat11 : compression sans perte pour l'inference GPU qui reduit
+// les LLM a 70 % de leur taille" (fr.news.hada.io), << Decompression adaptee
+// a l'inference GPU >>: the weight matrix is decompressed to BF16 right
+// before its matrix multiplication and discarded after it.
+//
+// Shapes: X [T, in] (activations, row-major), W [out, in] (nn.Linear weight,
+// row-major), Y [T, out] FP32.  T is small (1..256 tokens), so the product
+// is computed transposed (Y^T = W X^T): the UMMA M dimension is 128 rows of
+// W, N is T rounded up to 16, K advances 16 per instruction.
+//
+// One CTA computes a 128-row tile of W over a range of K (split-K when there
+// are too few row tiles to fill the SMs; partial tiles are added into Y,
+// which the launcher zeroes first).  128 threads: one thread issues TMA
+// loads (W and X tiles, 128-byte swizzle, no multicast) into a ring of
+// shared-memory stages, one thread issues tcgen05.mma into an FP32
+// accumulator in tensor memory and releases each stage with tcgen05.commit,
+// and all four warps read the accumulator back (tcgen05.ld) and write Y.
+// Every wait is bounded; a timed-out wait sets an error bit and the CTA
+// still frees its tensor memory before leaving.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+#include <stdint.h>
+
+#include <atomic>
+#include <mutex>
+
+#include "df11.h"
+
+namespace {
+
+constexpr uint32_t kBlockM = 128;      // rows of W per tile (UMMA M)
+constexpr uint32_t kBlockK = 64;       // K per stage: 64 BF16 = one 128-byte swizzle row
+constexpr uint32_t kUmmaK = 16;        // K per tcgen05.mma (kind::f16)
+constexpr uint32_t kThreads = 128;
+constexpr uint32_t kMaxStages = 8;
+constexpr uint32_t kSmemBudget = 200u * 1024u;
+constexpr uint32_t kGemmErrTimeout = 0x20u;
+constexpr uint32_t kSpin = 1u << 24;   // bounded waits
+
+struct GemmArgs {
+    float *y;
+    uint32_t *err;
+    uint32_t T, out, in;
+    uint32_t n_pad;      // UMMA N: T rounded up to 16
+    uint32_t k_tiles;    // in / 64
+    uint32_t splits;     // CTAs per row tile along K
+    uint32_t stages;
+    uint32_t tmem_cols;  // power of two >= 32 and >= n_pad
+    uint32_t atomic_out; // 1: add into Y (split-K), 0: store
+};
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+    uint32_t done = 0;
+    for (uint32_t it = 0; it < kSpin && !done; ++it) {
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(done)
+            : "r"(bar), "r"(parity)
+            : "memory");
+    }
+    return done != 0;
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, uint32_t bar, int32_t x,
+                                            int32_t y) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];" ::"r"(
+            dst),
+        "l"(map), "r"(bar), "r"(x), "r"(y)
+        : "memory");
+}
+
+// Shared-memory matrix descriptor for a K-major tile written by TMA with the
+// 128-byte swizzle: rows of 128 bytes, 8-row groups 1024 bytes apart.
+__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr) {
+    uint64_t d = 0;
+    d |= (uint64_t)((addr >> 4) & 0x3FFFu);        // start address
+    d |= (uint64_t)1u << 16;                       // leading byte offset (unused with swizzle)
+    d |= (uint64_t)(1024u >> 4) << 32;             // stride byte offset: 8 rows x 128 B
+    d |= (uint64_t)1u << 46;                       // descriptor version (sm_100)
+    d |= (uint64_t)2u << 61;                       // layout: 128-byte swizzle
+    return d;
+}
+
+// Instruction descriptor: BF16 x BF16 -> FP32, both operands K-major.
+__device__ __forceinline__ uint32_t instr_desc_bf16(uint32_t n, uint32_t m) {
+    return (1u << 4)            // D format F32
+           | (1u << 7)          // A format BF16
+           | (1u << 10)         // B format BF16
+           | ((n >> 3) << 17)   // N / 8
+           | ((m >> 4) << 24);  // M / 16
+}
+
+__device__ __forceinline__ void umma_bf16(uint32_t tmem_d, uint64_t da, uint64_t db, uint32_t idesc,
+                                          uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+        "l"(da), "l"(db), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+__device__ __forceinline__ void umma_commit(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+                 : "memory");
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    df11_gemm_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUtensorMap map_x,
+                     const GemmArgs g) {
+    extern __shared__ __align__(1024) uint8_t smem[];
+    const uint32_t tid = threadIdx.x, warp = tid >> 5, lane = tid & 31u;
+    const uint32_t a_bytes = kBlockM * kBlockK * 2u;
+    const uint32_t b_bytes = g.n_pad * kBlockK * 2u;
+    const uint32_t stage_bytes = (a_bytes + b_bytes + 1023u) & ~1023u;
+    // smem: [stages x (A | B)] [full[S]] [empty[S]] [acc_full] [tmem address]
+    const uint32_t base = (smem_u32(smem) + 1023u) & ~1023u;
+    const uint32_t bars = base + g.stages * stage_bytes;
+    const uint32_t full0 = bars, empty0 = bars + 8u * kMaxStages, acc_full = bars + 16u * kMaxStages;
+    const uint32_t tmem_slot = acc_full + 8u;
+    uint8_t *tmem_slot_ptr = smem + (tmem_slot - smem_u32(smem));
+
+    const uint32_t m_tile = blockIdx.x / g.splits, split = blockIdx.x % g.splits;
+    const uint32_t kt_per = (g.k_tiles + g.splits - 1u) / g.splits;
+    const uint32_t kt0 = split * kt_per;
+    const uint32_t kt1 = min(g.k_tiles, kt0 + kt_per);
+    uint32_t err = 0;
+
+    if (tid == 0) {
+        for (uint32_t s = 0; s < g.stages; ++s) {
+            asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(full0 + 8u * s) : "memory");
+            asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(empty0 + 8u * s) : "memory");
+        }
+        asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(acc_full) : "memory");
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 2) {  // one full warp allocates the accumulator columns
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(tmem_slot),
+                     "r"(g.tmem_cols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    __syncthreads();
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    const uint32_t tmem_d = *reinterpret_cast<volatile uint32_t *>(tmem_slot_ptr);
+    const uint32_t n_kt = kt1 > kt0 ? kt1 - kt0 : 0u;
+
+    if (warp == 0 && lane == 0) {
+        // ---- producer: TMA loads of W (128 x 64) and X (n_pad x 64) tiles
+        for (uint32_t i = 0; i < n_kt; ++i) {
+            const uint32_t s = i % g.stages, use = i / g.stages;
+            if (!mbar_wait(empty0 + 8u * s, (use & 1u) ^ 1u)) { err |= kGemmErrTimeout; break; }
+            const uint32_t sa = base + s * stage_bytes, sbb = sa + a_bytes;
+            asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(full0 + 8u * s),
+                         "r"(a_bytes + b_bytes)
+                         : "memory");
+            const int32_t k = (int32_t)((kt0 + i) * kBlockK);
+            tma_load_2d(sa, &map_w, full0 + 8u * s, k, (int32_t)(m_tile * kBlockM));
+            tma_load_2d(sbb, &map_x, full0 + 8u * s, k, 0);
+        }
+    } else if (warp == 1 && lane == 0) {
+        // ---- MMA issuer: 4 UMMAs of K = 16 per stage, then release the stage
+        const uint32_t idesc = instr_desc_bf16(g.n_pad, kBlockM);
+        for (uint32_t i = 0; i < n_kt; ++i) {
+            const uint32_t s = i % g.stages, use = i / g.stages;
+            if (!mbar_wait(full0 + 8u * s, use & 1u)) { err |= kGemmErrTimeout; break; }
+            asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+            const uint32_t sa = base + s * stage_bytes, sbb = sa + a_bytes;
+#pragma unroll
+            for (uint32_t kk = 0; kk < kBlockK / kUmmaK; ++kk) {
+                // advancing K by 16 BF16 = 32 bytes inside the swizzled row
+                umma_bf16(tmem_d, smem_desc_sw128(sa + kk * 32u), smem_desc_sw128(sbb + kk * 32u), idesc,
+                          (i | kk) != 0u ? 1u : 0u);
+            }
+            umma_commit(empty0 + 8u * s);
+        }
+        umma_commit(acc_full);  // fires once every issued MMA has completed
+    }
+    __syncwarp();
+
+    // ---- epilogue: warp w owns accumulator lanes 32w..32w+31 (rows of W)
+    const bool have = n_kt > 0 && mbar_wait(acc_full, 0u);
+    if (n_kt > 0 && !have) err |= kGemmErrTimeout;
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    const uint32_t row = m_tile * kBlockM + warp * 32u + lane;
+    for (uint32_t c0 = 0; c0 < g.n_pad; c0 += 16u) {
+        uint32_t v[16];
+        asm volatile(
+            "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
+            "%14, %15}, [%16];"
+            : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+              "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
+            : "r"(tmem_d + ((warp * 32u) << 16) + c0));
+        asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+        if (have) {
+#pragma unroll
+            for (uint32_t j = 0; j < 16; ++j) {
+                const uint32_t t = c0 + j;
+                if (t < g.T) {
+                    float *dst = g.y + (uint64_t)t * g.out + row;
+                    if (g.atomic_out) atomicAdd(dst, __uint_as_float(v[j]));
+                    else *dst = __uint_as_float(v[j]);
+                }
+            }
+        }
+    }
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    __syncthreads();
+    if (warp == 2) {
+        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_d), "r"(g.tmem_cols)
+                     : "memory");
+    }
+    if (err && g.err) atomicOr(g.err, err);
+}
+
+// ---------------------------------------------------------------- host
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+std::atomic<int> g_gemm_attr[64];
+
+bool get_encoder() {
+    std::call_once(g_encode_once, [] {
+        void *fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    });
+    return g_encode != nullptr;
+}
+
+// 2-D BF16 tensor map over a row-major [rows, cols] matrix, box [box_rows, 64]
+// with the 128-byte swizzle; rows past the end read as zero.
+bool make_map(CUtensorMap *m, const void *ptr, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+    const cuuint64_t dims[2] = {cols, rows};
+    const cuuint64_t strides[1] = {cols * 2u};
+    const cuuint32_t box[2] = {kBlockK, box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    return g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(ptr), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+extern "C" df11_status df11_gemm_bf16(const uint16_t *x, const uint16_t *w, float *y, uint32_t T, uint32_t out,
+                                      uint32_t in, uint32_t *err_word, void *stream) {
+    if (!x || !w || !y) return DF11_ERR_INVALID_ARG;
+    if (T == 0 || T > 256 || out == 0 || out % kBlockM != 0 || in == 0 || in % kBlockK != 0)
+        return DF11_ERR_UNSUPPORTED;
+    if (((uintptr_t)x & 15u) || ((uintptr_t)w & 15u) || ((uintptr_t)y & 3u)) return DF11_ERR_INVALID_ARG;
+    if (!get_encoder()) return DF11_ERR_CUDA;
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return DF11_ERR_CUDA;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return DF11_ERR_CUDA;
+
+    GemmArgs g;
+    g.y = y;
+    g.err = err_word;
+    g.T = T;
+    g.out = out;
+    g.in = in;
+    g.n_pad = (T + 15u) & ~15u;
+    g.k_tiles = in / kBlockK;
+    g.tmem_cols = 32;
+    while (g.tmem_cols < g.n_pad) g.tmem_cols <<= 1;
+    const uint32_t m_tiles = out / kBlockM;
+    uint32_t splits = (uint32_t)sms / m_tiles;
+    if (splits < 1) splits = 1;
+    if (splits > g.k_tiles) splits = g.k_tiles;
+    // no empty split: every CTA gets at least one K tile
+    const uint32_t kt_per = (g.k_tiles + splits - 1) / splits;
+    splits = (g.k_tiles + kt_per - 1) / kt_per;
+    g.splits = splits;
+    g.atomic_out = splits > 1 ? 1u : 0u;
+    const uint32_t stage_bytes = ((kBlockM + g.n_pad) * kBlockK * 2u + 1023u) & ~1023u;
+    g.stages = kSmemBudget / stage_bytes;
+    if (g.stages > kMaxStages) g.stages = kMaxStages;
+    if (g.stages < 2) return DF11_ERR_UNSUPPORTED;
+    const uint32_t smem = 1024u + g.stages * stage_bytes + 8u * (2u * kMaxStages + 2u);
+
+    CUtensorMap mw, mx;
+    if (!make_map(&mw, w, out, in, kBlockM) || !make_map(&mx, x, T, in, g.n_pad)) return DF11_ERR_CUDA;
+    if (!g_gemm_attr[dev].load(std::memory_order_acquire)) {
+        if (cudaFuncSetAttribute(df11_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)(1024u + kSmemBudget + 8u * (2u * kMaxStages + 2u))) != cudaSuccess)
+            return DF11_ERR_CUDA;
+        g_gemm_attr[dev].store(1, std::memory_order_release);
+    }
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (g.atomic_out && cudaMemsetAsync(y, 0, (size_t)T * out * sizeof(float), s) != cudaSuccess)
+        return DF11_ERR_CUDA;
+    df11_gemm_kernel<<<m_tiles * splits, kThreads, smem, s>>>(mw, mx, g);
+    if (cudaGetLastError() != cudaSuccess) return DF11_ERR_CUDA;
+    return DF11_OK;
+}

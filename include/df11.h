@@ -190,6 +190,20 @@ df11_status df11_decode(const df11_tensor *t, uint16_t *out, uint32_t *err_word,
 df11_status df11_decode_block(const df11_tensor *blk, const uint64_t *mat_offsets, uint32_t k,
                               uint16_t *scratch, uint32_t *err_word, void *stream);
 
+/* Consumer of a decoded weight matrix: Y = X * W^T with BF16 inputs and FP32
+ * accumulation on the tensor cores (tcgen05), the matrix multiplication the
+ * decompressed weights feed ("Decompression adaptee a l'inference GPU": a
+ * matrix is decompressed right before its multiplication and discarded after).
+ *  x: DEVICE [T, in] BF16 (uint16 bits), row-major, 16-byte aligned
+ *  w: DEVICE [out, in] BF16, row-major (nn.Linear layout; e.g. a view of a
+ *     decoded block's scratch buffer), 16-byte aligned
+ *  y: DEVICE [T, out] FP32, row-major; fully overwritten
+ *  Limits: 1 <= T <= 256, out a multiple of 128, in a multiple of 64;
+ *  otherwise DF11_ERR_UNSUPPORTED.  err_word as in df11_decode (a wait that
+ *  timed out sets bit 0x20); may be NULL.  Asynchronous on `stream`. */
+df11_status df11_gemm_bf16(const uint16_t *x, const uint16_t *w, float *y, uint32_t T, uint32_t out,
+                           uint32_t in, uint32_t *err_word, void *stream);
+
 /* Copies *err_word to the host after the stream's work so far completes
  * (synchronises the stream) and returns DF11_ERR_CORRUPT if any bit is set. */
 df11_status df11_read_error(const uint32_t *err_word, void *stream, uint32_t *host_value);

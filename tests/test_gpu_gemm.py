@@ -1,0 +1,81 @@
+"""The consumer GEMM (tcgen05, FP32 accumulation) against a CPU GEMM: the
+relative Frobenius error must stay within 2e-3.  Inputs are BF16, so every
+product is exact in FP32 and the two sides differ only in summation order."""
+import numpy as np
+import pytest
+
+import workloads
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+import huffman_decode_02_b200 as df11  # noqa: E402
+
+TOL = 2e-3
+
+
+def _dev():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    return torch.device("cuda:0")
+
+
+def _bf16(a: np.ndarray) -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16)
+
+
+def _rel_fro(y, ref):
+    return float(np.linalg.norm(y - ref) / np.linalg.norm(ref))
+
+
+def _check(T, out, inn, seed):
+    dev = _dev()
+    rng = np.random.default_rng(seed)
+    x = workloads.round_to_bf16(rng.standard_normal((T, inn), dtype=np.float32))
+    w = workloads.round_to_bf16(rng.standard_normal((out, inn), dtype=np.float32) * np.float32(0.02))
+    xt, wt = _bf16(x), _bf16(w)
+    ref = xt.double() @ wt.double().T  # CPU reference
+    y = df11.gemm(xt.to(dev), wt.to(dev))
+    torch.cuda.synchronize()
+    assert y.shape == (T, out) and y.dtype == torch.float32
+    assert _rel_fro(y.cpu().double().numpy(), ref.numpy()) <= TOL
+
+
+@pytest.mark.parametrize("T", [1, 16, 64, 256])
+def test_gemm_q_proj_shape(T):
+    _check(T, 4096, 4096, seed=1000 + T)
+
+
+@pytest.mark.parametrize("T,out,inn", [(5, 1024, 4096), (33, 128, 64), (256, 14336, 4096), (16, 4096, 14336),
+                                       (200, 256, 128)])
+def test_gemm_other_shapes(T, out, inn):
+    _check(T, out, inn, seed=T + out)
+
+
+def test_gemm_rejects_unsupported():
+    dev = _dev()
+    x = torch.zeros(4, 100, dtype=torch.bfloat16, device=dev)
+    w = torch.zeros(128, 100, dtype=torch.bfloat16, device=dev)
+    with pytest.raises(df11.DF11Error):
+        df11.gemm(x, w)  # in not a multiple of 64
+    x = torch.zeros(300, 64, dtype=torch.bfloat16, device=dev)
+    w = torch.zeros(128, 64, dtype=torch.bfloat16, device=dev)
+    with pytest.raises(df11.DF11Error):
+        df11.gemm(x, w)  # T > 256
+
+
+def test_decode_then_gemm_from_scratch():
+    """Decode a small block into a scratch buffer, multiply straight from the
+    matrix views (the decode -> consumer path)."""
+    dev = _dev()
+    mats = [workloads.normal_matrix(512, 256, 0.02, seed=1), workloads.normal_matrix(256, 512, 0.03, seed=2)]
+    blk = df11.encode_multi(mats).to(dev)
+    scratch = df11.decode_block(blk)
+    views = blk.views(scratch)
+    rng = np.random.default_rng(9)
+    for w, v in zip(mats, views):
+        x = workloads.round_to_bf16(rng.standard_normal((64, w.shape[1]), dtype=np.float32))
+        xt = _bf16(x)
+        y = df11.gemm(xt.to(dev), v.contiguous())
+        ref = xt.double() @ _bf16(w).double().T
+        assert _rel_fro(y.cpu().double().numpy(), ref.numpy()) <= TOL
