@@ -46,6 +46,9 @@ WORKLOADS = {
                    lambda r: [workloads.heavy_tail_matrix(seed=4 + r)]),
     "down-proj": ("single 4096x14336 matrix, N(0, 0.03^2), seed = rank (profiling size)",
                   lambda r: [workloads.normal_matrix(4096, 14336, 0.03, seed=r)]),
+    "decode-gemm": ("32 llama3.1-8b blocks (seeds 32*rank + 0..31), each decoded into one reused BF16 scratch, "
+                    "then every matrix multiplied by N(0,1) BF16 activations [T, in], T in {1,16,64,256} "
+                    "(seed 1000 + T), FP32-accumulate GEMM on tcgen05", None),
 }
 WORKLOAD = WORKLOADS["llama8b-block"][0]
 
@@ -190,6 +193,133 @@ def run_reference(args, rank: int, world: int):
     print(json.dumps(line), flush=True)
 
 
+def _encode_block_worker(seed: int, cap: int):
+    """Generates and encodes one block in a worker process; returns the
+    compressed arrays and a checksum of the original bits."""
+    import huffman_decode_02_b200 as df11
+    mats = workloads.llama8b_block(seed=seed)
+    blk = df11.encode_multi(mats, df11.Params(max_code_len=cap))
+    flat = np.concatenate([m.reshape(-1) for m in mats]).astype(np.int64)
+    idx = np.arange(flat.size, dtype=np.int64) & 0xFFFF
+    chk = (int(flat.sum()), int((flat * idx).sum()))
+    return bytes(blk.desc), {k: np.asarray(v) for k, v in blk.arrays.items()}, blk.shapes, blk.offsets, chk
+
+
+def run_decode_gemm(args, rank: int, world: int):
+    """Decode -> consumer GEMM over a sequence of blocks: per T, the decode
+    time, the GEMM time and the total per block, next to plain BF16 GEMMs
+    (torch.matmul on the same decoded weights) as the uncompressed baseline."""
+    import multiprocessing as mp
+    seeds = [args.blocks * rank + b for b in range(args.blocks)]
+    workers = max(1, min(len(seeds), (os.cpu_count() or 1) // 2, 16))
+    t0 = time.time()
+    with mp.get_context("spawn").Pool(workers) as pool:  # before any CUDA call
+        enc = pool.starmap(_encode_block_worker, [(sd, args.max_code_len) for sd in seeds])
+    encode_s = time.time() - t0
+
+    import torch
+    import torch.distributed as dist
+
+    import huffman_decode_02_b200 as df11
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=dev)
+    blocks = []
+    for desc, arrays, shapes, offsets, chk in enc:
+        t = df11.DF11Tensor(df11._Tensor.from_buffer_copy(desc), arrays, "cpu", shapes, offsets)
+        blocks.append((t.to(dev), chk))
+    del enc
+    n = blocks[0][0].n_elems
+    scratch = torch.empty(n, dtype=torch.bfloat16, device=dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    idx = torch.arange(n, device=dev, dtype=torch.int64) & 0xFFFF
+    ok = True
+    for d, chk in blocks:  # every block decodes to its original bits (checksums)
+        df11.decode_block(d, scratch, err, stream)
+        v = scratch.view(torch.int16).to(torch.int64) & 0xFFFF
+        ok &= (int(v.sum()), int((v * idx).sum())) == chk
+        del v
+    del idx
+    assert df11.read_error(err, stream) == 0
+    views = blocks[0][0].views(scratch)
+    gemm_mats = views[:7]  # q, k, v, o, gate, up, down (the norms are not GEMM operands)
+    ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+
+    def timed(fn, steps):
+        fn()
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+        a, b = ev(), ev()
+        a.record(stream)
+        for _ in range(steps):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        ms = a.elapsed_time(b) / steps
+        return max_over_ranks(ms, dist, dev) if world > 1 else ms
+
+    per_T = {}
+    nb = len(blocks)
+    w_bytes = sum(int(w.numel()) * 2 for w in gemm_mats)
+    for T in (1, 16, 64, 256):
+        g = torch.Generator().manual_seed(1000 + T)
+        xs = {k: torch.randn(T, k, generator=g).to(torch.bfloat16).to(dev) for k in {w.shape[1] for w in gemm_mats}}
+        ys = [torch.empty(T, w.shape[0], dtype=torch.float32, device=dev) for w in gemm_mats]
+        # numerics of this configuration: sampled columns vs an FP64 GEMM
+        rel = 0.0
+        for w, y in zip(gemm_mats, ys):
+            df11.gemm(xs[w.shape[1]], w, y, err, stream)
+            cols = torch.arange(0, w.shape[0], max(1, w.shape[0] // 256), device=dev)
+            ref = xs[w.shape[1]].double() @ w[cols].double().T
+            rel = max(rel, float((y[:, cols].double() - ref).norm() / ref.norm()))
+
+        def dec_all():
+            for d, _ in blocks:
+                df11.decode_block(d, scratch, err, stream)
+
+        def gemm_all():
+            for _ in range(nb):
+                for w, y in zip(gemm_mats, ys):
+                    df11.gemm(xs[w.shape[1]], w, y, err, stream)
+
+        def both():
+            for d, _ in blocks:
+                df11.decode_block(d, scratch, err, stream)
+                for w, y in zip(gemm_mats, ys):
+                    df11.gemm(xs[w.shape[1]], w, y, err, stream)
+
+        def bf16_all():
+            for _ in range(nb):
+                for w in gemm_mats:
+                    torch.matmul(xs[w.shape[1]], w.T)
+
+        t_dec, t_gemm, t_both, t_bf16 = (timed(f, args.steps) / nb for f in (dec_all, gemm_all, both, bf16_all))
+        x_bytes = sum(T * w.shape[1] * 2 + T * w.shape[0] * 4 for w in gemm_mats)
+        per_T[str(T)] = {"decode_us": t_dec * 1e3, "gemm_us": t_gemm * 1e3, "total_us": t_both * 1e3,
+                         "bf16_gemm_us": t_bf16 * 1e3, "slowdown_vs_bf16": t_both / t_bf16,
+                         "gemm_gbs": (w_bytes + x_bytes) / (t_gemm * 1e-3) / 1e9, "gemm_rel_fro": rel}
+    assert df11.read_error(err, stream) == 0
+    if rank == 0:
+        desc = WORKLOADS["decode-gemm"][0]
+        line = {"metric": "decode->GEMM time per llama3.1-8b block", "value": per_T["1"]["total_us"], "unit": "us",
+                "n_gpus": world, "steps": args.steps, "warmup": 1, "higher_is_better": False, "scaling": "weak",
+                "vs_baseline": None, "dtype": "bf16 x bf16 -> f32 (GEMM), u32 (decode)", "data": "synthetic",
+                "config": {"workload": desc, "blocks_per_rank": nb, "n_elems_per_block": n,
+                           "value_is": "total per block at T=1",
+                           "l2": "436 MB scratch and 300 MB compressed per block, larger than L2; no flush"},
+                "checksums_ok": ok, "per_T": per_T, "host_encode_s": round(encode_s, 1),
+                "gpu_launches_per_block": 8}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -200,6 +330,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="llama8b-block")
     ap.add_argument("--max-code-len", type=int, default=12, help="length cap of the exponent code")
+    ap.add_argument("--blocks", type=int, default=32, help="blocks of the decode-gemm workload")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -208,6 +339,9 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         run_reference(args, rank, world)
+        return
+    if args.workload == "decode-gemm":
+        run_decode_gemm(args, rank, world)
         return
 
     import torch

@@ -79,3 +79,34 @@ def test_decode_then_gemm_from_scratch():
         y = df11.gemm(xt.to(dev), v.contiguous())
         ref = xt.double() @ _bf16(w).double().T
         assert _rel_fro(y.cpu().double().numpy(), ref.numpy()) <= TOL
+
+
+@pytest.mark.slow
+def test_config5_decode_then_gemm_full_blocks():
+    """Llama-8B-shaped blocks (seeds 0 and 31 of the 32-block sequence) decoded
+    one after the other into the same scratch, each matrix multiplied by
+    N(0,1) BF16 activations [T, in] (seed 1000 + T) for T in {1, 16, 64, 256};
+    512 sampled output columns per product are checked against an FP64 CPU
+    GEMM of the original weights."""
+    dev = _dev()
+    names = ["q", "k", "v", "o", "gate", "up", "down"]
+    scratch = None
+    rng_cols = np.random.default_rng(5)
+    for seed in (0, 31):
+        mats = workloads.llama8b_block(seed=seed)
+        blk = df11.encode_multi(mats).to(dev)
+        if scratch is None:
+            scratch = torch.empty(blk.n_elems, dtype=torch.bfloat16, device=dev)
+        df11.decode_block(blk, scratch)
+        views = blk.views(scratch)
+        for T in (1, 16, 64, 256):
+            xs = {}
+            for name, w, v in zip(names, mats, views):
+                inn = w.shape[1]
+                if inn not in xs:
+                    r = np.random.default_rng(1000 + T)
+                    xs[inn] = _bf16(workloads.round_to_bf16(r.standard_normal((T, inn), dtype=np.float32)))
+                y = df11.gemm(xs[inn].to(dev), v).cpu().double().numpy()
+                cols = rng_cols.choice(w.shape[0], 512, replace=False)
+                ref = (xs[inn].double() @ _bf16(w[cols]).double().T).numpy()
+                assert _rel_fro(y[:, cols], ref) <= TOL, (seed, T, name)
