@@ -19,12 +19,13 @@
 //  * Persistent CTAs, one per SM (1024 threads = 8 groups of 128).  Each
 //    group decodes one format block (256 format threads x 8 bytes) at a
 //    time and strides over the blocks.  The compact decode tables arrive by
-//    one TMA bulk copy (cp.async.bulk, no multicast) and are replicated in
-//    shared memory so that each lane reads its own copy (near
-//    conflict-free random lookups).  Each group's next-block inputs (stream
-//    bytes, gaps, block starts) and first sign/mantissa vectors are fetched
-//    by bulk copies on per-group mbarriers, so no register holds prefetched
-//    data across the decode loops.
+//    one TMA bulk copy (cp.async.bulk, no multicast); the count table is
+//    kept in two interleaved copies (lane l reads copy l mod 2).
+//  * Per group, bulk copies on mbarriers bring the next block's inputs
+//    (stream bytes, gaps, block starts) and the current block's whole
+//    sign/mantissa range into shared memory, so the merge reads nothing
+//    from global memory and no register holds prefetched data across the
+//    decode loops.
 //  * The exponent buffer holds 8192 symbols per group; tensors whose blocks
 //    hold more codes (average code under 2 bits) use a second instance with
 //    4 groups of 16 KB buffers.
@@ -38,21 +39,19 @@
 //    gap) are set to 1: a run of ones shorter than the longest code is never
 //    a whole code of a canonical code, so a table lookup can never take a
 //    code that belongs to the next thread.
-//  * Pass 1 counts with a 14-bit count table (several codes per lookup);
+//  * Pass 1 counts with a 12-bit count table (several codes per lookup);
 //    one add per lookup updates both the code count and the bits taken,
-//    the entry's low bits are the shift amount, and a code longer than the
-//    window leaves the loop through its condition (flag bit), so the loop
-//    body is a lookup, an add, three funnel shifts and a compare.
+//    and the entry's low bits are the shift amount.
 //  * Pass 2 decodes with a 12-bit table of up to four symbols per entry and
-//    stops on the code count pass 1 found.  Codes longer than the window
-//    fall back to canonical limits.
+//    stops on the code count pass 1 found; the symbol bytes are OR-ed into
+//    the clear buffer (a word is touched only when it receives a symbol).
+//    Codes longer than the window fall back to canonical limits.
 //  * Warp shuffle scan + one cross-warp step (named barrier per group).
+//    Two group barriers per block: the merge clears the buffer chunks it
+//    reads, so the next block needs no barrier of its own before decoding.
 //  * Exponents are kept rotated by one bit, so the merge with the
 //    sign/mantissa bytes is two bit-selects and two byte-permutes per four
-//    weights; loads and stores are 128-bit.  The next block's stream words,
-//    gaps and block starts, and this block's first sign/mantissa vectors,
-//    are loaded before the decode loops so their latency hides behind the
-//    arithmetic.
+//    weights; stores are 32 bytes per thread (whole sectors per warp).
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -72,17 +71,17 @@ using namespace df11;
 //   kOffSymRep               symbol table, kSymCopies copies interleaved:
 //                            entry i of copy c at u64 (i * kSymCopies + c)
 //   kOffGroups               per group: exponent buffer, warp totals, staged
-//                            inputs of the next block, the first
-//                            sign/mantissa vectors of this one, 2 mbarriers
+//                            inputs of the next block, this block's
+//                            sign/mantissa bytes, 2 mbarriers
 //   table mbarrier
-// Lane l reads copy (l mod copies), so the 32 random lookups of a warp fall
-// in different banks: a lookup costs one or two shared-memory wavefronts
-// instead of the 3..8 of a single table.
+// Lane l reads copy (l mod copies).  Random lookups still meet bank
+// conflicts (a warp's lookup costs several wavefronts); more copies cut
+// them little and take the room the staged sign/mantissa bytes need.
 #ifndef DF11_COUNT_COPIES
-#define DF11_COUNT_COPIES 4
+#define DF11_COUNT_COPIES 2
 #endif
 #ifndef DF11_SYM_COPIES
-#define DF11_SYM_COPIES 2
+#define DF11_SYM_COPIES 1
 #endif
 constexpr uint32_t kCountCopies = DF11_COUNT_COPIES;
 constexpr uint32_t kSymCopies = DF11_SYM_COPIES;
@@ -95,7 +94,6 @@ constexpr uint32_t kOffSymRep = kOffCountRep + 4u * kCountCopies * (1u << kW1Max
 constexpr uint32_t kOffGroups = kOffSymRep + 8u * kSymCopies * (1u << kW2Max);
 constexpr uint32_t kEncStage = kThreadsPerBlockFmt * kBytesPerThread + 16u;  // + next block's first 16
 constexpr uint32_t kGapStage = kThreadsPerBlockFmt * 5u / 8u + 16u;          // + next block's first gaps
-constexpr uint32_t kSmStage = 16u * kGroupThreads;                           // one vector per thread
 constexpr uint32_t kFull = 0xFFFFFFFFu;
 #ifndef DF11_LOOP_CAP
 #define DF11_LOOP_CAP 128
@@ -117,10 +115,9 @@ struct Cfg {
     static constexpr uint32_t kGrpEnc = kGrpWtot + 16u;
     static constexpr uint32_t kGrpGap = kGrpEnc + kEncStage;
     static constexpr uint32_t kGrpBs = kGrpGap + kGapStage;
-    static constexpr uint32_t kGrpSm = kGrpBs + 32u;
-    // the first sign/mantissa vectors are staged when shared memory allows
-    static constexpr bool kStageSm = kOffGroups + G * (kGrpSm + kSmStage + 16u) + 16u <= 227u * 1024u;
-    static constexpr uint32_t kGrpMbar = kGrpSm + (kStageSm ? kSmStage : 0u);
+    static constexpr uint32_t kGrpSm = kGrpBs + 32u;  // the block's sign/mantissa bytes
+    static constexpr uint32_t kSmBytes = S + 16u;
+    static constexpr uint32_t kGrpMbar = kGrpSm + kSmBytes;
     static constexpr uint32_t kGroupBytes = kGrpMbar + 16u;
     static constexpr uint32_t kSmemBytes = kOffGroups + G * kGroupBytes + 16u;
     static_assert(S % 16 == 0, "whole chunks");
@@ -146,15 +143,15 @@ struct DecodeArgs {
     uint64_t total_bits;
     uint64_t n_threads;
     uint64_t n_blocks;
+    uint32_t out_al32;  // out is 32-byte aligned: whole-chunk stores are 32 bytes
 };
 
 // ----------------------------------------------------------------- PTX
-__device__ __forceinline__ uint4 ld_stream_u4(const void *p) {
-    uint4 r;
-    asm("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
-        : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
-        : "l"(p));
-    return r;
+// 32-byte store (sm_100): one warp instruction writes 1 KB of whole sectors.
+__device__ __forceinline__ void st_u8x32(void *p, const uint32_t o[8]) {
+    asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(o[0]), "r"(o[1]), "r"(o[2]),
+                 "r"(o[3]), "r"(o[4]), "r"(o[5]), "r"(o[6]), "r"(o[7])
+                 : "memory");
 }
 __device__ __forceinline__ void st_u4(void *p, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
     asm volatile("st.global.v4.b32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(a), "r"(b), "r"(c), "r"(d)
@@ -287,6 +284,16 @@ __device__ __forceinline__ void merge_edges(const uint8_t *sm, uint16_t *out, ui
         const uint32_t lo8 = (r & 0x80u) | (sm8 & 0x7Fu);
         out[g] = (uint16_t)(lo8 | (hi8 << 8));
     }
+}
+// merge_edges, then clears the two edge chunks (whole warp, converged).
+__device__ __forceinline__ void merge_edges_clear(const uint8_t *sm, uint16_t *out, uint32_t sb, uint32_t base,
+                                                  uint32_t c_full, uint32_t span, uint32_t s, uint32_t e,
+                                                  uint32_t lane) {
+    merge_edges(sm, out, sb, base, c_full, span, s, e, lane);
+    __syncwarp();
+    const bool head = s != base;
+    const bool tail = (span & 15u) != 0u && !(head && c_full == 0u);
+    if ((lane == 0u && head) || (lane == 16u && tail)) sts_zero16(sb + 16u * (lane == 0u ? 0u : c_full));
 }
 
 // One decode chain: the 96-bit window (hi, lo, fl) of a format thread and
@@ -422,13 +429,15 @@ __device__ __forceinline__ void decode_pass(const Chain &A, const Chain &B, uint
         const uint32_t shA = (bA & 3u) << 3, shB = (bB & 3u) << 3;
         uint32_t *wA = buf + (bA >> 2), *wB = buf + (bB >> 2);
         // (an escape entry has no symbol bytes: its stores OR zero)
+        // the second word only when symbol bytes reach it (OR with zero is a no-op)
+        const uint32_t hiA = __funnelshift_l(eA.x, 0u, shA), hiB = __funnelshift_l(eB.x, 0u, shB);
         if (actA) {
             atomicOr(wA, eA.x << shA);
-            if (shA) atomicOr(wA + 1, __funnelshift_l(eA.x, 0u, shA));
+            if (hiA) atomicOr(wA + 1, hiA);
         }
         if (actB) {
             atomicOr(wB, eB.x << shB);
-            if (shB) atomicOr(wB + 1, __funnelshift_l(eB.x, 0u, shB));
+            if (hiB) atomicOr(wB + 1, hiB);
         }
         pA += mA;
         pB += mB;
@@ -442,25 +451,27 @@ __device__ __forceinline__ void decode_pass(const Chain &A, const Chain &B, uint
 }
 
 // Merges chunks c_first, c_first + 128, ... < c_end (chunk c covers output
-// elements base + 16c .. +16, at buffer offset 16c) with sign/mantissa.
-__device__ __forceinline__ void merge_chunks(const uint8_t *sm, uint16_t *out, uint32_t sb, uint32_t base,
-                                             uint32_t c_first, uint32_t c_end, uint4 smv) {
-    if (c_first >= c_end) return;
-    const uint8_t *smp = sm + (uint64_t)base + 16ull * c_first;
-    uint16_t *dst = out + (uint64_t)base + 16ull * c_first;
-    uint32_t ex_addr = sb + 16u * c_first;
-    for (uint32_t c = c_first;;) {
-        const uint4 ex = lds_u4(ex_addr);
+// elements base + 16c .. +16, at buffer offset 16c) with their sign/mantissa
+// bytes, staged in shared memory from chunk c_lo on at `sm_s`, and clears
+// each buffer chunk it reads (the decoding pass ORs into a clear buffer).
+// Stores are 32 bytes per thread when `out` is 32-byte aligned (one warp
+// instruction writes 1 KB of whole sectors), else two 16-byte stores.
+__device__ __forceinline__ void merge_chunks(uint16_t *out, uint32_t sb, uint32_t base, uint32_t c_first,
+                                             uint32_t c_end, uint32_t sm_s, uint32_t c_lo, uint32_t al32) {
+    for (uint32_t c = c_first; c < c_end; c += kGroupThreads) {
+        const uint4 smv = lds_u4(sm_s + 16u * (c - c_lo));
+        const uint4 ex = lds_u4(sb + 16u * c);
+        sts_zero16(sb + 16u * c);
         uint32_t o[8];
         merge16(smv, ex, o);
-        st_u4(dst, o[0], o[1], o[2], o[3]);
-        st_u4(dst + 8, o[4], o[5], o[6], o[7]);
-        c += kGroupThreads;
-        if (c >= c_end) break;
-        smp += 16u * kGroupThreads;
-        dst += 16u * kGroupThreads;
-        ex_addr += 16u * kGroupThreads;
-        smv = ld_stream_u4(smp);
+        uint16_t *dst = out + (uint64_t)base + 16ull * c;
+        if (al32) {
+            st_u8x32(dst, o);
+        } else
+        {
+            st_u4(dst, o[0], o[1], o[2], o[3]);
+            st_u4(dst + 8, o[4], o[5], o[6], o[7]);
+        }
     }
 }
 
@@ -571,6 +582,9 @@ __global__ void __launch_bounds__(C::kCtaThreads, 1) df11_decode_kernel(const De
     }
     const uint32_t sh1 = 32u - w1, sh2 = 32u - w2;
 
+    // The exponent buffer starts clear; the merge clears what it reads.
+    for (uint32_t c = lt; c < C::kSbufBytes / 16u; c += kGroupThreads) sts_zero16(sb + 16u * c);
+
     // ---- the group's mbarriers (inputs of the next block; first
     // sign/mantissa vectors of this one) and its first block's inputs
     if (lt == 0) {
@@ -595,18 +609,6 @@ __global__ void __launch_bounds__(C::kCtaThreads, 1) df11_decode_kernel(const De
         const uint32_t c_lo = (s != base) ? 1u : 0u;
         const uint32_t c_full = span >> 4;  // chunks [c_lo, c_full) lie wholly inside [s, e)
         const uint32_t c0 = c_lo + lt;
-        if (C::kStageSm && lt == 0) {
-            // this block's first sign/mantissa vectors (one per thread), up to
-            // the end of the block's last chunk; always at least 16 bytes
-            const uint32_t from = range_ok ? base + 16u * c_lo : 0u;
-            const uint32_t upto = range_ok ? ((e + 15u) & ~15u) : 16u;
-            const uint32_t bytes = upto > from ? min(kSmStage, upto - from) : 16u;
-            const uint32_t src = upto > from ? from : (range_ok ? base : 0u);
-            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-            mbar_expect(mb_sm, bytes);
-            bulk_g2s(grp + C::kGrpSm, a.sm + src, bytes, mb_sm);
-        }
-
         // ---- the two chains: format threads tA and tA + 1
         const uint4 v = lds_u4(grp + C::kGrpEnc + 16u * lt);
         const uint32_t nextw = lds_u32(grp + C::kGrpEnc + 16u * lt + 16u);
@@ -631,11 +633,6 @@ __global__ void __launch_bounds__(C::kCtaThreads, 1) df11_decode_kernel(const De
         uint32_t cA, cB;
         count_pass<kLong>(A, B, cnt_lane, sh1, s_lim, w1 + 1u, max_len, cA, cB, my_err);
 
-        // ---- clear the buffer span (the decoding pass ORs into it); the scan
-        // barrier orders this before any write of the decoding pass
-        // (OR-stores reach buffer index span + 2 at most: bytes [0, span + 4))
-        for (uint32_t c = lt; c < (span + 19u) >> 4; c += kGroupThreads) sts_zero16(sb + 16u * c);
-
         // ---- block scan: warp inclusive scan, then across the group's warps
         const uint32_t cnt = cA + cB;
         uint32_t incl = cnt;
@@ -650,6 +647,19 @@ __global__ void __launch_bounds__(C::kCtaThreads, 1) df11_decode_kernel(const De
         // every thread has read this block's staged inputs: fetch the next
         const uint64_t nxt = blk + stride;
         if (lt == 0 && nxt < a.n_blocks) issue_inputs<C>(a, nxt, grp, mb_in);
+        // and this block's sign/mantissa bytes (chunks c_lo .. the block's
+        // last chunk; always at least 16 bytes).  Every thread of the group
+        // has passed its previous merge, so the staging area is free.
+        if (lt == 0) {
+            const uint32_t from = range_ok ? base + 16u * c_lo : 0u;
+            const uint32_t upto = range_ok ? ((e + 15u) & ~15u) : 16u;
+            const uint32_t bytes = upto > from ? min(C::kSmBytes, upto - from) : 16u;
+            const uint32_t src = upto > from ? from : (range_ok ? base : 0u);
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            mbar_expect(mb_sm, bytes);
+            bulk_g2s(grp + C::kGrpSm, a.sm + src, bytes, mb_sm);
+        }
+
         uint32_t wsum = (lane < kWarps) ? lds_u32(wtot + 4u * lane) : 0u;
 #pragma unroll
         for (uint32_t d = 1; d < kWarps; d <<= 1) {
@@ -670,19 +680,15 @@ __global__ void __launch_bounds__(C::kCtaThreads, 1) df11_decode_kernel(const De
         group_barrier(group);
 
         // ---- merge with sign/mantissa and store, 16 weights per step
-        if (C::kStageSm) {
-            if (!wait_phase(mb_sm, ph_sm)) my_err |= kKernErrTimeout;
-            ph_sm ^= 1u;
-        }
+        if (!wait_phase(mb_sm, ph_sm)) my_err |= kKernErrTimeout;
+        ph_sm ^= 1u;
         if (ok) {
-            uint4 smv0 = make_uint4(0, 0, 0, 0);
-            if (c0 < c_full)
-                smv0 = C::kStageSm ? lds_u4(grp + C::kGrpSm + 16u * lt)
-                                   : ld_stream_u4(a.sm + (uint64_t)base + 16ull * c0);
-            merge_chunks(a.sm, a.out, sb, base, c0, c_full, smv0);
-            if (warp == 0) merge_edges(a.sm, a.out, sb, base, c_full, span, s, e, lane);
+            merge_chunks(a.out, sb, base, c0, c_full, grp + C::kGrpSm, c_lo, a.out_al32);
+            if (warp == 0) merge_edges_clear(a.sm, a.out, sb, base, c_full, span, s, e, lane);
         }
-        group_barrier(group);
+        // No barrier here: the next block's buffer writes and staging copies
+        // come after its scan barrier, which every thread reaches only after
+        // this merge.
     }
     if (my_err && a.err) atomicOr(a.err, my_err);
 }
@@ -750,6 +756,7 @@ df11_status launch_decode(const df11_tensor *t, uint16_t *out, uint32_t *err_wor
     a.total_bits = t->total_bits;
     a.n_threads = t->n_threads;
     a.n_blocks = t->n_blocks;
+    a.out_al32 = ((uintptr_t)out & 31u) == 0 ? 1u : 0u;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     // a block's buffer span is at most its code count + 15; codes no longer
     // than both table windows never take the long-code path
