@@ -14,7 +14,10 @@
 //
 // One CTA computes a 128-row tile of W over a range of K (split-K when there
 // are too few row tiles to fill the SMs; partial tiles are added into Y,
-// which the launcher zeroes first).  128 threads: one thread issues TMA
+// which the launcher zeroes first).  A stage holds one or two 64-wide K
+// sub-tiles: two when T <= 128, so that each W row is read 256 contiguous
+// bytes at a time (better DRAM locality for the weight stream), one when
+// the X tiles are large (a deeper ring).  128 threads: one thread issues TMA
 // loads (W and X tiles, 128-byte swizzle, no multicast) into a ring of
 // shared-memory stages, one thread issues tcgen05.mma into an FP32
 // accumulator in tensor memory and releases each stage with tcgen05.commit,
@@ -34,7 +37,7 @@
 namespace {
 
 constexpr uint32_t kBlockM = 128;      // rows of W per tile (UMMA M)
-constexpr uint32_t kBlockK = 64;       // K per stage: 64 BF16 = one 128-byte swizzle row
+constexpr uint32_t kBlockK = 64;       // K per sub-tile: 64 BF16 = one 128-byte swizzle row
 constexpr uint32_t kUmmaK = 16;        // K per tcgen05.mma (kind::f16)
 constexpr uint32_t kThreads = 128;
 constexpr uint32_t kMaxStages = 8;
@@ -47,7 +50,8 @@ struct GemmArgs {
     uint32_t *err;
     uint32_t T, out, in;
     uint32_t n_pad;      // UMMA N: T rounded up to 16
-    uint32_t k_tiles;    // in / 64
+    uint32_t sub;        // 64-wide K sub-tiles per stage (1 or 2)
+    uint32_t k_tiles;    // K stages: in / (64 sub)
     uint32_t splits;     // CTAs per row tile along K
     uint32_t stages;
     uint32_t tmem_cols;  // power of two >= 32 and >= n_pad
@@ -120,8 +124,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                      const GemmArgs g) {
     extern __shared__ __align__(1024) uint8_t smem[];
     const uint32_t tid = threadIdx.x, warp = tid >> 5, lane = tid & 31u;
-    const uint32_t a_bytes = kBlockM * kBlockK * 2u;
-    const uint32_t b_bytes = g.n_pad * kBlockK * 2u;
+    const uint32_t a_sub = kBlockM * kBlockK * 2u, b_sub = g.n_pad * kBlockK * 2u;
+    const uint32_t a_bytes = g.sub * a_sub;
+    const uint32_t b_bytes = g.sub * b_sub;
     const uint32_t stage_bytes = (a_bytes + b_bytes + 1023u) & ~1023u;
     // smem: [stages x (A | B)] [full[S]] [empty[S]] [acc_full] [tmem address]
     const uint32_t base = (smem_u32(smem) + 1023u) & ~1023u;
@@ -165,9 +170,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(full0 + 8u * s),
                          "r"(a_bytes + b_bytes)
                          : "memory");
-            const int32_t k = (int32_t)((kt0 + i) * kBlockK);
-            tma_load_2d(sa, &map_w, full0 + 8u * s, k, (int32_t)(m_tile * kBlockM));
-            tma_load_2d(sbb, &map_x, full0 + 8u * s, k, 0);
+            for (uint32_t j = 0; j < g.sub; ++j) {
+                const int32_t k = (int32_t)(((kt0 + i) * g.sub + j) * kBlockK);
+                tma_load_2d(sa + j * a_sub, &map_w, full0 + 8u * s, k, (int32_t)(m_tile * kBlockM));
+                tma_load_2d(sbb + j * b_sub, &map_x, full0 + 8u * s, k, 0);
+            }
         }
     } else if (warp == 1 && lane == 0) {
         // ---- MMA issuer: 4 UMMAs of K = 16 per stage, then release the stage
@@ -177,11 +184,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!mbar_wait(full0 + 8u * s, use & 1u)) { err |= kGemmErrTimeout; break; }
             asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
             const uint32_t sa = base + s * stage_bytes, sbb = sa + a_bytes;
+            for (uint32_t j = 0; j < g.sub; ++j) {
 #pragma unroll
-            for (uint32_t kk = 0; kk < kBlockK / kUmmaK; ++kk) {
-                // advancing K by 16 BF16 = 32 bytes inside the swizzled row
-                umma_bf16(tmem_d, smem_desc_sw128(sa + kk * 32u), smem_desc_sw128(sbb + kk * 32u), idesc,
-                          (i | kk) != 0u ? 1u : 0u);
+                for (uint32_t kk = 0; kk < kBlockK / kUmmaK; ++kk) {
+                    // advancing K by 16 BF16 = 32 bytes inside the swizzled row
+                    umma_bf16(tmem_d, smem_desc_sw128(sa + j * a_sub + kk * 32u),
+                              smem_desc_sw128(sbb + j * b_sub + kk * 32u), idesc, (i | j | kk) != 0u ? 1u : 0u);
+                }
             }
             umma_commit(empty0 + 8u * s);
         }
@@ -273,7 +282,8 @@ extern "C" df11_status df11_gemm_bf16(const uint16_t *x, const uint16_t *w, floa
     g.out = out;
     g.in = in;
     g.n_pad = (T + 15u) & ~15u;
-    g.k_tiles = in / kBlockK;
+    g.sub = (g.n_pad <= 128u && in % (2u * kBlockK) == 0u) ? 2u : 1u;
+    g.k_tiles = in / (g.sub * kBlockK);
     g.tmem_cols = 32;
     while (g.tmem_cols < g.n_pad) g.tmem_cols <<= 1;
     const uint32_t m_tiles = out / kBlockM;
@@ -285,7 +295,7 @@ extern "C" df11_status df11_gemm_bf16(const uint16_t *x, const uint16_t *w, floa
     splits = (g.k_tiles + kt_per - 1) / kt_per;
     g.splits = splits;
     g.atomic_out = splits > 1 ? 1u : 0u;
-    const uint32_t stage_bytes = ((kBlockM + g.n_pad) * kBlockK * 2u + 1023u) & ~1023u;
+    const uint32_t stage_bytes = (g.sub * (kBlockM + g.n_pad) * kBlockK * 2u + 1023u) & ~1023u;
     g.stages = kSmemBudget / stage_bytes;
     if (g.stages > kMaxStages) g.stages = kMaxStages;
     if (g.stages < 2) return DF11_ERR_UNSUPPORTED;
