@@ -49,6 +49,9 @@ WORKLOADS = {
     "decode-gemm": ("32 llama3.1-8b blocks (seeds 32*rank + 0..31), each decoded into one reused BF16 scratch, "
                     "then every matrix multiplied by N(0,1) BF16 activations [T, in], T in {1,16,64,256} "
                     "(seed 1000 + T), FP32-accumulate GEMM on tcgen05", None),
+    "offload": ("llama3.1-8b blocks (seeds 0..B-1, default 4) kept in pinned host memory and streamed over PCIe "
+                "block by block, repeated; each decoded on the GPU and multiplied by BF16 activations [1, in]; "
+                "compared with streaming the same blocks as plain BF16", None),
 }
 WORKLOAD = WORKLOADS["llama8b-block"][0]
 
@@ -193,6 +196,12 @@ def run_reference(args, rank: int, world: int):
     print(json.dumps(line), flush=True)
 
 
+def _encode_block_raw_worker(seed: int, cap: int):
+    """As `_encode_block_worker`, also returning the original matrices."""
+    out = _encode_block_worker(seed, cap)
+    return out + (workloads.llama8b_block(seed=seed),)
+
+
 def _encode_block_worker(seed: int, cap: int):
     """Generates and encodes one block in a worker process; returns the
     compressed arrays and a checksum of the original bits."""
@@ -320,6 +329,96 @@ def run_decode_gemm(args, rank: int, world: int):
         dist.destroy_process_group()
 
 
+def run_offload(args, rank: int, world: int):
+    """Blocks streamed from pinned host memory: compressed (copy, decode,
+    consume) against plain BF16 (copy, consume), both double-buffered so the
+    copy of block b+1 overlaps the GPU work of block b.  The consumer is the
+    block's seven GEMMs at T = 1."""
+    import multiprocessing as mp
+    nb = args.blocks if args.blocks_given else 4
+    seeds = [nb * rank + b for b in range(nb)]
+    with mp.get_context("spawn").Pool(max(1, min(nb, (os.cpu_count() or 1) // 2, 8))) as pool:
+        enc = pool.starmap(_encode_block_raw_worker, [(sd, args.max_code_len) for sd in seeds])
+
+    import torch
+    import torch.distributed as dist
+
+    import huffman_decode_02_b200 as df11
+    from huffman_decode_02_b200.offload import BlockStreamer, RawStreamer
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=dev)
+    blocks, raws, chks = [], [], []
+    for desc, arrays, shapes, offsets, chk, mats in enc:
+        pinned = {k: torch.empty(max(a.size, 16), dtype=torch.uint8, pin_memory=True) for k, a in arrays.items()}
+        for k, a in arrays.items():
+            pinned[k][: a.size].copy_(torch.from_numpy(a.view(np.uint8)))
+        blocks.append(df11.DF11Tensor(df11._Tensor.from_buffer_copy(desc), pinned, "cpu", shapes, offsets))
+        raws.append(mats)
+        chks.append(chk)
+    del enc
+    streamer = BlockStreamer(blocks, dev)
+    raw = RawStreamer(raws, dev)
+    del raws
+    gemm_shapes = [tuple(s) for s in blocks[0].shapes[:7]]
+    g = torch.Generator().manual_seed(1001)
+    xs = {k: torch.randn(1, k, generator=g).to(torch.bfloat16).to(dev) for k in {s[1] for s in gemm_shapes}}
+    ys = {"df11": [torch.empty(1, s[0], dtype=torch.float32, device=dev) for s in gemm_shapes],
+          "bf16": [torch.empty(1, s[0], dtype=torch.float32, device=dev) for s in gemm_shapes]}
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+
+    def consumer(key):
+        def f(bi, views):
+            for w, y in zip(views[:7], ys[key]):
+                df11.gemm(xs[w.shape[1]], w, y, err)
+        return f
+
+    stream = torch.cuda.current_stream(dev)
+    order = list(range(nb)) * args.repeat
+
+    def timed(run):
+        run(list(range(nb)))  # warm-up pass over every block
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        run(order)
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        ms = a.elapsed_time(b) / len(order)
+        return max_over_ranks(ms, dist, dev) if world > 1 else ms
+
+    ms_df11 = timed(lambda o: streamer.run(o, consumer("df11")))
+    streamer.check()
+    v = streamer.scratch[: blocks[order[-1]].n_elems].view(torch.int16).to(torch.int64) & 0xFFFF
+    idx = torch.arange(v.numel(), device=dev, dtype=torch.int64) & 0xFFFF
+    ok = (int(v.sum()), int((v * idx).sum())) == chks[order[-1]]
+    del v, idx
+    ms_bf16 = timed(lambda o: raw.run(o, consumer("bf16")))
+    assert df11.read_error(err) == 0
+    rel = max(float((a - b).norm() / b.norm()) for a, b in zip(ys["df11"], ys["bf16"]))
+    if rank == 0:
+        h2d_c = sum(streamer.h2d_bytes) / nb
+        h2d_r = sum(raw.h2d_bytes) / nb
+        line = {"metric": "offloaded decode->GEMM time per llama3.1-8b block streamed from host memory",
+                "value": ms_df11, "unit": "ms", "n_gpus": world, "steps": len(order), "warmup": nb,
+                "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
+                "dtype": "u32 (decode), bf16 x bf16 -> f32 (GEMM, T=1)", "data": "synthetic",
+                "config": {"workload": WORKLOADS["offload"][0], "blocks_per_rank": nb, "repeat": args.repeat},
+                "bf16_offload_ms_per_block": ms_bf16, "speedup_vs_bf16_offload": ms_bf16 / ms_df11,
+                "h2d_bytes_per_block": {"df11": h2d_c, "bf16": h2d_r},
+                "h2d_gbs": {"df11": h2d_c / ms_df11 / 1e6, "bf16": h2d_r / ms_bf16 / 1e6},
+                "checksum_ok": ok, "gemm_rel_diff_df11_vs_bf16": rel}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -330,8 +429,12 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="llama8b-block")
     ap.add_argument("--max-code-len", type=int, default=12, help="length cap of the exponent code")
-    ap.add_argument("--blocks", type=int, default=32, help="blocks of the decode-gemm workload")
+    ap.add_argument("--blocks", type=int, default=None, help="blocks of the decode-gemm (32) / offload (4) workloads")
+    ap.add_argument("--repeat", type=int, default=4, help="passes over the blocks in the offload workload")
     args = ap.parse_args()
+    args.blocks_given = args.blocks is not None
+    if args.blocks is None:
+        args.blocks = 32
     args.warmup = max(args.warmup, 3)
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -342,6 +445,9 @@ def main():
         return
     if args.workload == "decode-gemm":
         run_decode_gemm(args, rank, world)
+        return
+    if args.workload == "offload":
+        run_offload(args, rank, world)
         return
 
     import torch

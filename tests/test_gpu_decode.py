@@ -202,3 +202,20 @@ def test_config4_heavy_tail_full_size(cap):
     ref = _oracle_decode(t)
     np.testing.assert_array_equal(got, ref)
     np.testing.assert_array_equal(ref, w.reshape(-1))
+
+
+@pytest.mark.parametrize("offset_elems", [8, 16])
+def test_output_alignment_paths(offset_elems):
+    """Whole-chunk stores are 32 bytes when the output is 32-byte aligned and
+    two 16-byte stores otherwise: both paths bit-exact, nothing written
+    outside the output range."""
+    dev = _dev()
+    w = workloads.normal_matrix(777, 301, 0.02, seed=12)
+    d = df11.encode(w).to(dev)
+    buf = torch.full((w.size + 64,), -1, dtype=torch.int16, device=dev)
+    out = buf[offset_elems: offset_elems + w.size].view(torch.bfloat16)
+    df11.decode(d, out)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(_bits(out), w.reshape(-1))
+    rest = torch.cat([buf[:offset_elems], buf[offset_elems + w.size:]])
+    assert bool((rest == -1).all())
