@@ -46,6 +46,9 @@ WORKLOADS = {
                    lambda r: [workloads.heavy_tail_matrix(seed=4 + r)]),
     "down-proj": ("single 4096x14336 matrix, N(0, 0.03^2), seed = rank (profiling size)",
                   lambda r: [workloads.normal_matrix(4096, 14336, 0.03, seed=r)]),
+    "lm-head": ("llama3.1-8b LM head / embedding shape 128256x4096 (525M weights), N(0, 0.02^2), seed = 5 + rank; "
+                "also a 256-row gather (embedding lookup) timed", lambda r: [workloads.normal_matrix(128256, 4096, 0.02,
+                                                                                              seed=5 + r)]),
     "decode-gemm": ("32 llama3.1-8b blocks (seeds 32*rank + 0..31), each decoded into one reused BF16 scratch, "
                     "then every matrix multiplied by N(0,1) BF16 activations [T, in], T in {1,16,64,256} "
                     "(seed 1000 + T), FP32-accumulate GEMM on tcgen05", None),
@@ -544,6 +547,28 @@ def main():
     e2e_ok = bool(np.array_equal(host_out.view(torch.int16).numpy().view(np.uint16)[:1_000_000],
                                  mats[0].reshape(-1)[:1_000_000]))
 
+    row_gather = None
+    if args.workload == "lm-head":  # embedding lookup: only the rows a batch of tokens needs
+        g = torch.Generator().manual_seed(11)
+        rows = torch.randint(0, mats[0].shape[0], (256,), generator=g, dtype=torch.int32).to(dev)
+        outr = torch.empty(256, mats[0].shape[1], dtype=torch.bfloat16, device=dev)
+        for _ in range(3):
+            df11.decode_rows(d, mats[0].shape[1], rows, outr, err, stream)
+        torch.cuda.synchronize(dev)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(20):
+            df11.decode_rows(d, mats[0].shape[1], rows, outr, err, stream)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        assert df11.read_error(err, stream) == 0
+        us = e0.elapsed_time(e1) * 1e3 / 20
+        ridx = rows.cpu().numpy()
+        ok_rows = bool(np.array_equal(outr.view(torch.int16).cpu().numpy().view(np.uint16), mats[0][ridx]))
+        row_gather = {"rows": 256, "row_len": int(mats[0].shape[1]), "us_per_call": us,
+                      "full_decode_us": ms_step * 1e3, "bit_exact": ok_rows}
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, secs, sample = oracle_decode_rate(mats)
@@ -584,6 +609,8 @@ def main():
             "clocks": clocks,
             "cpu_baseline": cpu,
         }
+        if row_gather is not None:
+            line["row_gather"] = row_gather
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()

@@ -30,8 +30,8 @@ from . import build as _build
 
 __all__ = [
     "DF11Error", "CorruptStreamError", "Params", "DF11Tensor", "encode", "encode_multi",
-    "decode", "decode_block", "gemm", "read_error", "exponent_histogram", "lib_path", "sm_count",
-    "KERR_COUNT_MISMATCH", "KERR_BAD_CODE", "KERR_BAD_BLOCK", "KERR_OVERRUN", "KERR_TIMEOUT",
+    "decode", "decode_block", "decode_rows", "gemm", "read_error", "exponent_histogram", "lib_path", "sm_count",
+    "KERR_COUNT_MISMATCH", "KERR_BAD_CODE", "KERR_BAD_BLOCK", "KERR_OVERRUN", "KERR_TIMEOUT", "KERR_BAD_ROW",
 ]
 
 KERR_COUNT_MISMATCH = 0x1
@@ -39,6 +39,7 @@ KERR_BAD_CODE = 0x2
 KERR_BAD_BLOCK = 0x4
 KERR_OVERRUN = 0x8
 KERR_TIMEOUT = 0x10
+KERR_BAD_ROW = 0x40
 
 _STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported parameter", 3: "tensor too large",
            4: "corrupt compressed data", 5: "CUDA error", 6: "out of host memory"}
@@ -107,6 +108,7 @@ def _lib():
     lib.df11_read_error.argtypes = [vp, vp, P(u32)]
     lib.df11_device_sm_count.argtypes = [P(ctypes.c_int)]
     lib.df11_gemm_bf16.argtypes = [vp, vp, vp, u32, u32, u32, vp, vp]
+    lib.df11_decode_rows.argtypes = [P(_Tensor), ctypes.c_uint64, vp, u32, vp, vp, vp]
     if lib.df11_abi_version() != 2 or lib.df11_sizeof_tensor() != ctypes.sizeof(_Tensor):
         raise ImportError("libdf11.so ABI does not match this binding")
     _LIB = lib
@@ -347,6 +349,29 @@ def decode_block(t: DF11Tensor, scratch=None, err=None, stream=None):
     if own_err:
         read_error(err, stream)
     return scratch
+
+
+def decode_rows(t: DF11Tensor, row_len: int, rows, out=None, err=None, stream=None):
+    """Decodes only the requested rows of a device-resident compressed
+    [R, row_len] matrix (an embedding table): out[i] = row rows[i], as a
+    [len(rows), row_len] BF16 tensor.  `rows` is an int32 CUDA tensor."""
+    import torch
+    _check_device(t)
+    if rows.dtype not in (torch.int32,) or rows.device.type != "cuda" or rows.dim() != 1:
+        raise TypeError("rows must be a 1-D int32 CUDA tensor")
+    rows = rows.contiguous()
+    n = int(rows.numel())
+    if out is None:
+        out = torch.empty(n, int(row_len), dtype=torch.bfloat16, device=t.device)
+    own_err = err is None
+    if own_err:
+        err = _new_err(t.device)
+    _check(_lib().df11_decode_rows(ctypes.byref(t._bind()), int(row_len), ctypes.c_void_p(rows.data_ptr()), n,
+                                   ctypes.c_void_p(out.data_ptr()), ctypes.c_void_p(err.data_ptr()),
+                                   _stream_handle(stream)), "decode_rows")
+    if own_err:
+        read_error(err, stream)
+    return out
 
 
 def gemm(x, w, out=None, err=None, stream=None):

@@ -118,7 +118,8 @@ struct Cfg {
     static constexpr uint32_t kGrpSm = kGrpBs + 32u;  // the block's sign/mantissa bytes
     static constexpr uint32_t kSmBytes = S + 16u;
     static constexpr uint32_t kGrpMbar = kGrpSm + kSmBytes;
-    static constexpr uint32_t kGroupBytes = kGrpMbar + 16u;
+    static constexpr uint32_t kGrpAux = kGrpMbar + 16u;  // row gather: the row's block range
+    static constexpr uint32_t kGroupBytes = kGrpAux + 16u;
     static constexpr uint32_t kSmemBytes = kOffGroups + G * kGroupBytes + 16u;
     static_assert(S % 16 == 0, "whole chunks");
     static_assert(((S + 19u) >> 4) * 16u <= kSbufBytes, "zeroing stays inside the buffer");
@@ -488,35 +489,15 @@ __device__ __forceinline__ void issue_inputs(const DecodeArgs &a, uint64_t blk, 
     bulk_g2s(grp + C::kGrpBs, reinterpret_cast<const uint8_t *>(a.bstart) + ((4ull * blk) & ~15ull), 32u, mbar);
 }
 
-// kLong: compiled with the long-code path (codes longer than the table
-// windows); without it the loops carry no escape handling at all.
-template <class C, bool kLong>
-__global__ void __launch_bounds__(C::kCtaThreads, 1) df11_decode_kernel(const DecodeArgs a) {
-    extern __shared__ __align__(128) uint8_t smem[];
-    const uint32_t s_base = smem_addr(smem);
-    const uint32_t s_lim = s_base + kOffLim;
-    const uint32_t s_offs = s_base + kOffOffs;
-    const uint32_t s_symrot = s_base + kOffSymRot;
+// Stages the decode tables by one bulk copy, validates every entry and
+// replicates them (whole CTA).  Returns false, uniformly over the CTA and with
+// the error reported, when they did not arrive in time or are malformed;
+// nothing has been written to global memory then.
+template <class C>
+__device__ __forceinline__ bool load_tables(const uint8_t *lut, uint32_t *err_out, uint8_t *smem, uint32_t s_base,
+                                            uint32_t tid) {
     const uint32_t s_tmbar = s_base + kOffGroups + C::kGroups * C::kGroupBytes;
     const uint32_t s_stage = s_base + kOffGroups;  // compact tables land here first
-
-    const uint32_t tid = threadIdx.x;
-    const uint32_t group = tid / kGroupThreads;
-    const uint32_t lt = tid % kGroupThreads;  // thread within the group
-    const uint32_t lane = tid & 31u;
-    const uint32_t warp = lt >> 5;            // warp within the group
-    const uint32_t grp = s_base + kOffGroups + group * C::kGroupBytes;
-    const uint32_t sb = grp;                  // exponent buffer
-    const uint32_t wtot = grp + C::kGrpWtot;  // 4 warp totals
-    const uint32_t mb_in = grp + C::kGrpMbar, mb_sm = grp + C::kGrpMbar + 8u;
-    const uint32_t *cnt_lane = reinterpret_cast<const uint32_t *>(smem + kOffCountRep) + (lane % kCountCopies);
-    const uint2 *sym_lane = reinterpret_cast<const uint2 *>(smem + kOffSymRep) + (lane % kSymCopies);
-    uint32_t *buf = reinterpret_cast<uint32_t *>(smem + kOffGroups + group * C::kGroupBytes);
-    uint32_t my_err = 0;
-
-    const uint64_t stride = (uint64_t)gridDim.x * C::kGroups;
-    uint64_t blk = (uint64_t)blockIdx.x * C::kGroups + group;
-
     // ---- decode tables: one bulk copy, then validate and replicate
     if (tid == 0) {
         mbar_init(s_tmbar);
@@ -525,7 +506,7 @@ __global__ void __launch_bounds__(C::kCtaThreads, 1) df11_decode_kernel(const De
     __syncthreads();
     if (tid == 0) {
         mbar_expect(s_tmbar, kLutBytes);
-        bulk_g2s(s_stage, a.lut, kLutBytes, s_tmbar);
+        bulk_g2s(s_stage, lut, kLutBytes, s_tmbar);
     }
     const bool staged = wait_phase(s_tmbar, 0u);
     if (__syncthreads_or(!staged)) {
@@ -533,10 +514,10 @@ __global__ void __launch_bounds__(C::kCtaThreads, 1) df11_decode_kernel(const De
         // flight into this CTA's shared memory, then report and stop.
         if (tid == 0) {
             wait_phase(s_tmbar, 0u);
-            if (a.err) atomicOr(a.err, kKernErrTimeout);
+            if (err_out) atomicOr(err_out, kKernErrTimeout);
         }
         __syncthreads();
-        return;
+        return false;
     }
     const LutHeader *hdr = reinterpret_cast<const LutHeader *>(smem + kOffGroups + kOffHeader);
     const uint32_t w1 = hdr->w1, w2 = hdr->w2, max_len = hdr->max_len;
@@ -576,10 +557,43 @@ __global__ void __launch_bounds__(C::kCtaThreads, 1) df11_decode_kernel(const De
         // codes, so each lookup makes progress: the decode loops then end
         // after at most 95 lookups plus 95 long codes whatever the stream.
         if (__syncthreads_or(bad)) {
-            if (tid == 0 && a.err) atomicOr(a.err, DF11_KERR_BAD_CODE);
-            return;  // uniform over the CTA: nothing was written to global memory
+            if (tid == 0 && err_out) atomicOr(err_out, DF11_KERR_BAD_CODE);
+            return false;  // uniform over the CTA: nothing was written to global memory
         }
     }
+    __syncthreads();  // the replicated tables are complete before any lookup
+    return true;
+}
+
+// kLong: compiled with the long-code path (codes longer than the table
+// windows); without it the loops carry no escape handling at all.
+template <class C, bool kLong>
+__global__ void __launch_bounds__(C::kCtaThreads, 1) df11_decode_kernel(const DecodeArgs a) {
+    extern __shared__ __align__(128) uint8_t smem[];
+    const uint32_t s_base = smem_addr(smem);
+    const uint32_t s_lim = s_base + kOffLim;
+    const uint32_t s_offs = s_base + kOffOffs;
+    const uint32_t s_symrot = s_base + kOffSymRot;
+    const uint32_t tid = threadIdx.x;
+    const uint32_t group = tid / kGroupThreads;
+    const uint32_t lt = tid % kGroupThreads;  // thread within the group
+    const uint32_t lane = tid & 31u;
+    const uint32_t warp = lt >> 5;            // warp within the group
+    const uint32_t grp = s_base + kOffGroups + group * C::kGroupBytes;
+    const uint32_t sb = grp;                  // exponent buffer
+    const uint32_t wtot = grp + C::kGrpWtot;  // 4 warp totals
+    const uint32_t mb_in = grp + C::kGrpMbar, mb_sm = grp + C::kGrpMbar + 8u;
+    const uint32_t *cnt_lane = reinterpret_cast<const uint32_t *>(smem + kOffCountRep) + (lane % kCountCopies);
+    const uint2 *sym_lane = reinterpret_cast<const uint2 *>(smem + kOffSymRep) + (lane % kSymCopies);
+    uint32_t *buf = reinterpret_cast<uint32_t *>(smem + kOffGroups + group * C::kGroupBytes);
+    uint32_t my_err = 0;
+
+    const uint64_t stride = (uint64_t)gridDim.x * C::kGroups;
+    uint64_t blk = (uint64_t)blockIdx.x * C::kGroups + group;
+
+    if (!load_tables<C>(a.lut, a.err, smem, s_base, tid)) return;
+    const LutHeader *hdr = reinterpret_cast<const LutHeader *>(smem + kOffHeader);
+    const uint32_t w1 = hdr->w1, w2 = hdr->w2, max_len = hdr->max_len;
     const uint32_t sh1 = 32u - w1, sh2 = 32u - w2;
 
     // The exponent buffer starts clear; the merge clears what it reads.
@@ -693,13 +707,181 @@ __global__ void __launch_bounds__(C::kCtaThreads, 1) df11_decode_kernel(const De
     if (my_err && a.err) atomicOr(a.err, my_err);
 }
 
+
+// ----------------------------------------------------------------- row gather
+struct GatherArgs {
+    DecodeArgs d;           // the compressed matrix (d.out unused)
+    const uint32_t *rows;   // requested row indices
+    uint16_t *out;          // n_rows x row_len
+    uint64_t row_len;
+    uint64_t n_rows_total;  // n_elems / row_len
+    uint32_t n_rows;
+};
+
+// Largest b in [0, n_blocks) with bs[b] <= x, by one warp (32-way search,
+// ceil(log32 n_blocks) rounds of one load per lane).  bs[0] is 0 for valid
+// data; with corrupt starts the result is still some block in range (the
+// per-block range checks then catch the inconsistency).
+__device__ __forceinline__ uint64_t find_block(const uint32_t *bs, uint64_t n_blocks, uint64_t x, uint32_t lane) {
+    uint64_t lo = 0, hi = n_blocks;  // the answer lies in [lo, hi)
+    while (hi - lo > 1u) {
+        const uint64_t step = (hi - lo + 31u) / 32u;
+        const uint64_t p = lo + (uint64_t)lane * step;
+        const bool le = p < hi && (uint64_t)__ldg(bs + p) <= x;
+        const uint32_t m = __ballot_sync(kFull, le) | 1u;  // lane 0 probes lo itself
+        const uint64_t j = 31u - __clz(m);
+        lo += j * step;
+        hi = min(hi, lo + step);
+    }
+    return lo;
+}
+
+// One group per requested row (grid-stride over rows): the format blocks
+// covering the row are staged, decoded as in df11_decode_kernel and merged
+// element by element into the output row.  Three group barriers per block
+// (inputs and buffer are reused synchronously; this path decodes a few
+// blocks per row, not the whole tensor).
+template <class C, bool kLong>
+__global__ void __launch_bounds__(C::kCtaThreads, 1) df11_gather_kernel(const GatherArgs ga) {
+    const DecodeArgs &a = ga.d;
+    extern __shared__ __align__(128) uint8_t smem[];
+    const uint32_t s_base = smem_addr(smem);
+    const uint32_t s_lim = s_base + kOffLim;
+    const uint32_t s_offs = s_base + kOffOffs;
+    const uint32_t s_symrot = s_base + kOffSymRot;
+    const uint32_t tid = threadIdx.x;
+    const uint32_t group = tid / kGroupThreads;
+    const uint32_t lt = tid % kGroupThreads;
+    const uint32_t lane = tid & 31u;
+    const uint32_t warp = lt >> 5;
+    const uint32_t grp = s_base + kOffGroups + group * C::kGroupBytes;
+    const uint32_t sb = grp;
+    const uint32_t wtot = grp + C::kGrpWtot;
+    const uint32_t mb_in = grp + C::kGrpMbar;
+    const uint32_t aux = grp + C::kGrpAux;
+    const uint32_t *cnt_lane = reinterpret_cast<const uint32_t *>(smem + kOffCountRep) + (lane % kCountCopies);
+    const uint2 *sym_lane = reinterpret_cast<const uint2 *>(smem + kOffSymRep) + (lane % kSymCopies);
+    uint32_t *buf = reinterpret_cast<uint32_t *>(smem + kOffGroups + group * C::kGroupBytes);
+    uint32_t my_err = 0;
+
+    if (!load_tables<C>(a.lut, a.err, smem, s_base, tid)) return;
+    const LutHeader *hdr = reinterpret_cast<const LutHeader *>(smem + kOffHeader);
+    const uint32_t w1 = hdr->w1, w2 = hdr->w2, max_len = hdr->max_len;
+    const uint32_t sh1 = 32u - w1, sh2 = 32u - w2;
+
+    for (uint32_t c = lt; c < C::kSbufBytes / 16u; c += kGroupThreads) sts_zero16(sb + 16u * c);
+    if (lt == 0) {
+        mbar_init(mb_in);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    group_barrier(group);
+    uint32_t ph_in = 0;
+
+    for (uint64_t i = (uint64_t)blockIdx.x * C::kGroups + group; i < ga.n_rows;
+         i += (uint64_t)gridDim.x * C::kGroups) {
+        const uint64_t row = __ldg(ga.rows + i);
+        const bool row_ok = row < ga.n_rows_total;
+        const uint64_t lo = row * ga.row_len, hi = lo + ga.row_len;
+        if (warp == 0 && row_ok) {
+            const uint64_t b0 = find_block(a.bstart, a.n_blocks, lo, lane);
+            const uint64_t b1 = find_block(a.bstart, a.n_blocks, hi - 1u, lane);
+            if (lane == 0) {
+                sts_u32(aux, (uint32_t)b0);
+                sts_u32(aux + 4u, (uint32_t)b1);
+            }
+        }
+        group_barrier(group);
+        const uint32_t b0 = lds_u32(aux), b1 = lds_u32(aux + 4u);
+        if (!row_ok || b1 < b0) {
+            if (lt == 0) my_err |= row_ok ? DF11_KERR_BAD_BLOCK : DF11_KERR_BAD_ROW;
+            group_barrier(group);  // the range words are read before the next row writes them
+            continue;
+        }
+        uint16_t *orow = ga.out + i * ga.row_len;
+        for (uint64_t blk = b0; blk <= b1; ++blk) {
+            if (lt == 0) issue_inputs<C>(a, blk, grp, mb_in);
+            if (!wait_phase(mb_in, ph_in)) my_err |= kKernErrTimeout;
+            ph_in ^= 1u;
+            const uint64_t tA = blk * (uint64_t)kThreadsPerBlockFmt + 2u * lt;
+            const uint32_t bs_off = (uint32_t)((4ull * blk) & 15ull);
+            const uint32_t s = lds_u32(grp + C::kGrpBs + bs_off), e = lds_u32(grp + C::kGrpBs + bs_off + 4u);
+            const uint32_t base = s & ~15u;
+            const bool range_ok = (e >= s) && ((uint64_t)e <= a.n_elems) && (e - base <= C::kBufSyms);
+            const uint32_t span = range_ok ? e - base : 0u;
+
+            const uint4 v = lds_u4(grp + C::kGrpEnc + 16u * lt);
+            const uint32_t nextw = lds_u32(grp + C::kGrpEnc + 16u * lt + 16u);
+            const uint32_t gq = (10u * lt) >> 5;
+            const uint32_t g_hi = lds_u32(grp + C::kGrpGap + 4u * gq), g_lo = lds_u32(grp + C::kGrpGap + 4u * gq + 4u);
+            const uint32_t gb = __funnelshift_l(bswap32(g_lo), bswap32(g_hi), (10u * lt) & 31u);
+            uint32_t gapA = gb >> 27, gapB = (gb >> 22) & 31u;
+            const uint32_t gapC = (gb >> 17) & 31u;
+            int32_t endA, endB;
+            if (tA >= a.n_threads) { gapA = 0; endA = 0; }
+            else if (tA + 1 == a.n_threads) endA = (int32_t)(a.total_bits - 64ull * tA);
+            else endA = 64 + (int32_t)gapB;
+            if (tA + 1 >= a.n_threads) { gapB = 0; endB = 0; }
+            else if (tA + 2 == a.n_threads) endB = (int32_t)(a.total_bits - 64ull * (tA + 1));
+            else endB = 64 + (int32_t)gapC;
+            const Chain A = make_chain(bswap32(v.x), bswap32(v.y), bswap32(v.z), gapA, endA, my_err);
+            const Chain B = make_chain(bswap32(v.z), bswap32(v.w), bswap32(nextw), gapB, endB, my_err);
+
+            uint32_t cA, cB;
+            count_pass<kLong>(A, B, cnt_lane, sh1, s_lim, w1 + 1u, max_len, cA, cB, my_err);
+            const uint32_t cnt = cA + cB;
+            uint32_t incl = cnt;
+#pragma unroll
+            for (uint32_t d = 1; d < 32; d <<= 1) {
+                const uint32_t x = __shfl_up_sync(kFull, incl, d);
+                if (lane >= d) incl += x;
+            }
+            constexpr uint32_t kWarps = kGroupThreads / 32;
+            if (lane == 31u) sts_u32(wtot + 4u * warp, incl);
+            group_barrier(group);
+            uint32_t wsum = (lane < kWarps) ? lds_u32(wtot + 4u * lane) : 0u;
+#pragma unroll
+            for (uint32_t d = 1; d < kWarps; d <<= 1) {
+                const uint32_t x = __shfl_up_sync(kFull, wsum, d);
+                if (lane >= d) wsum += x;
+            }
+            const uint32_t total = __shfl_sync(kFull, wsum, kWarps - 1u);
+            const uint32_t wpre = __shfl_sync(kFull, wsum, (warp + kWarps - 1u) % kWarps) * (warp != 0u ? 1u : 0u);
+            const bool ok = range_ok && (total == e - s);
+            if (!ok && lt == 0) my_err |= range_ok ? DF11_KERR_COUNT_MISMATCH : DF11_KERR_BAD_BLOCK;
+            if (ok) {
+                const uint32_t startA = (s - base) + wpre + incl - cnt;
+                decode_pass<kLong>(A, B, startA, cA, startA + cA, cB, buf, sb, sym_lane, sh2, s_lim, s_offs,
+                                   s_symrot, w2 + 1u, max_len);
+            }
+            group_barrier(group);
+            if (ok) {  // the row's part of this block, element by element
+                const uint64_t g0 = max((uint64_t)s, lo), g1 = min((uint64_t)e, hi);
+                for (uint64_t g = g0 + lt; g < g1; g += kGroupThreads) {
+                    const uint32_t sm8 = __ldg(a.sm + g);
+                    const uint32_t r = lds_u8(sb + (uint32_t)(g - base));
+                    const uint32_t hi8 = (sm8 & 0x80u) | (r & 0x7Fu);
+                    const uint32_t lo8 = (r & 0x80u) | (sm8 & 0x7Fu);
+                    orow[g - lo] = (uint16_t)(lo8 | (hi8 << 8));
+                }
+            }
+            group_barrier(group);  // every read of the buffer and the staged inputs is done
+            for (uint32_t c = lt; c < (span + 19u) >> 4; c += kGroupThreads) sts_zero16(sb + 16u * c);
+        }
+        group_barrier(group);  // the range words are read before the next row writes them
+    }
+    if (my_err && a.err) atomicOr(a.err, my_err);
+}
+
 // ----------------------------------------------------------------- host
 std::atomic<int> g_sm_count[64];
 std::atomic<int> g_attr_set[64];
 
 template <class C, bool kLong>
 cudaError_t set_smem_attr() {
-    return cudaFuncSetAttribute(df11_decode_kernel<C, kLong>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(df11_decode_kernel<C, kLong>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)C::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    return cudaFuncSetAttribute(df11_gather_kernel<C, kLong>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 (int)C::kSmemBytes);
 }
 
@@ -732,42 +914,98 @@ void launch(const DecodeArgs &a, uint64_t n_blocks, int sms, cudaStream_t stream
     df11_decode_kernel<C, kLong><<<grid, C::kCtaThreads, C::kSmemBytes, stream>>>(a);
 }
 
-df11_status launch_decode(const df11_tensor *t, uint16_t *out, uint32_t *err_word, void *stream) {
-    if (!t) return DF11_ERR_INVALID_ARG;
-    df11_status st = df11_validate(t);
-    if (st != DF11_OK) return st;
-    if (t->n_elems == 0) return DF11_OK;  // nothing to write; out may be NULL
-    if (!out || !t->enc || !t->sm || !t->gaps || !t->block_start || !t->lut) return DF11_ERR_INVALID_ARG;
+// Checks a device tensor for a decode launch and fills the kernel arguments.
+df11_status prepare_args(const df11_tensor *t, DecodeArgs &a) {
+    if (!t->enc || !t->sm || !t->gaps || !t->block_start || !t->lut) return DF11_ERR_INVALID_ARG;
     if (!aligned16(t->enc) || !aligned16(t->sm) || !aligned16(t->gaps) || !aligned16(t->lut) ||
-        !aligned16(t->block_start) || !aligned16(out))
+        !aligned16(t->block_start))
         return DF11_ERR_INVALID_ARG;
-    int sms = 0;
-    st = prepare_device(&sms);
-    if (st != DF11_OK) return st;
-    DecodeArgs a;
     a.enc = t->enc;
     a.sm = t->sm;
     a.gaps = t->gaps;
     a.bstart = t->block_start;
     a.lut = t->lut;
-    a.out = out;
-    a.err = err_word;
+    a.out = nullptr;
+    a.err = nullptr;
     a.n_elems = t->n_elems;
     a.total_bits = t->total_bits;
     a.n_threads = t->n_threads;
     a.n_blocks = t->n_blocks;
-    a.out_al32 = ((uintptr_t)out & 31u) == 0 ? 1u : 0u;
-    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    // a block's buffer span is at most its code count + 15; codes no longer
-    // than both table windows never take the long-code path
+    a.out_al32 = 0;
+    return DF11_OK;
+}
+
+// Which instance decodes a tensor: codes no longer than both table windows
+// never take the long-code path; a block's buffer span is at most its code
+// count + 15.
+void pick_instance(const df11_tensor *t, bool &wide, bool &lng) {
     uint32_t max_len = 0;
     for (int k = 0; k < 256; ++k) max_len = t->code_len[k] > max_len ? t->code_len[k] : max_len;
-    const bool lng = max_len > (uint32_t)(kW1Max < kW2Max ? kW1Max : kW2Max);
-    const bool wide = t->max_block_codes + 15u <= CfgWide::kBufSyms;
+    lng = max_len > (uint32_t)(kW1Max < kW2Max ? kW1Max : kW2Max);
+    wide = t->max_block_codes + 15u <= CfgWide::kBufSyms;
+}
+
+df11_status launch_decode(const df11_tensor *t, uint16_t *out, uint32_t *err_word, void *stream) {
+    if (!t) return DF11_ERR_INVALID_ARG;
+    df11_status st = df11_validate(t);
+    if (st != DF11_OK) return st;
+    if (t->n_elems == 0) return DF11_OK;  // nothing to write; out may be NULL
+    if (!out || !aligned16(out)) return DF11_ERR_INVALID_ARG;
+    DecodeArgs a;
+    st = prepare_args(t, a);
+    if (st != DF11_OK) return st;
+    int sms = 0;
+    st = prepare_device(&sms);
+    if (st != DF11_OK) return st;
+    a.out = out;
+    a.err = err_word;
+    a.out_al32 = ((uintptr_t)out & 31u) == 0 ? 1u : 0u;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    bool wide, lng;
+    pick_instance(t, wide, lng);
     if (wide && !lng) launch<CfgWide, false>(a, t->n_blocks, sms, s);
     else if (wide) launch<CfgWide, true>(a, t->n_blocks, sms, s);
     else if (!lng) launch<CfgDense, false>(a, t->n_blocks, sms, s);
     else launch<CfgDense, true>(a, t->n_blocks, sms, s);
+    if (cudaGetLastError() != cudaSuccess) return DF11_ERR_CUDA;
+    return DF11_OK;
+}
+
+template <class C, bool kLong>
+void launch_gather(const GatherArgs &g, int sms, cudaStream_t stream) {
+    const uint64_t ctas_needed = (g.n_rows + C::kGroups - 1) / C::kGroups;
+    const unsigned grid = (unsigned)(ctas_needed < (uint64_t)sms ? ctas_needed : (uint64_t)sms);
+    df11_gather_kernel<C, kLong><<<grid, C::kCtaThreads, C::kSmemBytes, stream>>>(g);
+}
+
+df11_status launch_rows(const df11_tensor *t, uint64_t row_len, const uint32_t *rows, uint32_t n_rows, uint16_t *out,
+                        uint32_t *err_word, void *stream) {
+    if (!t) return DF11_ERR_INVALID_ARG;
+    df11_status st = df11_validate(t);
+    if (st != DF11_OK) return st;
+    if (row_len == 0 || t->n_elems % row_len != 0) return DF11_ERR_INVALID_ARG;
+    if (n_rows == 0) return DF11_OK;
+    if (!rows || !out || ((uintptr_t)out & 1u) || ((uintptr_t)rows & 3u) || t->n_elems == 0)
+        return DF11_ERR_INVALID_ARG;
+    GatherArgs g;
+    st = prepare_args(t, g.d);
+    if (st != DF11_OK) return st;
+    int sms = 0;
+    st = prepare_device(&sms);
+    if (st != DF11_OK) return st;
+    g.d.err = err_word;
+    g.rows = rows;
+    g.out = out;
+    g.row_len = row_len;
+    g.n_rows_total = t->n_elems / row_len;
+    g.n_rows = n_rows;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    bool wide, lng;
+    pick_instance(t, wide, lng);
+    if (wide && !lng) launch_gather<CfgWide, false>(g, sms, s);
+    else if (wide) launch_gather<CfgWide, true>(g, sms, s);
+    else if (!lng) launch_gather<CfgDense, false>(g, sms, s);
+    else launch_gather<CfgDense, true>(g, sms, s);
     if (cudaGetLastError() != cudaSuccess) return DF11_ERR_CUDA;
     return DF11_OK;
 }
@@ -787,6 +1025,11 @@ df11_status df11_decode_block(const df11_tensor *blk, const uint64_t *mat_offset
     for (uint32_t j = 0; j < k; ++j)
         if (mat_offsets[j + 1] < mat_offsets[j]) return DF11_ERR_INVALID_ARG;
     return launch_decode(blk, scratch, err_word, stream);
+}
+
+df11_status df11_decode_rows(const df11_tensor *t, uint64_t row_len, const uint32_t *rows, uint32_t n_rows,
+                             uint16_t *out, uint32_t *err_word, void *stream) {
+    return launch_rows(t, row_len, rows, n_rows, out, err_word, stream);
 }
 
 df11_status df11_read_error(const uint32_t *err_word, void *stream, uint32_t *host_value) {

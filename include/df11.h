@@ -52,6 +52,7 @@ typedef enum df11_status {
 #define DF11_KERR_BAD_CODE 0x2u       /* a bit pattern that is no code        */
 #define DF11_KERR_BAD_BLOCK 0x4u      /* block_start not monotone / too big   */
 #define DF11_KERR_OVERRUN 0x8u        /* a thread's codes run past its end    */
+#define DF11_KERR_BAD_ROW 0x40u       /* a requested row index is out of range */
 
 /* Encoder parameters.
  *  max_code_len      -- length cap L_MAX for the exponent code, 1..32.  The
@@ -189,6 +190,22 @@ df11_status df11_decode(const df11_tensor *t, uint16_t *out, uint32_t *err_word,
  * scratch[mat_offsets[j] .. mat_offsets[j+1]).  err_word as in df11_decode. */
 df11_status df11_decode_block(const df11_tensor *blk, const uint64_t *mat_offsets, uint32_t k,
                               uint16_t *scratch, uint32_t *err_word, void *stream);
+
+/* Row gather: decodes only rows rows[0..n_rows) of a compressed [R, row_len]
+ * matrix (an embedding table: the rows a batch of token ids needs) into out,
+ * row i of out = row rows[i] of the matrix (n_rows x row_len BF16 values,
+ * row-major, 2-byte aligned device memory).  The pages name the embedding and
+ * LM-head matrices among those DF11 compresses ("Le format DFloat11"); the
+ * format keeps only each thread block's first output index ("Noyau GPU en deux
+ * etapes et metadonnees auxiliaires"), so the kernel finds the thread blocks
+ * covering a row by searching those indices, decodes them in full (count
+ * pass, scan, decode pass) and writes only the row's elements.
+ *  rows: DEVICE uint32 row indices (repeats allowed); an index >= R sets
+ *        DF11_KERR_BAD_ROW and leaves that output row unwritten.
+ *  row_len: > 0 and dividing t->n_elems; else DF11_ERR_INVALID_ARG.
+ *  n_rows == 0 is a no-op.  err_word as in df11_decode.  One launch. */
+df11_status df11_decode_rows(const df11_tensor *t, uint64_t row_len, const uint32_t *rows, uint32_t n_rows,
+                             uint16_t *out, uint32_t *err_word, void *stream);
 
 /* Consumer of a decoded weight matrix: Y = X * W^T with BF16 inputs and FP32
  * accumulation on the tensor cores (tcgen05), the matrix multiplication the
