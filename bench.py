@@ -425,7 +425,7 @@ def run_offload(args, rank: int, world: int):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=3000)
+    ap.add_argument("--steps", type=int, default=8000)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["df11", "reference"], default="df11")
     ap.add_argument("--e2e-steps", type=int, default=5)
