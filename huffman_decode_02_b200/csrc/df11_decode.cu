@@ -68,8 +68,8 @@ using namespace df11;
 //   [0, 768)                 table header, canonical limits, symbol list
 //   kOffCountRep             count table, kCountCopies copies interleaved:
 //                            entry i of copy c at word (i * kCountCopies + c)
-//   kOffSymRep               symbol table, kSymCopies copies interleaved:
-//                            entry i of copy c at u64 (i * kSymCopies + c)
+//   kOffSymRep               symbol table, C::kSymCopies copies interleaved:
+//                            entry i of copy c at u64 (i * copies + c)
 //   kOffGroups               per group: exponent buffer, warp totals, staged
 //                            inputs of the next block, this block's
 //                            sign/mantissa bytes, 2 mbarriers
@@ -80,18 +80,12 @@ using namespace df11;
 #ifndef DF11_COUNT_COPIES
 #define DF11_COUNT_COPIES 2
 #endif
-#ifndef DF11_SYM_COPIES
-#define DF11_SYM_COPIES 1
-#endif
 constexpr uint32_t kCountCopies = DF11_COUNT_COPIES;
-constexpr uint32_t kSymCopies = DF11_SYM_COPIES;
 constexpr uint32_t log2u(uint32_t x) { return x <= 1u ? 0u : 1u + log2u(x >> 1); }
 constexpr uint32_t kCountShift = log2u(4u * kCountCopies);  // byte stride of one replicated entry
-constexpr uint32_t kSymShift = log2u(8u * kSymCopies);
-static_assert((1u << kCountShift) == 4u * kCountCopies && (1u << kSymShift) == 8u * kSymCopies, "power of two");
+static_assert((1u << kCountShift) == 4u * kCountCopies, "power of two");
 constexpr uint32_t kOffCountRep = 768;
 constexpr uint32_t kOffSymRep = kOffCountRep + 4u * kCountCopies * (1u << kW1Max);
-constexpr uint32_t kOffGroups = kOffSymRep + 8u * kSymCopies * (1u << kW2Max);
 constexpr uint32_t kEncStage = kThreadsPerBlockFmt * kBytesPerThread + 16u;  // + next block's first 16
 constexpr uint32_t kGapStage = kThreadsPerBlockFmt * 5u / 8u + 16u;          // + next block's first gaps
 constexpr uint32_t kFull = 0xFFFFFFFFu;
@@ -105,8 +99,10 @@ static_assert(kLutBytes % 16 == 0, "bulk copy size");
 
 // Per-instance layout: G groups per CTA, buffers of S symbols (+ 16: the
 // 16-element chunk alignment of the block start is at most 15).
-template <int G, int S>
+template <int G, int S, int SC>
 struct Cfg {
+    static constexpr uint32_t kSymCopies = SC;  // symbol-table copies (lane l reads copy l mod SC)
+    static constexpr uint32_t kOffGroups = kOffSymRep + 8u * SC * (1u << kW2Max);
     static constexpr uint32_t kGroups = G;
     static constexpr uint32_t kBufSyms = S;
     static constexpr uint32_t kCtaThreads = G * kGroupThreads;
@@ -123,14 +119,16 @@ struct Cfg {
     static constexpr uint32_t kSmemBytes = kOffGroups + G * kGroupBytes + 16u;
     static_assert(S % 16 == 0, "whole chunks");
     static_assert(((S + 19u) >> 4) * 16u <= kSbufBytes, "zeroing stays inside the buffer");
+    static_assert(SC == 1 || SC == 2, "one or two symbol-table copies");
     static_assert(kGroupBytes % 16 == 0 && kGrpEnc % 16 == 0 && kGrpGap % 16 == 0 && kGrpBs % 16 == 0 &&
                       kGrpSm % 16 == 0,
                   "bulk copy destinations are 16-byte aligned");
     static_assert(kLutBytes <= G * kGroupBytes, "tables stage in the group area");
     static_assert(kSmemBytes <= 227u * 1024u, "fits one CTA's shared memory");
 };
-using CfgWide = Cfg<8, 8192>;    // blocks of up to 8192 - 15 codes (any LLM-like data)
-using CfgDense = Cfg<4, 16400>;  // any block (1-bit codes: 16384 per block)
+using CfgTypical = Cfg<8, 6400, 2>;  // blocks of up to 6400 - 15 codes: two symbol-table copies fit
+using CfgWide = Cfg<8, 8192, 1>;     // blocks of up to 8192 - 15 codes (any LLM-like data)
+using CfgDense = Cfg<4, 16400, 1>;   // any block (1-bit codes: 16384 per block)
 
 struct DecodeArgs {
     const uint8_t *enc;
@@ -404,7 +402,7 @@ __device__ __forceinline__ void count_pass(const Chain &A, const Chain &B, const
 // unused symbol bytes of a table entry are zero.  Stops on the code counts
 // of the count pass.  `sym` points at this lane's copy of the symbol table
 // (entry i at sym[i * kSymCopies]).
-template <bool kLong>
+template <bool kLong, uint32_t kSymCopies>
 __device__ __forceinline__ void decode_pass(const Chain &A, const Chain &B, uint32_t startA, uint32_t cA,
                                             uint32_t startB, uint32_t cB, uint32_t *buf, uint32_t sb,
                                             const uint2 *sym, uint32_t sh2, uint32_t s_lim, uint32_t s_offs,
@@ -496,6 +494,8 @@ __device__ __forceinline__ void issue_inputs(const DecodeArgs &a, uint64_t blk, 
 template <class C>
 __device__ __forceinline__ bool load_tables(const uint8_t *lut, uint32_t *err_out, uint8_t *smem, uint32_t s_base,
                                             uint32_t tid) {
+    constexpr uint32_t kOffGroups = C::kOffGroups;
+    constexpr uint32_t kSymCopies = C::kSymCopies;
     const uint32_t s_tmbar = s_base + kOffGroups + C::kGroups * C::kGroupBytes;
     const uint32_t s_stage = s_base + kOffGroups;  // compact tables land here first
     // ---- decode tables: one bulk copy, then validate and replicate
@@ -579,13 +579,13 @@ __global__ void __launch_bounds__(C::kCtaThreads, 1) df11_decode_kernel(const De
     const uint32_t lt = tid % kGroupThreads;  // thread within the group
     const uint32_t lane = tid & 31u;
     const uint32_t warp = lt >> 5;            // warp within the group
-    const uint32_t grp = s_base + kOffGroups + group * C::kGroupBytes;
+    const uint32_t grp = s_base + C::kOffGroups + group * C::kGroupBytes;
     const uint32_t sb = grp;                  // exponent buffer
     const uint32_t wtot = grp + C::kGrpWtot;  // 4 warp totals
     const uint32_t mb_in = grp + C::kGrpMbar, mb_sm = grp + C::kGrpMbar + 8u;
     const uint32_t *cnt_lane = reinterpret_cast<const uint32_t *>(smem + kOffCountRep) + (lane % kCountCopies);
-    const uint2 *sym_lane = reinterpret_cast<const uint2 *>(smem + kOffSymRep) + (lane % kSymCopies);
-    uint32_t *buf = reinterpret_cast<uint32_t *>(smem + kOffGroups + group * C::kGroupBytes);
+    const uint2 *sym_lane = reinterpret_cast<const uint2 *>(smem + kOffSymRep) + (lane % C::kSymCopies);
+    uint32_t *buf = reinterpret_cast<uint32_t *>(smem + C::kOffGroups + group * C::kGroupBytes);
     uint32_t my_err = 0;
 
     const uint64_t stride = (uint64_t)gridDim.x * C::kGroups;
@@ -688,7 +688,7 @@ __global__ void __launch_bounds__(C::kCtaThreads, 1) df11_decode_kernel(const De
         // ---- pass 2: decode both chains again into the buffer
         if (ok) {
             const uint32_t startA = (s - base) + wpre + incl - cnt;  // buffer index of A's first code
-            decode_pass<kLong>(A, B, startA, cA, startA + cA, cB, buf, sb, sym_lane, sh2, s_lim, s_offs, s_symrot,
+            decode_pass<kLong, C::kSymCopies>(A, B, startA, cA, startA + cA, cB, buf, sb, sym_lane, sh2, s_lim, s_offs, s_symrot,
                         w2 + 1u, max_len);
         }
         group_barrier(group);
@@ -754,14 +754,14 @@ __global__ void __launch_bounds__(C::kCtaThreads, 1) df11_gather_kernel(const Ga
     const uint32_t lt = tid % kGroupThreads;
     const uint32_t lane = tid & 31u;
     const uint32_t warp = lt >> 5;
-    const uint32_t grp = s_base + kOffGroups + group * C::kGroupBytes;
+    const uint32_t grp = s_base + C::kOffGroups + group * C::kGroupBytes;
     const uint32_t sb = grp;
     const uint32_t wtot = grp + C::kGrpWtot;
     const uint32_t mb_in = grp + C::kGrpMbar;
     const uint32_t aux = grp + C::kGrpAux;
     const uint32_t *cnt_lane = reinterpret_cast<const uint32_t *>(smem + kOffCountRep) + (lane % kCountCopies);
-    const uint2 *sym_lane = reinterpret_cast<const uint2 *>(smem + kOffSymRep) + (lane % kSymCopies);
-    uint32_t *buf = reinterpret_cast<uint32_t *>(smem + kOffGroups + group * C::kGroupBytes);
+    const uint2 *sym_lane = reinterpret_cast<const uint2 *>(smem + kOffSymRep) + (lane % C::kSymCopies);
+    uint32_t *buf = reinterpret_cast<uint32_t *>(smem + C::kOffGroups + group * C::kGroupBytes);
     uint32_t my_err = 0;
 
     if (!load_tables<C>(a.lut, a.err, smem, s_base, tid)) return;
@@ -850,7 +850,7 @@ __global__ void __launch_bounds__(C::kCtaThreads, 1) df11_gather_kernel(const Ga
             if (!ok && lt == 0) my_err |= range_ok ? DF11_KERR_COUNT_MISMATCH : DF11_KERR_BAD_BLOCK;
             if (ok) {
                 const uint32_t startA = (s - base) + wpre + incl - cnt;
-                decode_pass<kLong>(A, B, startA, cA, startA + cA, cB, buf, sb, sym_lane, sh2, s_lim, s_offs,
+                decode_pass<kLong, C::kSymCopies>(A, B, startA, cA, startA + cA, cB, buf, sb, sym_lane, sh2, s_lim, s_offs,
                                    s_symrot, w2 + 1u, max_len);
             }
             group_barrier(group);
@@ -896,7 +896,8 @@ df11_status prepare_device(int *sm_count) {
         g_sm_count[dev].store(sms, std::memory_order_relaxed);
     }
     if (!g_attr_set[dev].load(std::memory_order_acquire)) {
-        if (set_smem_attr<CfgWide, false>() != cudaSuccess || set_smem_attr<CfgWide, true>() != cudaSuccess ||
+        if (set_smem_attr<CfgTypical, false>() != cudaSuccess || set_smem_attr<CfgTypical, true>() != cudaSuccess ||
+            set_smem_attr<CfgWide, false>() != cudaSuccess || set_smem_attr<CfgWide, true>() != cudaSuccess ||
             set_smem_attr<CfgDense, false>() != cudaSuccess || set_smem_attr<CfgDense, true>() != cudaSuccess)
             return DF11_ERR_CUDA;
         g_attr_set[dev].store(1, std::memory_order_release);
@@ -937,12 +938,15 @@ df11_status prepare_args(const df11_tensor *t, DecodeArgs &a) {
 
 // Which instance decodes a tensor: codes no longer than both table windows
 // never take the long-code path; a block's buffer span is at most its code
-// count + 15.
-void pick_instance(const df11_tensor *t, bool &wide, bool &lng) {
+// count + 15, and the instance with the smallest buffers that holds it is
+// taken (smaller buffers leave room for a second symbol-table copy).
+enum class Inst { kTypical, kWide, kDense };
+void pick_instance(const df11_tensor *t, Inst &inst, bool &lng) {
     uint32_t max_len = 0;
     for (int k = 0; k < 256; ++k) max_len = t->code_len[k] > max_len ? t->code_len[k] : max_len;
     lng = max_len > (uint32_t)(kW1Max < kW2Max ? kW1Max : kW2Max);
-    wide = t->max_block_codes + 15u <= CfgWide::kBufSyms;
+    const uint64_t need = (uint64_t)t->max_block_codes + 15u;
+    inst = need <= CfgTypical::kBufSyms ? Inst::kTypical : need <= CfgWide::kBufSyms ? Inst::kWide : Inst::kDense;
 }
 
 df11_status launch_decode(const df11_tensor *t, uint16_t *out, uint32_t *err_word, void *stream) {
@@ -961,12 +965,19 @@ df11_status launch_decode(const df11_tensor *t, uint16_t *out, uint32_t *err_wor
     a.err = err_word;
     a.out_al32 = ((uintptr_t)out & 31u) == 0 ? 1u : 0u;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    bool wide, lng;
-    pick_instance(t, wide, lng);
-    if (wide && !lng) launch<CfgWide, false>(a, t->n_blocks, sms, s);
-    else if (wide) launch<CfgWide, true>(a, t->n_blocks, sms, s);
-    else if (!lng) launch<CfgDense, false>(a, t->n_blocks, sms, s);
-    else launch<CfgDense, true>(a, t->n_blocks, sms, s);
+    Inst inst;
+    bool lng;
+    pick_instance(t, inst, lng);
+    if (inst == Inst::kTypical) {
+        if (lng) launch<CfgTypical, true>(a, t->n_blocks, sms, s);
+        else launch<CfgTypical, false>(a, t->n_blocks, sms, s);
+    } else if (inst == Inst::kWide) {
+        if (lng) launch<CfgWide, true>(a, t->n_blocks, sms, s);
+        else launch<CfgWide, false>(a, t->n_blocks, sms, s);
+    } else {
+        if (lng) launch<CfgDense, true>(a, t->n_blocks, sms, s);
+        else launch<CfgDense, false>(a, t->n_blocks, sms, s);
+    }
     if (cudaGetLastError() != cudaSuccess) return DF11_ERR_CUDA;
     return DF11_OK;
 }
@@ -1000,12 +1011,19 @@ df11_status launch_rows(const df11_tensor *t, uint64_t row_len, const uint32_t *
     g.n_rows_total = t->n_elems / row_len;
     g.n_rows = n_rows;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    bool wide, lng;
-    pick_instance(t, wide, lng);
-    if (wide && !lng) launch_gather<CfgWide, false>(g, sms, s);
-    else if (wide) launch_gather<CfgWide, true>(g, sms, s);
-    else if (!lng) launch_gather<CfgDense, false>(g, sms, s);
-    else launch_gather<CfgDense, true>(g, sms, s);
+    Inst inst;
+    bool lng;
+    pick_instance(t, inst, lng);
+    if (inst == Inst::kTypical) {
+        if (lng) launch_gather<CfgTypical, true>(g, sms, s);
+        else launch_gather<CfgTypical, false>(g, sms, s);
+    } else if (inst == Inst::kWide) {
+        if (lng) launch_gather<CfgWide, true>(g, sms, s);
+        else launch_gather<CfgWide, false>(g, sms, s);
+    } else {
+        if (lng) launch_gather<CfgDense, true>(g, sms, s);
+        else launch_gather<CfgDense, false>(g, sms, s);
+    }
     if (cudaGetLastError() != cudaSuccess) return DF11_ERR_CUDA;
     return DF11_OK;
 }
