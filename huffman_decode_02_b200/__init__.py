@@ -30,7 +30,7 @@ from . import build as _build
 
 __all__ = [
     "DF11Error", "CorruptStreamError", "Params", "DF11Tensor", "encode", "encode_multi",
-    "decode", "decode_block", "decode_rows", "gemm", "read_error", "exponent_histogram", "lib_path", "sm_count",
+    "encode_device", "decode", "decode_block", "decode_rows", "gemm", "read_error", "exponent_histogram", "lib_path", "sm_count",
     "KERR_COUNT_MISMATCH", "KERR_BAD_CODE", "KERR_BAD_BLOCK", "KERR_OVERRUN", "KERR_TIMEOUT", "KERR_BAD_ROW",
 ]
 
@@ -109,6 +109,10 @@ def _lib():
     lib.df11_device_sm_count.argtypes = [P(ctypes.c_int)]
     lib.df11_gemm_bf16.argtypes = [vp, vp, vp, u32, u32, u32, vp, vp]
     lib.df11_decode_rows.argtypes = [P(_Tensor), ctypes.c_uint64, vp, u32, vp, vp, vp]
+    lib.df11_encode_device_scratch_bytes.argtypes = [u64]
+    lib.df11_encode_device_scratch_bytes.restype = u64
+    lib.df11_encode_device_size.argtypes = [vp, u64, P(_Params), P(T), vp, u64, vp]
+    lib.df11_encode_device.argtypes = [vp, u64, P(T), vp, u64, vp]
     if lib.df11_abi_version() != 2 or lib.df11_sizeof_tensor() != ctypes.sizeof(_Tensor):
         raise ImportError("libdf11.so ABI does not match this binding")
     _LIB = lib
@@ -284,6 +288,50 @@ def encode_multi(mats: Sequence, params: Params | None = None, pinned: bool = Fa
     arrs = [_as_u16(m) for m in mats]
     shapes = [tuple(getattr(m, "shape", ())) for m in mats]
     return _encode_impl(arrs, shapes, params, pinned)
+
+
+def encode_device(mats, params: Params | None = None, stream=None) -> DF11Tensor:
+    """Encodes weights already on the GPU (a CUDA BF16 tensor, or a list of
+    them encoded as one block with one shared table) with the device encoder;
+    returns a device-resident DF11Tensor, byte-identical to what `encode` /
+    `encode_multi` produce for the same weights."""
+    import torch
+    single = isinstance(mats, torch.Tensor)
+    mats = [mats] if single else list(mats)
+    if not mats:
+        raise ValueError("no matrices")
+    dev = mats[0].device
+    for m in mats:
+        if m.device != dev or m.device.type != "cuda" or m.dtype not in (torch.bfloat16, torch.int16):
+            raise TypeError("encode_device expects CUDA BF16 tensors on one device")
+    shapes = [tuple(m.shape) for m in mats]
+    offsets = [0]
+    for m in mats:
+        offsets.append(offsets[-1] + m.numel())
+    n = offsets[-1]
+    if single and mats[0].is_contiguous() and mats[0].data_ptr() % 16 == 0:
+        flat = mats[0].reshape(-1).view(torch.int16)
+    else:  # one buffer for the whole block (device-to-device copies)
+        flat = torch.empty(max(n, 8), dtype=torch.int16, device=dev)
+        for m, o in zip(mats, offsets):
+            flat[o: o + m.numel()].copy_(m.reshape(-1).view(torch.int16))
+    lib = _lib()
+    sb = int(lib.df11_encode_device_scratch_bytes(n))
+    scratch = torch.empty(max(sb, 16), dtype=torch.uint8, device=dev)
+    desc = _Tensor()
+    pc = (params or Params())._c()
+    h = _stream_handle(stream)
+    _check(lib.df11_encode_device_size(ctypes.c_void_p(flat.data_ptr()), n, ctypes.byref(pc), ctypes.byref(desc),
+                                       ctypes.c_void_p(scratch.data_ptr()), sb, h), "encode_device (size)")
+    arrays = {name: torch.empty(max(int(getattr(desc, name + "_bytes")), 16), dtype=torch.uint8, device=dev)
+              for name in _ARRAYS}
+    for name in _ARRAYS:
+        setattr(desc, name, arrays[name].data_ptr())
+    _check(lib.df11_encode_device(ctypes.c_void_p(flat.data_ptr()), n, ctypes.byref(desc),
+                                  ctypes.c_void_p(scratch.data_ptr()), sb, h), "encode_device")
+    for name in _ARRAYS:
+        setattr(desc, name, None)
+    return DF11Tensor(desc, arrays, str(dev), shapes if not single else [shapes[0]], offsets)
 
 
 def exponent_histogram(mats: Iterable) -> np.ndarray:

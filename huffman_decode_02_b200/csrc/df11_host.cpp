@@ -329,6 +329,17 @@ df11_status fill_sizes(const Sequence &seq, const df11_params *params, df11_tens
     if (seq.n > 0xFFFFFFFFull) return DF11_ERR_TOO_LARGE;
     uint64_t count[256];
     histogram(seq, count);
+    return df11::plan_from_histogram(count, seq.n, p, t);
+}
+
+}  // namespace
+
+// Code lengths, sizes and scalar fields of a tensor from its exponent
+// histogram (shared by the host encoder and the device encoder).
+df11_status df11::plan_from_histogram(const uint64_t count[256], uint64_t n, const df11_params &p, df11_tensor *t) {
+    uint64_t total = 0;
+    for (int s = 0; s < 256; ++s) total += count[s];
+    if (total != n) return DF11_ERR_INVALID_ARG;
     uint8_t len[256];
     huffman_lengths(count, len);
     int mx = 0;
@@ -340,7 +351,7 @@ df11_status fill_sizes(const Sequence &seq, const df11_params *params, df11_tens
     for (int s = 0; s < 256; ++s) bits += count[s] * len[s];
     const uint64_t span = 8ull * kBytesPerThread;
     std::memset(t, 0, offsetof(df11_tensor, enc));
-    t->n_elems = seq.n;
+    t->n_elems = n;
     t->total_bits = bits;
     t->n_threads = (bits + span - 1) / span;
     t->n_blocks = (t->n_threads + kThreadsPerBlockFmt - 1) / kThreadsPerBlockFmt;
@@ -348,12 +359,21 @@ df11_status fill_sizes(const Sequence &seq, const df11_params *params, df11_tens
     std::memcpy(t->code_len, len, 256);
     const uint64_t padded_threads = t->n_blocks * kThreadsPerBlockFmt;
     t->enc_bytes = padded_threads * kBytesPerThread + 16;
-    t->sm_bytes = ((seq.n + 15) / 16) * 16 + 16;
+    t->sm_bytes = ((n + 15) / 16) * 16 + 16;
     t->gaps_bytes = ((padded_threads * 5 + 7) / 8 + 15) / 16 * 16 + 16;
     t->block_start_bytes = ((t->n_blocks + 1) * 4 + 15) / 16 * 16 + 16;
     t->lut_bytes = df11::kLutBytes;
     return DF11_OK;
 }
+
+void df11::host_build_luts(const uint8_t len[256], uint8_t *lut) { build_luts(len, lut); }
+void df11::host_canonical_codes(const uint8_t len[256], uint32_t code[256]) {
+    uint64_t first[34];
+    uint32_t cnt[34];
+    canonical_codes(len, code, first, cnt);
+}
+
+namespace {
 
 // ------------------------------------------------------------ packing
 df11_status fill_arrays(const Sequence &seq, df11_tensor *t) {

@@ -24,6 +24,8 @@
 
 #include <stdint.h>
 
+#include "df11.h"
+
 #if defined(__CUDACC__)
 #define DF11_HD __host__ __device__
 #else
@@ -106,5 +108,10 @@ constexpr int kGroupsPerCta = 8;          // format blocks decoded side by side 
 constexpr int kCtaThreads = kGroupThreads * kGroupsPerCta;
 // Worst case codes per format block: every code 1 bit long.
 constexpr int kMaxCodesPerBlock = kThreadsPerBlockFmt * kBytesPerThread * 8;
+
+// Host planner pieces shared by the host and device encoders (df11_host.cpp).
+df11_status plan_from_histogram(const uint64_t count[256], uint64_t n, const df11_params &p, df11_tensor *t);
+void host_build_luts(const uint8_t len[256], uint8_t *lut);
+void host_canonical_codes(const uint8_t len[256], uint32_t code[256]);
 
 }  // namespace df11

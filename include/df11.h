@@ -171,6 +171,34 @@ df11_status df11_encode_multi(const uint16_t *const *mats, const uint64_t *sizes
  * (no array contents are read). */
 df11_status df11_validate(const df11_tensor *t);
 
+/* --------------------------------------------------------- device encoder */
+
+/* The encoder for weights already in device memory: the exponent histogram
+ * and the packing (EncodedExponent, PackedSignMantissa, Gaps, block output
+ * positions: "Le format DFloat11", "Noyau GPU en deux etapes et metadonnees
+ * auxiliaires") run on the GPU; the code lengths (<= 256 symbols) and the
+ * decode tables are computed on the host by the same planner as
+ * df11_encode, so the arrays are byte-identical to the host encoder's.
+ *
+ * Scratch: caller-owned device memory of df11_encode_device_scratch_bytes(n)
+ * bytes, 16-byte aligned (the library allocates no device memory). */
+uint64_t df11_encode_device_scratch_bytes(uint64_t n);
+
+/* Size pass: w is a DEVICE array of n BF16 values (16-byte aligned; a block's
+ * matrices concatenated).  Runs the histogram on `stream`, synchronises it,
+ * plans the code and fills *hdr (sizes, code lengths, counts) as
+ * df11_encode_size does; array pointers are left NULL. */
+df11_status df11_encode_device_size(const uint16_t *w, uint64_t n, const df11_params *params, df11_tensor *hdr,
+                                    void *scratch, uint64_t scratch_bytes, void *stream);
+
+/* Fill pass: io from df11_encode_device_size with its five array pointers set
+ * to caller-allocated DEVICE buffers of the planned sizes (16-byte aligned).
+ * Packs everything on `stream` (the decode tables are copied from the host)
+ * and synchronises it; sets io->max_block_codes.  DF11_ERR_INVALID_ARG if
+ * w no longer matches the planned code (e.g. changed since the size pass). */
+df11_status df11_encode_device(const uint16_t *w, uint64_t n, df11_tensor *io, void *scratch, uint64_t scratch_bytes,
+                               void *stream);
+
 /* ---------------------------------------------------------------- device */
 
 /* Decodes one compressed tensor into out (n_elems BF16 values, as uint16,
