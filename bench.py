@@ -52,6 +52,8 @@ WORKLOADS = {
     "decode-gemm": ("32 llama3.1-8b blocks (seeds 32*rank + 0..31), each decoded into one reused BF16 scratch, "
                     "then every matrix multiplied by N(0,1) BF16 activations [T, in], T in {1,16,64,256} "
                     "(seed 1000 + T), FP32-accumulate GEMM on tcgen05", None),
+    "encode-device": ("llama3.1-8b transformer block (218,112,000 BF16 weights, seed = rank) already in device memory, "
+                      "encoded on the GPU (histogram + packing; code lengths on the host)", None),
     "offload": ("llama3.1-8b blocks (seeds 0..B-1, default 4) kept in pinned host memory and streamed over PCIe "
                 "block by block, repeated; each decoded on the GPU and multiplied by BF16 activations [1, in]; "
                 "compared with streaming the same blocks as plain BF16", None),
@@ -422,6 +424,60 @@ def run_offload(args, rank: int, world: int):
         dist.destroy_process_group()
 
 
+def run_encode_device(args, rank: int, world: int):
+    """The device encoder on a block already in device memory: wall time per
+    encode (size pass with its host round trip for the histogram, then the
+    fill pass; both synchronise), against the host encoder on the same block."""
+    import torch
+    import torch.distributed as dist
+
+    import huffman_decode_02_b200 as df11
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=dev)
+    mats = workloads.llama8b_block(seed=rank_seed(rank))
+    flat_h = np.concatenate([m.reshape(-1) for m in mats])
+    flat = torch.from_numpy(flat_h.view(np.int16)).to(dev).view(torch.bfloat16)
+    d = df11.encode_device(flat)  # warm-up (allocator, module load)
+    for _ in range(max(0, args.warmup - 1)):
+        d = df11.encode_device(flat)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        d = df11.encode_device(flat)
+    torch.cuda.synchronize(dev)
+    secs = (time.perf_counter() - t0) / args.steps
+    if world > 1:
+        t = torch.tensor([secs], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        secs = float(t.item())
+    t0 = time.perf_counter()
+    h = df11.encode(flat_h)
+    host_s = time.perf_counter() - t0
+    same = all(bool(np.array_equal(h.host_array(k).view(np.uint8)[: h.nbytes(k)],
+                                   d.host_array(k).view(np.uint8)[: d.nbytes(k)])) for k in ("enc", "sm", "gaps",
+                                                                                         "block_start", "lut"))
+    ok = bool(np.array_equal(df11.decode(d).view(torch.int16).cpu().numpy().view(np.uint16), flat_h))
+    if rank == 0:
+        n = int(flat_h.size)
+        line = {"metric": "device encode throughput (BF16 weights in device memory -> DF11 arrays)",
+                "value": world * 2.0 * n / secs / 1e9, "unit": "GB/s of BF16 input", "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": secs * 1e3, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "u32", "data": "synthetic",
+                "config": {"workload": WORKLOADS["encode-device"][0], "n_elems_per_rank": n,
+                           "timing": "wall clock per encode (the API synchronises twice), max over ranks"},
+                "host_encoder_ms": host_s * 1e3, "identical_to_host_encoder": same, "roundtrip_bit_exact": ok}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -451,6 +507,9 @@ def main():
         return
     if args.workload == "offload":
         run_offload(args, rank, world)
+        return
+    if args.workload == "encode-device":
+        run_encode_device(args, rank, world)
         return
 
     import torch
