@@ -30,7 +30,7 @@ from . import build as _build
 
 __all__ = [
     "DF11Error", "CorruptStreamError", "Params", "DF11Tensor", "encode", "encode_multi",
-    "encode_device", "decode", "decode_block", "decode_rows", "gemm", "read_error", "exponent_histogram", "lib_path", "sm_count",
+    "encode_device", "encode_device_noalloc", "decode", "decode_block", "decode_rows", "gemm", "read_error", "exponent_histogram", "lib_path", "sm_count",
     "KERR_COUNT_MISMATCH", "KERR_BAD_CODE", "KERR_BAD_BLOCK", "KERR_OVERRUN", "KERR_TIMEOUT", "KERR_BAD_ROW",
 ]
 
@@ -113,6 +113,9 @@ def _lib():
     lib.df11_encode_device_scratch_bytes.restype = u64
     lib.df11_encode_device_size.argtypes = [vp, u64, P(_Params), P(T), vp, u64, vp]
     lib.df11_encode_device.argtypes = [vp, u64, P(T), vp, u64, vp]
+    lib.df11_encode_device_noalloc_max_elems.restype = u64
+    lib.df11_encode_device_size_noalloc.argtypes = [vp, u64, P(_Params), P(T), vp]
+    lib.df11_encode_device_noalloc.argtypes = [vp, u64, P(T), vp]
     if lib.df11_abi_version() != 2 or lib.df11_sizeof_tensor() != ctypes.sizeof(_Tensor):
         raise ImportError("libdf11.so ABI does not match this binding")
     _LIB = lib
@@ -332,6 +335,34 @@ def encode_device(mats, params: Params | None = None, stream=None) -> DF11Tensor
     for name in _ARRAYS:
         setattr(desc, name, None)
     return DF11Tensor(desc, arrays, str(dev), shapes if not single else [shapes[0]], offsets)
+
+
+def encode_device_noalloc(w, params: Params | None = None, stream=None) -> DF11Tensor:
+    """`encode_device` for one contiguous 16-byte-aligned CUDA BF16 tensor
+    through the library's no-allocation entry points: the encoder's scratch
+    is a fixed array inside libdf11 (inputs up to
+    df11_encode_device_noalloc_max_elems() weights; calls must not overlap on
+    a device).  The compressed arrays themselves are still allocated here."""
+    import torch
+    if not (isinstance(w, torch.Tensor) and w.device.type == "cuda" and w.is_contiguous()
+            and w.dtype in (torch.bfloat16, torch.int16)):
+        raise TypeError("encode_device_noalloc expects one contiguous CUDA BF16 tensor")
+    lib = _lib()
+    n = int(w.numel())
+    desc = _Tensor()
+    pc = (params or Params())._c()
+    h = _stream_handle(stream)
+    _check(lib.df11_encode_device_size_noalloc(ctypes.c_void_p(w.data_ptr()), n, ctypes.byref(pc),
+                                               ctypes.byref(desc), h), "encode_device_noalloc (size)")
+    arrays = {name: torch.empty(max(int(getattr(desc, name + "_bytes")), 16), dtype=torch.uint8, device=w.device)
+              for name in _ARRAYS}
+    for name in _ARRAYS:
+        setattr(desc, name, arrays[name].data_ptr())
+    _check(lib.df11_encode_device_noalloc(ctypes.c_void_p(w.data_ptr()), n, ctypes.byref(desc), h),
+           "encode_device_noalloc")
+    for name in _ARRAYS:
+        setattr(desc, name, None)
+    return DF11Tensor(desc, arrays, str(w.device), [tuple(w.shape)], [0, n])
 
 
 def exponent_histogram(mats: Iterable) -> np.ndarray:

@@ -28,6 +28,7 @@
 #include <stdint.h>
 
 #include <algorithm>
+#include <atomic>
 #include <vector>
 
 #include "df11.h"
@@ -49,11 +50,11 @@ struct CodeTables {
 
 // Scratch layout: exponent counts (256 x u64), tile offsets (n_tiles + 1 x
 // u64), the largest block's code count (u32) and the total bits (u64).
-uint64_t n_tiles_of(uint64_t n) { return (n + kTile - 1) / kTile; }
+constexpr uint64_t n_tiles_of(uint64_t n) { return (n + kTile - 1) / kTile; }
 constexpr uint64_t kOffCounts = 0;
 constexpr uint64_t kOffTiles = 2048;
-uint64_t off_tail(uint64_t n) { return kOffTiles + 8u * (n_tiles_of(n) + 1u); }
-uint64_t scratch_need(uint64_t n) { return ((off_tail(n) + 16u + 15u) / 16u) * 16u; }
+constexpr uint64_t off_tail(uint64_t n) { return kOffTiles + 8u * (n_tiles_of(n) + 1u); }
+constexpr uint64_t scratch_need(uint64_t n) { return ((off_tail(n) + 16u + 15u) / 16u) * 16u; }
 
 __device__ __forceinline__ uint32_t exponent_of(uint32_t w) { return (w >> 7) & 0xFFu; }
 
@@ -385,6 +386,59 @@ df11_status df11_encode_device(const uint16_t *w, uint64_t n, df11_tensor *io, v
     if (total != io->total_bits) return DF11_ERR_INVALID_ARG;  // the input changed since the size pass
     io->max_block_codes = most;
     return DF11_OK;
+}
+
+}  // extern "C"
+
+// ------------------------------------------------------------ no-alloc entry points
+// The same encoder with its scratch in a fixed array of this library
+// instead of caller memory, for callers that must not allocate device memory
+// (see df11.h).  Inputs of up to kNoAllocMaxElems weights.
+namespace {
+
+constexpr uint64_t kNoAllocMaxElems = 1ull << 28;
+constexpr uint64_t kNoAllocScratchBytes = scratch_need(kNoAllocMaxElems);
+__device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+std::atomic<uintptr_t> g_noalloc_addr[64];
+
+// Device address of the fixed scratch on the current device, resolved once
+// per device (cudaGetSymbolAddress with that device current).
+df11_status noalloc_scratch(void **out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return DF11_ERR_CUDA;
+    if (dev < 0 || dev >= 64) return DF11_ERR_UNSUPPORTED;
+    uintptr_t a = g_noalloc_addr[dev].load(std::memory_order_acquire);
+    if (a == 0) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return DF11_ERR_CUDA;
+        a = reinterpret_cast<uintptr_t>(p);
+        g_noalloc_addr[dev].store(a, std::memory_order_release);
+    }
+    *out = reinterpret_cast<void *>(a);
+    return DF11_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+uint64_t df11_encode_device_noalloc_max_elems(void) { return kNoAllocMaxElems; }
+
+df11_status df11_encode_device_size_noalloc(const uint16_t *w, uint64_t n, const df11_params *params,
+                                            df11_tensor *hdr, void *stream) {
+    if (n > kNoAllocMaxElems) return DF11_ERR_TOO_LARGE;
+    void *scratch = nullptr;
+    const df11_status st = noalloc_scratch(&scratch);
+    if (st != DF11_OK) return st;
+    return df11_encode_device_size(w, n, params, hdr, scratch, kNoAllocScratchBytes, stream);
+}
+
+df11_status df11_encode_device_noalloc(const uint16_t *w, uint64_t n, df11_tensor *io, void *stream) {
+    if (n > kNoAllocMaxElems) return DF11_ERR_TOO_LARGE;
+    void *scratch = nullptr;
+    const df11_status st = noalloc_scratch(&scratch);
+    if (st != DF11_OK) return st;
+    return df11_encode_device(w, n, io, scratch, kNoAllocScratchBytes, stream);
 }
 
 }  // extern "C"

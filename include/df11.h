@@ -199,6 +199,28 @@ df11_status df11_encode_device_size(const uint16_t *w, uint64_t n, const df11_pa
 df11_status df11_encode_device(const uint16_t *w, uint64_t n, df11_tensor *io, void *scratch, uint64_t scratch_bytes,
                                void *stream);
 
+/* The device encoder without caller scratch.  The pages describe no
+ * counterpart of these calls: they are a convenience of this library for
+ * callers that must not allocate device memory around an encode -- e.g. a
+ * runtime that owns all device memory through a fixed pool, or a serving
+ * process re-encoding weights in place on a full GPU, where cudaMalloc would
+ * fail or synchronise the device.  The scratch is a fixed array inside
+ * libdf11 (about 258 KB per device), so:
+ *  - n is limited to df11_encode_device_noalloc_max_elems() (2^28 weights, a
+ *    whole Llama-3.1-8B block); larger inputs return DF11_ERR_TOO_LARGE
+ *    before any GPU work;
+ *  - the first call on a device resolves the array's address
+ *    (cudaGetSymbolAddress with that device current): make it before any
+ *    stream capture;
+ *  - calls that overlap on one device (other host threads or streams) share
+ *    that array and race: serialise them per device.
+ * Everything the encoder needs cleared is cleared by each call.  Otherwise
+ * as df11_encode_device_size / df11_encode_device. */
+uint64_t df11_encode_device_noalloc_max_elems(void);
+df11_status df11_encode_device_size_noalloc(const uint16_t *w, uint64_t n, const df11_params *params,
+                                            df11_tensor *hdr, void *stream);
+df11_status df11_encode_device_noalloc(const uint16_t *w, uint64_t n, df11_tensor *io, void *stream);
+
 /* ---------------------------------------------------------------- device */
 
 /* Decodes one compressed tensor into out (n_elems BF16 values, as uint16,
