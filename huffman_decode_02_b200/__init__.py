@@ -87,8 +87,7 @@ def _lib():
         return _LIB
     path = _build.LIB_PATH
     if not os.path.exists(path):
-        raise ImportError(f"libdf11.so is not built ({path}); run __graft_entry__.build() or "
-                          "python -m huffman_decode_02_b200.build")
+        raise ImportError(f"libdf11.so is not built ({path}); run python -m huffman_decode_02_b200.build")
     lib = ctypes.CDLL(path)
     P, T, u64, u32, vp = ctypes.POINTER, _Tensor, ctypes.c_uint64, ctypes.c_uint32, ctypes.c_void_p
     u16pp = P(P(ctypes.c_uint16))

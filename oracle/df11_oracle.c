@@ -24,7 +24,7 @@
  *  - Canonical code assignment by (length, symbol) as defined in RFC 1951
  *    section 3.2.2.
  *
- * Readings of points the pages leave open (listed again in the design doc):
+ * Readings of points the pages leave open:
  *  - Exponent bits are packed MSB-first inside each byte, bytes in increasing
  *    address order; the last partial byte is zero-filled.
  *  - The sign/mantissa byte of a weight is (sign << 7) | mantissa.

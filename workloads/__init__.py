@@ -8,7 +8,7 @@ pages discuss (Llama-3.1-8B / 70B) and with weight-like value distributions.
 
 All arrays are returned as ``numpy.uint16`` BF16 bit patterns.
 
-Recipes (each one is also written out in the design doc):
+Recipes:
 
 * ``normal_matrix(rows, cols, std, seed)`` -- i.i.d. N(0, std^2) float32,
   rounded to BF16.  1024x1024 / seed 0 and 4096x4096 / seed 1 are the
