@@ -234,6 +234,101 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (err && g.err) atomicOr(g.err, err);
 }
 
+// ---------------------------------------------------------------- T <= 4
+// With T <= 4 tokens every weight feeds at most 8 flops: the product is a
+// matrix-vector stream bound by reading W, and the tensor-core tiling (128
+// rows x 64 columns per load) reads W with poor DRAM locality.  This kernel
+// streams W along contiguous rows instead: a CTA of 8 warps takes R rows,
+// S = 8 / R warps share a row's K range, each lane loads 16 bytes (8 weights)
+// per step with several loads in flight, multiplies them by X (read through
+// the cache: X is small and shared by every CTA) in FP32, and the partial sums
+// are reduced by warp shuffles and then across the row's warps in shared
+// memory.  One writer per output: no atomics, no zeroing, deterministic.
+constexpr uint32_t kGemvThreads = 256;
+
+__device__ __forceinline__ uint4 ld_stream_u4(const void *p) {
+    uint4 r;
+    asm("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+        : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+        : "l"(p));
+    return r;
+}
+
+// 8 BF16 products (two per 32-bit word) added into acc.
+__device__ __forceinline__ float dot8(const uint4 a, const uint4 b, float acc) {
+    const uint32_t A[4] = {a.x, a.y, a.z, a.w}, B[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        acc = fmaf(__uint_as_float(A[i] << 16), __uint_as_float(B[i] << 16), acc);
+        acc = fmaf(__uint_as_float(A[i] & 0xFFFF0000u), __uint_as_float(B[i] & 0xFFFF0000u), acc);
+    }
+    return acc;
+}
+
+template <int T, int R>
+__global__ void __launch_bounds__(kGemvThreads) gemv_kernel(const uint16_t *x, const uint16_t *w, float *y,
+                                                            uint32_t out, uint32_t in) {
+    constexpr uint32_t S = 8 / R;  // warps per row
+    __shared__ float part[8][T];
+    const uint32_t warp = threadIdx.x >> 5, lane = threadIdx.x & 31u;
+    const uint32_t row = blockIdx.x * R + (warp % R);
+    const uint32_t split = warp / R;
+    const uint32_t n8 = in / (8u * S);  // 16-byte chunks in this warp's K range
+    const uint32_t k0 = split * n8;     // first chunk
+    const uint4 *wr = reinterpret_cast<const uint4 *>(w + (uint64_t)row * in) + k0;
+    const uint4 *xr = reinterpret_cast<const uint4 *>(x) + k0;
+    const uint32_t xstride = in / 8u;   // chunks per token row of X
+    float acc[T];
+#pragma unroll
+    for (int t = 0; t < T; ++t) acc[t] = 0.f;
+    uint32_t c = lane;
+    for (; c + 96u < n8; c += 128u) {  // four loads of W in flight per lane
+        const uint4 w0 = ld_stream_u4(wr + c), w1 = ld_stream_u4(wr + c + 32u);
+        const uint4 w2 = ld_stream_u4(wr + c + 64u), w3 = ld_stream_u4(wr + c + 96u);
+#pragma unroll
+        for (int t = 0; t < T; ++t) {
+            const uint4 *xt = xr + (uint64_t)t * xstride + c;
+            acc[t] = dot8(w0, __ldg(xt), acc[t]);
+            acc[t] = dot8(w1, __ldg(xt + 32u), acc[t]);
+            acc[t] = dot8(w2, __ldg(xt + 64u), acc[t]);
+            acc[t] = dot8(w3, __ldg(xt + 96u), acc[t]);
+        }
+    }
+    for (; c < n8; c += 32u) {
+        const uint4 w0 = ld_stream_u4(wr + c);
+#pragma unroll
+        for (int t = 0; t < T; ++t) acc[t] = dot8(w0, __ldg(xr + (uint64_t)t * xstride + c), acc[t]);
+    }
+#pragma unroll
+    for (int t = 0; t < T; ++t) {
+        float v = acc[t];
+#pragma unroll
+        for (uint32_t d = 16; d > 0; d >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, d);
+        if (lane == 0) part[warp][t] = v;
+    }
+    __syncthreads();
+    if (threadIdx.x < (uint32_t)(R * T)) {
+        const uint32_t r = threadIdx.x % R, t = threadIdx.x / R;
+        float v = 0.f;
+#pragma unroll
+        for (uint32_t sp = 0; sp < S; ++sp) v += part[sp * R + r][t];
+        y[(uint64_t)t * out + blockIdx.x * R + r] = v;
+    }
+}
+
+template <int T>
+void launch_gemv(const uint16_t *x, const uint16_t *w, float *y, uint32_t out, uint32_t in, int sms,
+                 cudaStream_t s) {
+    // rows per CTA: enough CTAs (about 6 per SM) for the loads in flight
+    uint32_t r = out / (6u * (uint32_t)sms);
+    r = r >= 8u ? 8u : r >= 4u ? 4u : r >= 2u ? 2u : 1u;
+    const unsigned grid = out / r;
+    if (r == 8u) gemv_kernel<T, 8><<<grid, kGemvThreads, 0, s>>>(x, w, y, out, in);
+    else if (r == 4u) gemv_kernel<T, 4><<<grid, kGemvThreads, 0, s>>>(x, w, y, out, in);
+    else if (r == 2u) gemv_kernel<T, 2><<<grid, kGemvThreads, 0, s>>>(x, w, y, out, in);
+    else gemv_kernel<T, 1><<<grid, kGemvThreads, 0, s>>>(x, w, y, out, in);
+}
+
 // ---------------------------------------------------------------- host
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 std::once_flag g_encode_once;
@@ -274,6 +369,16 @@ extern "C" df11_status df11_gemm_bf16(const uint16_t *x, const uint16_t *w, floa
     int dev = 0, sms = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return DF11_ERR_CUDA;
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return DF11_ERR_CUDA;
+
+    if (T <= 4u) {  // matrix-vector stream on the CUDA cores
+        cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+        if (T == 1u) launch_gemv<1>(x, w, y, out, in, sms, s);
+        else if (T == 2u) launch_gemv<2>(x, w, y, out, in, sms, s);
+        else if (T == 3u) launch_gemv<3>(x, w, y, out, in, sms, s);
+        else launch_gemv<4>(x, w, y, out, in, sms, s);
+        if (cudaGetLastError() != cudaSuccess) return DF11_ERR_CUDA;
+        return DF11_OK;
+    }
 
     GemmArgs g;
     g.y = y;

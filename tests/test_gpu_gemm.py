@@ -1,5 +1,6 @@
-"""The consumer GEMM (tcgen05, FP32 accumulation) against a CPU GEMM: the
-relative Frobenius error must stay within 2e-3.  Inputs are BF16, so every
+"""The consumer GEMM (tcgen05 for T > 4, a CUDA-core matrix-vector stream
+for T <= 4; FP32 accumulation) against a CPU GEMM: the relative Frobenius
+error must stay within 2e-3.  Inputs are BF16, so every
 product is exact in FP32 and the two sides differ only in summation order."""
 import numpy as np
 import pytest
@@ -47,7 +48,8 @@ def test_gemm_q_proj_shape(T):
 
 
 @pytest.mark.parametrize("T,out,inn", [(5, 1024, 4096), (33, 128, 64), (256, 14336, 4096), (16, 4096, 14336),
-                                       (200, 256, 128)])
+                                       (200, 256, 128), (1, 14336, 4096), (2, 4096, 14336), (3, 1024, 4096),
+                                       (4, 128, 64), (4, 256, 128)])
 def test_gemm_other_shapes(T, out, inn):
     _check(T, out, inn, seed=T + out)
 
