@@ -30,7 +30,7 @@ from . import build as _build
 
 __all__ = [
     "DF11Error", "CorruptStreamError", "Params", "DF11Tensor", "encode", "encode_multi",
-    "encode_device", "encode_device_noalloc", "decode", "decode_block", "decode_rows", "gemm", "read_error", "exponent_histogram", "lib_path", "sm_count",
+    "encode_device", "encode_device_noalloc", "save", "load", "decode", "decode_block", "decode_rows", "gemm", "read_error", "exponent_histogram", "lib_path", "sm_count",
     "KERR_COUNT_MISMATCH", "KERR_BAD_CODE", "KERR_BAD_BLOCK", "KERR_OVERRUN", "KERR_TIMEOUT", "KERR_BAD_ROW",
 ]
 
@@ -362,6 +362,56 @@ def encode_device_noalloc(w, params: Params | None = None, stream=None) -> DF11T
     for name in _ARRAYS:
         setattr(desc, name, None)
     return DF11Tensor(desc, arrays, str(w.device), [tuple(w.shape)], [0, n])
+
+
+_FILE_MAGIC = b"DF11T001"
+
+
+def save(t: DF11Tensor, path: str) -> None:
+    """Writes a compressed tensor (host or device) to `path` as an .npz
+    archive: the descriptor bytes (array pointers cleared), the five arrays
+    and the matrix shapes and offsets.  Nothing is decoded."""
+    desc = _Tensor.from_buffer_copy(t.desc)
+    for name in _ARRAYS:
+        setattr(desc, name, None)
+    arrays = {name: t.host_array(name).view(np.uint8).reshape(-1)[: t.nbytes(name)] for name in _ARRAYS}
+    shapes = np.array([len(s) for s in t.shapes] + [d for s in t.shapes for d in s], dtype=np.int64)
+    np.savez(path, magic=np.frombuffer(_FILE_MAGIC, dtype=np.uint8), desc=np.frombuffer(bytes(desc), dtype=np.uint8),
+             offsets=np.asarray(t.offsets, dtype=np.int64), shapes=shapes, **arrays)
+
+
+def load(path: str, pinned: bool = False) -> DF11Tensor:
+    """Reads a tensor written by `save` into host memory (pinned torch
+    buffers if `pinned`); the descriptor is checked by df11_validate."""
+    with np.load(path) as z:
+        if bytes(z["magic"]) != _FILE_MAGIC:
+            raise ValueError("not a DF11 tensor file")
+        raw = bytes(z["desc"])
+        if len(raw) != ctypes.sizeof(_Tensor):
+            raise ValueError("descriptor size does not match this library")
+        desc = _Tensor.from_buffer_copy(raw)
+        arrays = {}
+        for name in _ARRAYS:
+            a = z[name]
+            if a.size != int(getattr(desc, name + "_bytes")):
+                raise ValueError(f"array {name} has the wrong size")
+            buf = _alloc_host(a.size, pinned)
+            if pinned:
+                import torch
+                buf[: a.size].copy_(torch.from_numpy(np.ascontiguousarray(a)))
+            else:
+                buf[: a.size] = a
+            arrays[name] = buf
+        offsets = [int(v) for v in z["offsets"]]
+        sh = [int(v) for v in z["shapes"]]
+    k = len(offsets) - 1
+    ndims, dims = sh[:k], sh[k:]
+    shapes, pos = [], 0
+    for nd in ndims:
+        shapes.append(tuple(dims[pos: pos + nd]))
+        pos += nd
+    _check(_lib().df11_validate(ctypes.byref(desc)), "load")
+    return DF11Tensor(desc, arrays, "cpu", shapes, offsets)
 
 
 def exponent_histogram(mats: Iterable) -> np.ndarray:

@@ -255,3 +255,26 @@ def test_table_walk_reproduces_exponents(name):
     assert np.array_equal(np.diff(bs[: t.n_blocks + 1]), per_block)
     if name == "long_codes":
         assert t.code_len.max() > 14
+
+
+def test_save_load_round_trip(tmp_path):
+    """A compressed block written and read back: identical descriptor and
+    arrays, same matrix shapes and offsets, and the oracle decodes the loaded
+    stream to the original weights."""
+    mats = [workloads.normal_matrix(64, 48, 0.02, seed=3), workloads.normal_matrix(5, 7, 0.5, seed=4)]
+    t = df11.encode_multi(mats)
+    path = str(tmp_path / "blk.npz")
+    df11.save(t, path)
+    u = df11.load(path)
+    assert bytes(u.desc)[:8] == bytes(t.desc)[:8] and u.n_elems == t.n_elems and u.total_bits == t.total_bits
+    assert u.shapes == [(64, 48), (5, 7)] and u.offsets == t.offsets
+    for k in ("enc", "sm", "gaps", "block_start", "lut"):
+        np.testing.assert_array_equal(u.host_array(k).view(np.uint8)[: u.nbytes(k)],
+                                      t.host_array(k).view(np.uint8)[: t.nbytes(k)])
+    out = oracle.decode(u.host_array("enc"), u.total_bits, u.host_array("sm"), u.n_elems, u.code_len)
+    np.testing.assert_array_equal(out, np.concatenate([m.reshape(-1) for m in mats]))
+    with open(path, "r+b") as f:  # a damaged file is refused
+        f.seek(0)
+        f.write(b"\0" * 16)
+    with pytest.raises(Exception):
+        df11.load(path)
