@@ -1,8 +1,14 @@
 """Builds libdf11.so in-tree with nvcc for sm_100a.
 
-Sources: csrc/df11_host.cpp (host encoder / planner) and csrc/df11_decode.cu
-(decode kernel + launchers), plus csrc/df11_gemm.cu when present.  The CUDA
-runtime is linked statically, so the library needs only the driver.
+Sources: every csrc/*.cu and csrc/*.cpp (host encoder / planner, decode and
+row-gather kernels, device encoder, consumer GEMM).  The CUDA runtime is
+linked statically, so the library needs only the driver.
+
+`build(debug=True)` builds libdf11_debug.so from the same sources with
+DF11_DEBUG_CHECKS: every data-dependent shared-memory index and global
+store address of the decode kernels is checked before the access (a failed
+check skips it and is counted; read with df11_debug_bounds_errors).  It is
+for tests; the product library is libdf11.so.
 """
 from __future__ import annotations
 
@@ -16,6 +22,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB_PATH = os.path.join(HERE, "libdf11.so")
+DEBUG_LIB_PATH = os.path.join(HERE, "libdf11_debug.so")
 
 NVCC_FLAGS = [
     "-std=c++17", "-O3", "-lineinfo",
@@ -34,25 +41,27 @@ def sources() -> list[str]:
     return sorted(glob.glob(os.path.join(CSRC, "*.cu")) + glob.glob(os.path.join(CSRC, "*.cpp")))
 
 
-def _stale() -> bool:
-    if not os.path.exists(LIB_PATH):
+def _stale(path: str) -> bool:
+    if not os.path.exists(path):
         return True
-    t = os.path.getmtime(LIB_PATH)
+    t = os.path.getmtime(path)
     deps = sources() + glob.glob(os.path.join(CSRC, "*.h")) + glob.glob(os.path.join(INCLUDE, "*.h"))
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and not _stale():
-        return LIB_PATH
-    tmp = LIB_PATH + f".tmp{os.getpid()}"
-    cmd = [_nvcc(), *NVCC_FLAGS, "-I" + INCLUDE, "-I" + CSRC, *sources(), "-o", tmp]
+def build(force: bool = False, verbose: bool = False, debug: bool = False) -> str:
+    path = DEBUG_LIB_PATH if debug else LIB_PATH
+    if not force and not _stale(path):
+        return path
+    tmp = path + f".tmp{os.getpid()}"
+    extra = ["-DDF11_DEBUG_CHECKS"] if debug else []
+    cmd = [_nvcc(), *NVCC_FLAGS, *extra, "-I" + INCLUDE, "-I" + CSRC, *sources(), "-o", tmp]
     if verbose:
         print(" ".join(cmd), file=sys.stderr)
     subprocess.check_call(cmd)
-    os.replace(tmp, LIB_PATH)
-    return LIB_PATH
+    os.replace(tmp, path)
+    return path
 
 
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv, verbose=True))
+    print(build(force="--force" in sys.argv, verbose=True, debug="--debug" in sys.argv))

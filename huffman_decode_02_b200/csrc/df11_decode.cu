@@ -95,6 +95,18 @@ constexpr uint32_t kFull = 0xFFFFFFFFu;
 constexpr uint32_t kLoopCap = DF11_LOOP_CAP;  // lookups per decode loop (95 suffice)
 constexpr uint32_t kKernErrTimeout = 0x10u;  // an asynchronous copy did not complete in time
 static_assert(kGroupThreads == 128, "group scan assumes four warps");
+
+// Debug builds (DF11_DEBUG_CHECKS, libdf11_debug.so) check every
+// data-dependent shared-memory index and global store address against its
+// array before the access; a failed check skips the access and is counted in
+// a device word the host reads back.  In the product build the checks are
+// the constant `true` and generate no code.
+#ifdef DF11_DEBUG_CHECKS
+__device__ uint32_t g_df11_bounds_errors;
+#define DF11_BOUNDS_OK(cond) ((cond) || (atomicAdd(&g_df11_bounds_errors, 1u), false))
+#else
+#define DF11_BOUNDS_OK(cond) true
+#endif
 static_assert(kLutBytes % 16 == 0, "bulk copy size");
 
 // Per-instance layout: G groups per CTA, buffers of S symbols (+ 16: the
@@ -275,7 +287,7 @@ __device__ __forceinline__ void merge_edges(const uint8_t *sm, uint16_t *out, ui
     const uint32_t c = (lane < 16u) ? 0u : c_full;
     const bool mine = (lane < 16u) ? head : tail;
     const uint32_t g = base + 16u * c + (lane & 15u);
-    if (mine && g >= s && g < e) {
+    if (mine && g >= s && g < e && DF11_BOUNDS_OK(g - base < kMaxCodesPerBlock + 16u)) {
         const uint32_t sm8 = __ldg(sm + g);
         const uint32_t r = lds_u8(sb + (g - base));
         // r = rotated exponent: high byte (s & 0x80) | (r & 0x7F), low byte (r & 0x80) | (s & 0x7F)
@@ -342,6 +354,7 @@ __device__ __forceinline__ uint32_t count_long_code(uint32_t acc, uint32_t lim, 
 // Same for the decoding pass: ORs the long code's symbol into the buffer at
 // index p, shifts the window and returns the meta word of 1 code with a
 // zero shift amount; an invalid pattern stops the chain at pend.
+template <uint32_t kBufBytes>
 __device__ __forceinline__ uint32_t decode_long_code(uint32_t pacc, uint32_t pend, uint32_t &hi, uint32_t &lo,
                                                      uint32_t &fl, uint32_t sb, uint32_t s_lim, uint32_t s_offs,
                                                      uint32_t s_symrot, uint32_t from, uint32_t max_len) {
@@ -349,7 +362,8 @@ __device__ __forceinline__ uint32_t decode_long_code(uint32_t pacc, uint32_t pen
     if (l == 0u) return (pend - pacc + 31u) & ~31u;  // reported by the count pass
     const uint32_t idx = (hi >> (32u - l)) + lds_u32(s_offs + 4u * l);
     const uint32_t p = pacc >> 8;
-    red_or(sb + (p & ~3u), lds_u8(s_symrot + (idx & 255u)) << (8u * (p & 3u)));
+    if (DF11_BOUNDS_OK((p & ~3u) + 4u <= kBufBytes))
+        red_or(sb + (p & ~3u), lds_u8(s_symrot + (idx & 255u)) << (8u * (p & 3u)));
     shift_window_clamped(hi, lo, fl, l);
     return 1u << 8;
 }
@@ -371,8 +385,8 @@ __device__ __forceinline__ void count_pass(const Chain &A, const Chain &B, const
     uint32_t guard = kLoopCap;
     while (((aA < limA) | (aB < limB)) && guard != 0u) {
         --guard;
-        uint32_t eA = cnt[(hA >> sh1) * kCountCopies];
-        uint32_t eB = cnt[(hB >> sh1) * kCountCopies];
+        uint32_t eA = DF11_BOUNDS_OK((hA >> sh1) < (1u << kW1Max)) ? cnt[(hA >> sh1) * kCountCopies] : kEscape;
+        uint32_t eB = DF11_BOUNDS_OK((hB >> sh1) < (1u << kW1Max)) ? cnt[(hB >> sh1) * kCountCopies] : kEscape;
         eA = (aA < limA) ? eA : 0u;
         eB = (aB < limB) ? eB : 0u;
         // Long codes exist only when the code is longer than the window; an
@@ -402,7 +416,7 @@ __device__ __forceinline__ void count_pass(const Chain &A, const Chain &B, const
 // unused symbol bytes of a table entry are zero.  Stops on the code counts
 // of the count pass.  `sym` points at this lane's copy of the symbol table
 // (entry i at sym[i * kSymCopies]).
-template <bool kLong, uint32_t kSymCopies>
+template <bool kLong, uint32_t kSymCopies, uint32_t kBufBytes>
 __device__ __forceinline__ void decode_pass(const Chain &A, const Chain &B, uint32_t startA, uint32_t cA,
                                             uint32_t startB, uint32_t cB, uint32_t *buf, uint32_t sb,
                                             const uint2 *sym, uint32_t sh2, uint32_t s_lim, uint32_t s_offs,
@@ -413,16 +427,18 @@ __device__ __forceinline__ void decode_pass(const Chain &A, const Chain &B, uint
     uint32_t guard = kLoopCap;  // as in the count pass
     while (((pA < endPA) | (pB < endPB)) && guard != 0u) {
         --guard;
-        const uint2 eA = sym[(hA >> sh2) * kSymCopies];
-        const uint2 eB = sym[(hB >> sh2) * kSymCopies];
+        const uint2 eA = DF11_BOUNDS_OK((hA >> sh2) < (1u << kW2Max)) ? sym[(hA >> sh2) * kSymCopies]
+                                                                      : make_uint2(0u, kEscape);
+        const uint2 eB = DF11_BOUNDS_OK((hB >> sh2) < (1u << kW2Max)) ? sym[(hB >> sh2) * kSymCopies]
+                                                                      : make_uint2(0u, kEscape);
         const bool actA = pA < endPA, actB = pB < endPB;
         uint32_t mA = actA ? eA.y : 0u;
         uint32_t mB = actB ? eB.y : 0u;
         if (kLong && (mA | mB) >= kEscape) {  // rare: a long code
             if (mA == kEscape)
-                mA = decode_long_code(pA, endPA, hA, lA, fA, sb, s_lim, s_offs, s_symrot, from, max_len);
+                mA = decode_long_code<kBufBytes>(pA, endPA, hA, lA, fA, sb, s_lim, s_offs, s_symrot, from, max_len);
             if (mB == kEscape)
-                mB = decode_long_code(pB, endPB, hB, lB, fB, sb, s_lim, s_offs, s_symrot, from, max_len);
+                mB = decode_long_code<kBufBytes>(pB, endPB, hB, lB, fB, sb, s_lim, s_offs, s_symrot, from, max_len);
         }
         const uint32_t bA = pA >> 8, bB = pB >> 8;
         const uint32_t shA = (bA & 3u) << 3, shB = (bB & 3u) << 3;
@@ -430,11 +446,11 @@ __device__ __forceinline__ void decode_pass(const Chain &A, const Chain &B, uint
         // (an escape entry has no symbol bytes: its stores OR zero)
         // the second word only when symbol bytes reach it (OR with zero is a no-op)
         const uint32_t hiA = __funnelshift_l(eA.x, 0u, shA), hiB = __funnelshift_l(eB.x, 0u, shB);
-        if (actA) {
+        if (actA && DF11_BOUNDS_OK(4u * ((bA >> 2) + 2u) <= kBufBytes)) {
             atomicOr(wA, eA.x << shA);
             if (hiA) atomicOr(wA + 1, hiA);
         }
-        if (actB) {
+        if (actB && DF11_BOUNDS_OK(4u * ((bB >> 2) + 2u) <= kBufBytes)) {
             atomicOr(wB, eB.x << shB);
             if (hiB) atomicOr(wB + 1, hiB);
         }
@@ -455,9 +471,14 @@ __device__ __forceinline__ void decode_pass(const Chain &A, const Chain &B, uint
 // each buffer chunk it reads (the decoding pass ORs into a clear buffer).
 // Stores are 32 bytes per thread when `out` is 32-byte aligned (one warp
 // instruction writes 1 KB of whole sectors), else two 16-byte stores.
+template <uint32_t kBufBytes>
 __device__ __forceinline__ void merge_chunks(uint16_t *out, uint32_t sb, uint32_t base, uint32_t c_first,
-                                             uint32_t c_end, uint32_t sm_s, uint32_t c_lo, uint32_t al32) {
+                                             uint32_t c_end, uint32_t sm_s, uint32_t c_lo, uint32_t al32,
+                                             uint64_t n_elems) {
     for (uint32_t c = c_first; c < c_end; c += kGroupThreads) {
+        if (!DF11_BOUNDS_OK(16u * (c + 1u) <= kBufBytes && (uint64_t)base + 16ull * (c + 1u) <= n_elems &&
+                            c >= c_lo && 16u * (c - c_lo + 1u) <= kBufBytes))
+            continue;
         const uint4 smv = lds_u4(sm_s + 16u * (c - c_lo));
         const uint4 ex = lds_u4(sb + 16u * c);
         sts_zero16(sb + 16u * c);
@@ -688,7 +709,7 @@ __global__ void __launch_bounds__(C::kCtaThreads, 1) df11_decode_kernel(const De
         // ---- pass 2: decode both chains again into the buffer
         if (ok) {
             const uint32_t startA = (s - base) + wpre + incl - cnt;  // buffer index of A's first code
-            decode_pass<kLong, C::kSymCopies>(A, B, startA, cA, startA + cA, cB, buf, sb, sym_lane, sh2, s_lim, s_offs, s_symrot,
+            decode_pass<kLong, C::kSymCopies, C::kSbufBytes>(A, B, startA, cA, startA + cA, cB, buf, sb, sym_lane, sh2, s_lim, s_offs, s_symrot,
                         w2 + 1u, max_len);
         }
         group_barrier(group);
@@ -697,7 +718,7 @@ __global__ void __launch_bounds__(C::kCtaThreads, 1) df11_decode_kernel(const De
         if (!wait_phase(mb_sm, ph_sm)) my_err |= kKernErrTimeout;
         ph_sm ^= 1u;
         if (ok) {
-            merge_chunks(a.out, sb, base, c0, c_full, grp + C::kGrpSm, c_lo, a.out_al32);
+            merge_chunks<C::kSbufBytes>(a.out, sb, base, c0, c_full, grp + C::kGrpSm, c_lo, a.out_al32, a.n_elems);
             if (warp == 0) merge_edges_clear(a.sm, a.out, sb, base, c_full, span, s, e, lane);
         }
         // No barrier here: the next block's buffer writes and staging copies
@@ -850,13 +871,14 @@ __global__ void __launch_bounds__(C::kCtaThreads, 1) df11_gather_kernel(const Ga
             if (!ok && lt == 0) my_err |= range_ok ? DF11_KERR_COUNT_MISMATCH : DF11_KERR_BAD_BLOCK;
             if (ok) {
                 const uint32_t startA = (s - base) + wpre + incl - cnt;
-                decode_pass<kLong, C::kSymCopies>(A, B, startA, cA, startA + cA, cB, buf, sb, sym_lane, sh2, s_lim, s_offs,
+                decode_pass<kLong, C::kSymCopies, C::kSbufBytes>(A, B, startA, cA, startA + cA, cB, buf, sb, sym_lane, sh2, s_lim, s_offs,
                                    s_symrot, w2 + 1u, max_len);
             }
             group_barrier(group);
             if (ok) {  // the row's part of this block, element by element
                 const uint64_t g0 = max((uint64_t)s, lo), g1 = min((uint64_t)e, hi);
                 for (uint64_t g = g0 + lt; g < g1; g += kGroupThreads) {
+                    if (!DF11_BOUNDS_OK(g - lo < ga.row_len && g - base < C::kSbufBytes && g < a.n_elems)) continue;
                     const uint32_t sm8 = __ldg(a.sm + g);
                     const uint32_t r = lds_u8(sb + (uint32_t)(g - base));
                     const uint32_t hi8 = (sm8 & 0x80u) | (r & 0x7Fu);
@@ -1049,6 +1071,21 @@ df11_status df11_decode_rows(const df11_tensor *t, uint64_t row_len, const uint3
                              uint16_t *out, uint32_t *err_word, void *stream) {
     return launch_rows(t, row_len, rows, n_rows, out, err_word, stream);
 }
+
+#ifdef DF11_DEBUG_CHECKS
+// Debug builds only (not part of the product ABI): the number of failed
+// bounds checks since the last reset; synchronises the device.
+uint32_t df11_debug_bounds_errors(int reset) {
+    uint32_t v = 0;
+    if (cudaDeviceSynchronize() != cudaSuccess) return 0xFFFFFFFFu;
+    if (cudaMemcpyFromSymbol(&v, g_df11_bounds_errors, sizeof(v)) != cudaSuccess) return 0xFFFFFFFFu;
+    if (reset) {
+        const uint32_t z = 0;
+        if (cudaMemcpyToSymbol(g_df11_bounds_errors, &z, sizeof(z)) != cudaSuccess) return 0xFFFFFFFFu;
+    }
+    return v;
+}
+#endif
 
 df11_status df11_read_error(const uint32_t *err_word, void *stream, uint32_t *host_value) {
     if (!err_word || !host_value) return DF11_ERR_INVALID_ARG;
