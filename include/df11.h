@@ -10,6 +10,7 @@
  *    LLM a 70 % de leur taille" (fr.news.hada.io).  Sections used:
  *      << La marge de compression restante dans l'exposant BFloat16 >>
  *      << Le format DFloat11 >>
+ *      << Decompression adaptee a l'inference GPU >>
  *      << Decodage fonde sur des LUT hierarchiques >>
  *      << Noyau GPU en deux etapes et metadonnees auxiliaires >>
  *      << Decompression par bloc transformer >>
@@ -25,7 +26,9 @@
  *  - Device calls are asynchronous on the given stream and return launch /
  *    argument errors immediately.  Data corruption found by a kernel is
  *    reported by OR-ing bits into a caller-owned device word (err_word).
- *  - Thread safety: calls share no mutable global state.
+ *  - Thread safety: calls share no mutable global state, except the
+ *    no-allocation encoder calls, which share one fixed scratch array per
+ *    device (see there).
  */
 #ifndef DF11_H
 #define DF11_H
@@ -258,9 +261,12 @@ df11_status df11_decode_rows(const df11_tensor *t, uint64_t row_len, const uint3
                              uint16_t *out, uint32_t *err_word, void *stream);
 
 /* Consumer of a decoded weight matrix: Y = X * W^T with BF16 inputs and FP32
- * accumulation on the tensor cores (tcgen05), the matrix multiplication the
- * decompressed weights feed ("Decompression adaptee a l'inference GPU": a
- * matrix is decompressed right before its multiplication and discarded after).
+ * accumulation, the matrix multiplication the decompressed weights feed
+ * ("Decompression adaptee a l'inference GPU": a matrix is decompressed right
+ * before its multiplication and discarded after).  T > 4 runs on the tensor
+ * cores (tcgen05; split-K partial sums are added with FP32 atomics, so the
+ * last bits may differ run to run); T <= 4 is a matrix-vector stream on the
+ * CUDA cores (bound by reading W; deterministic).
  *  x: DEVICE [T, in] BF16 (uint16 bits), row-major, 16-byte aligned
  *  w: DEVICE [out, in] BF16, row-major (nn.Linear layout; e.g. a view of a
  *     decoded block's scratch buffer), 16-byte aligned
