@@ -1,5 +1,6 @@
 // df11_decode.cu -- the DF11 decode kernel for sm_100a and its launchers
-// (df11_decode, df11_decode_block).
+// (df11_decode, df11_decode_block), and the row-gather kernel that decodes
+// only the thread blocks covering requested rows (df11_decode_rows).
 //
 // Sources: "DFloat11 : compression sans perte pour l'inference GPU qui reduit
 // les LLM a 70 % de leur taille" (fr.news.hada.io):
@@ -20,15 +21,18 @@
 //    group decodes one format block (256 format threads x 8 bytes) at a
 //    time and strides over the blocks.  The compact decode tables arrive by
 //    one TMA bulk copy (cp.async.bulk, no multicast); the count table is
-//    kept in two interleaved copies (lane l reads copy l mod 2).
+//    kept in two interleaved copies (lane l reads copy l mod 2), the symbol
+//    table in two or one (per instance).
 //  * Per group, bulk copies on mbarriers bring the next block's inputs
 //    (stream bytes, gaps, block starts) and the current block's whole
 //    sign/mantissa range into shared memory, so the merge reads nothing
 //    from global memory and no register holds prefetched data across the
 //    decode loops.
-//  * The exponent buffer holds 8192 symbols per group; tensors whose blocks
-//    hold more codes (average code under 2 bits) use a second instance with
-//    4 groups of 16 KB buffers.
+//  * The exponent buffer holds 6400 symbols per group when every block of
+//    the tensor fits (LLM-like weights: the room left gives the symbol table
+//    its second copy), else 8192; tensors whose blocks hold more codes
+//    (average code under 2 bits) use an instance with 4 groups of 16 KB
+//    buffers.
 //  * Every CUDA thread runs two format threads side by side (two
 //    independent decode chains in one loop): each lookup is a dependent
 //    shift -> index -> shared load chain, and two chains per thread hide
