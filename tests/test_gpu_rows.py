@@ -96,3 +96,25 @@ def test_lm_head_full_decode_and_gather():
     rows = rng.integers(0, 128256, 256).astype(np.int32)
     out = df11.decode_rows(d, 4096, torch.from_numpy(rows).to(dev))
     np.testing.assert_array_equal(_rows_bits(out), w[rows])
+
+
+@pytest.mark.parametrize("kind", ["dense", "wide"])
+def test_rows_other_instances(kind):
+    """Gather through the instances for blocks with more codes: 1-bit codes
+    (a two-valued matrix, up to 16384 codes per block) and a five-exponent
+    matrix (about 7500 codes per block)."""
+    dev = _dev()
+    rng = np.random.default_rng(17)
+    if kind == "dense":
+        e = rng.choice([100, 126], p=[0.2, 0.8], size=(4000, 96))
+    else:
+        e = rng.choice([120, 121, 122, 123, 124], p=[0.3, 0.3, 0.2, 0.1, 0.1], size=(4000, 96))
+    w = ((e << 7) | rng.integers(0, 128, e.shape) | (rng.integers(0, 2, e.shape) << 15)).astype(np.uint16)
+    t = df11.encode(w)
+    need = t.desc.max_block_codes + 15
+    assert (need > 8192) if kind == "dense" else (6400 < need <= 8192)
+    d = t.to(dev)
+    rows = torch.from_numpy(rng.integers(0, 4000, 300).astype(np.int32)).to(dev)
+    out = df11.decode_rows(d, 96, rows)
+    np.testing.assert_array_equal(_rows_bits(out), w[rows.cpu().numpy()])
+    np.testing.assert_array_equal(_rows_bits(df11.decode(d)).reshape(w.shape), w)
