@@ -238,8 +238,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 // With T <= 4 tokens every weight feeds at most 8 flops: the product is a
 // matrix-vector stream bound by reading W, and the tensor-core tiling (128
 // rows x 64 columns per load) reads W with poor DRAM locality.  This kernel
-// streams W along contiguous rows instead: a CTA of 8 warps takes R rows,
-// S = 8 / R warps share a row's K range, each lane loads 16 bytes (8 weights)
+// streams W along contiguous rows instead: a CTA of 8 warps takes R = 1 or
+// 2 rows, S = 8 / R warps share a row's K range, each lane loads 16 bytes (8 weights)
 // per step with several loads in flight, multiplies them by X (read through
 // the cache: X is small and shared by every CTA) in FP32, and the partial sums
 // are reduced by warp shuffles and then across the row's warps in shared
@@ -319,13 +319,12 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(const uint16_t *x, c
 template <int T>
 void launch_gemv(const uint16_t *x, const uint16_t *w, float *y, uint32_t out, uint32_t in, int sms,
                  cudaStream_t s) {
-    // rows per CTA: enough CTAs (about 6 per SM) for the loads in flight
-    uint32_t r = out / (6u * (uint32_t)sms);
-    r = r >= 8u ? 8u : r >= 4u ? 4u : r >= 2u ? 2u : 1u;
+    // rows per CTA: one when there are few rows (about 6 CTAs per SM), else
+    // two, so that at least four warps share a row's K range (measured:
+    // 4 or 8 rows per CTA, i.e. fewer warps per row, stream W more slowly)
+    const uint32_t r = out >= 12u * (uint32_t)sms ? 2u : 1u;
     const unsigned grid = out / r;
-    if (r == 8u) gemv_kernel<T, 8><<<grid, kGemvThreads, 0, s>>>(x, w, y, out, in);
-    else if (r == 4u) gemv_kernel<T, 4><<<grid, kGemvThreads, 0, s>>>(x, w, y, out, in);
-    else if (r == 2u) gemv_kernel<T, 2><<<grid, kGemvThreads, 0, s>>>(x, w, y, out, in);
+    if (r == 2u) gemv_kernel<T, 2><<<grid, kGemvThreads, 0, s>>>(x, w, y, out, in);
     else gemv_kernel<T, 1><<<grid, kGemvThreads, 0, s>>>(x, w, y, out, in);
 }
 
