@@ -690,10 +690,12 @@ __global__ void __launch_bounds__(C::kCtaThreads, 1) df11_decode_kernel(const De
         // last chunk; always at least 16 bytes).  Every thread of the group
         // has passed its previous merge, so the staging area is free.
         if (lt == 0) {
-            const uint32_t from = range_ok ? base + 16u * c_lo : 0u;
-            const uint32_t upto = range_ok ? ((e + 15u) & ~15u) : 16u;
-            const uint32_t bytes = upto > from ? min(C::kSmBytes, upto - from) : 16u;
-            const uint32_t src = upto > from ? from : (range_ok ? base : 0u);
+            // (64-bit: the end of the last chunk passes 2^32 when the tensor
+            // holds nearly 2^32 elements)
+            const uint64_t from = range_ok ? (uint64_t)base + 16u * c_lo : 0u;
+            const uint64_t upto = range_ok ? (((uint64_t)e + 15u) & ~15ull) : 16u;
+            const uint32_t bytes = upto > from ? (uint32_t)min((uint64_t)C::kSmBytes, upto - from) : 16u;
+            const uint64_t src = upto > from ? from : (range_ok ? base : 0u);
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             mbar_expect(mb_sm, bytes);
             bulk_g2s(grp + C::kGrpSm, a.sm + src, bytes, mb_sm);

@@ -219,3 +219,28 @@ def test_output_alignment_paths(offset_elems):
     np.testing.assert_array_equal(_bits(out), w.reshape(-1))
     rest = torch.cat([buf[:offset_elems], buf[offset_elems + w.size:]])
     assert bool((rest == -1).all())
+
+
+@pytest.mark.slow
+def test_maximum_size_tensor():
+    """The largest tensor the format holds: 2^32 - 1 elements (u32 block
+    output positions), 8.6 GB of BF16.  The weights repeat a 4096 x 4096
+    Gaussian matrix, so the histogram and code are those of the matrix; the
+    decoded tensor is compared with the input on 20 M sampled positions and
+    on its last 4 M elements, and the last block start must be right below
+    2^32."""
+    dev = _dev()
+    n = (1 << 32) - 1
+    base = workloads.normal_matrix(4096, 4096, 0.02, seed=2).reshape(-1)
+    w = np.tile(base, n // base.size + 1)[:n]
+    t = df11.encode(w)
+    bs = t.host_array("block_start")
+    assert int(bs[t.n_blocks]) == n and int(bs[t.n_blocks - 1]) > n - 20_000
+    d = t.to(dev)
+    del t
+    out = df11.decode(d)
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(6)
+    idx = np.concatenate([rng.integers(0, n, 20_000_000), np.arange(n - 4_000_000, n)])
+    got = out.view(torch.int16)[torch.from_numpy(idx).to(dev)].cpu().numpy().view(np.uint16)
+    np.testing.assert_array_equal(got, w[idx])
