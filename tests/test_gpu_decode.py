@@ -244,3 +244,14 @@ def test_maximum_size_tensor():
     idx = np.concatenate([rng.integers(0, n, 20_000_000), np.arange(n - 4_000_000, n)])
     got = out.view(torch.int16)[torch.from_numpy(idx).to(dev)].cpu().numpy().view(np.uint16)
     np.testing.assert_array_equal(got, w[idx])
+    del out
+    # row gather at the far end (65537 divides 2^32 - 1): rows 0, the middle and the last
+    rows = np.array([0, 32768, 65533, 65534], dtype=np.int32)
+    got = df11.decode_rows(d, 65537, torch.from_numpy(rows).to(dev))
+    np.testing.assert_array_equal(got.view(torch.int16).cpu().numpy().view(np.uint16),
+                                  w.reshape(65535, 65537)[rows])
+    # the device encoder on the same weights: arrays identical to the host encoder's
+    e = df11.encode_device(torch.from_numpy(w.view(np.int16)).to(dev).view(torch.bfloat16))
+    for k in ("enc", "sm", "gaps", "block_start", "lut"):
+        nb = d.nbytes(k)
+        assert e.nbytes(k) == nb and torch.equal(e.arrays[k][:nb], d.arrays[k][:nb]), k
