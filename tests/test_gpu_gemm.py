@@ -112,3 +112,19 @@ def test_config5_decode_then_gemm_full_blocks():
                 cols = rng_cols.choice(w.shape[0], 512, replace=False)
                 ref = (xs[inn].double() @ _bf16(w[cols]).double().T).numpy()
                 assert _rel_fro(y[:, cols], ref) <= TOL, (seed, T, name)
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("T", [1, 16])
+def test_gemm_lm_head_shape(T):
+    """The LM-head shape (128256 x 4096): the widest grid of either path
+    (64128 GEMV CTAs at T = 1; 1002 row tiles on tcgen05 at T = 16).  1024
+    sampled output columns against an FP64 CPU GEMM."""
+    dev = _dev()
+    g = torch.Generator(device=dev).manual_seed(40 + T)
+    w = (torch.randn(128256, 4096, device=dev, generator=g) * 0.02).to(torch.bfloat16)
+    x = torch.randn(T, 4096, device=dev, generator=g).to(torch.bfloat16)
+    y = df11.gemm(x, w)
+    cols = torch.from_numpy(np.random.default_rng(T).choice(128256, 1024, replace=False)).to(dev)
+    ref = (x.double() @ w[cols].double().T).cpu().numpy()
+    assert _rel_fro(y[:, cols].double().cpu().numpy(), ref) <= TOL
