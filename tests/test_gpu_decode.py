@@ -255,3 +255,29 @@ def test_maximum_size_tensor():
     for k in ("enc", "sm", "gaps", "block_start", "lut"):
         nb = d.nbytes(k)
         assert e.nbytes(k) == nb and torch.equal(e.arrays[k][:nb], d.arrays[k][:nb]), k
+
+
+def test_two_streams_at_once():
+    """Two decodes in flight on two streams (no shared device state): both
+    bit-exact."""
+    dev = _dev()
+    w1 = workloads.normal_matrix(3000, 1024, 0.02, seed=21)
+    rng = np.random.default_rng(22)
+    x = (rng.standard_t(3, (2000, 1024)) * 0.015).astype(np.float32)
+    x[rng.random(x.shape) < 0.001] *= 1000.0
+    w2 = workloads.round_to_bf16(x)  # heavy tail: long codes
+    d1 = df11.encode(w1).to(dev)
+    d2 = df11.encode(w2, df11.Params(max_code_len=32)).to(dev)
+    s1, s2 = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+    o1 = torch.empty(w1.size, dtype=torch.bfloat16, device=dev)
+    o2 = torch.empty(w2.size, dtype=torch.bfloat16, device=dev)
+    e1 = torch.zeros(1, dtype=torch.int32, device=dev)
+    e2 = torch.zeros(1, dtype=torch.int32, device=dev)
+    torch.cuda.synchronize()
+    for _ in range(4):
+        df11.decode(d1, o1, e1, stream=s1)
+        df11.decode(d2, o2, e2, stream=s2)
+    torch.cuda.synchronize()
+    assert df11.read_error(e1, s1) == 0 and df11.read_error(e2, s2) == 0
+    np.testing.assert_array_equal(_bits(o1), w1.reshape(-1))
+    np.testing.assert_array_equal(_bits(o2), w2.reshape(-1))

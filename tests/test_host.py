@@ -278,3 +278,25 @@ def test_save_load_round_trip(tmp_path):
         f.write(b"\0" * 16)
     with pytest.raises(Exception):
         df11.load(path)
+
+
+def test_concurrent_host_encodes_match_sequential():
+    """Encodes from several host threads at once (the library keeps no shared
+    mutable state) give the same arrays as one after another."""
+    import threading
+    mats = [workloads.normal_matrix(300 + 37 * i, 211, 0.02 + 0.005 * i, seed=50 + i) for i in range(4)]
+    seq = [df11.encode(m) for m in mats]
+    got = [None] * len(mats)
+
+    def run(i):
+        got[i] = df11.encode(mats[i])
+
+    threads = [threading.Thread(target=run, args=(i,)) for i in range(len(mats))]
+    for th in threads:
+        th.start()
+    for th in threads:
+        th.join()
+    for a, b in zip(seq, got):
+        assert a.total_bits == b.total_bits and a.n_blocks == b.n_blocks
+        for k in ("enc", "sm", "gaps", "block_start", "lut"):
+            np.testing.assert_array_equal(a.host_array(k)[: a.nbytes(k)], b.host_array(k)[: b.nbytes(k)])
