@@ -52,6 +52,9 @@ WORKLOADS = {
     "decode-gemm": ("32 llama3.1-8b blocks (seeds 32*rank + 0..31), each decoded into one reused BF16 scratch, "
                     "then every matrix multiplied by N(0,1) BF16 activations [T, in], T in {1,16,64,256} "
                     "(seed 1000 + T), FP32-accumulate GEMM on tcgen05", None),
+    "decode-gemv": ("llama3.1-8b transformer block (218,112,000 BF16 weights, seed = rank), all seven matrices "
+                    "multiplied by N(0,1) BF16 activations [T, in] (seed 1000 + T) in ONE fused decode -> "
+                    "matrix-vector launch (weights never written to memory); T from --T (1..4)", None),
     "encode-device": ("llama3.1-8b transformer block (218,112,000 BF16 weights, seed = rank) already in device memory, "
                       "encoded on the GPU (histogram + packing; code lengths on the host)", None),
     "offload": ("llama3.1-8b blocks (seeds 0..B-1, default 4) kept in pinned host memory and streamed over PCIe "
@@ -121,6 +124,16 @@ class ClockSampler:
         return {"sm_mhz": statistics.median(sm) if sm else None,
                 "sm_max_mhz": max(mx) if mx else None,
                 "reasons": reasons, "samples": len(rows)}
+
+
+def _bus_id(dev) -> str | None:
+    """PCI bus id of a torch CUDA device in nvidia-smi's form."""
+    try:
+        import torch
+        p = torch.cuda.get_device_properties(dev)
+        return f"{p.pci_domain_id:08x}:{p.pci_bus_id:02x}:{p.pci_device_id:02x}.0"
+    except Exception:
+        return None
 
 
 def rank_seed(rank: int) -> int:
@@ -280,7 +293,7 @@ def run_decode_gemm(args, rank: int, world: int):
     per_T = {}
     nb = len(blocks)
     w_bytes = sum(int(w.numel()) * 2 for w in gemm_mats)
-    for T in (1, 16, 64, 256):
+    for T in (1, 4, 16, 64, 256):
         g = torch.Generator().manual_seed(1000 + T)
         xs = {k: torch.randn(T, k, generator=g).to(torch.bfloat16).to(dev) for k in {w.shape[1] for w in gemm_mats}}
         ys = [torch.empty(T, w.shape[0], dtype=torch.float32, device=dev) for w in gemm_mats]
@@ -317,6 +330,34 @@ def run_decode_gemm(args, rank: int, world: int):
         per_T[str(T)] = {"decode_us": t_dec * 1e3, "gemm_us": t_gemm * 1e3, "total_us": t_both * 1e3,
                          "bf16_gemm_us": t_bf16 * 1e3, "slowdown_vs_bf16": t_both / t_bf16,
                          "gemm_gbs": (w_bytes + x_bytes) / (t_gemm * 1e-3) / 1e9, "gemm_rel_fro": rel}
+        if T <= 4:
+            # fused decode -> matrix-vector products: per block, one zeroing of
+            # the seven outputs and one launch for all seven matrices; the
+            # decoded weights never reach memory
+            rows_tot = sum(int(w.shape[0]) for w in gemm_mats)
+            ybuf = torch.empty(T * rows_tot, dtype=torch.float32, device=dev)
+            xs_f, ys_f, off = {}, {}, 0
+            for j, w in enumerate(gemm_mats):
+                xs_f[j] = xs[w.shape[1]]
+                ys_f[j] = ybuf[off: off + T * w.shape[0]].view(T, w.shape[0])
+                off += T * w.shape[0]
+            ybuf.zero_()
+            df11.decode_gemv(blocks[-1][0], xs_f, ys_f, err, stream)  # the block the scratch holds
+            frel = 0.0
+            for j, w in enumerate(gemm_mats):
+                cols = torch.arange(0, w.shape[0], max(1, w.shape[0] // 256), device=dev)
+                ref = xs[w.shape[1]].double() @ w[cols].double().T
+                frel = max(frel, float((ys_f[j][:, cols].double() - ref).norm() / ref.norm()))
+
+            def fused_all():
+                for d, _ in blocks:
+                    ybuf.zero_()
+                    df11.decode_gemv(d, xs_f, ys_f, err, stream)
+
+            t_fused = timed(fused_all, args.steps) / nb
+            per_T[str(T)].update({"fused_us": t_fused * 1e3, "fused_vs_bf16": t_fused / t_bf16,
+                                  "fused_speedup_vs_unfused": t_both / t_fused, "fused_rel_fro": frel,
+                                  "fused_launches_per_block": 2})
     assert df11.read_error(err, stream) == 0
     if rank == 0:
         desc = WORKLOADS["decode-gemm"][0]
@@ -327,6 +368,7 @@ def run_decode_gemm(args, rank: int, world: int):
                            "value_is": "total per block at T=1",
                            "l2": "436 MB scratch and 300 MB compressed per block, larger than L2; no flush"},
                 "checksums_ok": ok, "per_T": per_T, "host_encode_s": round(encode_s, 1),
+                "fused_us_T1": per_T["1"].get("fused_us"),
                 "gpu_launches_per_block": 8}
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -424,6 +466,112 @@ def run_offload(args, rank: int, world: int):
         dist.destroy_process_group()
 
 
+def run_decode_gemv(args, rank: int, world: int):
+    """Fused decode -> matrix-vector products on one block: per step the seven
+    outputs are zeroed and one launch decodes the block and multiplies every
+    matrix by its activations.  Timed next to the unfused path (block decode
+    into the scratch, then the seven T <= 4 GEMMs)."""
+    import torch
+    import torch.distributed as dist
+
+    import huffman_decode_02_b200 as df11
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=dev)
+    T = args.T
+    mats = workloads.llama8b_block(seed=rank_seed(rank))
+    blk = df11.encode_multi(mats, df11.Params(max_code_len=args.max_code_len))
+    d = blk.to(dev)
+    idx = [j for j, m in enumerate(mats) if m.ndim == 2]
+    g = torch.Generator().manual_seed(1000 + T)
+    xs_in = {k: torch.randn(T, k, generator=g).to(torch.bfloat16) for k in sorted({mats[j].shape[1] for j in idx})}
+    xs = {j: xs_in[mats[j].shape[1]].to(dev) for j in idx}
+    rows_tot = sum(mats[j].shape[0] for j in idx)
+    ybuf = torch.zeros(T * rows_tot, dtype=torch.float32, device=dev)
+    ys, off = {}, 0
+    for j in idx:
+        ys[j] = ybuf[off: off + T * mats[j].shape[0]].view(T, mats[j].shape[0])
+        off += T * mats[j].shape[0]
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def fused():
+        ybuf.zero_()
+        df11.decode_gemv(d, xs, ys, err, stream)
+
+    # numerics: 256 sampled rows of every matrix against FP64
+    fused()
+    rng = np.random.default_rng(11)
+    rel = 0.0
+    for j in idx:
+        r = np.sort(rng.choice(mats[j].shape[0], 256, replace=False))
+        w = torch.from_numpy(mats[j][r].view(np.int16)).view(torch.bfloat16).double()
+        ref = xs_in[mats[j].shape[1]].double() @ w.T
+        got = ys[j].cpu().double()[:, r]
+        rel = max(rel, float((got - ref).norm() / ref.norm()))
+    assert df11.read_error(err, stream) == 0
+    scratch = torch.empty(d.n_elems, dtype=torch.bfloat16, device=dev)
+    views = d.views(scratch)
+    yu = {j: torch.empty(T, mats[j].shape[0], dtype=torch.float32, device=dev) for j in idx}
+
+    def unfused():
+        df11.decode_block(d, scratch, err, stream)
+        for j in idx:
+            df11.gemm(xs[j], views[j], yu[j], err, stream)
+
+    ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+
+    def timed(fn, steps):
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+        a, b = ev(), ev()
+        a.record(stream)
+        for _ in range(steps):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        ms = a.elapsed_time(b) / steps
+        return max_over_ranks(ms, dist, dev) if world > 1 else ms
+
+    sampler = ClockSampler(_bus_id(dev))
+    sampler.start()
+    time.sleep(0.25)  # let nvidia-smi start sampling before the timed region
+    ms_fused = timed(fused, args.steps)
+    clocks = sampler.stop()
+    ms_unfused = timed(unfused, max(1, args.steps // 4))
+    assert df11.read_error(err, stream) == 0
+    if rank == 0:
+        peak, peak_kind = _peaks()
+        comp = sum(d.nbytes(k) for k in ("enc", "sm", "gaps", "block_start", "lut"))
+        io = sum(T * mats[j].shape[1] * 2 + T * mats[j].shape[0] * 4 for j in idx)
+        alg = comp + io
+        achieved = alg / (ms_fused * 1e-3) / 1e9
+        line = {"metric": "fused decode -> matrix-vector time per llama3.1-8b block", "value": ms_fused * 1e3,
+                "unit": "us", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": ms_fused, "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
+                "dtype": "bf16 x bf16 -> f32 (decode u32)", "data": "synthetic",
+                "config": {"workload": WORKLOADS["decode-gemv"][0], "T": T, "n_elems_per_rank": d.n_elems,
+                           "l2": f"inputs larger than L2 ({comp / 1e6:.0f} MB compressed per step), no flush",
+                           "timing": "K steps (zeroing of y + one fused launch) between CUDA events"},
+                "rel_fro_sampled_rows": rel,
+                "unfused_us": ms_unfused * 1e3, "speedup_vs_unfused": ms_unfused / ms_fused,
+                "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                             "frac": achieved / peak, "traffic": None,
+                             "peak_kind": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs, copy burst)",
+                             "algorithmic_bytes_per_launch": alg},
+                "gpu_launches": args.steps, "clocks": clocks}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
 def run_encode_device(args, rank: int, world: int):
     """The device encoder on a block already in device memory: wall time per
     encode (size pass with its host round trip for the histogram, then the
@@ -490,6 +638,7 @@ def main():
     ap.add_argument("--max-code-len", type=int, default=12, help="length cap of the exponent code")
     ap.add_argument("--blocks", type=int, default=None, help="blocks of the decode-gemm (32) / offload (4) workloads")
     ap.add_argument("--repeat", type=int, default=4, help="passes over the blocks in the offload workload")
+    ap.add_argument("--T", type=int, default=1, help="batch of the decode-gemv workload (1..4)")
     args = ap.parse_args()
     args.blocks_given = args.blocks is not None
     if args.blocks is None:
@@ -507,6 +656,9 @@ def main():
         return
     if args.workload == "offload":
         run_offload(args, rank, world)
+        return
+    if args.workload == "decode-gemv":
+        run_decode_gemv(args, rank, world)
         return
     if args.workload == "encode-device":
         run_encode_device(args, rank, world)
@@ -544,13 +696,7 @@ def main():
         df11.decode_block(d, scratch, err, stream)
     torch.cuda.synchronize(dev)
 
-    bus = None
-    try:
-        p = torch.cuda.get_device_properties(dev)
-        bus = f"{p.pci_domain_id:08x}:{p.pci_bus_id:02x}:{p.pci_device_id:02x}.0"
-    except Exception:
-        pass
-    sampler = ClockSampler(bus)
+    sampler = ClockSampler(_bus_id(dev))
     sampler.start()
     time.sleep(0.25)  # let nvidia-smi start sampling before the timed region
     if world > 1:

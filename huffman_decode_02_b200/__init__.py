@@ -30,7 +30,7 @@ from . import build as _build
 
 __all__ = [
     "DF11Error", "CorruptStreamError", "Params", "DF11Tensor", "encode", "encode_multi",
-    "encode_device", "encode_device_noalloc", "save", "load", "decode", "decode_block", "decode_rows", "gemm", "read_error", "exponent_histogram", "lib_path", "sm_count",
+    "encode_device", "encode_device_noalloc", "save", "load", "decode", "decode_block", "decode_rows", "decode_gemv", "gemm", "read_error", "exponent_histogram", "lib_path", "sm_count",
     "KERR_COUNT_MISMATCH", "KERR_BAD_CODE", "KERR_BAD_BLOCK", "KERR_OVERRUN", "KERR_TIMEOUT", "KERR_BAD_ROW",
 ]
 
@@ -73,6 +73,11 @@ class _Tensor(ctypes.Structure):
                 ("block_start", ctypes.c_void_p), ("lut", ctypes.c_void_p)]
 
 
+class _GemvMat(ctypes.Structure):
+    _fields_ = [("elem_offset", ctypes.c_uint64), ("rows", ctypes.c_uint32), ("cols", ctypes.c_uint32),
+                ("x", ctypes.c_void_p), ("y", ctypes.c_void_p)]
+
+
 _ARRAYS = ("enc", "sm", "gaps", "block_start", "lut")
 _LIB = None
 
@@ -108,6 +113,7 @@ def _lib():
     lib.df11_device_sm_count.argtypes = [P(ctypes.c_int)]
     lib.df11_gemm_bf16.argtypes = [vp, vp, vp, u32, u32, u32, vp, vp]
     lib.df11_decode_rows.argtypes = [P(_Tensor), ctypes.c_uint64, vp, u32, vp, vp, vp]
+    lib.df11_decode_gemv.argtypes = [P(_Tensor), P(_GemvMat), u32, u32, vp, vp]
     lib.df11_encode_device_scratch_bytes.argtypes = [u64]
     lib.df11_encode_device_scratch_bytes.restype = u64
     lib.df11_encode_device_size.argtypes = [vp, u64, P(_Params), P(T), vp, u64, vp]
@@ -500,6 +506,50 @@ def decode_rows(t: DF11Tensor, row_len: int, rows, out=None, err=None, stream=No
     if own_err:
         read_error(err, stream)
     return out
+
+
+def decode_gemv(t: DF11Tensor, xs: dict, ys: dict | None = None, err=None, stream=None) -> dict:
+    """Fused decode and matrix-vector products for batches T <= 4 (one
+    launch): for each matrix index j in ``xs`` (indices into ``t.shapes``; a
+    2-D [out, in] matrix), y_j = x_j @ W_j^T with W_j decoded on the fly and
+    never written to memory.  ``xs[j]``: [T, in] bfloat16 CUDA tensors, one
+    T for all.  ``ys[j]`` ([T, out] float32), when given, are added into;
+    otherwise zero-filled outputs are allocated.  Returns {j: y_j}."""
+    import torch
+    _check_device(t)
+    if not xs:
+        return {}
+    order = sorted(xs)
+    T = None
+    if ys is None:
+        ys = {}
+    mats = (_GemvMat * len(order))()
+    for i, j in enumerate(order):
+        shape = t.shapes[j]
+        if len(shape) != 2:
+            raise ValueError(f"matrix {j} is not 2-D")
+        rows, cols = int(shape[0]), int(shape[1])
+        x = xs[j]
+        if x.dtype != torch.bfloat16 or x.dim() != 2 or x.shape[1] != cols or not x.is_contiguous():
+            raise TypeError(f"x for matrix {j} must be a contiguous [T, {cols}] bfloat16 tensor")
+        if T is None:
+            T = int(x.shape[0])
+        elif int(x.shape[0]) != T:
+            raise ValueError("every x must have the same batch T")
+        if j not in ys:
+            ys[j] = torch.zeros(T, rows, dtype=torch.float32, device=t.device)
+        y = ys[j]
+        if y.dtype != torch.float32 or tuple(y.shape) != (T, rows) or not y.is_contiguous():
+            raise TypeError(f"y for matrix {j} must be a contiguous [{T}, {rows}] float32 tensor")
+        mats[i] = _GemvMat(int(t.offsets[j]), rows, cols, x.data_ptr(), y.data_ptr())
+    own_err = err is None
+    if own_err:
+        err = _new_err(t.device)
+    _check(_lib().df11_decode_gemv(ctypes.byref(t._bind()), mats, len(order), T, ctypes.c_void_p(err.data_ptr()),
+                                   _stream_handle(stream)), "decode_gemv")
+    if own_err:
+        read_error(err, stream)
+    return {j: ys[j] for j in order}
 
 
 def gemm(x, w, out=None, err=None, stream=None):

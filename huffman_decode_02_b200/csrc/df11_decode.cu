@@ -590,10 +590,34 @@ __device__ __forceinline__ bool load_tables(const uint8_t *lut, uint32_t *err_ou
     return true;
 }
 
+// Where a decoded block goes: StoreSink writes it as BF16 (the decoder);
+// the fused matrix-vector product below multiplies it into y instead.  A
+// sink takes the whole chunks of a block (`chunks`, every thread of the
+// group) and its two edge chunks (`edges`, warp 0), and clears every buffer
+// chunk it reads.
+struct StoreSink {
+    uint16_t *out;
+    const uint8_t *sm;
+    uint64_t n_elems;
+    uint32_t al32;
+    template <uint32_t kBufBytes>
+    __device__ __forceinline__ void chunks(uint32_t sb, uint32_t base, uint32_t c_first, uint32_t c_end,
+                                           uint32_t sm_s, uint32_t c_lo) {
+        merge_chunks<kBufBytes>(out, sb, base, c_first, c_end, sm_s, c_lo, al32, n_elems);
+    }
+    __device__ __forceinline__ void edges(uint32_t sb, uint32_t base, uint32_t c_full, uint32_t span, uint32_t s,
+                                          uint32_t e, uint32_t lane) {
+        merge_edges_clear(sm, out, sb, base, c_full, span, s, e, lane);
+    }
+};
+
+// The persistent decode loop of one CTA: loads the tables, then each group
+// decodes format blocks blk_first + (CTA * groups + group) + k * stride,
+// below blk_end, and hands every decoded block to the sink.
 // kLong: compiled with the long-code path (codes longer than the table
 // windows); without it the loops carry no escape handling at all.
-template <class C, bool kLong>
-__global__ void __launch_bounds__(C::kCtaThreads, 1) df11_decode_kernel(const DecodeArgs a) {
+template <class C, bool kLong, class Sink>
+__device__ __forceinline__ void decode_blocks(const DecodeArgs &a, Sink &sink, uint64_t blk_first, uint64_t blk_end) {
     extern __shared__ __align__(128) uint8_t smem[];
     const uint32_t s_base = smem_addr(smem);
     const uint32_t s_lim = s_base + kOffLim;
@@ -614,7 +638,7 @@ __global__ void __launch_bounds__(C::kCtaThreads, 1) df11_decode_kernel(const De
     uint32_t my_err = 0;
 
     const uint64_t stride = (uint64_t)gridDim.x * C::kGroups;
-    uint64_t blk = (uint64_t)blockIdx.x * C::kGroups + group;
+    uint64_t blk = blk_first + (uint64_t)blockIdx.x * C::kGroups + group;
 
     if (!load_tables<C>(a.lut, a.err, smem, s_base, tid)) return;
     const LutHeader *hdr = reinterpret_cast<const LutHeader *>(smem + kOffHeader);
@@ -630,12 +654,12 @@ __global__ void __launch_bounds__(C::kCtaThreads, 1) df11_decode_kernel(const De
         mbar_init(mb_in);
         mbar_init(mb_sm);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-        if (blk < a.n_blocks) issue_inputs<C>(a, blk, grp, mb_in);
+        if (blk < blk_end) issue_inputs<C>(a, blk, grp, mb_in);
     }
     group_barrier(group);
     uint32_t ph_in = 0, ph_sm = 0;
 
-    for (; blk < a.n_blocks; blk += stride) {
+    for (; blk < blk_end; blk += stride) {
         if (!wait_phase(mb_in, ph_in)) my_err |= kKernErrTimeout;
         ph_in ^= 1u;
         const uint64_t tA = blk * (uint64_t)kThreadsPerBlockFmt + 2u * lt;
@@ -685,7 +709,7 @@ __global__ void __launch_bounds__(C::kCtaThreads, 1) df11_decode_kernel(const De
         group_barrier(group);
         // every thread has read this block's staged inputs: fetch the next
         const uint64_t nxt = blk + stride;
-        if (lt == 0 && nxt < a.n_blocks) issue_inputs<C>(a, nxt, grp, mb_in);
+        if (lt == 0 && nxt < blk_end) issue_inputs<C>(a, nxt, grp, mb_in);
         // and this block's sign/mantissa bytes (chunks c_lo .. the block's
         // last chunk; always at least 16 bytes).  Every thread of the group
         // has passed its previous merge, so the staging area is free.
@@ -724,14 +748,20 @@ __global__ void __launch_bounds__(C::kCtaThreads, 1) df11_decode_kernel(const De
         if (!wait_phase(mb_sm, ph_sm)) my_err |= kKernErrTimeout;
         ph_sm ^= 1u;
         if (ok) {
-            merge_chunks<C::kSbufBytes>(a.out, sb, base, c0, c_full, grp + C::kGrpSm, c_lo, a.out_al32, a.n_elems);
-            if (warp == 0) merge_edges_clear(a.sm, a.out, sb, base, c_full, span, s, e, lane);
+            sink.template chunks<C::kSbufBytes>(sb, base, c0, c_full, grp + C::kGrpSm, c_lo);
+            if (warp == 0) sink.edges(sb, base, c_full, span, s, e, lane);
         }
         // No barrier here: the next block's buffer writes and staging copies
         // come after its scan barrier, which every thread reaches only after
         // this merge.
     }
     if (my_err && a.err) atomicOr(a.err, my_err);
+}
+
+template <class C, bool kLong>
+__global__ void __launch_bounds__(C::kCtaThreads, 1) df11_decode_kernel(const DecodeArgs a) {
+    StoreSink sink{a.out, a.sm, a.n_elems, a.out_al32};
+    decode_blocks<C, kLong>(a, sink, 0u, a.n_blocks);
 }
 
 
@@ -900,17 +930,315 @@ __global__ void __launch_bounds__(C::kCtaThreads, 1) df11_gather_kernel(const Ga
     if (my_err && a.err) atomicOr(a.err, my_err);
 }
 
+// ------------------------------------------------- fused decode -> matrix-vector
+// Decompressing a matrix right before its multiplication ("Decompression
+// adaptee a l'inference GPU") taken to the end for small batches: the merge
+// multiplies each decoded chunk by the activations instead of storing it, so
+// the BF16 weights never reach global memory.  For T <= 4 the product is a
+// matrix-vector stream (at most 8 flops per weight), which fits in the merge
+// on the CUDA cores.  Each listed matrix j of the tensor gets
+// y_j[t][r] += sum_c W_j[r][c] * x_j[t][c] (FP32; each warp reduces its
+// partial sums per row and adds them with FP32 atomics).
+constexpr uint32_t kMaxGemvMats = 16;
+constexpr uint32_t kNoRow = 0xFFFFFFFFu;
+
+struct GemvMat {
+    uint32_t off, end;      // elements [off, end) of the tensor; both multiples of 16
+    uint32_t rows, cols;    // cols a multiple of 16
+    uint32_t magic, shift;  // chunk q = (g - off) / 16 (< 2^28) lies in row (q * magic) >> shift
+    const uint16_t *x;      // [T][cols] BF16
+    float *y;               // [T][rows] FP32, accumulated into
+};
+
+struct GemvArgs {
+    DecodeArgs d;
+    GemvMat m[kMaxGemvMats];  // ordered by offset, not overlapping
+    uint32_t n_mats, T;
+    uint32_t e_first, e_last;  // first and last element of the matrices
+};
+
+// lo += w.lo * x.lo and hi += w.hi * x.hi for two BF16 pairs, with FP32
+// accumulators (mixed-precision FMA: the product is exact, one rounding).
+__device__ __forceinline__ void fma2_bf16(float &lo, float &hi, uint32_t w, uint32_t x) {
+    asm("{\n\t.reg .b16 wl, wh, xl, xh;\n\t"
+        "mov.b32 {wl, wh}, %2;\n\t"
+        "mov.b32 {xl, xh}, %3;\n\t"
+        "fma.rn.f32.bf16 %0, wl, xl, %0;\n\t"
+        "fma.rn.f32.bf16 %1, wh, xh, %1;\n\t}"
+        : "+f"(lo), "+f"(hi)
+        : "r"(w), "r"(x));
+}
+
+// Accumulates 16 BF16 weights (8 words, element order) times 16 BF16
+// activations into (lo, hi).
+__device__ __forceinline__ void dot16(const uint32_t w[8], const uint4 xa, const uint4 xb, float &lo, float &hi) {
+    const uint32_t X[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
+#pragma unroll
+    for (int i = 0; i < 8; ++i) fma2_bf16(lo, hi, w[i], X[i]);
+}
+
+__device__ __forceinline__ uint32_t gemv_row(uint32_t local, uint32_t magic, uint32_t shift) {
+    return (uint32_t)(((uint64_t)(local >> 4) * magic) >> shift);
+}
+
+// Adds a warp's per-lane sums into y: one atomic per run of lanes holding the
+// same key.  Equal keys must sit in contiguous lanes (the callers' element
+// order guarantees it); a lane with key kNoRow holds nothing.  Whole warp,
+// converged.  key0 / yrow: the key and output row of each lane.
+template <uint32_t TM>
+__device__ __forceinline__ void flush_runs(const float (&lo)[TM], const float (&hi)[TM], uint32_t key,
+                                           float *const yrow, uint32_t rows, uint32_t T, uint32_t lane) {
+    const uint32_t k0 = __shfl_sync(kFull, key, 0);
+    if (__all_sync(kFull, key == k0)) {  // the common case: one run
+        if (k0 == kNoRow) return;
+#pragma unroll
+        for (uint32_t t = 0; t < TM; ++t) {
+            float v = lo[t] + hi[t];
+#pragma unroll
+            for (uint32_t d = 16; d >= 1; d >>= 1) v += __shfl_xor_sync(kFull, v, d);
+            if (lane == 0 && t < T) atomicAdd(yrow + (uint64_t)t * rows, v);
+        }
+        return;
+    }
+    // suffix sums inside each run, then the run's first lane adds
+    uint32_t same = 0;  // bit k: lane + 2^k holds the same key
+#pragma unroll
+    for (uint32_t k = 0; k < 5; ++k) {
+        const uint32_t o = __shfl_down_sync(kFull, key, 1u << k);
+        if (lane + (1u << k) < 32u && o == key) same |= 1u << k;
+    }
+    const uint32_t prev = __shfl_up_sync(kFull, key, 1);
+    const bool first = (lane == 0 || prev != key) && key != kNoRow;
+#pragma unroll
+    for (uint32_t t = 0; t < TM; ++t) {
+        float v = lo[t] + hi[t];
+#pragma unroll
+        for (uint32_t k = 0; k < 5; ++k) {
+            const float o = __shfl_down_sync(kFull, v, 1u << k);
+            if (same & (1u << k)) v += o;
+        }
+        if (first && t < T) atomicAdd(yrow + (uint64_t)t * rows, v);
+    }
+}
+
+// The fused sink: decoded chunks are multiplied into y instead of stored.
+// Each warp takes a contiguous quarter of the block's whole chunks (lane l
+// the chunk at l + 32 i), so its successive 512-weight pieces mostly stay in
+// one row: lanes accumulate until some lane's row changes, then the warp
+// adds its sums into y.  `m` is the first matrix that can still hold the
+// warp's elements (they only grow: chunks within a block, then blocks by
+// stride).
+template <uint32_t TM>
+struct GemvSink {
+    const GemvArgs &g;
+    uint32_t m;
+
+    template <uint32_t kBufBytes>
+    __device__ __forceinline__ void chunks(uint32_t sb, uint32_t base, uint32_t /*c_first*/, uint32_t c_end,
+                                           uint32_t sm_s, uint32_t c_lo) {
+        const uint32_t lane = threadIdx.x & 31u, warp = (threadIdx.x >> 5) % (kGroupThreads / 32u);
+        const uint32_t n = c_end > c_lo ? c_end - c_lo : 0u;
+        const uint32_t per = ((n + 3u) / 4u + 31u) & ~31u;  // whole warp iterations
+        const uint32_t w_lo = c_lo + min(n, warp * per), w_hi = c_lo + min(n, (warp + 1u) * per);
+        if (w_lo >= w_hi) return;  // warp-uniform
+        const uint32_t g_lo = base + 16u * w_lo, g_hi = base + 16u * w_hi;
+        while (m < g.n_mats && g_lo >= g.m[m].end) ++m;
+        if (m < g.n_mats && g_lo >= g.m[m].off && g_hi <= g.m[m].end)
+            one_matrix<kBufBytes>(sb, base, w_lo, w_hi, sm_s, c_lo, lane);
+        else
+            any_matrices<kBufBytes>(sb, base, w_lo, w_hi, sm_s, c_lo, lane);
+    }
+
+    // All of the warp's chunks lie in matrix m (the common case).
+    template <uint32_t kBufBytes>
+    __device__ __forceinline__ void one_matrix(uint32_t sb, uint32_t base, uint32_t w_lo, uint32_t w_hi,
+                                               uint32_t sm_s, uint32_t c_lo, uint32_t lane) {
+        const GemvMat &M = g.m[m];
+        const uint32_t off = M.off, cols = M.cols, magic = M.magic, shift = M.shift, rows = M.rows, T = g.T;
+        const uint16_t *const x = M.x;
+        float lo[TM], hi[TM];
+#pragma unroll
+        for (uint32_t t = 0; t < TM; ++t) lo[t] = hi[t] = 0.f;
+        uint32_t held = kNoRow;  // row of the sums this lane holds
+        for (uint32_t cw = w_lo; cw < w_hi; cw += 32u) {  // warp-uniform trip count
+            const uint32_t c = cw + lane;
+            const bool act = c < w_hi && DF11_BOUNDS_OK(16u * (c + 1u) <= kBufBytes &&
+                                                        (uint64_t)base + 16ull * (c + 1u) <= g.d.n_elems &&
+                                                        c >= c_lo && 16u * (c - c_lo + 1u) <= kBufBytes);
+            uint4 smv, ex;
+            uint32_t local = 0, row = kNoRow;
+            if (act) {
+                smv = lds_u4(sm_s + 16u * (c - c_lo));
+                ex = lds_u4(sb + 16u * c);
+                sts_zero16(sb + 16u * c);
+                local = base + 16u * c - off;
+                row = gemv_row(local, magic, shift);
+            }
+            // Rows grow with the lane within a step and from step to step, and
+            // a lane that is idle once stays idle: so after this flush rule the
+            // lanes holding one row are always contiguous.
+            if (__any_sync(kFull, act && held != kNoRow && row != held)) {
+                flush_runs<TM>(lo, hi, held, M.y + (held == kNoRow ? 0u : held), rows, T, lane);
+#pragma unroll
+                for (uint32_t t = 0; t < TM; ++t) lo[t] = hi[t] = 0.f;
+                held = kNoRow;
+            }
+            if (act) {
+                uint32_t w[8];
+                merge16(smv, ex, w);
+                const uint16_t *xp = x + (local - row * cols);
+#pragma unroll
+                for (uint32_t t = 0; t < TM; ++t) {
+                    if (t < T) {
+                        const uint4 *xv = reinterpret_cast<const uint4 *>(xp + (uint64_t)t * cols);
+                        dot16(w, __ldg(xv), __ldg(xv + 1), lo[t], hi[t]);
+                    }
+                }
+                held = row;
+            }
+        }
+        flush_runs<TM>(lo, hi, held, M.y + (held == kNoRow ? 0u : held), rows, T, lane);
+    }
+
+    // The warp's chunks meet a matrix boundary or elements of no matrix:
+    // each chunk finds its matrix, and the warp adds its sums every step.
+    template <uint32_t kBufBytes>
+    __device__ __forceinline__ void any_matrices(uint32_t sb, uint32_t base, uint32_t w_lo, uint32_t w_hi,
+                                                 uint32_t sm_s, uint32_t c_lo, uint32_t lane) {
+        uint32_t mm = m;
+        for (uint32_t cw = w_lo; cw < w_hi; cw += 32u) {  // warp-uniform trip count
+            const uint32_t c = cw + lane;
+            float lo[TM], hi[TM];
+#pragma unroll
+            for (uint32_t t = 0; t < TM; ++t) lo[t] = hi[t] = 0.f;
+            uint32_t key = kNoRow, rows = 0;
+            float *yrow = nullptr;
+            if (c < w_hi && DF11_BOUNDS_OK(16u * (c + 1u) <= kBufBytes &&
+                                           (uint64_t)base + 16ull * (c + 1u) <= g.d.n_elems && c >= c_lo &&
+                                           16u * (c - c_lo + 1u) <= kBufBytes)) {
+                const uint4 smv = lds_u4(sm_s + 16u * (c - c_lo));
+                const uint4 ex = lds_u4(sb + 16u * c);
+                sts_zero16(sb + 16u * c);
+                const uint32_t g0 = base + 16u * c;
+                while (mm < g.n_mats && g0 >= g.m[mm].end) ++mm;
+                if (mm < g.n_mats && g0 >= g.m[mm].off) {
+                    const GemvMat &M = g.m[mm];
+                    uint32_t w[8];
+                    merge16(smv, ex, w);
+                    const uint32_t local = g0 - M.off;
+                    const uint32_t row = gemv_row(local, M.magic, M.shift);
+                    const uint16_t *xp = M.x + (local - row * M.cols);
+#pragma unroll
+                    for (uint32_t t = 0; t < TM; ++t) {
+                        if (t < g.T) {
+                            const uint4 *xv = reinterpret_cast<const uint4 *>(xp + (uint64_t)t * M.cols);
+                            dot16(w, __ldg(xv), __ldg(xv + 1), lo[t], hi[t]);
+                        }
+                    }
+                    // the key orders (matrix, row) pairs as the elements do
+                    key = M.off / 16u + row;
+                    rows = M.rows;
+                    yrow = M.y + row;
+                }
+            }
+            // (a lane's y row and row stride travel with its key)
+            flush_any<TM>(lo, hi, key, yrow, rows, lane);
+        }
+    }
+
+    // flush_runs for lanes whose runs may belong to different matrices: the
+    // run's first lane adds with its own row pointer and stride.
+    template <uint32_t TM2>
+    __device__ __forceinline__ void flush_any(const float (&lo)[TM2], const float (&hi)[TM2], uint32_t key,
+                                              float *yrow, uint32_t rows, uint32_t lane) {
+        uint32_t same = 0;
+#pragma unroll
+        for (uint32_t k = 0; k < 5; ++k) {
+            const uint32_t o = __shfl_down_sync(kFull, key, 1u << k);
+            if (lane + (1u << k) < 32u && o == key) same |= 1u << k;
+        }
+        const uint32_t prev = __shfl_up_sync(kFull, key, 1);
+        const bool first = (lane == 0 || prev != key) && key != kNoRow;
+#pragma unroll
+        for (uint32_t t = 0; t < TM2; ++t) {
+            float v = lo[t] + hi[t];
+#pragma unroll
+            for (uint32_t k = 0; k < 5; ++k) {
+                const float o = __shfl_down_sync(kFull, v, 1u << k);
+                if (same & (1u << k)) v += o;
+            }
+            if (first && t < g.T) atomicAdd(yrow + (uint64_t)t * rows, v);
+        }
+    }
+
+    // The block's two edge chunks (warp 0, converged): lanes 0..15 the first,
+    // 16..31 the last, one element each; each half-warp's sum is added once
+    // (a chunk lies in one row of one matrix or in none).
+    __device__ __forceinline__ void edges(uint32_t sb, uint32_t base, uint32_t c_full, uint32_t span, uint32_t s,
+                                          uint32_t e, uint32_t lane) {
+        const bool head = s != base;
+        const bool tail = (span & 15u) != 0u && !(head && c_full == 0u);
+        const uint32_t c = (lane < 16u) ? 0u : c_full;
+        const bool mine = (lane < 16u) ? head : tail;
+        const uint32_t gc = base + 16u * c;  // the chunk's first element
+        uint32_t mm = 0;
+        while (mm < g.n_mats && gc >= g.m[mm].end) ++mm;
+        const bool in_mat = mine && mm < g.n_mats && gc >= g.m[mm].off;
+        float p[TM];
+#pragma unroll
+        for (uint32_t t = 0; t < TM; ++t) p[t] = 0.f;
+        uint32_t row = 0;
+        if (in_mat) {
+            const GemvMat &M = g.m[mm];
+            row = gemv_row(gc - M.off, M.magic, M.shift);
+            const uint32_t gel = gc + (lane & 15u);
+            if (gel >= s && gel < e && DF11_BOUNDS_OK(gel - base < kMaxCodesPerBlock + 16u)) {
+                const uint32_t sm8 = __ldg(g.d.sm + gel);
+                const uint32_t r = lds_u8(sb + (gel - base));
+                const uint32_t hi8 = (sm8 & 0x80u) | (r & 0x7Fu);
+                const uint32_t lo8 = (r & 0x80u) | (sm8 & 0x7Fu);
+                const float wv = __uint_as_float((lo8 | (hi8 << 8)) << 16);
+                const uint32_t col = (gel - M.off) - row * M.cols;
+#pragma unroll
+                for (uint32_t t = 0; t < TM; ++t)
+                    if (t < g.T) p[t] = wv * __uint_as_float((uint32_t)__ldg(M.x + (uint64_t)t * M.cols + col) << 16);
+            }
+        }
+#pragma unroll
+        for (uint32_t t = 0; t < TM; ++t) {
+#pragma unroll
+            for (uint32_t d = 8; d >= 1; d >>= 1) p[t] += __shfl_xor_sync(kFull, p[t], d);
+            if ((lane & 15u) == 0u && in_mat && t < g.T)
+                atomicAdd(g.m[mm].y + (uint64_t)t * g.m[mm].rows + row, p[t]);
+        }
+        __syncwarp();
+        if ((lane == 0u && head) || (lane == 16u && tail)) sts_zero16(sb + 16u * (lane == 0u ? 0u : c_full));
+    }
+};
+
+// TM: the largest batch the instance handles (1, or 4 for T = 2..4).
+template <class C, bool kLong, uint32_t TM>
+__global__ void __launch_bounds__(C::kCtaThreads, 1) df11_decode_gemv_kernel(const __grid_constant__ GemvArgs g) {
+    // the format blocks that hold the matrices' elements (each warp finds them)
+    const uint32_t lane = threadIdx.x & 31u;
+    const uint64_t b0 = find_block(g.d.bstart, g.d.n_blocks, g.e_first, lane);
+    const uint64_t b1 = find_block(g.d.bstart, g.d.n_blocks, g.e_last, lane) + 1u;
+    GemvSink<TM> sink{g, 0u};
+    decode_blocks<C, kLong>(g.d, sink, b0, b1);
+}
+
 // ----------------------------------------------------------------- host
 std::atomic<int> g_sm_count[64];
 std::atomic<int> g_attr_set[64];
 
 template <class C, bool kLong>
 cudaError_t set_smem_attr() {
-    cudaError_t e = cudaFuncSetAttribute(df11_decode_kernel<C, kLong>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)C::kSmemBytes);
-    if (e != cudaSuccess) return e;
-    return cudaFuncSetAttribute(df11_gather_kernel<C, kLong>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                (int)C::kSmemBytes);
+    const cudaFuncAttribute kAttr = cudaFuncAttributeMaxDynamicSharedMemorySize;
+    cudaError_t e = cudaFuncSetAttribute(df11_decode_kernel<C, kLong>, kAttr, (int)C::kSmemBytes);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(df11_gather_kernel<C, kLong>, kAttr, (int)C::kSmemBytes);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(df11_decode_gemv_kernel<C, kLong, 1>, kAttr, (int)C::kSmemBytes);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(df11_decode_gemv_kernel<C, kLong, 4>, kAttr, (int)C::kSmemBytes);
+    return e;
 }
 
 df11_status prepare_device(int *sm_count) {
@@ -1056,6 +1384,93 @@ df11_status launch_rows(const df11_tensor *t, uint64_t row_len, const uint32_t *
     return DF11_OK;
 }
 
+template <class C, bool kLong, uint32_t TM>
+void launch_gemv_inst(const GemvArgs &g, uint64_t blocks_est, int sms, cudaStream_t stream) {
+    const uint64_t ctas_needed = (blocks_est + C::kGroups - 1) / C::kGroups;
+    const unsigned grid = (unsigned)(ctas_needed < (uint64_t)sms ? ctas_needed : (uint64_t)sms);
+    df11_decode_gemv_kernel<C, kLong, TM><<<grid, C::kCtaThreads, C::kSmemBytes, stream>>>(g);
+}
+
+template <uint32_t TM>
+void launch_gemv_tm(const GemvArgs &g, Inst inst, bool lng, uint64_t blocks_est, int sms, cudaStream_t s) {
+    if (inst == Inst::kTypical) {
+        if (lng) launch_gemv_inst<CfgTypical, true, TM>(g, blocks_est, sms, s);
+        else launch_gemv_inst<CfgTypical, false, TM>(g, blocks_est, sms, s);
+    } else if (inst == Inst::kWide) {
+        if (lng) launch_gemv_inst<CfgWide, true, TM>(g, blocks_est, sms, s);
+        else launch_gemv_inst<CfgWide, false, TM>(g, blocks_est, sms, s);
+    } else {
+        if (lng) launch_gemv_inst<CfgDense, true, TM>(g, blocks_est, sms, s);
+        else launch_gemv_inst<CfgDense, false, TM>(g, blocks_est, sms, s);
+    }
+}
+
+// Multiply-shift division by d (1 <= d < 2^28) for dividends q < 2^28: with
+// l = ceil(log2 d), shift = 28 + l and magic = ceil(2^shift / d) (< 2^29),
+// the error magic * d - 2^shift is below d <= 2^l, so q times it stays below
+// 2^shift and floor(q * magic / 2^shift) = floor(q / d) (Granlund and
+// Montgomery, "Division by invariant integers using multiplication", 1994).
+void div_magic(uint32_t d, uint32_t &magic, uint32_t &shift) {
+    uint32_t l = 0;
+    while ((1ull << l) < d) ++l;
+    shift = 28u + l;
+    magic = (uint32_t)(((1ull << shift) + d - 1u) / d);
+}
+
+df11_status launch_gemv(const df11_tensor *t, const df11_gemv_mat *mats, uint32_t n_mats, uint32_t T,
+                        uint32_t *err_word, void *stream) {
+    if (!t) return DF11_ERR_INVALID_ARG;
+    df11_status st = df11_validate(t);
+    if (st != DF11_OK) return st;
+    if (n_mats == 0) return DF11_OK;
+    if (!mats) return DF11_ERR_INVALID_ARG;
+    if (n_mats > kMaxGemvMats || T < 1u || T > 4u) return DF11_ERR_UNSUPPORTED;
+    GemvArgs g;
+    st = prepare_args(t, g.d);
+    if (st != DF11_OK) return st;
+    uint64_t prev_end = 0;
+    for (uint32_t j = 0; j < n_mats; ++j) {
+        const df11_gemv_mat &mj = mats[j];
+        if (mj.rows == 0 || mj.cols == 0 || (mj.cols & 15u) || (mj.elem_offset & 15u) || !mj.x || !mj.y ||
+            !aligned16(mj.x) || ((uintptr_t)mj.y & 3u))
+            return DF11_ERR_INVALID_ARG;
+        const uint64_t size = (uint64_t)mj.rows * mj.cols;
+        if (mj.elem_offset < prev_end || mj.elem_offset > t->n_elems || size > t->n_elems - mj.elem_offset)
+            return DF11_ERR_INVALID_ARG;
+        GemvMat &M = g.m[j];
+        M.off = (uint32_t)mj.elem_offset;  // n_elems < 2^32 (df11_validate)
+        M.end = (uint32_t)(mj.elem_offset + size);
+        M.x = mj.x;
+        M.y = mj.y;
+        M.rows = mj.rows;
+        M.cols = mj.cols;
+        div_magic(mj.cols / 16u, M.magic, M.shift);
+        prev_end = mj.elem_offset + size;
+    }
+    for (uint32_t j = n_mats; j < kMaxGemvMats; ++j) g.m[j] = GemvMat{};
+    g.n_mats = n_mats;
+    g.T = T;
+    g.e_first = g.m[0].off;
+    g.e_last = g.m[n_mats - 1].end - 1u;
+    g.d.err = err_word;
+    int sms = 0;
+    st = prepare_device(&sms);
+    if (st != DF11_OK) return st;
+    // blocks the matrices span, estimated from the mean block size (the
+    // persistent CTAs stride over the exact range the kernel finds)
+    const uint64_t span = (uint64_t)g.e_last + 1u - g.e_first;
+    const uint64_t blocks_est =
+        (uint64_t)((double)span * (double)t->n_blocks / (double)t->n_elems) + 2u;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    Inst inst;
+    bool lng;
+    pick_instance(t, inst, lng);
+    if (T == 1u) launch_gemv_tm<1>(g, inst, lng, blocks_est, sms, s);
+    else launch_gemv_tm<4>(g, inst, lng, blocks_est, sms, s);
+    if (cudaGetLastError() != cudaSuccess) return DF11_ERR_CUDA;
+    return DF11_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -1076,6 +1491,11 @@ df11_status df11_decode_block(const df11_tensor *blk, const uint64_t *mat_offset
 df11_status df11_decode_rows(const df11_tensor *t, uint64_t row_len, const uint32_t *rows, uint32_t n_rows,
                              uint16_t *out, uint32_t *err_word, void *stream) {
     return launch_rows(t, row_len, rows, n_rows, out, err_word, stream);
+}
+
+df11_status df11_decode_gemv(const df11_tensor *t, const df11_gemv_mat *mats, uint32_t n_mats, uint32_t T,
+                             uint32_t *err_word, void *stream) {
+    return launch_gemv(t, mats, n_mats, T, err_word, stream);
 }
 
 #ifdef DF11_DEBUG_CHECKS

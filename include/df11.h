@@ -260,6 +260,40 @@ df11_status df11_decode_block(const df11_tensor *blk, const uint64_t *mat_offset
 df11_status df11_decode_rows(const df11_tensor *t, uint64_t row_len, const uint32_t *rows, uint32_t n_rows,
                              uint16_t *out, uint32_t *err_word, void *stream);
 
+/* One matrix of a compressed tensor for df11_decode_gemv. */
+typedef struct df11_gemv_mat {
+    uint64_t elem_offset; /* first element of the [rows, cols] row-major matrix
+                             in the tensor (e.g. a df11_decode_block offset);
+                             a multiple of 16 */
+    uint32_t rows;        /* out features, >= 1 */
+    uint32_t cols;        /* in features, a multiple of 16 */
+    const uint16_t *x;    /* DEVICE [T, cols] BF16 activations, row-major,
+                             16-byte aligned */
+    float *y;             /* DEVICE [T, rows] FP32, row-major: x * W^T is ADDED
+                             (zero it first for a plain product), 4-byte
+                             aligned */
+} df11_gemv_mat;
+
+/* Fused decode and matrix-vector products for small batches (1 <= T <= 4):
+ * for each listed matrix, y += x * W^T, with W decoded on the fly and never
+ * written to memory.  The pages decompress each matrix right before its
+ * multiplication and discard it after ("Decompression adaptee a l'inference
+ * GPU"); here the merge step multiplies every decoded 16-weight chunk by x
+ * instead of storing it, so only the compressed arrays are read.  Only the
+ * thread blocks that hold the listed matrices are decoded.
+ *  mats: HOST array of n_mats descriptors (<= 16), ordered by elem_offset,
+ *        not overlapping, each inside [0, t->n_elems); n_mats == 0 is a
+ *        no-op.  Elements outside the listed matrices are decoded (where
+ *        they share a thread block) but not used.
+ *  FP32 accumulation (BF16 x BF16 products are exact); each warp's partial
+ *  sum of a row is added into y with an FP32 atomic, so the last bits of y
+ *  may differ run to run.
+ *  Errors: DF11_ERR_UNSUPPORTED for T outside 1..4 or more than 16 matrices;
+ *  DF11_ERR_INVALID_ARG for a bad descriptor (size, order, alignment, NULL).
+ *  err_word as in df11_decode.  One launch, asynchronous on `stream`. */
+df11_status df11_decode_gemv(const df11_tensor *t, const df11_gemv_mat *mats, uint32_t n_mats, uint32_t T,
+                             uint32_t *err_word, void *stream);
+
 /* Consumer of a decoded weight matrix: Y = X * W^T with BF16 inputs and FP32
  * accumulation, the matrix multiplication the decompressed weights feed
  * ("Decompression adaptee a l'inference GPU": a matrix is decompressed right

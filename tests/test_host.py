@@ -300,3 +300,53 @@ def test_concurrent_host_encodes_match_sequential():
         assert a.total_bits == b.total_bits and a.n_blocks == b.n_blocks
         for k in ("enc", "sm", "gaps", "block_start", "lut"):
             np.testing.assert_array_equal(a.host_array(k)[: a.nbytes(k)], b.host_array(k)[: b.nbytes(k)])
+
+
+def _aligned_copy(a: np.ndarray) -> tuple[np.ndarray, np.ndarray]:
+    """A 16-byte aligned copy of a's bytes (returns the view and its owner)."""
+    raw = a.view(np.uint8).reshape(-1)
+    buf = np.zeros(raw.size + 32, dtype=np.uint8)
+    k = (-buf.ctypes.data) % 16
+    view = buf[k: k + raw.size]
+    view[:] = raw
+    return view, buf
+
+
+def test_decode_gemv_argument_checks():
+    """df11_decode_gemv rejects bad calls before any GPU work (so these run
+    without a GPU): batch outside 1..4 and more than 16 matrices are
+    unsupported; misaligned, overlapping, out-of-order or out-of-range
+    matrices and NULL vectors are invalid arguments; no matrices is a no-op."""
+    lib = df11._lib()
+    mats = [workloads.normal_matrix(64, 32, 0.02, seed=1), workloads.normal_matrix(32, 64, 0.02, seed=2)]
+    t = df11.encode_multi(mats)
+    d = t._bind()
+    keep = []
+    for name in ("enc", "sm", "gaps", "block_start", "lut"):
+        v, owner = _aligned_copy(t.host_array(name))
+        keep.append(owner)
+        setattr(d, name, v.ctypes.data)
+    xbuf, xown = _aligned_copy(np.zeros(4 * 64 + 8, dtype=np.uint16))
+    ybuf = np.zeros(4 * 64 + 4, dtype=np.float32)
+    X, Y = xbuf.ctypes.data, ybuf.ctypes.data
+
+    def call(descs, T=1, n=None):
+        arr = (df11._GemvMat * max(1, len(descs)))(*[df11._GemvMat(*m) for m in descs])
+        return lib.df11_decode_gemv(ctypes.byref(d), arr, len(descs) if n is None else n, T, None, None)
+
+    good = [(0, 64, 32, X, Y), (2048, 32, 64, X, Y)]
+    assert call(good, n=0) == 0
+    assert call(good, T=0) == 2 and call(good, T=5) == 2
+    assert call([(0, 1, 16, X, Y)] * 17) == 2
+    assert call([(8, 64, 32, X, Y)]) == 1                      # offset not a multiple of 16
+    assert call([(0, 64, 24, X, Y)]) == 1                      # cols not a multiple of 16
+    assert call([(0, 0, 32, X, Y)]) == 1                       # no rows
+    assert call([(0, 64, 32, None, Y)]) == 1                   # NULL x
+    assert call([(0, 64, 32, X, None)]) == 1                   # NULL y
+    assert call([(0, 64, 32, X + 2, Y)]) == 1                  # x not 16-byte aligned
+    assert call([(0, 64, 32, X, Y + 2)]) == 1                  # y not 4-byte aligned
+    assert call([good[1], good[0]]) == 1                       # out of order
+    assert call([(0, 64, 32, X, Y), (2032, 32, 64, X, Y)]) == 1  # overlapping
+    assert call([(2048, 33, 64, X, Y)]) == 1                   # past the tensor's end
+    assert call([(0, 0xFFFFFFFF, 0xFFFFFFF0, X, Y)]) == 1      # size far past the end
+    del keep, xown
