@@ -1,4 +1,5 @@
-"""The decode, block-decode and row-gather kernels built with every
+"""The decode, block-decode, row-gather and fused decode -> matrix-vector
+kernels built with every
 data-dependent shared-memory index and global store address checked
 (libdf11_debug.so): on adversarial inputs, all length caps, ragged sizes and
 the long-code path, no check fails and the output stays bit-exact."""
@@ -64,6 +65,12 @@ def test_decode_paths_without_bounds_errors(debug_lib):
             rows = torch.arange(0, w.size // 64, 7, dtype=torch.int32, device=dev)
             got = _bits(df11.decode_rows(d, 64, rows))
             np.testing.assert_array_equal(got, w.reshape(-1, 64)[rows.cpu().numpy()], err_msg=name)
+            # and the fused matrix-vector product (T = 1 and 3; values are
+            # checked elsewhere, adversarial inputs hold NaN and Inf)
+            for T in (1, 3):
+                x = torch.randn(T, 64, generator=torch.Generator().manual_seed(T)).to(torch.bfloat16).to(dev)
+                df11.decode_gemv(df11.DF11Tensor(d.desc, d.arrays, d.device, [(w.size // 64, 64)], [0, w.size]),
+                                 {0: x})
         assert debug_lib.df11_debug_bounds_errors(1) == 0, name
     mats = [workloads.normal_matrix(r, c, s, seed=i) for i, (r, c, s) in
             enumerate([(512, 256, 0.02), (64, 128, 0.03), (3, 7, 0.5)])]
@@ -71,4 +78,12 @@ def test_decode_paths_without_bounds_errors(debug_lib):
     scratch = df11.decode_block(blk)
     for m, v in zip(mats, blk.views(scratch)):
         np.testing.assert_array_equal(_bits(v).reshape(m.shape), m)
+    for T in (1, 4):  # the fused product over the two 2-D matrices (in = 256, 128)
+        xs = {j: torch.randn(T, mats[j].shape[1], generator=torch.Generator().manual_seed(j)).to(torch.bfloat16)
+              .to(dev) for j in (0, 1)}
+        ys = df11.decode_gemv(blk, xs)
+        for j in (0, 1):
+            w64 = torch.from_numpy(mats[j].view(np.int16)).view(torch.bfloat16).double()
+            ref = xs[j].cpu().double() @ w64.T
+            assert float((ys[j].cpu().double() - ref).norm() / ref.norm()) < 1e-5
     assert debug_lib.df11_debug_bounds_errors(1) == 0
