@@ -55,6 +55,9 @@ WORKLOADS = {
     "decode-gemv": ("llama3.1-8b transformer block (218,112,000 BF16 weights, seed = rank), all seven matrices "
                     "multiplied by N(0,1) BF16 activations [T, in] (seed 1000 + T) in ONE fused decode -> "
                     "matrix-vector launch (weights never written to memory); T from --T (1..4)", None),
+    "gemm": ("consumer GEMM Y = X W^T on one weight shape (default 14336x4096, the gate/up projection), "
+             "W N(0, 0.02^2) BF16 in three copies used in turn (351 MB, larger than L2), X N(0,1) BF16 [T, in]",
+             None),
     "encode-device": ("llama3.1-8b transformer block (218,112,000 BF16 weights, seed = rank) already in device memory, "
                       "encoded on the GPU (histogram + packing; code lengths on the host)", None),
     "offload": ("llama3.1-8b blocks (seeds 0..B-1, default 4) kept in pinned host memory and streamed over PCIe "
@@ -572,6 +575,76 @@ def run_decode_gemv(args, rank: int, world: int):
         dist.destroy_process_group()
 
 
+def run_gemm(args, rank: int, world: int):
+    """The consumer GEMM alone on one shape: CUDA-core matrix-vector stream for
+    T <= 4, tcgen05 kernel above; three copies of W are used in turn so every
+    launch reads W from HBM."""
+    import torch
+    import torch.distributed as dist
+
+    import huffman_decode_02_b200 as df11
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=dev)
+    out, inn = (int(v) for v in args.shape.lower().split("x"))
+    T = args.T
+    g = torch.Generator(device=dev).manual_seed(rank)
+    ws = [(torch.randn(out, inn, device=dev, generator=g) * 0.02).to(torch.bfloat16) for _ in range(3)]
+    x = torch.randn(T, inn, device=dev, generator=g).to(torch.bfloat16)
+    y = torch.empty(T, out, dtype=torch.float32, device=dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    df11.gemm(x, ws[0], y, err, stream)
+    rows = torch.arange(0, out, max(1, out // 256), device=dev)
+    ref = x.double().cpu() @ ws[0][rows].double().cpu().T
+    rel = float((y[:, rows].double().cpu() - ref).norm() / ref.norm())
+    for i in range(args.warmup):
+        df11.gemm(x, ws[i % 3], y, err, stream)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for i in range(args.steps):
+        df11.gemm(x, ws[i % 3], y, err, stream)
+    b.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = a.elapsed_time(b) / args.steps
+    if world > 1:
+        ms = max_over_ranks(ms, dist, dev)
+    assert df11.read_error(err, stream) == 0
+    if rank == 0:
+        hbm, hbm_kind = _peaks()
+        try:
+            with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+                tf_peak, tf_kind = float(json.load(f)["bf16_tflops"]), "measured"
+        except Exception:
+            tf_peak, tf_kind = 1590.0, "fallback"
+        nbytes = 2 * out * inn + 2 * T * inn + 4 * T * out
+        flops = 2.0 * T * out * inn
+        gbs, tfs = nbytes / (ms * 1e-3) / 1e9, flops / (ms * 1e-3) / 1e12
+        hbm_bound = nbytes / hbm >= flops / (tf_peak * 1e3)  # both in us per unit
+        roof = ({"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
+                 "peak_kind": f"{hbm_kind} (MEASURED_PEAKS.json hbm_gbs, copy burst)"} if hbm_bound else
+                {"bound": "tensor", "achieved": tfs, "peak": tf_peak, "unit": "TFLOP/s", "frac": tfs / tf_peak,
+                 "peak_kind": f"{tf_kind} (MEASURED_PEAKS.json bf16_tflops, cuBLAS burst)"})
+        roof.update({"traffic": None, "algorithmic_bytes_per_launch": nbytes, "flops_per_launch": flops})
+        line = {"metric": "consumer GEMM time", "value": ms * 1e3, "unit": "us", "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": False,
+                "scaling": "weak", "vs_baseline": None, "dtype": "bf16 x bf16 -> f32", "data": "synthetic",
+                "config": {"workload": WORKLOADS["gemm"][0], "shape": [out, inn], "T": T,
+                           "kernel": "CUDA-core matrix-vector stream" if T <= 4 else "tcgen05",
+                           "l2": "W in three copies used in turn (3 x 2 out in bytes > L2), no flush"},
+                "rel_fro_sampled_rows": rel, "roofline": roof, "gpu_launches": args.steps}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
 def run_encode_device(args, rank: int, world: int):
     """The device encoder on a block already in device memory: wall time per
     encode (size pass with its host round trip for the histogram, then the
@@ -638,7 +711,8 @@ def main():
     ap.add_argument("--max-code-len", type=int, default=12, help="length cap of the exponent code")
     ap.add_argument("--blocks", type=int, default=None, help="blocks of the decode-gemm (32) / offload (4) workloads")
     ap.add_argument("--repeat", type=int, default=4, help="passes over the blocks in the offload workload")
-    ap.add_argument("--T", type=int, default=1, help="batch of the decode-gemv workload (1..4)")
+    ap.add_argument("--T", type=int, default=1, help="batch of the decode-gemv (1..4) and gemm (1..256) workloads")
+    ap.add_argument("--shape", default="14336x4096", help="OUTxIN of the gemm workload")
     args = ap.parse_args()
     args.blocks_given = args.blocks is not None
     if args.blocks is None:
@@ -659,6 +733,9 @@ def main():
         return
     if args.workload == "decode-gemv":
         run_decode_gemv(args, rank, world)
+        return
+    if args.workload == "gemm":
+        run_gemm(args, rank, world)
         return
     if args.workload == "encode-device":
         run_encode_device(args, rank, world)
