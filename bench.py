@@ -548,6 +548,16 @@ def run_decode_gemv(args, rank: int, world: int):
     ms_fused = timed(fused, args.steps)
     clocks = sampler.stop()
     ms_unfused = timed(unfused, max(1, args.steps // 4))
+    # a forward pass's order: one call per group of matrices that share an
+    # input (q/k/v, o, gate/up, down), each decoding only its thread blocks
+    groups = [g for g in ([0, 1, 2], [3], [4, 5], [6]) if all(j in xs for j in g)]
+
+    def forward_order():
+        ybuf.zero_()
+        for grp in groups:
+            df11.decode_gemv(d, {j: xs[j] for j in grp}, {j: ys[j] for j in grp}, err, stream)
+
+    ms_forward = timed(forward_order, max(1, args.steps // 4))
     assert df11.read_error(err, stream) == 0
     if rank == 0:
         peak, peak_kind = _peaks()
@@ -564,6 +574,7 @@ def run_decode_gemv(args, rank: int, world: int):
                            "timing": "K steps (zeroing of y + one fused launch) between CUDA events"},
                 "rel_fro_sampled_rows": rel,
                 "unfused_us": ms_unfused * 1e3, "speedup_vs_unfused": ms_unfused / ms_fused,
+                "forward_order_us": ms_forward * 1e3, "forward_order_calls": len(groups),
                 "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                              "frac": achieved / peak, "traffic": None,
                              "peak_kind": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs, copy burst)",
