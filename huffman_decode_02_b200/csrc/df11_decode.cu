@@ -982,9 +982,10 @@ __device__ __forceinline__ uint32_t gemv_row(uint32_t local, uint32_t magic, uin
 }
 
 // Adds a warp's per-lane sums into y: one atomic per run of lanes holding the
-// same key.  Equal keys must sit in contiguous lanes (the callers' element
+// same key (the row), at that run's `yrow` (y + row) for each t (stride
+// `rows`).  Equal keys must sit in contiguous lanes (the caller's element
 // order guarantees it); a lane with key kNoRow holds nothing.  Whole warp,
-// converged.  key0 / yrow: the key and output row of each lane.
+// converged.
 template <uint32_t TM>
 __device__ __forceinline__ void flush_runs(const float (&lo)[TM], const float (&hi)[TM], uint32_t key,
                                            float *const yrow, uint32_t rows, uint32_t T, uint32_t lane) {
