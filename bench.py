@@ -293,6 +293,8 @@ def run_decode_gemm(args, rank: int, world: int):
         ms = a.elapsed_time(b) / steps
         return max_over_ranks(ms, dist, dev) if world > 1 else ms
 
+    from huffman_decode_02_b200.pipeline import BlockPipeline
+    pipe = BlockPipeline([d for d, _ in blocks], dev)  # two more scratch buffers
     per_T = {}
     nb = len(blocks)
     w_bytes = sum(int(w.numel()) * 2 for w in gemm_mats)
@@ -328,10 +330,16 @@ def run_decode_gemm(args, rank: int, world: int):
                 for w in gemm_mats:
                     torch.matmul(xs[w.shape[1]], w.T)
 
-        t_dec, t_gemm, t_both, t_bf16 = (timed(f, args.steps) / nb for f in (dec_all, gemm_all, both, bf16_all))
+        def piped():  # decode of block b+1 on a side stream overlaps the GEMMs of block b
+            pipe.run(range(nb), lambda bi, views: [df11.gemm(xs[w.shape[1]], v, y, err, stream)
+                                                   for w, v, y in zip(gemm_mats, views[:7], ys)], stream)
+
+        t_dec, t_gemm, t_both, t_bf16, t_pipe = (timed(f, args.steps) / nb
+                                                 for f in (dec_all, gemm_all, both, bf16_all, piped))
         x_bytes = sum(T * w.shape[1] * 2 + T * w.shape[0] * 4 for w in gemm_mats)
         per_T[str(T)] = {"decode_us": t_dec * 1e3, "gemm_us": t_gemm * 1e3, "total_us": t_both * 1e3,
                          "bf16_gemm_us": t_bf16 * 1e3, "slowdown_vs_bf16": t_both / t_bf16,
+                         "pipelined_total_us": t_pipe * 1e3,
                          "gemm_gbs": (w_bytes + x_bytes) / (t_gemm * 1e-3) / 1e9, "gemm_rel_fro": rel}
         if T <= 4:
             # fused decode -> matrix-vector products: per block, one zeroing of
@@ -362,6 +370,7 @@ def run_decode_gemm(args, rank: int, world: int):
                                   "fused_speedup_vs_unfused": t_both / t_fused, "fused_rel_fro": frel,
                                   "fused_launches_per_block": 2})
     assert df11.read_error(err, stream) == 0
+    pipe.check(stream)
     if rank == 0:
         desc = WORKLOADS["decode-gemm"][0]
         line = {"metric": "decode->GEMM time per llama3.1-8b block", "value": per_T["1"]["total_us"], "unit": "us",
