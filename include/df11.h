@@ -29,6 +29,12 @@
  *  - Thread safety: calls share no mutable global state, except the
  *    no-allocation encoder calls, which share one fixed scratch array per
  *    device (see there).
+ *  - CUDA graphs: df11_decode, df11_decode_block, df11_decode_gemv and
+ *    df11_gemm_bf16 only enqueue work on the given stream (kernels, and a
+ *    memset for split-K GEMMs), so they can be captured into a CUDA graph
+ *    and replayed.  The first call on a device must come before any capture
+ *    (it makes one-time settings), and df11_read_error synchronises the
+ *    stream, so it stays outside the graph.
  */
 #ifndef DF11_H
 #define DF11_H
