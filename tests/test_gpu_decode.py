@@ -228,7 +228,8 @@ def test_maximum_size_tensor():
     Gaussian matrix, so the histogram and code are those of the matrix; the
     decoded tensor is compared with the input on 20 M sampled positions and
     on its last 4 M elements, and the last block start must be right below
-    2^32."""
+    2^32.  The row gather, the fused matrix-vector product and the device
+    encoder run on the same tensor."""
     dev = _dev()
     n = (1 << 32) - 1
     base = workloads.normal_matrix(4096, 4096, 0.02, seed=2).reshape(-1)
@@ -250,6 +251,22 @@ def test_maximum_size_tensor():
     got = df11.decode_rows(d, 65537, torch.from_numpy(rows).to(dev))
     np.testing.assert_array_equal(got.view(torch.int16).cpu().numpy().view(np.uint16),
                                   w.reshape(65535, 65537)[rows])
+    # the fused matrix-vector product over the whole range (a [1048575, 4096]
+    # matrix: chunk indices up to 2^28 - 256) and over a 1024 x 4096 matrix
+    # that ends within 16 elements of 2^32 - 1; sampled rows (the last ones
+    # among them) against FP64, within the FP32 rounding bound
+    xb = workloads.round_to_bf16(rng.standard_normal((1, 4096), dtype=np.float32))
+    x64 = torch.from_numpy(xb.view(np.int16)).view(torch.bfloat16).double()
+    far = ((n - 1024 * 4096) // 16) * 16
+    for off, rows_m in ((0, n // 4096), (far, 1024)):
+        view = df11.DF11Tensor(d.desc, d.arrays, d.device, [(rows_m, 4096)], [off, off + rows_m * 4096])
+        y = df11.decode_gemv(view, {0: torch.from_numpy(xb.view(np.int16)).view(torch.bfloat16).to(dev)})[0]
+        r = np.unique(np.concatenate([rng.integers(0, rows_m, 300), np.arange(rows_m - 8, rows_m)]))
+        W = torch.from_numpy(np.stack([w[off + int(i) * 4096: off + (int(i) + 1) * 4096] for i in r])
+                             .view(np.int16)).view(torch.bfloat16).double()
+        ref, mag = x64 @ W.T, x64.abs() @ W.abs().T
+        got = y.cpu().double()[:, torch.from_numpy(r)]
+        assert bool(torch.all((got - ref).abs() <= (4096 + 32) * 2.0 ** -24 * mag + 1e-30)), off
     # the device encoder on the same weights: arrays identical to the host encoder's
     e = df11.encode_device(torch.from_numpy(w.view(np.int16)).to(dev).view(torch.bfloat16))
     for k in ("enc", "sm", "gaps", "block_start", "lut"):
