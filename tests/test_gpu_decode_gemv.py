@@ -216,3 +216,18 @@ def test_fused_llama_block(T):
         yj = df11.decode_gemv(d, {j: xs[j]})[j]
         rows = np.sort(rng.choice(mats[j].shape[0], 256, replace=False))
         _check(yj, mats[j], xs_np[mats[j].shape[1]], rows=rows)
+
+
+@pytest.mark.slow
+def test_fused_lm_head_shape():
+    """The LM-head / embedding shape (128256 x 4096, 525 M weights, one
+    matrix): T = 1 and 4, 512 sampled rows (the last ones among them)."""
+    dev = _dev()
+    w = workloads.normal_matrix(128256, 4096, 0.02, seed=5)
+    d = df11.encode(w).to(dev)
+    rng = np.random.default_rng(13)
+    rows = np.unique(np.concatenate([rng.choice(128256, 504, replace=False), np.arange(128248, 128256)]))
+    for T in (1, 4):
+        xb = _x(T, 4096, 50 + T)
+        y = df11.decode_gemv(d, {0: _bf16(xb).to(dev)})[0]
+        _check(y, w, xb, rows=rows)
