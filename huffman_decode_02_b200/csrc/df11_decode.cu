@@ -28,7 +28,7 @@
 //    sign/mantissa range into shared memory, so the merge reads nothing
 //    from global memory and no register holds prefetched data across the
 //    decode loops.
-//  * The exponent buffer holds 6400 symbols per group when every block of
+//  * The exponent buffer holds 7152 symbols per group when every block of
 //    the tensor fits (LLM-like weights: the room left gives the symbol table
 //    its second copy), else 8192; tensors whose blocks hold more codes
 //    (average code under 2 bits) use an instance with 4 groups of 16 KB
@@ -142,7 +142,9 @@ struct Cfg {
     static_assert(kLutBytes <= G * kGroupBytes, "tables stage in the group area");
     static_assert(kSmemBytes <= 227u * 1024u, "fits one CTA's shared memory");
 };
-using CfgTypical = Cfg<8, 6400, 2>;  // blocks of up to 6400 - 15 codes: two symbol-table copies fit
+// (S = 7152 is the largest buffer with which 8 groups and two symbol-table
+// copies fit: 232,336 of the 232,448 bytes a CTA may use)
+using CfgTypical = Cfg<8, 7152, 2>;  // blocks of up to 7152 - 15 codes: two symbol-table copies fit
 using CfgWide = Cfg<8, 8192, 1>;     // blocks of up to 8192 - 15 codes (any LLM-like data)
 using CfgDense = Cfg<4, 16400, 1>;   // any block (1-bit codes: 16384 per block)
 

@@ -112,7 +112,7 @@ def test_rows_other_instances(kind):
     w = ((e << 7) | rng.integers(0, 128, e.shape) | (rng.integers(0, 2, e.shape) << 15)).astype(np.uint16)
     t = df11.encode(w)
     need = t.desc.max_block_codes + 15
-    assert (need > 8192) if kind == "dense" else (6400 < need <= 8192)
+    assert (need > 8192) if kind == "dense" else (7152 < need <= 8192)
     d = t.to(dev)
     rows = torch.from_numpy(rng.integers(0, 4000, 300).astype(np.int32)).to(dev)
     out = df11.decode_rows(d, 96, rows)
