@@ -1219,7 +1219,7 @@ struct GemvSink {
     }
 };
 
-// TM: the largest batch the instance handles (1, or 4 for T = 2..4).
+// TM: the largest batch the instance handles (1, 2, or 4 for T = 3..4).
 template <class C, bool kLong, uint32_t TM>
 __global__ void __launch_bounds__(C::kCtaThreads, 1) df11_decode_gemv_kernel(const __grid_constant__ GemvArgs g) {
     // the format blocks that hold the matrices' elements (each warp finds them)
@@ -1240,6 +1240,7 @@ cudaError_t set_smem_attr() {
     cudaError_t e = cudaFuncSetAttribute(df11_decode_kernel<C, kLong>, kAttr, (int)C::kSmemBytes);
     if (e == cudaSuccess) e = cudaFuncSetAttribute(df11_gather_kernel<C, kLong>, kAttr, (int)C::kSmemBytes);
     if (e == cudaSuccess) e = cudaFuncSetAttribute(df11_decode_gemv_kernel<C, kLong, 1>, kAttr, (int)C::kSmemBytes);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(df11_decode_gemv_kernel<C, kLong, 2>, kAttr, (int)C::kSmemBytes);
     if (e == cudaSuccess) e = cudaFuncSetAttribute(df11_decode_gemv_kernel<C, kLong, 4>, kAttr, (int)C::kSmemBytes);
     return e;
 }
@@ -1469,6 +1470,7 @@ df11_status launch_gemv(const df11_tensor *t, const df11_gemv_mat *mats, uint32_
     bool lng;
     pick_instance(t, inst, lng);
     if (T == 1u) launch_gemv_tm<1>(g, inst, lng, blocks_est, sms, s);
+    else if (T == 2u) launch_gemv_tm<2>(g, inst, lng, blocks_est, sms, s);
     else launch_gemv_tm<4>(g, inst, lng, blocks_est, sms, s);
     if (cudaGetLastError() != cudaSuccess) return DF11_ERR_CUDA;
     return DF11_OK;

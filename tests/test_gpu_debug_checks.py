@@ -65,9 +65,9 @@ def test_decode_paths_without_bounds_errors(debug_lib):
             rows = torch.arange(0, w.size // 64, 7, dtype=torch.int32, device=dev)
             got = _bits(df11.decode_rows(d, 64, rows))
             np.testing.assert_array_equal(got, w.reshape(-1, 64)[rows.cpu().numpy()], err_msg=name)
-            # and the fused matrix-vector product (T = 1 and 3; values are
+            # and the fused matrix-vector product (T = 1, 2 and 3; values are
             # checked elsewhere, adversarial inputs hold NaN and Inf)
-            for T in (1, 3):
+            for T in (1, 2, 3):
                 x = torch.randn(T, 64, generator=torch.Generator().manual_seed(T)).to(torch.bfloat16).to(dev)
                 df11.decode_gemv(df11.DF11Tensor(d.desc, d.arrays, d.device, [(w.size // 64, 64)], [0, w.size]),
                                  {0: x})
