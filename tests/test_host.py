@@ -350,3 +350,24 @@ def test_decode_gemv_argument_checks():
     assert call([(2048, 33, 64, X, Y)]) == 1                   # past the tensor's end
     assert call([(0, 0xFFFFFFFF, 0xFFFFFFF0, X, Y)]) == 1      # size far past the end
     del keep, xown
+
+
+def test_header_compiles_as_plain_c(tmp_path):
+    """include/df11.h is a C ABI: it compiles as C99 with -pedantic -Werror
+    and every struct the calls take can be declared from C."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "use_df11.c"
+    src.write_text('#include "df11.h"\n'
+                   "int main(void) {\n"
+                   "    df11_params p; df11_tensor t; df11_gemv_mat m;\n"
+                   "    (void)p; (void)t; (void)m;\n"
+                   "    return 0;\n"
+                   "}\n")
+    r = subprocess.run([gcc, "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror", "-I",
+                        os.path.join(ROOT, "include"), "-c", str(src), "-o", str(tmp_path / "use_df11.o")],
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
