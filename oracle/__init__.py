@@ -21,7 +21,9 @@ Functions (each cites its passage in ``df11_oracle.c``):
   -- gaps, per-thread counts and block starts recomputed from a stream.
 * ``pack_gaps(gaps)`` -- 5-bit packing of gaps.
 * ``exponent_stats(count, lengths)`` -- entropy, distinct values, mean length.
-* ``kraft_sum_2p32(lengths)``, ``is_prefix_free(lengths)``.
+* ``kraft_sum_2p32(lengths)``, ``is_prefix_free(lengths)`` (the canonical
+  code of the lengths), ``codes_prefix_free(codes, lengths)`` (an explicit
+  code set).
 
 Parity: pinned by the ``-m "not gpu"`` tests in ``tests/test_oracle.py``
 (identity on every input, brute-force optimality, closed forms, textbook
@@ -92,6 +94,7 @@ def _load():
     lib.orc_total_bits.restype = u64
     lib.orc_encode.argtypes = [_u16p, u64, _u8p, _u8p, u64, _u8p, _u64p]
     lib.orc_is_prefix_free.argtypes = [_u8p]
+    lib.orc_codes_prefix_free.argtypes = [_u32p, _u8p]
     lib.orc_decode.argtypes = [_u8p, u64, _u8p, u64, _u8p, _u16p]
     lib.orc_aux.argtypes = [_u8p, u64, u64, _u8p, ctypes.c_uint32, ctypes.c_uint32,
                             _u8p, _u32p, _u32p, _u64p, _u64p]
@@ -167,6 +170,18 @@ def kraft_sum_2p32(lengths) -> int:
 def is_prefix_free(lengths) -> bool:
     l8 = np.ascontiguousarray(lengths, dtype=np.uint8)
     return bool(_load().orc_is_prefix_free(_ptr(l8, _u8p)))
+
+
+def codes_prefix_free(codes, lengths) -> bool:
+    """Tree-insertion check of an explicit code set: codes[s] holds
+    lengths[s] bits (most significant first); lengths[s] == 0 means no code."""
+    c32 = np.zeros(256, dtype=np.uint32)
+    l8 = np.zeros(256, dtype=np.uint8)
+    c = np.asarray(codes, dtype=np.uint64).reshape(-1)
+    ln = np.asarray(lengths, dtype=np.int64).reshape(-1)
+    c32[: c.size] = c.astype(np.uint32)
+    l8[: ln.size] = ln.astype(np.uint8)
+    return bool(_load().orc_codes_prefix_free(_ptr(c32, _u32p), _ptr(l8, _u8p)))
 
 
 def total_bits(w, lengths) -> int:

@@ -292,10 +292,13 @@ typedef struct {
     int n_nodes;
 } orc_tree;
 
-static orc_tree *build_tree(const uint8_t len[256], int *rc) {
-    uint32_t code[256];
-    *rc = orc_canonical_codes(len, code);
-    if (*rc) return NULL;
+/* Inserts every code into a binary tree, one bit at a time from its most
+ * significant bit.  A code set is prefix-free exactly when no insertion
+ * walks through a node that is already a leaf, and no code ends on a node
+ * that is already a leaf or already has children. */
+static orc_tree *build_tree_from_codes(const uint32_t code[256], const uint8_t len[256], int *rc) {
+    for (int s = 0; s < 256; ++s)
+        if (len[s] > 32) { *rc = ORC_ERR_ARG; return NULL; }
     orc_tree *t = (orc_tree *)malloc(sizeof(orc_tree));
     if (!t) { *rc = ORC_ERR_NOMEM; return NULL; }
     t->n_nodes = 1;
@@ -324,8 +327,26 @@ static orc_tree *build_tree(const uint8_t len[256], int *rc) {
     return t;
 }
 
-/* Prefix-freeness check by tree insertion: no code ends at or passes
- * through another code's leaf. */
+/* The decoding tree of the canonical code the lengths define. */
+static orc_tree *build_tree(const uint8_t len[256], int *rc) {
+    uint32_t code[256];
+    *rc = orc_canonical_codes(len, code);
+    if (*rc) return NULL;
+    return build_tree_from_codes(code, len, rc);
+}
+
+/* Prefix-freeness of an explicit code set (code[s] holds len[s] bits, most
+ * significant first; len[s] == 0: no code), by tree insertion. */
+int orc_codes_prefix_free(const uint32_t code[256], const uint8_t len[256]) {
+    int rc;
+    orc_tree *t = build_tree_from_codes(code, len, &rc);
+    if (t) free(t);
+    return rc == ORC_OK;
+}
+
+/* Prefix-freeness of the canonical code of the given lengths: false when
+ * the lengths admit no prefix code (Kraft sum above 1, or a length above
+ * 32), else the tree-insertion check of the canonical codes. */
 int orc_is_prefix_free(const uint8_t len[256]) {
     int rc;
     orc_tree *t = build_tree(len, &rc);

@@ -230,6 +230,72 @@ def test_roundtrip_identity_and_kraft(name):
         assert out.dtype == np.uint16 and np.array_equal(out, w)
 
 
+def _lengths(values):
+    out = np.zeros(256, dtype=np.uint8)
+    out[: len(values)] = values
+    return out
+
+
+@pytest.mark.parametrize("bad", [[1, 1, 1], [1, 2, 2, 2], [2, 2, 2, 2, 3], [1, 1, 2]])
+def test_over_full_lengths_are_rejected(bad):
+    """Lengths whose Kraft sum exceeds 1 admit no prefix code: the canonical
+    assignment refuses them and the prefix check says no.  {1,1,1} sums to
+    3/2 and {1,2,2,2} to 5/4."""
+    lengths = _lengths(bad)
+    assert oracle.kraft_sum_2p32(lengths) > 1 << 32
+    assert not oracle.is_prefix_free(lengths)
+    with pytest.raises(oracle.OracleError):
+        oracle.canonical_codes(lengths)
+
+
+def test_shortening_one_length_of_a_complete_code_overflows_kraft():
+    """Every length vector of a complete code (Kraft sum exactly 1) turns
+    into an over-full one when any single length is shortened by one bit."""
+    w = workloads.normal_matrix(64, 64, 0.02, seed=5)
+    lengths = oracle.package_merge_lengths(oracle.histogram(w), 32)
+    assert oracle.kraft_sum_2p32(lengths) == 1 << 32
+    for s in np.flatnonzero(lengths):
+        if lengths[s] < 2:
+            continue
+        short = lengths.copy()
+        short[s] -= 1
+        assert oracle.kraft_sum_2p32(short) > 1 << 32
+        assert not oracle.is_prefix_free(short)
+        with pytest.raises(oracle.OracleError):
+            oracle.canonical_codes(short)
+
+
+def test_length_above_32_is_rejected():
+    lengths = _lengths([1, 2, 33])
+    assert not oracle.is_prefix_free(lengths)
+    with pytest.raises(oracle.OracleError):
+        oracle.canonical_codes(lengths)
+
+
+@pytest.mark.parametrize("codes,lengths,ok", [
+    # RFC 1951 section 3.2.2 example: A..H with lengths 3,3,3,3,3,2,4,4
+    ([0b010, 0b011, 0b100, 0b101, 0b110, 0b00, 0b1110, 0b1111], [3, 3, 3, 3, 3, 2, 4, 4], True),
+    ([0b0, 0b10, 0b11], [1, 2, 2], True),
+    ([0b0, 0b01], [1, 2], False),            # "0" is a prefix of "01"
+    ([0b01, 0b0], [2, 1], False),            # same, longer code inserted first
+    ([0b10, 0b101, 0b11], [2, 3, 2], False),  # "10" is a prefix of "101"
+    ([0b110, 0b110], [3, 3], False),         # the same code twice
+    ([0b1, 0b0111, 0b0110, 0b010], [1, 4, 4, 3], True),
+    ([0b1, 0b0111, 0b01111], [1, 4, 5], False),  # "0111" is a prefix of "01111"
+])
+def test_explicit_code_sets_prefix_check(codes, lengths, ok):
+    """The tree-insertion check on explicit code sets, including ones whose
+    lengths satisfy Kraft but whose codes collide; canonical codes from
+    lengths alone can never reach these cases."""
+    assert oracle.codes_prefix_free(codes, lengths) is ok
+
+
+def test_canonical_codes_of_lengths_pass_the_explicit_check(golden_dir):
+    g = _load(golden_dir, "rfc1951_canonical.json")
+    lengths = _lengths(g["lengths"])
+    assert oracle.codes_prefix_free(oracle.canonical_codes(lengths), lengths)
+
+
 def test_encoded_bits_match_independent_bitstring():
     """The stream is the concatenation of the canonical codes, MSB-first;
     rebuilt here with Python strings and numpy.packbits."""
