@@ -170,13 +170,24 @@ def _u16_ptr(a: np.ndarray):
     return a.ctypes.data_as(ctypes.POINTER(ctypes.c_uint16))
 
 
-def _stream_handle(stream) -> ctypes.c_void_p:
+def _stream_handle(stream, device=None) -> ctypes.c_void_p:
+    """The CUDA stream to launch on: `stream` if given, else the current
+    stream of `device` (of the current device when None)."""
     if stream is None:
         import torch
-        return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+        return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
     if isinstance(stream, int):
         return ctypes.c_void_p(stream)
     return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _on(device):
+    """Makes `device` the current CUDA device for the duration of a library
+    call: the C entry points launch on the current device, so the data's own
+    device must be current (another device's memory would be read without
+    peer access)."""
+    import torch
+    return torch.cuda.device(torch.device(device))
 
 
 class DF11Tensor:
@@ -328,15 +339,17 @@ def encode_device(mats, params: Params | None = None, stream=None) -> DF11Tensor
     scratch = torch.empty(max(sb, 16), dtype=torch.uint8, device=dev)
     desc = _Tensor()
     pc = (params or Params())._c()
-    h = _stream_handle(stream)
-    _check(lib.df11_encode_device_size(ctypes.c_void_p(flat.data_ptr()), n, ctypes.byref(pc), ctypes.byref(desc),
-                                       ctypes.c_void_p(scratch.data_ptr()), sb, h), "encode_device (size)")
-    arrays = {name: torch.empty(max(int(getattr(desc, name + "_bytes")), 16), dtype=torch.uint8, device=dev)
-              for name in _ARRAYS}
-    for name in _ARRAYS:
-        setattr(desc, name, arrays[name].data_ptr())
-    _check(lib.df11_encode_device(ctypes.c_void_p(flat.data_ptr()), n, ctypes.byref(desc),
-                                  ctypes.c_void_p(scratch.data_ptr()), sb, h), "encode_device")
+    with _on(dev):
+        h = _stream_handle(stream, dev)
+        _check(lib.df11_encode_device_size(ctypes.c_void_p(flat.data_ptr()), n, ctypes.byref(pc),
+                                           ctypes.byref(desc), ctypes.c_void_p(scratch.data_ptr()), sb, h),
+               "encode_device (size)")
+        arrays = {name: torch.empty(max(int(getattr(desc, name + "_bytes")), 16), dtype=torch.uint8, device=dev)
+                  for name in _ARRAYS}
+        for name in _ARRAYS:
+            setattr(desc, name, arrays[name].data_ptr())
+        _check(lib.df11_encode_device(ctypes.c_void_p(flat.data_ptr()), n, ctypes.byref(desc),
+                                      ctypes.c_void_p(scratch.data_ptr()), sb, h), "encode_device")
     for name in _ARRAYS:
         setattr(desc, name, None)
     return DF11Tensor(desc, arrays, str(dev), shapes if not single else [shapes[0]], offsets)
@@ -356,15 +369,16 @@ def encode_device_noalloc(w, params: Params | None = None, stream=None) -> DF11T
     n = int(w.numel())
     desc = _Tensor()
     pc = (params or Params())._c()
-    h = _stream_handle(stream)
-    _check(lib.df11_encode_device_size_noalloc(ctypes.c_void_p(w.data_ptr()), n, ctypes.byref(pc),
-                                               ctypes.byref(desc), h), "encode_device_noalloc (size)")
-    arrays = {name: torch.empty(max(int(getattr(desc, name + "_bytes")), 16), dtype=torch.uint8, device=w.device)
-              for name in _ARRAYS}
-    for name in _ARRAYS:
-        setattr(desc, name, arrays[name].data_ptr())
-    _check(lib.df11_encode_device_noalloc(ctypes.c_void_p(w.data_ptr()), n, ctypes.byref(desc), h),
-           "encode_device_noalloc")
+    with _on(w.device):
+        h = _stream_handle(stream, w.device)
+        _check(lib.df11_encode_device_size_noalloc(ctypes.c_void_p(w.data_ptr()), n, ctypes.byref(pc),
+                                                   ctypes.byref(desc), h), "encode_device_noalloc (size)")
+        arrays = {name: torch.empty(max(int(getattr(desc, name + "_bytes")), 16), dtype=torch.uint8,
+                                    device=w.device) for name in _ARRAYS}
+        for name in _ARRAYS:
+            setattr(desc, name, arrays[name].data_ptr())
+        _check(lib.df11_encode_device_noalloc(ctypes.c_void_p(w.data_ptr()), n, ctypes.byref(desc), h),
+               "encode_device_noalloc")
     for name in _ARRAYS:
         setattr(desc, name, None)
     return DF11Tensor(desc, arrays, str(w.device), [tuple(w.shape)], [0, n])
@@ -454,8 +468,9 @@ def decode(t: DF11Tensor, out=None, err=None, stream=None):
     if own_err:
         err = _new_err(t.device)
     d = t._bind()
-    _check(_lib().df11_decode(ctypes.byref(d), ctypes.c_void_p(out.data_ptr()),
-                              ctypes.c_void_p(err.data_ptr()), _stream_handle(stream)), "decode")
+    with _on(t.device):
+        _check(_lib().df11_decode(ctypes.byref(d), ctypes.c_void_p(out.data_ptr()),
+                                  ctypes.c_void_p(err.data_ptr()), _stream_handle(stream, t.device)), "decode")
     if own_err:
         read_error(err, stream)
     return out
@@ -476,10 +491,11 @@ def decode_block(t: DF11Tensor, scratch=None, err=None, stream=None):
         err = _new_err(t.device)
     offs = (ctypes.c_uint64 * len(t.offsets))(*t.offsets)
     d = t._bind()
-    _check(_lib().df11_decode_block(ctypes.byref(d), offs, len(t.offsets) - 1,
-                                    ctypes.c_void_p(scratch.data_ptr()),
-                                    ctypes.c_void_p(err.data_ptr()), _stream_handle(stream)),
-           "decode_block")
+    with _on(t.device):
+        _check(_lib().df11_decode_block(ctypes.byref(d), offs, len(t.offsets) - 1,
+                                        ctypes.c_void_p(scratch.data_ptr()),
+                                        ctypes.c_void_p(err.data_ptr()), _stream_handle(stream, t.device)),
+               "decode_block")
     if own_err:
         read_error(err, stream)
     return scratch
@@ -500,9 +516,10 @@ def decode_rows(t: DF11Tensor, row_len: int, rows, out=None, err=None, stream=No
     own_err = err is None
     if own_err:
         err = _new_err(t.device)
-    _check(_lib().df11_decode_rows(ctypes.byref(t._bind()), int(row_len), ctypes.c_void_p(rows.data_ptr()), n,
-                                   ctypes.c_void_p(out.data_ptr()), ctypes.c_void_p(err.data_ptr()),
-                                   _stream_handle(stream)), "decode_rows")
+    with _on(t.device):
+        _check(_lib().df11_decode_rows(ctypes.byref(t._bind()), int(row_len), ctypes.c_void_p(rows.data_ptr()), n,
+                                       ctypes.c_void_p(out.data_ptr()), ctypes.c_void_p(err.data_ptr()),
+                                       _stream_handle(stream, t.device)), "decode_rows")
     if own_err:
         read_error(err, stream)
     return out
@@ -545,8 +562,10 @@ def decode_gemv(t: DF11Tensor, xs: dict, ys: dict | None = None, err=None, strea
     own_err = err is None
     if own_err:
         err = _new_err(t.device)
-    _check(_lib().df11_decode_gemv(ctypes.byref(t._bind()), mats, len(order), T, ctypes.c_void_p(err.data_ptr()),
-                                   _stream_handle(stream)), "decode_gemv")
+    with _on(t.device):
+        _check(_lib().df11_decode_gemv(ctypes.byref(t._bind()), mats, len(order), T,
+                                       ctypes.c_void_p(err.data_ptr()), _stream_handle(stream, t.device)),
+               "decode_gemv")
     if own_err:
         read_error(err, stream)
     return {j: ys[j] for j in order}
@@ -569,9 +588,12 @@ def gemm(x, w, out=None, err=None, stream=None):
     own_err = err is None
     if own_err:
         err = _new_err(x.device)
-    _check(_lib().df11_gemm_bf16(ctypes.c_void_p(x.data_ptr()), ctypes.c_void_p(w.data_ptr()),
-                                 ctypes.c_void_p(out.data_ptr()), T, n, k, ctypes.c_void_p(err.data_ptr()),
-                                 _stream_handle(stream)), "gemm")
+    if x.device != w.device or out.device != x.device:
+        raise ValueError("gemm expects x, w and out on one device")
+    with _on(x.device):
+        _check(_lib().df11_gemm_bf16(ctypes.c_void_p(x.data_ptr()), ctypes.c_void_p(w.data_ptr()),
+                                     ctypes.c_void_p(out.data_ptr()), T, n, k, ctypes.c_void_p(err.data_ptr()),
+                                     _stream_handle(stream, x.device)), "gemm")
     if own_err:
         read_error(err, stream)
     return out
@@ -581,7 +603,9 @@ def read_error(err, stream=None) -> int:
     """Reads the kernel error word (synchronises the stream); raises
     CorruptStreamError if any bit is set."""
     v = ctypes.c_uint32(0)
-    st = _lib().df11_read_error(ctypes.c_void_p(err.data_ptr()), _stream_handle(stream), ctypes.byref(v))
+    with _on(err.device):
+        st = _lib().df11_read_error(ctypes.c_void_p(err.data_ptr()), _stream_handle(stream, err.device),
+                                    ctypes.byref(v))
     if st == 4:
         raise CorruptStreamError(4, f"decode kernel reported error bits 0x{v.value:x}")
     _check(st, "read_error")

@@ -276,6 +276,21 @@ df11_status check_params(const df11_params *params, df11_params &p) {
     return DF11_OK;
 }
 
+// The weights must live on the current device: the kernels launch there and
+// would otherwise read another device's memory (a fault without peer access).
+df11_status check_on_current_device(const void *w) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return DF11_ERR_CUDA;
+    cudaPointerAttributes at{};
+    if (cudaPointerGetAttributes(&at, w) != cudaSuccess) {
+        (void)cudaGetLastError();  // clear the (non-sticky) error so later launch checks do not see it
+        return DF11_ERR_INVALID_ARG;
+    }
+    if ((at.type != cudaMemoryTypeDevice && at.type != cudaMemoryTypeManaged) || at.device != dev)
+        return DF11_ERR_INVALID_ARG;
+    return DF11_OK;
+}
+
 int sm_count() {
     int dev = 0, sms = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return 0;
@@ -300,6 +315,8 @@ df11_status df11_encode_device_size(const uint16_t *w, uint64_t n, const df11_pa
     if (n > 0) {
         if (((uintptr_t)w & 15u) || ((uintptr_t)scratch & 15u) || scratch_bytes < scratch_need(n))
             return DF11_ERR_INVALID_ARG;
+        st = check_on_current_device(w);
+        if (st != DF11_OK) return st;
         const int sms = sm_count();
         if (sms <= 0) return DF11_ERR_CUDA;
         cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -333,6 +350,12 @@ df11_status df11_encode_device(const uint16_t *w, uint64_t n, df11_tensor *io, v
         const df11_status vst = df11_validate(&chk);
         if (vst != DF11_OK) return vst;
     }
+    if (n > 0) {  // before anything is enqueued
+        if (!w || ((uintptr_t)w & 15u) || !scratch || ((uintptr_t)scratch & 15u) || scratch_bytes < scratch_need(n))
+            return DF11_ERR_INVALID_ARG;
+        const df11_status dst = check_on_current_device(w);
+        if (dst != DF11_OK) return dst;
+    }
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (cudaMemsetAsync(io->enc, 0, io->enc_bytes, s) != cudaSuccess ||
         cudaMemsetAsync(io->sm, 0, io->sm_bytes, s) != cudaSuccess ||
@@ -346,8 +369,6 @@ df11_status df11_encode_device(const uint16_t *w, uint64_t n, df11_tensor *io, v
     uint32_t most = 0;
     uint64_t total = 0;
     if (n > 0) {
-        if (!w || ((uintptr_t)w & 15u) || !scratch || ((uintptr_t)scratch & 15u) || scratch_bytes < scratch_need(n))
-            return DF11_ERR_INVALID_ARG;
         const int sms = sm_count();
         if (sms <= 0) return DF11_ERR_CUDA;
         CodeTables ct;
@@ -398,23 +419,21 @@ namespace {
 
 constexpr uint64_t kNoAllocMaxElems = 1ull << 28;
 constexpr uint64_t kNoAllocScratchBytes = scratch_need(kNoAllocMaxElems);
+static_assert(kNoAllocScratchBytes == 264224u, "the size the header states");
 __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
-std::atomic<uintptr_t> g_noalloc_addr[64];
 
-// Device address of the fixed scratch on the current device, resolved once
-// per device (cudaGetSymbolAddress with that device current).
+// Device address of the fixed scratch in the current device's context.  In
+// host code the array's name is only a host-side stand-in, so the address is
+// looked up with cudaGetSymbolAddress, with the device current, on every
+// call: a device reset or a re-created primary context reloads the module and
+// may move the array, and a cached address would then point at freed memory.
+// (The lookup is a host-side table query; the first one on a device loads
+// the library's device code, which is why the first call must come before
+// any stream capture.)
 df11_status noalloc_scratch(void **out) {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return DF11_ERR_CUDA;
-    if (dev < 0 || dev >= 64) return DF11_ERR_UNSUPPORTED;
-    uintptr_t a = g_noalloc_addr[dev].load(std::memory_order_acquire);
-    if (a == 0) {
-        void *p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return DF11_ERR_CUDA;
-        a = reinterpret_cast<uintptr_t>(p);
-        g_noalloc_addr[dev].store(a, std::memory_order_release);
-    }
-    *out = reinterpret_cast<void *>(a);
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return DF11_ERR_CUDA;
+    *out = p;
     return DF11_OK;
 }
 

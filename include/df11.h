@@ -194,7 +194,7 @@ df11_status df11_validate(const df11_tensor *t);
 uint64_t df11_encode_device_scratch_bytes(uint64_t n);
 
 /* Size pass: w is a DEVICE array of n BF16 values (16-byte aligned; a block's
- * matrices concatenated).  Runs the histogram on `stream`, synchronises it,
+ * matrices concatenated) on the current device (else DF11_ERR_INVALID_ARG).  Runs the histogram on `stream`, synchronises it,
  * plans the code and fills *hdr (sizes, code lengths, counts) as
  * df11_encode_size does; array pointers are left NULL. */
 df11_status df11_encode_device_size(const uint16_t *w, uint64_t n, const df11_params *params, df11_tensor *hdr,
@@ -214,13 +214,17 @@ df11_status df11_encode_device(const uint16_t *w, uint64_t n, df11_tensor *io, v
  * runtime that owns all device memory through a fixed pool, or a serving
  * process re-encoding weights in place on a full GPU, where cudaMalloc would
  * fail or synchronise the device.  The scratch is a fixed array inside
- * libdf11 (about 258 KB per device), so:
+ * libdf11 (264,224 B = 258 KiB on every device that loads the library,
+ * held until exit), so:
  *  - n is limited to df11_encode_device_noalloc_max_elems() (2^28 weights, a
  *    whole Llama-3.1-8B block); larger inputs return DF11_ERR_TOO_LARGE
  *    before any GPU work;
- *  - the first call on a device resolves the array's address
- *    (cudaGetSymbolAddress with that device current): make it before any
- *    stream capture;
+ *  - every call looks up the array's address in the current device's
+ *    context (cudaGetSymbolAddress), so a device reset or a re-created
+ *    context is picked up; the first call on a device also loads the
+ *    library's device code, so make it before any stream capture;
+ *  - w must be device memory of the current device (else
+ *    DF11_ERR_INVALID_ARG);
  *  - calls that overlap on one device (other host threads or streams) share
  *    that array and race: serialise them per device.
  * Everything the encoder needs cleared is cleared by each call.  Otherwise

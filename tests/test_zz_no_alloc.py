@@ -58,3 +58,44 @@ def test_too_large_refused_before_gpu_work():
     st = lib.df11_encode_device_size_noalloc(ctypes.c_void_p(buf.data_ptr()), cap + 1, ctypes.byref(pc),
                                              ctypes.byref(desc), ctypes.c_void_p(0))
     assert st == 3  # DF11_ERR_TOO_LARGE
+
+
+def test_too_large_refused_by_the_fill_call():
+    """The fill call checks its own size limit too (before any GPU work)."""
+    dev = _dev()
+    lib = df11._lib()
+    cap = int(lib.df11_encode_device_noalloc_max_elems())
+    buf = torch.zeros(16, dtype=torch.int16, device=dev)
+    desc = df11._Tensor()
+    st = lib.df11_encode_device_noalloc(ctypes.c_void_p(buf.data_ptr()), cap + 1, ctypes.byref(desc),
+                                        ctypes.c_void_p(0))
+    assert st == 3  # DF11_ERR_TOO_LARGE
+
+
+def test_host_pointer_refused():
+    """Weights must be memory of the current device; a host pointer is an
+    argument error, reported before anything is enqueued."""
+    _dev()
+    lib = df11._lib()
+    host = np.zeros(4096, dtype=np.uint16)
+    desc = df11._Tensor()
+    pc = df11.Params()._c()
+    st = lib.df11_encode_device_size_noalloc(ctypes.c_void_p(host.ctypes.data), host.size, ctypes.byref(pc),
+                                             ctypes.byref(desc), ctypes.c_void_p(0))
+    assert st == 1  # DF11_ERR_INVALID_ARG
+
+
+@pytest.mark.slow
+def test_llama_block_near_capacity_matches_caller_scratch():
+    """A whole Llama-3.1-8B-shaped block (218,112,000 weights, 81 % of the
+    fixed scratch's 2^28-weight limit, so the tile-offset region is filled
+    far into its end) encoded without allocation, byte for byte against the
+    caller-scratch encoder."""
+    dev = _dev()
+    mats = workloads.llama8b_block(seed=0)
+    flat = np.concatenate([np.ascontiguousarray(m).reshape(-1) for m in mats])
+    t = torch.from_numpy(flat.view(np.int16)).to(dev).view(torch.bfloat16)
+    got = df11.encode_device_noalloc(t)
+    _same(df11.encode_device(t), got)
+    del got
+    torch.cuda.empty_cache()
