@@ -68,9 +68,9 @@ class _Tensor(ctypes.Structure):
                 ("reserved2", ctypes.c_uint32), ("code_len", ctypes.c_uint8 * 256),
                 ("enc_bytes", ctypes.c_uint64), ("sm_bytes", ctypes.c_uint64),
                 ("gaps_bytes", ctypes.c_uint64), ("block_start_bytes", ctypes.c_uint64),
-                ("lut_bytes", ctypes.c_uint64),
+                ("lut_bytes", ctypes.c_uint64), ("counts_bytes", ctypes.c_uint64),
                 ("enc", ctypes.c_void_p), ("sm", ctypes.c_void_p), ("gaps", ctypes.c_void_p),
-                ("block_start", ctypes.c_void_p), ("lut", ctypes.c_void_p)]
+                ("block_start", ctypes.c_void_p), ("lut", ctypes.c_void_p), ("counts", ctypes.c_void_p)]
 
 
 class _GemvMat(ctypes.Structure):
@@ -78,7 +78,9 @@ class _GemvMat(ctypes.Structure):
                 ("x", ctypes.c_void_p), ("y", ctypes.c_void_p)]
 
 
-_ARRAYS = ("enc", "sm", "gaps", "block_start", "lut")
+# The compressed arrays; "counts" (per-thread code counts) is optional: a
+# tensor without it decodes with the count pass.
+_ARRAYS = ("enc", "sm", "gaps", "block_start", "lut", "counts")
 _LIB = None
 
 
@@ -121,7 +123,7 @@ def _lib():
     lib.df11_encode_device_noalloc_max_elems.restype = u64
     lib.df11_encode_device_size_noalloc.argtypes = [vp, u64, P(_Params), P(T), vp]
     lib.df11_encode_device_noalloc.argtypes = [vp, u64, P(T), vp]
-    if lib.df11_abi_version() != 2 or lib.df11_sizeof_tensor() != ctypes.sizeof(_Tensor):
+    if lib.df11_abi_version() != 3 or lib.df11_sizeof_tensor() != ctypes.sizeof(_Tensor):
         raise ImportError("libdf11.so ABI does not match this binding")
     _LIB = lib
     return lib
@@ -216,14 +218,31 @@ class DF11Tensor:
     def nbytes(self, which: str) -> int:
         return int(getattr(self.desc, which + "_bytes"))
 
+    @property
+    def has_counts(self) -> bool:
+        return "counts" in self.arrays
+
     def compressed_bytes(self) -> int:
         """Bytes the stored format needs: exponent stream, sign/mantissa,
-        gaps, block starts and the 256-byte code-length table."""
+        gaps, block starts and the 256-byte code-length table (the pages'
+        arrays; the optional per-thread counts are `counts_bytes()`)."""
         return ((self.total_bits + 7) // 8 + self.n_elems + (5 * self.n_threads + 7) // 8
                 + 4 * (self.n_blocks + 1) + 256)
 
+    def counts_bytes(self) -> int:
+        """Bytes of the per-thread code counts (one per thread), 0 without them."""
+        return self.n_threads if self.has_counts else 0
+
     def bits_per_weight(self) -> float:
         return 8.0 * self.compressed_bytes() / max(1, self.n_elems)
+
+    def without_counts(self) -> "DF11Tensor":
+        """The same tensor without its per-thread counts (shares the arrays):
+        decoding it runs the count pass of the two-step kernel."""
+        arrays = {k: v for k, v in self.arrays.items() if k != "counts"}
+        desc = _Tensor.from_buffer_copy(self.desc)
+        desc.counts_bytes = 0
+        return DF11Tensor(desc, arrays, self.device, self.shapes, self.offsets)
 
     def host_array(self, which: str) -> np.ndarray:
         a = self.arrays[which]
@@ -236,8 +255,8 @@ class DF11Tensor:
     def _bind(self) -> _Tensor:
         d = _Tensor.from_buffer_copy(self.desc)
         for name in _ARRAYS:
-            a = self.arrays[name]
-            ptr = a.ctypes.data if isinstance(a, np.ndarray) else a.data_ptr()
+            a = self.arrays.get(name)
+            ptr = None if a is None else (a.ctypes.data if isinstance(a, np.ndarray) else a.data_ptr())
             setattr(d, name, ptr)
         return d
 
@@ -246,7 +265,7 @@ class DF11Tensor:
         import torch
         dev = torch.device(device)
         arrays = {}
-        for name in _ARRAYS:
+        for name in self.arrays:
             a = self.arrays[name]
             if isinstance(a, np.ndarray):
                 a = torch.from_numpy(a.view(np.uint8))
@@ -273,7 +292,8 @@ def _alloc_host(nbytes: int, pinned: bool):
     return raw[off: off + max(nbytes, 16)]
 
 
-def _encode_impl(mats: list[np.ndarray], shapes, params: Params | None, pinned: bool) -> DF11Tensor:
+def _encode_impl(mats: list[np.ndarray], shapes, params: Params | None, pinned: bool,
+                 counts: bool = True) -> DF11Tensor:
     lib = _lib()
     k = len(mats)
     ptrs = (ctypes.POINTER(ctypes.c_uint16) * max(1, k))(*[_u16_ptr(m) for m in mats])
@@ -281,32 +301,37 @@ def _encode_impl(mats: list[np.ndarray], shapes, params: Params | None, pinned: 
     desc = _Tensor()
     pc = (params or Params())._c()
     _check(lib.df11_encode_multi_size(ptrs, sizes, k, ctypes.byref(pc), ctypes.byref(desc)), "encode (size)")
-    arrays = {name: _alloc_host(int(getattr(desc, name + "_bytes")), pinned) for name in _ARRAYS}
-    for name in _ARRAYS:
+    names = _ARRAYS if counts else _ARRAYS[:-1]
+    arrays = {name: _alloc_host(int(getattr(desc, name + "_bytes")), pinned) for name in names}
+    for name in names:
         a = arrays[name]
         setattr(desc, name, a.ctypes.data if isinstance(a, np.ndarray) else a.data_ptr())
     _check(lib.df11_encode_multi(ptrs, sizes, k, ctypes.byref(desc)), "encode")
     for name in _ARRAYS:
         setattr(desc, name, None)
+    if not counts:
+        desc.counts_bytes = 0
     offsets = [0]
     for m in mats:
         offsets.append(offsets[-1] + m.size)
     return DF11Tensor(desc, arrays, "cpu", shapes, offsets)
 
 
-def encode(w, params: Params | None = None, pinned: bool = False) -> DF11Tensor:
+def encode(w, params: Params | None = None, pinned: bool = False, counts: bool = True) -> DF11Tensor:
     """Host encoder for one BF16 matrix (numpy uint16 bits or a CPU torch
-    tensor): histogram, length-limited canonical Huffman code, packing, aux."""
+    tensor): histogram, length-limited canonical Huffman code, packing, aux
+    (with the optional per-thread code counts unless ``counts`` is False)."""
     shape = tuple(getattr(w, "shape", ()))
-    return _encode_impl([_as_u16(w)], [shape], params, pinned)
+    return _encode_impl([_as_u16(w)], [shape], params, pinned, counts)
 
 
-def encode_multi(mats: Sequence, params: Params | None = None, pinned: bool = False) -> DF11Tensor:
+def encode_multi(mats: Sequence, params: Params | None = None, pinned: bool = False,
+                 counts: bool = True) -> DF11Tensor:
     """Encodes several matrices (a transformer block) as one stream with one
     shared table; ``DF11Tensor.offsets`` gives each matrix's element offset."""
     arrs = [_as_u16(m) for m in mats]
     shapes = [tuple(getattr(m, "shape", ())) for m in mats]
-    return _encode_impl(arrs, shapes, params, pinned)
+    return _encode_impl(arrs, shapes, params, pinned, counts)
 
 
 def encode_device(mats, params: Params | None = None, stream=None) -> DF11Tensor:
@@ -384,17 +409,18 @@ def encode_device_noalloc(w, params: Params | None = None, stream=None) -> DF11T
     return DF11Tensor(desc, arrays, str(w.device), [tuple(w.shape)], [0, n])
 
 
-_FILE_MAGIC = b"DF11T001"
+_FILE_MAGIC = b"DF11T002"
 
 
 def save(t: DF11Tensor, path: str) -> None:
     """Writes a compressed tensor (host or device) to `path` as an .npz
-    archive: the descriptor bytes (array pointers cleared), the five arrays
-    and the matrix shapes and offsets.  Nothing is decoded."""
+    archive: the descriptor bytes (array pointers cleared), the arrays (the
+    per-thread counts when the tensor has them) and the matrix shapes and
+    offsets.  Nothing is decoded."""
     desc = _Tensor.from_buffer_copy(t.desc)
     for name in _ARRAYS:
         setattr(desc, name, None)
-    arrays = {name: t.host_array(name).view(np.uint8).reshape(-1)[: t.nbytes(name)] for name in _ARRAYS}
+    arrays = {name: t.host_array(name).view(np.uint8).reshape(-1)[: t.nbytes(name)] for name in t.arrays}
     shapes = np.array([len(s) for s in t.shapes] + [d for s in t.shapes for d in s], dtype=np.int64)
     np.savez(path, magic=np.frombuffer(_FILE_MAGIC, dtype=np.uint8), desc=np.frombuffer(bytes(desc), dtype=np.uint8),
              offsets=np.asarray(t.offsets, dtype=np.int64), shapes=shapes, **arrays)
@@ -412,6 +438,9 @@ def load(path: str, pinned: bool = False) -> DF11Tensor:
         desc = _Tensor.from_buffer_copy(raw)
         arrays = {}
         for name in _ARRAYS:
+            if name == "counts" and "counts" not in z.files:
+                desc.counts_bytes = 0
+                continue
             a = z[name]
             if a.size != int(getattr(desc, name + "_bytes")):
                 raise ValueError(f"array {name} has the wrong size")

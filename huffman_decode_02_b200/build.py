@@ -50,15 +50,35 @@ def _stale(path: str) -> bool:
 
 
 def build(force: bool = False, verbose: bool = False, debug: bool = False) -> str:
+    """Compiles every source to an object file (in parallel, one nvcc per
+    source) under _build/, then links the shared library."""
     path = DEBUG_LIB_PATH if debug else LIB_PATH
     if not force and not _stale(path):
         return path
-    tmp = path + f".tmp{os.getpid()}"
+    tag = ("debug" if debug else "release") + f".{os.getpid()}"
+    obj_dir = os.path.join(HERE, "_build")
+    os.makedirs(obj_dir, exist_ok=True)
     extra = ["-DDF11_DEBUG_CHECKS"] if debug else []
-    cmd = [_nvcc(), *NVCC_FLAGS, *extra, "-I" + INCLUDE, "-I" + CSRC, *sources(), "-o", tmp]
+    compile_flags = [f for f in NVCC_FLAGS if f != "-shared"]
+    jobs = []
+    for src in sources():
+        obj = os.path.join(obj_dir, os.path.basename(src) + f".{tag}.o")
+        jobs.append((obj, [_nvcc(), *compile_flags, *extra, "-I" + INCLUDE, "-I" + CSRC, "-c", src, "-o", obj]))
+    procs = []
+    for _, cmd in jobs:
+        if verbose:
+            print(" ".join(cmd), file=sys.stderr)
+        procs.append(subprocess.Popen(cmd))
+    failed = [cmd for (_, cmd), p in zip(jobs, procs) if p.wait() != 0]
+    if failed:
+        raise subprocess.CalledProcessError(1, failed[0])
+    tmp = path + f".tmp{os.getpid()}"
+    link = [_nvcc(), *NVCC_FLAGS, *[obj for obj, _ in jobs], "-o", tmp]
     if verbose:
-        print(" ".join(cmd), file=sys.stderr)
-    subprocess.check_call(cmd)
+        print(" ".join(link), file=sys.stderr)
+    subprocess.check_call(link)
+    for obj, _ in jobs:
+        os.remove(obj)
     os.replace(tmp, path)
     return path
 

@@ -89,7 +89,6 @@ constexpr uint32_t log2u(uint32_t x) { return x <= 1u ? 0u : 1u + log2u(x >> 1);
 constexpr uint32_t kCountShift = log2u(4u * kCountCopies);  // byte stride of one replicated entry
 static_assert((1u << kCountShift) == 4u * kCountCopies, "power of two");
 constexpr uint32_t kOffCountRep = 768;
-constexpr uint32_t kOffSymRep = kOffCountRep + 4u * kCountCopies * (1u << kW1Max);
 constexpr uint32_t kEncStage = kThreadsPerBlockFmt * kBytesPerThread + 16u;  // + next block's first 16
 constexpr uint32_t kGapStage = kThreadsPerBlockFmt * 5u / 8u + 16u;          // + next block's first gaps
 constexpr uint32_t kFull = 0xFFFFFFFFu;
@@ -114,10 +113,16 @@ __device__ uint32_t g_df11_bounds_errors;
 static_assert(kLutBytes % 16 == 0, "bulk copy size");
 
 // Per-instance layout: G groups per CTA, buffers of S symbols (+ 16: the
-// 16-element chunk alignment of the block start is at most 15).
-template <int G, int S, int SC>
+// 16-element chunk alignment of the block start is at most 15), SC copies of
+// the symbol table.  CT: the instance runs the count pass and keeps the count
+// table (tensors without stored per-thread counts); without it, the counts
+// come from the tensor's `counts` array, staged per block, and the 32 KB of
+// the count table are free for buffers and table copies.
+template <int G, int S, int SC, bool CT = true>
 struct Cfg {
+    static constexpr bool kCountTable = CT;
     static constexpr uint32_t kSymCopies = SC;  // symbol-table copies (lane l reads copy l mod SC)
+    static constexpr uint32_t kOffSymRep = CT ? kOffCountRep + 4u * kCountCopies * (1u << kW1Max) : kOffCountRep;
     static constexpr uint32_t kOffGroups = kOffSymRep + 8u * SC * (1u << kW2Max);
     static constexpr uint32_t kGroups = G;
     static constexpr uint32_t kBufSyms = S;
@@ -127,7 +132,9 @@ struct Cfg {
     static constexpr uint32_t kGrpEnc = kGrpWtot + 16u;
     static constexpr uint32_t kGrpGap = kGrpEnc + kEncStage;
     static constexpr uint32_t kGrpBs = kGrpGap + kGapStage;
-    static constexpr uint32_t kGrpSm = kGrpBs + 32u;  // the block's sign/mantissa bytes
+    static constexpr uint32_t kGrpCnt = kGrpBs + 32u;  // the block's stored counts (instances without CT)
+    static constexpr uint32_t kCntStage = CT ? 0u : (uint32_t)kThreadsPerBlockFmt;
+    static constexpr uint32_t kGrpSm = kGrpCnt + kCntStage;  // the block's sign/mantissa bytes
     static constexpr uint32_t kSmBytes = S + 16u;
     static constexpr uint32_t kGrpMbar = kGrpSm + kSmBytes;
     static constexpr uint32_t kGrpAux = kGrpMbar + 16u;  // row gather: the row's block range
@@ -135,21 +142,33 @@ struct Cfg {
     static constexpr uint32_t kSmemBytes = kOffGroups + G * kGroupBytes + 16u;
     static_assert(S % 16 == 0, "whole chunks");
     static_assert(((S + 19u) >> 4) * 16u <= kSbufBytes, "zeroing stays inside the buffer");
-    static_assert(SC == 1 || SC == 2, "one or two symbol-table copies");
+    static_assert(SC >= 1 && SC <= 4, "one to four symbol-table copies");
     static_assert(kGroupBytes % 16 == 0 && kGrpEnc % 16 == 0 && kGrpGap % 16 == 0 && kGrpBs % 16 == 0 &&
-                      kGrpSm % 16 == 0,
+                      kGrpCnt % 16 == 0 && kGrpSm % 16 == 0,
                   "bulk copy destinations are 16-byte aligned");
     static_assert(kLutBytes <= G * kGroupBytes, "tables stage in the group area");
     static_assert(kSmemBytes <= 227u * 1024u, "fits one CTA's shared memory");
 };
 // (S = 7152 is the largest buffer with which 8 groups and two symbol-table
-// copies fit: 232,336 of the 232,448 bytes a CTA may use)
+// copies fit beside the count table: 232,336 of the 232,448 bytes a CTA may
+// use)
 using CfgTypical = Cfg<8, 7152, 2>;  // blocks of up to 7152 - 15 codes: two symbol-table copies fit
 using CfgWide = Cfg<8, 8192, 1>;     // blocks of up to 8192 - 15 codes (any LLM-like data)
 using CfgDense = Cfg<4, 16400, 1>;   // any block (1-bit codes: 16384 per block)
+// Stored counts (no count pass, no count table).
+#ifndef DF11_TYPICAL_C_SYMS
+#define DF11_TYPICAL_C_SYMS 7152
+#endif
+#ifndef DF11_TYPICAL_C_COPIES
+#define DF11_TYPICAL_C_COPIES 2
+#endif
+using CfgTypicalC = Cfg<8, DF11_TYPICAL_C_SYMS, DF11_TYPICAL_C_COPIES, false>;
+using CfgWideC = Cfg<8, 8192, 2, false>;
+using CfgDenseC = Cfg<4, 16400, 2, false>;
 
 struct DecodeArgs {
     const uint8_t *enc;
+    const uint8_t *counts;  // per-thread code counts (instances without the count pass)
     const uint8_t *sm;
     const uint8_t *gaps;
     const uint32_t *bstart;
@@ -359,18 +378,24 @@ __device__ __forceinline__ uint32_t count_long_code(uint32_t acc, uint32_t lim, 
 
 // Same for the decoding pass: ORs the long code's symbol into the buffer at
 // index p, shifts the window and returns the meta word of 1 code with a
-// zero shift amount; an invalid pattern stops the chain at pend.
+// zero shift amount (its length is added to `lbits`); an invalid pattern
+// stops the chain at pend.
 template <uint32_t kBufBytes>
 __device__ __forceinline__ uint32_t decode_long_code(uint32_t pacc, uint32_t pend, uint32_t &hi, uint32_t &lo,
-                                                     uint32_t &fl, uint32_t sb, uint32_t s_lim, uint32_t s_offs,
-                                                     uint32_t s_symrot, uint32_t from, uint32_t max_len) {
+                                                     uint32_t &fl, uint32_t &lbits, uint32_t sb, uint32_t s_lim,
+                                                     uint32_t s_offs, uint32_t s_symrot, uint32_t from,
+                                                     uint32_t max_len) {
     const uint32_t l = long_code_length(hi, s_lim, from, max_len);
-    if (l == 0u) return (pend - pacc + 31u) & ~31u;  // reported by the count pass
+    if (l == 0u) {
+        lbits += 0x100u;  // no code: the bit check below fails
+        return (pend - pacc + 31u) & ~31u;
+    }
     const uint32_t idx = (hi >> (32u - l)) + lds_u32(s_offs + 4u * l);
     const uint32_t p = pacc >> 8;
     if (DF11_BOUNDS_OK((p & ~3u) + 4u <= kBufBytes))
         red_or(sb + (p & ~3u), lds_u8(s_symrot + (idx & 255u)) << (8u * (p & 3u)));
     shift_window_clamped(hi, lo, fl, l);
+    lbits += l;
     return 1u << 8;
 }
 
@@ -420,15 +445,20 @@ __device__ __forceinline__ void count_pass(const Chain &A, const Chain &B, const
 // exponent into the group buffer `buf` (word-addressed).  Symbol bytes are
 // OR-ed into the (zeroed) buffer, one or two aligned words per lookup;
 // unused symbol bytes of a table entry are zero.  Stops on the code counts
-// of the count pass.  `sym` points at this lane's copy of the symbol table
-// (entry i at sym[i * kSymCopies]).
-template <bool kLong, uint32_t kSymCopies, uint32_t kBufBytes>
+// (of the count pass, or stored with the tensor).  `sym` points at this
+// lane's copy of the symbol table (entry i at sym[i * kSymCopies]).
+// kCheck (stored counts, no count pass to check the stream): after the
+// loop each chain must stand exactly on its code count and have taken
+// exactly its bits (the low byte of the position accumulator sums the bits
+// of the table entries, long codes are summed apart); else DF11_KERR_OVERRUN.
+template <bool kLong, bool kCheck, uint32_t kSymCopies, uint32_t kBufBytes>
 __device__ __forceinline__ void decode_pass(const Chain &A, const Chain &B, uint32_t startA, uint32_t cA,
                                             uint32_t startB, uint32_t cB, uint32_t *buf, uint32_t sb,
                                             const uint2 *sym, uint32_t sh2, uint32_t s_lim, uint32_t s_offs,
-                                            uint32_t s_symrot, uint32_t from, uint32_t max_len) {
+                                            uint32_t s_symrot, uint32_t from, uint32_t max_len, uint32_t &err) {
     uint32_t hA = A.hi, lA = A.lo, fA = A.fl, hB = B.hi, lB = B.lo, fB = B.fl;
     uint32_t pA = startA << 8, pB = startB << 8;
+    uint32_t lbA = 0, lbB = 0;  // bits of long codes
     const uint32_t endPA = (startA + cA) << 8, endPB = (startB + cB) << 8;
     uint32_t guard = kLoopCap;  // as in the count pass
     while (((pA < endPA) | (pB < endPB)) && guard != 0u) {
@@ -442,9 +472,11 @@ __device__ __forceinline__ void decode_pass(const Chain &A, const Chain &B, uint
         uint32_t mB = actB ? eB.y : 0u;
         if (kLong && (mA | mB) >= kEscape) {  // rare: a long code
             if (mA == kEscape)
-                mA = decode_long_code<kBufBytes>(pA, endPA, hA, lA, fA, sb, s_lim, s_offs, s_symrot, from, max_len);
+                mA = decode_long_code<kBufBytes>(pA, endPA, hA, lA, fA, lbA, sb, s_lim, s_offs, s_symrot, from,
+                                                 max_len);
             if (mB == kEscape)
-                mB = decode_long_code<kBufBytes>(pB, endPB, hB, lB, fB, sb, s_lim, s_offs, s_symrot, from, max_len);
+                mB = decode_long_code<kBufBytes>(pB, endPB, hB, lB, fB, lbB, sb, s_lim, s_offs, s_symrot, from,
+                                                 max_len);
         }
         const uint32_t bA = pA >> 8, bB = pB >> 8;
         const uint32_t shA = (bA & 3u) << 3, shB = (bB & 3u) << 3;
@@ -469,6 +501,8 @@ __device__ __forceinline__ void decode_pass(const Chain &A, const Chain &B, uint
         lB = __funnelshift_l(fB, lB, mB);
         fB = __funnelshift_l(kFull, fB, mB);
     }
+    if (kCheck && (pA != endPA + (uint32_t)A.rem0 - lbA || pB != endPB + (uint32_t)B.rem0 - lbB))
+        err |= DF11_KERR_OVERRUN;
 }
 
 // Merges chunks c_first, c_first + 128, ... < c_end (chunk c covers output
@@ -508,10 +542,28 @@ __device__ __forceinline__ void merge_chunks(uint16_t *out, uint32_t sb, uint32_
 template <class C>
 __device__ __forceinline__ void issue_inputs(const DecodeArgs &a, uint64_t blk, uint32_t grp, uint32_t mbar) {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-    mbar_expect(mbar, kEncStage + kGapStage + 32u);
+    mbar_expect(mbar, kEncStage + kGapStage + 32u + C::kCntStage);
     bulk_g2s(grp + C::kGrpEnc, a.enc + blk * (uint64_t)(kThreadsPerBlockFmt * kBytesPerThread), kEncStage, mbar);
     bulk_g2s(grp + C::kGrpGap, a.gaps + blk * (uint64_t)(kThreadsPerBlockFmt * 5u / 8u), kGapStage, mbar);
     bulk_g2s(grp + C::kGrpBs, reinterpret_cast<const uint8_t *>(a.bstart) + ((4ull * blk) & ~15ull), 32u, mbar);
+    if (!C::kCountTable)  // the block's 256 stored counts (one byte per thread)
+        bulk_g2s(grp + C::kGrpCnt, a.counts + blk * (uint64_t)kThreadsPerBlockFmt, C::kCntStage, mbar);
+}
+
+// The two chains' code counts: from the count pass, or from the stored
+// counts staged with the block's inputs.
+template <class C, bool kLong>
+__device__ __forceinline__ void chain_counts(const Chain &A, const Chain &B, uint32_t grp, uint32_t lt,
+                                             const uint32_t *cnt_lane, uint32_t sh1, uint32_t s_lim, uint32_t from,
+                                             uint32_t max_len, uint32_t &cA, uint32_t &cB, uint32_t &err) {
+    if (C::kCountTable) {
+        count_pass<kLong>(A, B, cnt_lane, sh1, s_lim, from, max_len, cA, cB, err);
+    } else {
+        uint32_t v;
+        asm volatile("ld.shared.u16 %0, [%1];" : "=r"(v) : "r"(grp + C::kGrpCnt + 2u * lt));
+        cA = v & 0xFFu;
+        cB = v >> 8;
+    }
 }
 
 // Stages the decode tables by one bulk copy, validates every entry and
@@ -532,8 +584,14 @@ __device__ __forceinline__ bool load_tables(const uint8_t *lut, uint32_t *err_ou
     }
     __syncthreads();
     if (tid == 0) {
-        mbar_expect(s_tmbar, kLutBytes);
-        bulk_g2s(s_stage, lut, kLutBytes, s_tmbar);
+        if (C::kCountTable) {
+            mbar_expect(s_tmbar, kLutBytes);
+            bulk_g2s(s_stage, lut, kLutBytes, s_tmbar);
+        } else {  // header, limits and symbols; then the symbol LUT (the count LUT is not used)
+            mbar_expect(s_tmbar, kOffCountLut + (kLutBytes - kOffSymLut));
+            bulk_g2s(s_stage, lut, kOffCountLut, s_tmbar);
+            bulk_g2s(s_stage + kOffSymLut, lut + kOffSymLut, kLutBytes - kOffSymLut, s_tmbar);
+        }
     }
     const bool staged = wait_phase(s_tmbar, 0u);
     if (__syncthreads_or(!staged)) {
@@ -560,9 +618,9 @@ __device__ __forceinline__ bool load_tables(const uint8_t *lut, uint32_t *err_ou
         // entry; the loops cover every (entry, copy), so every copy a lane can
         // read is written and validated here
         constexpr uint32_t kCW = kCountCopies < 4u ? kCountCopies : 4u;
-        constexpr uint32_t kSW = kSymCopies < 2u ? kSymCopies : 2u;
+        constexpr uint32_t kSW = kSymCopies % 2u == 0u ? 2u : 1u;
         static_assert(kCountCopies % kCW == 0u && kSymCopies % kSW == 0u, "copies fill whole stores");
-        for (uint32_t i = tid; i < (1u << kW1Max) * (kCountCopies / kCW); i += C::kCtaThreads) {
+        for (uint32_t i = tid; C::kCountTable && i < (1u << kW1Max) * (kCountCopies / kCW); i += C::kCtaThreads) {
             const uint32_t ent = lds_u32(s_stage + kOffCountLut + 4u * (i / (kCountCopies / kCW)));
             const uint32_t nb = count_entry_bits(ent), nc = count_entry_codes(ent);
             bad |= ent != kEscape && (ent != count_entry(nb, nc) || nb == 0u || nb > w1 || nc == 0u || nc > nb);
@@ -576,7 +634,7 @@ __device__ __forceinline__ bool load_tables(const uint8_t *lut, uint32_t *err_ou
             const uint32_t nb = sym_entry_bits(ent.y), nc = sym_entry_codes(ent.y);
             bad |= ent.y != kEscape && (ent.y != sym_entry_meta(nb, nc) || nb == 0u || nb > w2 || nc == 0u ||
                                         nc > (uint32_t)kSymsPerEntry || nc > nb);
-            const uint32_t dst = s_base + kOffSymRep + 8u * kSW * i;
+            const uint32_t dst = s_base + C::kOffSymRep + 8u * kSW * i;
             if (kSW == 2u) sts_u4(dst, ent.x, ent.y, ent.x, ent.y);
             else asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(dst), "r"(ent.x), "r"(ent.y) : "memory");
         }
@@ -635,7 +693,7 @@ __device__ __forceinline__ void decode_blocks(const DecodeArgs &a, Sink &sink, u
     const uint32_t wtot = grp + C::kGrpWtot;  // 4 warp totals
     const uint32_t mb_in = grp + C::kGrpMbar, mb_sm = grp + C::kGrpMbar + 8u;
     const uint32_t *cnt_lane = reinterpret_cast<const uint32_t *>(smem + kOffCountRep) + (lane % kCountCopies);
-    const uint2 *sym_lane = reinterpret_cast<const uint2 *>(smem + kOffSymRep) + (lane % C::kSymCopies);
+    const uint2 *sym_lane = reinterpret_cast<const uint2 *>(smem + C::kOffSymRep) + (lane % C::kSymCopies);
     uint32_t *buf = reinterpret_cast<uint32_t *>(smem + C::kOffGroups + group * C::kGroupBytes);
     uint32_t my_err = 0;
 
@@ -694,9 +752,9 @@ __device__ __forceinline__ void decode_blocks(const DecodeArgs &a, Sink &sink, u
         const Chain A = make_chain(bswap32(v.x), bswap32(v.y), bswap32(v.z), gapA, endA, my_err);
         const Chain B = make_chain(bswap32(v.z), bswap32(v.w), bswap32(nextw), gapB, endB, my_err);
 
-        // ---- pass 1: count the codes of both chains
+        // ---- pass 1: count the codes of both chains (or read the stored counts)
         uint32_t cA, cB;
-        count_pass<kLong>(A, B, cnt_lane, sh1, s_lim, w1 + 1u, max_len, cA, cB, my_err);
+        chain_counts<C, kLong>(A, B, grp, lt, cnt_lane, sh1, s_lim, w1 + 1u, max_len, cA, cB, my_err);
 
         // ---- block scan: warp inclusive scan, then across the group's warps
         const uint32_t cnt = cA + cB;
@@ -741,8 +799,9 @@ __device__ __forceinline__ void decode_blocks(const DecodeArgs &a, Sink &sink, u
         // ---- pass 2: decode both chains again into the buffer
         if (ok) {
             const uint32_t startA = (s - base) + wpre + incl - cnt;  // buffer index of A's first code
-            decode_pass<kLong, C::kSymCopies, C::kSbufBytes>(A, B, startA, cA, startA + cA, cB, buf, sb, sym_lane, sh2, s_lim, s_offs, s_symrot,
-                        w2 + 1u, max_len);
+            decode_pass<kLong, !C::kCountTable, C::kSymCopies, C::kSbufBytes>(
+                A, B, startA, cA, startA + cA, cB, buf, sb, sym_lane, sh2, s_lim, s_offs, s_symrot, w2 + 1u, max_len,
+                my_err);
         }
         group_barrier(group);
 
@@ -819,7 +878,7 @@ __global__ void __launch_bounds__(C::kCtaThreads, 1) df11_gather_kernel(const Ga
     const uint32_t mb_in = grp + C::kGrpMbar;
     const uint32_t aux = grp + C::kGrpAux;
     const uint32_t *cnt_lane = reinterpret_cast<const uint32_t *>(smem + kOffCountRep) + (lane % kCountCopies);
-    const uint2 *sym_lane = reinterpret_cast<const uint2 *>(smem + kOffSymRep) + (lane % C::kSymCopies);
+    const uint2 *sym_lane = reinterpret_cast<const uint2 *>(smem + C::kOffSymRep) + (lane % C::kSymCopies);
     uint32_t *buf = reinterpret_cast<uint32_t *>(smem + C::kOffGroups + group * C::kGroupBytes);
     uint32_t my_err = 0;
 
@@ -886,7 +945,7 @@ __global__ void __launch_bounds__(C::kCtaThreads, 1) df11_gather_kernel(const Ga
             const Chain B = make_chain(bswap32(v.z), bswap32(v.w), bswap32(nextw), gapB, endB, my_err);
 
             uint32_t cA, cB;
-            count_pass<kLong>(A, B, cnt_lane, sh1, s_lim, w1 + 1u, max_len, cA, cB, my_err);
+            chain_counts<C, kLong>(A, B, grp, lt, cnt_lane, sh1, s_lim, w1 + 1u, max_len, cA, cB, my_err);
             const uint32_t cnt = cA + cB;
             uint32_t incl = cnt;
 #pragma unroll
@@ -909,8 +968,9 @@ __global__ void __launch_bounds__(C::kCtaThreads, 1) df11_gather_kernel(const Ga
             if (!ok && lt == 0) my_err |= range_ok ? DF11_KERR_COUNT_MISMATCH : DF11_KERR_BAD_BLOCK;
             if (ok) {
                 const uint32_t startA = (s - base) + wpre + incl - cnt;
-                decode_pass<kLong, C::kSymCopies, C::kSbufBytes>(A, B, startA, cA, startA + cA, cB, buf, sb, sym_lane, sh2, s_lim, s_offs,
-                                   s_symrot, w2 + 1u, max_len);
+                decode_pass<kLong, !C::kCountTable, C::kSymCopies, C::kSbufBytes>(
+                    A, B, startA, cA, startA + cA, cB, buf, sb, sym_lane, sh2, s_lim, s_offs, s_symrot, w2 + 1u,
+                    max_len, my_err);
             }
             group_barrier(group);
             if (ok) {  // the row's part of this block, element by element
@@ -1258,7 +1318,10 @@ df11_status prepare_device(int *sm_count) {
     if (!g_attr_set[dev].load(std::memory_order_acquire)) {
         if (set_smem_attr<CfgTypical, false>() != cudaSuccess || set_smem_attr<CfgTypical, true>() != cudaSuccess ||
             set_smem_attr<CfgWide, false>() != cudaSuccess || set_smem_attr<CfgWide, true>() != cudaSuccess ||
-            set_smem_attr<CfgDense, false>() != cudaSuccess || set_smem_attr<CfgDense, true>() != cudaSuccess)
+            set_smem_attr<CfgDense, false>() != cudaSuccess || set_smem_attr<CfgDense, true>() != cudaSuccess ||
+            set_smem_attr<CfgTypicalC, false>() != cudaSuccess || set_smem_attr<CfgTypicalC, true>() != cudaSuccess ||
+            set_smem_attr<CfgWideC, false>() != cudaSuccess || set_smem_attr<CfgWideC, true>() != cudaSuccess ||
+            set_smem_attr<CfgDenseC, false>() != cudaSuccess || set_smem_attr<CfgDenseC, true>() != cudaSuccess)
             return DF11_ERR_CUDA;
         g_attr_set[dev].store(1, std::memory_order_release);
     }
@@ -1275,13 +1338,23 @@ void launch(const DecodeArgs &a, uint64_t n_blocks, int sms, cudaStream_t stream
     df11_decode_kernel<C, kLong><<<grid, C::kCtaThreads, C::kSmemBytes, stream>>>(a);
 }
 
+struct DecodeLaunch {
+    const DecodeArgs &a;
+    uint64_t n_blocks;
+    int sms;
+    cudaStream_t s;
+    template <class C, bool kLong>
+    void go() { launch<C, kLong>(a, n_blocks, sms, s); }
+};
+
 // Checks a device tensor for a decode launch and fills the kernel arguments.
 df11_status prepare_args(const df11_tensor *t, DecodeArgs &a) {
     if (!t->enc || !t->sm || !t->gaps || !t->block_start || !t->lut) return DF11_ERR_INVALID_ARG;
     if (!aligned16(t->enc) || !aligned16(t->sm) || !aligned16(t->gaps) || !aligned16(t->lut) ||
-        !aligned16(t->block_start))
+        !aligned16(t->block_start) || !aligned16(t->counts))
         return DF11_ERR_INVALID_ARG;
     a.enc = t->enc;
+    a.counts = t->counts;  // NULL: the kernel runs the count pass
     a.sm = t->sm;
     a.gaps = t->gaps;
     a.bstart = t->block_start;
@@ -1299,14 +1372,34 @@ df11_status prepare_args(const df11_tensor *t, DecodeArgs &a) {
 // Which instance decodes a tensor: codes no longer than both table windows
 // never take the long-code path; a block's buffer span is at most its code
 // count + 15, and the instance with the smallest buffers that holds it is
-// taken (smaller buffers leave room for a second symbol-table copy).
-enum class Inst { kTypical, kWide, kDense };
+// taken (smaller buffers leave room for a second symbol-table copy); a
+// tensor with stored per-thread counts takes the instances without the
+// count pass.
+enum class Inst { kTypical, kWide, kDense, kTypicalC, kWideC, kDenseC };
 void pick_instance(const df11_tensor *t, Inst &inst, bool &lng) {
     uint32_t max_len = 0;
     for (int k = 0; k < 256; ++k) max_len = t->code_len[k] > max_len ? t->code_len[k] : max_len;
     lng = max_len > (uint32_t)(kW1Max < kW2Max ? kW1Max : kW2Max);
     const uint64_t need = (uint64_t)t->max_block_codes + 15u;
-    inst = need <= CfgTypical::kBufSyms ? Inst::kTypical : need <= CfgWide::kBufSyms ? Inst::kWide : Inst::kDense;
+    if (t->counts)
+        inst = need <= CfgTypicalC::kBufSyms ? Inst::kTypicalC : need <= CfgWideC::kBufSyms ? Inst::kWideC
+                                                                                          : Inst::kDenseC;
+    else
+        inst = need <= CfgTypical::kBufSyms ? Inst::kTypical : need <= CfgWide::kBufSyms ? Inst::kWide
+                                                                                       : Inst::kDense;
+}
+
+// Calls f.go<C, kLong>() for the picked instance.
+template <class F>
+void dispatch(Inst inst, bool lng, F f) {
+    switch (inst) {
+        case Inst::kTypical: lng ? f.template go<CfgTypical, true>() : f.template go<CfgTypical, false>(); break;
+        case Inst::kWide: lng ? f.template go<CfgWide, true>() : f.template go<CfgWide, false>(); break;
+        case Inst::kDense: lng ? f.template go<CfgDense, true>() : f.template go<CfgDense, false>(); break;
+        case Inst::kTypicalC: lng ? f.template go<CfgTypicalC, true>() : f.template go<CfgTypicalC, false>(); break;
+        case Inst::kWideC: lng ? f.template go<CfgWideC, true>() : f.template go<CfgWideC, false>(); break;
+        case Inst::kDenseC: lng ? f.template go<CfgDenseC, true>() : f.template go<CfgDenseC, false>(); break;
+    }
 }
 
 df11_status launch_decode(const df11_tensor *t, uint16_t *out, uint32_t *err_word, void *stream) {
@@ -1328,16 +1421,7 @@ df11_status launch_decode(const df11_tensor *t, uint16_t *out, uint32_t *err_wor
     Inst inst;
     bool lng;
     pick_instance(t, inst, lng);
-    if (inst == Inst::kTypical) {
-        if (lng) launch<CfgTypical, true>(a, t->n_blocks, sms, s);
-        else launch<CfgTypical, false>(a, t->n_blocks, sms, s);
-    } else if (inst == Inst::kWide) {
-        if (lng) launch<CfgWide, true>(a, t->n_blocks, sms, s);
-        else launch<CfgWide, false>(a, t->n_blocks, sms, s);
-    } else {
-        if (lng) launch<CfgDense, true>(a, t->n_blocks, sms, s);
-        else launch<CfgDense, false>(a, t->n_blocks, sms, s);
-    }
+    dispatch(inst, lng, DecodeLaunch{a, t->n_blocks, sms, s});
     if (cudaGetLastError() != cudaSuccess) return DF11_ERR_CUDA;
     return DF11_OK;
 }
@@ -1348,6 +1432,14 @@ void launch_gather(const GatherArgs &g, int sms, cudaStream_t stream) {
     const unsigned grid = (unsigned)(ctas_needed < (uint64_t)sms ? ctas_needed : (uint64_t)sms);
     df11_gather_kernel<C, kLong><<<grid, C::kCtaThreads, C::kSmemBytes, stream>>>(g);
 }
+
+struct GatherLaunch {
+    const GatherArgs &g;
+    int sms;
+    cudaStream_t s;
+    template <class C, bool kLong>
+    void go() { launch_gather<C, kLong>(g, sms, s); }
+};
 
 df11_status launch_rows(const df11_tensor *t, uint64_t row_len, const uint32_t *rows, uint32_t n_rows, uint16_t *out,
                         uint32_t *err_word, void *stream) {
@@ -1374,16 +1466,7 @@ df11_status launch_rows(const df11_tensor *t, uint64_t row_len, const uint32_t *
     Inst inst;
     bool lng;
     pick_instance(t, inst, lng);
-    if (inst == Inst::kTypical) {
-        if (lng) launch_gather<CfgTypical, true>(g, sms, s);
-        else launch_gather<CfgTypical, false>(g, sms, s);
-    } else if (inst == Inst::kWide) {
-        if (lng) launch_gather<CfgWide, true>(g, sms, s);
-        else launch_gather<CfgWide, false>(g, sms, s);
-    } else {
-        if (lng) launch_gather<CfgDense, true>(g, sms, s);
-        else launch_gather<CfgDense, false>(g, sms, s);
-    }
+    dispatch(inst, lng, GatherLaunch{g, sms, s});
     if (cudaGetLastError() != cudaSuccess) return DF11_ERR_CUDA;
     return DF11_OK;
 }
@@ -1396,17 +1479,18 @@ void launch_gemv_inst(const GemvArgs &g, uint64_t blocks_est, int sms, cudaStrea
 }
 
 template <uint32_t TM>
+struct GemvLaunch {
+    const GemvArgs &g;
+    uint64_t blocks_est;
+    int sms;
+    cudaStream_t s;
+    template <class C, bool kLong>
+    void go() { launch_gemv_inst<C, kLong, TM>(g, blocks_est, sms, s); }
+};
+
+template <uint32_t TM>
 void launch_gemv_tm(const GemvArgs &g, Inst inst, bool lng, uint64_t blocks_est, int sms, cudaStream_t s) {
-    if (inst == Inst::kTypical) {
-        if (lng) launch_gemv_inst<CfgTypical, true, TM>(g, blocks_est, sms, s);
-        else launch_gemv_inst<CfgTypical, false, TM>(g, blocks_est, sms, s);
-    } else if (inst == Inst::kWide) {
-        if (lng) launch_gemv_inst<CfgWide, true, TM>(g, blocks_est, sms, s);
-        else launch_gemv_inst<CfgWide, false, TM>(g, blocks_est, sms, s);
-    } else {
-        if (lng) launch_gemv_inst<CfgDense, true, TM>(g, blocks_est, sms, s);
-        else launch_gemv_inst<CfgDense, false, TM>(g, blocks_est, sms, s);
-    }
+    dispatch(inst, lng, GemvLaunch<TM>{g, blocks_est, sms, s});
 }
 
 // Multiply-shift division by d (1 <= d < 2^28) for dividends q < 2^28: with

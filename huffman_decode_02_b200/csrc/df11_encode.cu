@@ -184,7 +184,14 @@ struct PackArgs {
     uint64_t n_threads, n_blocks;
     uint8_t *enc, *sm, *gaps;
     uint32_t *bstart;
+    uint32_t *counts;  // per-thread code counts, 4 per word (NULL: not written)
 };
+
+// Adds a run of n code starts in format thread t to its count byte (a count
+// never passes 64, so the bytes of a word never carry into each other).
+__device__ __forceinline__ void add_count(uint32_t *counts, uint64_t t, uint32_t n) {
+    if (counts && n) atomicAdd(counts + (t >> 2), n << (8u * (uint32_t)(t & 3u)));
+}
 
 __global__ void __launch_bounds__(kEncThreads) pack_kernel(const PackArgs a, const CodeTables ct) {
     __shared__ uint32_t code[256];
@@ -212,11 +219,19 @@ __global__ void __launch_bounds__(kEncThreads) pack_kernel(const PackArgs a, con
 
     uint64_t cur = 0, word = p >> 6;
     uint32_t used = (uint32_t)(p & 63u);
+    uint64_t run_t = p >> 6;  // format thread of the current run of code starts
+    uint32_t run_n = 0;
 #pragma unroll
     for (uint32_t j = 0; j < kPer; ++j) {
         if (j >= cnt) break;
         const uint32_t e = exponent_of(wv[j]);
         const uint32_t l = len[e], c = code[e];
+        if ((p >> 6) != run_t) {
+            add_count(a.counts, run_t, run_n);
+            run_t = p >> 6;
+            run_n = 0;
+        }
+        ++run_n;
         // the first code starting at or after a thread / block boundary
         if ((first_elem || (p >> 6) > (p_prev >> 6)) && (p >> 6) < a.n_threads)
             put_gap(a.gaps, p >> 6, (uint32_t)(p & 63u));
@@ -245,6 +260,7 @@ __global__ void __launch_bounds__(kEncThreads) pack_kernel(const PackArgs a, con
         p += l;
     }
     if (used) or_word64(a.enc, a.enc_words, word, cur);
+    add_count(a.counts, run_t, run_n);
     if (i0 + cnt == a.n) {
         // the end of the stream counts as a code start; then the sentinel
         if ((p >> 6) > (p_prev >> 6) && (p >> 6) < a.n_threads) put_gap(a.gaps, p >> 6, (uint32_t)(p & 63u));
@@ -331,7 +347,7 @@ df11_status df11_encode_device_size(const uint16_t *w, uint64_t n, const df11_pa
     }
     st = df11::plan_from_histogram(count, n, p, hdr);
     if (st != DF11_OK) return st;
-    hdr->enc = hdr->sm = hdr->gaps = hdr->lut = nullptr;
+    hdr->enc = hdr->sm = hdr->gaps = hdr->lut = hdr->counts = nullptr;
     hdr->block_start = nullptr;
     return DF11_OK;
 }
@@ -341,7 +357,7 @@ df11_status df11_encode_device(const uint16_t *w, uint64_t n, df11_tensor *io, v
     if (!io || io->n_elems != n) return DF11_ERR_INVALID_ARG;
     if (!io->enc || !io->sm || !io->gaps || !io->block_start || !io->lut) return DF11_ERR_INVALID_ARG;
     if (((uintptr_t)io->enc & 15u) || ((uintptr_t)io->sm & 15u) || ((uintptr_t)io->gaps & 15u) ||
-        ((uintptr_t)io->block_start & 15u) || ((uintptr_t)io->lut & 15u))
+        ((uintptr_t)io->block_start & 15u) || ((uintptr_t)io->lut & 15u) || ((uintptr_t)io->counts & 15u))
         return DF11_ERR_INVALID_ARG;
     // the scalar fields must be those df11_encode_device_size planned
     {
@@ -360,7 +376,8 @@ df11_status df11_encode_device(const uint16_t *w, uint64_t n, df11_tensor *io, v
     if (cudaMemsetAsync(io->enc, 0, io->enc_bytes, s) != cudaSuccess ||
         cudaMemsetAsync(io->sm, 0, io->sm_bytes, s) != cudaSuccess ||
         cudaMemsetAsync(io->gaps, 0, io->gaps_bytes, s) != cudaSuccess ||
-        cudaMemsetAsync(io->block_start, 0, io->block_start_bytes, s) != cudaSuccess)
+        cudaMemsetAsync(io->block_start, 0, io->block_start_bytes, s) != cudaSuccess ||
+        (io->counts && cudaMemsetAsync(io->counts, 0, io->counts_bytes, s) != cudaSuccess))
         return DF11_ERR_CUDA;
     std::vector<uint8_t> lut(io->lut_bytes);
     df11::host_build_luts(io->code_len, lut.data());
@@ -395,6 +412,7 @@ df11_status df11_encode_device(const uint16_t *w, uint64_t n, df11_tensor *io, v
         a.sm = io->sm;
         a.gaps = io->gaps;
         a.bstart = io->block_start;
+        a.counts = reinterpret_cast<uint32_t *>(io->counts);
         pack_kernel<<<(unsigned)n_tiles, kEncThreads, 0, s>>>(a, ct);
         const uint64_t fb = std::max<uint64_t>(1, std::min<uint64_t>((io->n_blocks + 255u) / 256u, 4u * (uint64_t)sms));
         finish_kernel<<<(unsigned)fb, 256, 0, s>>>(io->block_start, io->n_blocks, tile_off, n_tiles, most_d, total_d);

@@ -363,6 +363,7 @@ df11_status df11::plan_from_histogram(const uint64_t count[256], uint64_t n, con
     t->gaps_bytes = ((padded_threads * 5 + 7) / 8 + 15) / 16 * 16 + 16;
     t->block_start_bytes = ((t->n_blocks + 1) * 4 + 15) / 16 * 16 + 16;
     t->lut_bytes = df11::kLutBytes;
+    t->counts_bytes = padded_threads + 16;
     return DF11_OK;
 }
 
@@ -417,6 +418,14 @@ df11_status fill_arrays(const Sequence &seq, df11_tensor *t) {
     // afterwards: head = first byte when the chunk starts mid-byte, tail =
     // last partial byte when it ends mid-byte.
     std::vector<uint8_t> head(n_chunks, 0), tail(n_chunks, 0), head_set(n_chunks, 0);
+    // Per-thread code counts (when asked for): a chunk writes the counts of
+    // the threads only it starts codes in; its first and last runs (threads
+    // it may share with its neighbours) are kept aside and added afterwards.
+    uint8_t *counts = t->counts;
+    if (counts) std::memset(counts, 0, (size_t)t->counts_bytes);
+    constexpr uint64_t kNoThread = ~0ull;
+    std::vector<uint64_t> run_first_t(n_chunks, kNoThread), run_last_t(n_chunks, kNoThread);
+    std::vector<uint32_t> run_first_n(n_chunks, 0), run_last_n(n_chunks, 0);
     uint8_t *enc = t->enc;
     uint8_t *sm = t->sm;
     uint32_t *bstart = t->block_start;
@@ -430,11 +439,25 @@ df11_status fill_arrays(const Sequence &seq, df11_tensor *t) {
         unsigned nacc = (unsigned)(b0 & 7);
         uint8_t *dst = enc + (b0 >> 3);
         bool at_head = (b0 & 7) != 0;
+        uint64_t run_t = kNoThread;  // thread of the current run of code starts
+        uint32_t run_n = 0;
         seq.segments(lo, hi, [&](const uint16_t *p, uint64_t g0, uint64_t m) {
             for (uint64_t i = 0; i < m; ++i) {
                 const uint16_t w = p[i];
                 const unsigned e = exponent_of(w);
                 const unsigned l = len[e];
+                if (counts) {
+                    const uint64_t th = pos / span;
+                    if (th != run_t) {
+                        if (run_t != kNoThread) {
+                            if (run_first_t[c] == kNoThread) { run_first_t[c] = run_t; run_first_n[c] = run_n; }
+                            else counts[run_t] = (uint8_t)run_n;
+                        }
+                        run_t = th;
+                        run_n = 0;
+                    }
+                    ++run_n;
+                }
                 while (tn < n_threads && tn * span <= pos) { gaps[tn] = (uint8_t)(pos - tn * span); ++tn; }
                 while (bn < n_blocks && bn * block_span <= pos) { bstart[bn] = (uint32_t)(g0 + i); ++bn; }
                 sm[g0 + i] = (uint8_t)(((w >> 8) & 0x80u) | (w & 0x7Fu));
@@ -454,8 +477,17 @@ df11_status fill_arrays(const Sequence &seq, df11_tensor *t) {
         while (bn < n_blocks && bn * block_span < b1) { bstart[bn] = (uint32_t)hi; ++bn; }
         if (nacc) tail[c] = (uint8_t)(acc << (8 - nacc));
         else tail[c] = 0;
+        if (counts && run_t != kNoThread) {
+            if (run_first_t[c] == kNoThread) { run_first_t[c] = run_t; run_first_n[c] = run_n; }
+            else { run_last_t[c] = run_t; run_last_n[c] = run_n; }
+        }
         (void)dst;
     });
+    if (counts)
+        for (size_t c = 0; c < n_chunks; ++c) {
+            if (run_first_t[c] != kNoThread) counts[run_first_t[c]] = (uint8_t)(counts[run_first_t[c]] + run_first_n[c]);
+            if (run_last_t[c] != kNoThread) counts[run_last_t[c]] = (uint8_t)(counts[run_last_t[c]] + run_last_n[c]);
+        }
     // Shared bytes are never written whole by any chunk: clear them, then OR
     // in every partial contribution (a chunk that never completed its first
     // byte has all of its bits in its tail).
@@ -595,6 +627,7 @@ df11_status df11_validate(const df11_tensor *t) {
     if (t->gaps_bytes < (padded * 5 + 7) / 8 + 16) return DF11_ERR_INVALID_ARG;
     if (t->block_start_bytes < ((t->n_blocks + 1) * 4 + 15) / 16 * 16 + 16) return DF11_ERR_INVALID_ARG;
     if (t->lut_bytes < df11::kLutBytes) return DF11_ERR_INVALID_ARG;
+    if (t->counts && t->counts_bytes < padded + 16) return DF11_ERR_INVALID_ARG;
     if (t->max_block_codes > (uint32_t)df11::kMaxCodesPerBlock || t->reserved2 != 0) return DF11_ERR_CORRUPT;
     // Kraft: sum 2^-len <= 1 and lengths within the cap
     uint64_t kraft = 0;

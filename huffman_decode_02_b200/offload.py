@@ -30,11 +30,16 @@ def _torch():
     return torch
 
 
-def _slot_arrays(blocks: Sequence[DF11Tensor], device):
+def _common_arrays(blocks: Sequence[DF11Tensor]) -> list[str]:
+    """The arrays every block carries (the per-thread counts are optional)."""
+    return [k for k in _ARRAYS if all(k in b.arrays for b in blocks)]
+
+
+def _slot_arrays(blocks: Sequence[DF11Tensor], keys, device):
     """Two device slots, each large enough for any block's arrays."""
     torch = _torch()
-    size = {k: max(int(b.arrays[k].numel()) * b.arrays[k].element_size() for b in blocks) for k in _ARRAYS}
-    return [{k: torch.empty(max(size[k], 16), dtype=torch.uint8, device=device) for k in _ARRAYS} for _ in range(2)]
+    size = {k: max(int(b.arrays[k].numel()) * b.arrays[k].element_size() for b in blocks) for k in keys}
+    return [{k: torch.empty(max(size[k], 16), dtype=torch.uint8, device=device) for k in keys} for _ in range(2)]
 
 
 class BlockStreamer:
@@ -49,24 +54,29 @@ class BlockStreamer:
         for b in blocks:
             if b.device != "cpu":
                 raise ValueError("blocks must be host tensors (encode_multi(..., pinned=True))")
-            if not all(hasattr(b.arrays[k], "is_pinned") and b.arrays[k].is_pinned() for k in _ARRAYS):
+            if not all(hasattr(a, "is_pinned") and a.is_pinned() for a in b.arrays.values()):
                 raise ValueError("blocks must be in pinned host memory (encode_multi(..., pinned=True))")
         self.blocks = list(blocks)
+        self.keys = _common_arrays(self.blocks)
         self.device = torch.device(device)
-        self.slots = _slot_arrays(self.blocks, self.device)
+        self.slots = _slot_arrays(self.blocks, self.keys, self.device)
         n_max = max(b.n_elems for b in self.blocks)
         self.scratch = torch.empty(max(n_max, 8), dtype=torch.bfloat16, device=self.device)
         self.err = torch.zeros(1, dtype=torch.int32, device=self.device)
         self.copy_stream = torch.cuda.Stream(device=self.device)
-        self.h2d_bytes = [sum(int(b.arrays[k].numel()) * b.arrays[k].element_size() for k in _ARRAYS)
+        self.h2d_bytes = [sum(int(b.arrays[k].numel()) * b.arrays[k].element_size() for k in self.keys)
                           for b in self.blocks]
 
     def _device_view(self, b: DF11Tensor, slot: int) -> DF11Tensor:
-        arrays = {k: self.slots[slot][k][: int(b.arrays[k].numel()) * b.arrays[k].element_size()] for k in _ARRAYS}
-        return DF11Tensor(_Tensor.from_buffer_copy(b.desc), arrays, str(self.device), b.shapes, b.offsets)
+        arrays = {k: self.slots[slot][k][: int(b.arrays[k].numel()) * b.arrays[k].element_size()]
+                  for k in self.keys}
+        desc = _Tensor.from_buffer_copy(b.desc)
+        if "counts" not in self.keys:
+            desc.counts_bytes = 0
+        return DF11Tensor(desc, arrays, str(self.device), b.shapes, b.offsets)
 
     def _copy(self, b: DF11Tensor, slot: int):
-        for k in _ARRAYS:
+        for k in self.keys:
             src = b.arrays[k].view(_torch().uint8).reshape(-1)
             self.slots[slot][k][: src.numel()].copy_(src, non_blocking=True)
 

@@ -100,6 +100,16 @@ typedef struct df11_params {
  *  block_start u32 per thread block: index of the first element decoded by
  *              that block, plus a final entry equal to n_elems; zero-padded
  *              to block_start_bytes = round_up(4 * (n_blocks + 1), 16) + 16.
+ *  counts      OPTIONAL per-thread code counts, one byte per thread: how
+ *              many codes start in the thread's n bytes (0..64; threads past
+ *              the stream 0), n_blocks * T bytes, zero-padded to
+ *              counts_bytes = n_blocks * T + 16.  This is the number the
+ *              first pass of the two-step kernel finds ("Noyau GPU en deux
+ *              etapes et metadonnees auxiliaires"); stored, it lets the
+ *              decoder skip that pass (one decoding pass, then the block
+ *              prefix sum of the stored counts).  It is derived data: the
+ *              encoders write it when counts is non-NULL, and a decode with
+ *              counts == NULL runs the two passes of the pages.
  *  lut         decode tables derived from code_len (layout private to the
  *              library, lut_bytes long): a multi-code LUT on the first W
  *              bits of a window, a code-count LUT, and canonical limits for
@@ -111,8 +121,9 @@ typedef struct df11_params {
  *              span exceeds the buffer is reported as DF11_KERR_BAD_BLOCK).
  *
  * For the encode calls the pointers are HOST arrays the caller allocated
- * with the *_bytes sizes returned by the size call.  For the decode calls
- * they are DEVICE arrays holding the same bytes, each 16-byte aligned. */
+ * with the *_bytes sizes returned by the size call (counts may be NULL:
+ * not written).  For the decode calls they are DEVICE arrays holding the
+ * same bytes, each 16-byte aligned (counts may be NULL). */
 typedef struct df11_tensor {
     uint64_t n_elems;
     uint64_t total_bits; /* bits of code in enc (padding excluded) */
@@ -127,11 +138,13 @@ typedef struct df11_tensor {
     uint64_t gaps_bytes;
     uint64_t block_start_bytes;
     uint64_t lut_bytes;
+    uint64_t counts_bytes;
     uint8_t *enc;
     uint8_t *sm;
     uint8_t *gaps;
     uint32_t *block_start;
     uint8_t *lut;
+    uint8_t *counts; /* optional (NULL) */
 } df11_tensor;
 
 /* ------------------------------------------------------------------ host */
@@ -139,7 +152,7 @@ typedef struct df11_tensor {
 /* ABI version of this header (bumped on any layout change) and
  * sizeof(df11_tensor) as compiled into the library, so that bindings can
  * check their mirror of the struct. */
-#define DF11_ABI_VERSION 2u
+#define DF11_ABI_VERSION 3u
 uint32_t df11_abi_version(void);
 size_t df11_sizeof_tensor(void);
 
@@ -162,9 +175,10 @@ df11_status df11_exponent_histogram(const uint16_t *const *mats, const uint64_t 
 df11_status df11_encode_size(const uint16_t *bf16, uint64_t n, const df11_params *params,
                              df11_tensor *t);
 
-/* Fill pass: writes enc, sm, gaps, block_start and lut into the caller's
- * host arrays *t points to (sizes from df11_encode_size on the same data).
- * Arrays are fully written, padding included. */
+/* Fill pass: writes enc, sm, gaps, block_start, lut and (when non-NULL)
+ * counts into the caller's host arrays *t points to (sizes from
+ * df11_encode_size on the same data).  Arrays are fully written, padding
+ * included. */
 df11_status df11_encode(const uint16_t *bf16, uint64_t n, df11_tensor *t);
 
 /* Same two passes for k matrices encoded as ONE stream with ONE shared table
@@ -177,7 +191,8 @@ df11_status df11_encode_multi(const uint16_t *const *mats, const uint64_t *sizes
                               df11_tensor *t);
 
 /* Host-side consistency check of a tensor's scalar fields and sizes
- * (no array contents are read). */
+ * (no array contents are read; counts_bytes is checked only when counts is
+ * non-NULL). */
 df11_status df11_validate(const df11_tensor *t);
 
 /* --------------------------------------------------------- device encoder */
@@ -194,14 +209,16 @@ df11_status df11_validate(const df11_tensor *t);
 uint64_t df11_encode_device_scratch_bytes(uint64_t n);
 
 /* Size pass: w is a DEVICE array of n BF16 values (16-byte aligned; a block's
- * matrices concatenated) on the current device (else DF11_ERR_INVALID_ARG).  Runs the histogram on `stream`, synchronises it,
- * plans the code and fills *hdr (sizes, code lengths, counts) as
- * df11_encode_size does; array pointers are left NULL. */
+ * matrices concatenated) on the current device (else DF11_ERR_INVALID_ARG).
+ * Runs the histogram on `stream`, synchronises it, plans the code and fills
+ * *hdr (sizes, code lengths) as df11_encode_size does; array pointers are
+ * left NULL. */
 df11_status df11_encode_device_size(const uint16_t *w, uint64_t n, const df11_params *params, df11_tensor *hdr,
                                     void *scratch, uint64_t scratch_bytes, void *stream);
 
-/* Fill pass: io from df11_encode_device_size with its five array pointers set
- * to caller-allocated DEVICE buffers of the planned sizes (16-byte aligned).
+/* Fill pass: io from df11_encode_device_size with its array pointers set to
+ * caller-allocated DEVICE buffers of the planned sizes (16-byte aligned;
+ * counts may stay NULL, and is then not written).
  * Packs everything on `stream` (the decode tables are copied from the host)
  * and synchronises it; sets io->max_block_codes.  DF11_ERR_INVALID_ARG if
  * w no longer matches the planned code (e.g. changed since the size pass). */
@@ -262,7 +279,7 @@ df11_status df11_decode_block(const df11_tensor *blk, const uint64_t *mat_offset
  * format keeps only each thread block's first output index ("Noyau GPU en deux
  * etapes et metadonnees auxiliaires"), so the kernel finds the thread blocks
  * covering a row by searching those indices, decodes them in full (count
- * pass, scan, decode pass) and writes only the row's elements.
+ * pass or stored counts, scan, decoding pass) and writes only the row's elements.
  *  rows: DEVICE uint32 row indices (repeats allowed); an index >= R sets
  *        DF11_KERR_BAD_ROW and leaves that output row unwritten.
  *  row_len: > 0 and dividing t->n_elems; else DF11_ERR_INVALID_ARG.

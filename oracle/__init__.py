@@ -16,7 +16,9 @@ Functions (each cites its passage in ``df11_oracle.c``):
   length <= cap.
 * ``canonical_codes(lengths)`` -- canonical code values.
 * ``encode(w, lengths)`` -- (enc bytes, sign/mantissa bytes, total bits).
-* ``decode(enc, total_bits, sm, n, lengths)`` -- bit-serial tree walk.
+* ``decode(enc, total_bits, sm, n, lengths)`` -- bit-serial tree walk;
+  ``decode_range(enc, first_bit, end_bit, sm, n, lengths)`` -- the same on
+  one piece of a stream (a run of whole thread blocks).
 * ``aux(enc, total_bits, n, lengths, bytes_per_thread, threads_per_block)``
   -- gaps, per-thread counts and block starts recomputed from a stream.
 * ``pack_gaps(gaps)`` -- 5-bit packing of gaps.
@@ -96,6 +98,7 @@ def _load():
     lib.orc_is_prefix_free.argtypes = [_u8p]
     lib.orc_codes_prefix_free.argtypes = [_u32p, _u8p]
     lib.orc_decode.argtypes = [_u8p, u64, _u8p, u64, _u8p, _u16p]
+    lib.orc_decode_range.argtypes = [_u8p, u64, u64, _u8p, u64, _u8p, _u16p]
     lib.orc_aux.argtypes = [_u8p, u64, u64, _u8p, ctypes.c_uint32, ctypes.c_uint32,
                             _u8p, _u32p, _u32p, _u64p, _u64p]
     lib.orc_pack_gaps.argtypes = [_u8p, u64, _u8p, u64]
@@ -214,6 +217,25 @@ def decode(enc, total_bits_: int, sm, n: int, lengths) -> np.ndarray:
     out = np.zeros(max(1, n), dtype=np.uint16)
     _check(_load().orc_decode(_ptr(e, _u8p), int(total_bits_), _ptr(s, _u8p), int(n),
                               _ptr(l8, _u8p), _ptr(out, _u16p)), "decode")
+    return out[:n]
+
+
+def decode_range(enc, first_bit: int, end_bit: int, sm, n: int, lengths, out=None) -> np.ndarray:
+    """Decodes the n weights whose codes fill bits [first_bit, end_bit) of
+    ``enc``; ``sm`` holds those n weights' sign/mantissa bytes.  Writes into
+    ``out`` (uint16[n]) when given.  Releases the GIL while it runs (ctypes),
+    so pieces of one stream can be decoded on several host threads."""
+    e = np.ascontiguousarray(enc, dtype=np.uint8)
+    s = np.ascontiguousarray(sm, dtype=np.uint8)
+    l8 = np.ascontiguousarray(lengths, dtype=np.uint8)
+    if e.size == 0:
+        e = np.zeros(1, dtype=np.uint8)
+    if s.size == 0:
+        s = np.zeros(1, dtype=np.uint8)
+    if out is None:
+        out = np.zeros(max(1, n), dtype=np.uint16)
+    _check(_load().orc_decode_range(_ptr(e, _u8p), int(first_bit), int(end_bit), _ptr(s, _u8p), int(n),
+                                    _ptr(l8, _u8p), _ptr(out, _u16p)), "decode_range")
     return out[:n]
 
 

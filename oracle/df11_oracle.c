@@ -354,16 +354,22 @@ int orc_is_prefix_free(const uint8_t len[256]) {
     return rc == ORC_OK;
 }
 
-/* Decodes n weights.  Exponents come from the bit-serial tree walk, sign
- * and mantissa from their byte, and the BF16 word is reassembled.  Fails if
- * the stream hits a missing branch or does not end exactly at total_bits. */
-int orc_decode(const uint8_t *enc, uint64_t total_bits, const uint8_t *sm, uint64_t n,
-               const uint8_t len[256], uint16_t *out) {
+/* Decodes n weights whose codes occupy bits [first_bit, end_bit) of the
+ * stream.  Exponents come from the bit-serial tree walk, sign and mantissa
+ * from their byte, and the BF16 word is reassembled.  Fails if the stream
+ * hits a missing branch or does not end exactly at end_bit.  (A piece of a
+ * stream that starts at a thread block's first code -- its bit offset is
+ * the block's first bit plus its first thread's gap -- decodes on its own,
+ * which is what lets the GPU kernel's thread blocks work independently.) */
+int orc_decode_range(const uint8_t *enc, uint64_t first_bit, uint64_t end_bit, const uint8_t *sm, uint64_t n,
+                     const uint8_t len[256], uint16_t *out) {
     int rc;
-    if (n == 0) return total_bits == 0 ? ORC_OK : ORC_ERR_CORRUPT;
+    if (n == 0) return end_bit == first_bit ? ORC_OK : ORC_ERR_CORRUPT;
+    if (end_bit < first_bit) return ORC_ERR_ARG;
     orc_tree *t = build_tree(len, &rc);
     if (!t) return rc;
-    uint64_t pos = 0, i = 0;
+    const uint64_t total_bits = end_bit;
+    uint64_t pos = first_bit, i = 0;
     int node = 0;
     while (i < n) {
         if (pos >= total_bits) { free(t); return ORC_ERR_CORRUPT; }
@@ -378,6 +384,12 @@ int orc_decode(const uint8_t *enc, uint64_t total_bits, const uint8_t *sm, uint6
     }
     free(t);
     return pos == total_bits ? ORC_OK : ORC_ERR_CORRUPT;
+}
+
+/* Decodes a whole stream: n weights from bits [0, total_bits). */
+int orc_decode(const uint8_t *enc, uint64_t total_bits, const uint8_t *sm, uint64_t n,
+               const uint8_t len[256], uint16_t *out) {
+    return orc_decode_range(enc, 0, total_bits, sm, n, len, out);
 }
 
 /* ---------------------------------------------------------------------

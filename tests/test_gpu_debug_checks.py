@@ -57,9 +57,11 @@ def _cases():
 
 def test_decode_paths_without_bounds_errors(debug_lib):
     dev = _dev()
-    for name, w, p in _cases():
+    for name, w, p, counts in ((n, w, p, c) for n, w, p in _cases() for c in (True, False)):
         w = np.ascontiguousarray(w).reshape(-1).view(np.uint16)
         d = df11.encode(w, p).to(dev)
+        d = d if counts else d.without_counts()  # stored counts, and the count pass
+        name = f"{name}-{'counts' if counts else 'count-pass'}"
         np.testing.assert_array_equal(_bits(df11.decode(d)), w, err_msg=name)
         if w.size >= 64 and w.size % 64 == 0:  # as a 64-column matrix: row gather
             rows = torch.arange(0, w.size // 64, 7, dtype=torch.int32, device=dev)
@@ -75,9 +77,10 @@ def test_decode_paths_without_bounds_errors(debug_lib):
     mats = [workloads.normal_matrix(r, c, s, seed=i) for i, (r, c, s) in
             enumerate([(512, 256, 0.02), (64, 128, 0.03), (3, 7, 0.5)])]
     blk = df11.encode_multi(mats).to(dev)
-    scratch = df11.decode_block(blk)
-    for m, v in zip(mats, blk.views(scratch)):
-        np.testing.assert_array_equal(_bits(v).reshape(m.shape), m)
+    for b in (blk, blk.without_counts()):
+        scratch = df11.decode_block(b)
+        for m, v in zip(mats, b.views(scratch)):
+            np.testing.assert_array_equal(_bits(v).reshape(m.shape), m)
     for T in (1, 4):  # the fused product over the two 2-D matrices (in = 256, 128)
         xs = {j: torch.randn(T, mats[j].shape[1], generator=torch.Generator().manual_seed(j)).to(torch.bfloat16)
               .to(dev) for j in (0, 1)}

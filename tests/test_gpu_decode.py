@@ -33,19 +33,22 @@ def _oracle_decode(t: df11.DF11Tensor) -> np.ndarray:
 
 
 def _gpu_roundtrip(w, params=None, check_oracle=True):
+    """Both decode paths: with the stored per-thread counts (one decoding
+    pass) and without them (count pass, then decoding pass)."""
     dev = _dev()
     w = np.ascontiguousarray(w).reshape(-1).view(np.uint16)
     t = df11.encode(w, params)
+    assert t.has_counts
     d = t.to(dev)
-    out = df11.decode(d)
-    torch.cuda.synchronize()
-    got = _bits(out)
+    ref = _oracle_decode(t) if check_oracle else w
     if check_oracle:
-        ref = _oracle_decode(t)
         assert np.array_equal(ref, w)  # the oracle reproduces the input
+    got = None
+    for dd in (d, d.without_counts()):
+        out = df11.decode(dd)
+        torch.cuda.synchronize()
+        got = _bits(out)
         np.testing.assert_array_equal(got, ref)
-    else:
-        np.testing.assert_array_equal(got, w)
     return t, d, got
 
 
@@ -120,24 +123,48 @@ def test_decode_on_side_stream_and_repeat():
     np.testing.assert_array_equal(_bits(out), w.reshape(-1))
 
 
-def test_corrupt_block_start_is_reported():
+@pytest.mark.parametrize("counts", [True, False])
+def test_corrupt_block_start_is_reported(counts):
     dev = _dev()
     w = workloads.normal_matrix(512, 512, 0.02, seed=6)
     d = df11.encode(w).to(dev)
+    d = d if counts else d.without_counts()
     bs = d.arrays["block_start"].view(torch.int32)
     bs[3] += 5  # block 2 claims 5 more elements, block 3 5 fewer
     with pytest.raises(df11.CorruptStreamError):
         df11.decode(d)
 
 
-def test_corrupt_stream_bits_are_reported():
+@pytest.mark.parametrize("counts", [True, False])
+def test_corrupt_stream_bits_are_reported(counts):
     dev = _dev()
     w = workloads.normal_matrix(512, 512, 0.02, seed=8)
     d = df11.encode(w).to(dev)
+    d = d if counts else d.without_counts()
     enc = d.arrays["enc"]
     enc[1000:1100] ^= 0x5A  # scramble 100 bytes of codes
     with pytest.raises(df11.CorruptStreamError):
         df11.decode(d)
+
+
+@pytest.mark.parametrize("thread", [0, 5, 300, 1000])
+def test_corrupt_stored_count_is_reported(thread):
+    """A stored count off by one breaks its block's sum (reported by the
+    block check); two counts moved in opposite directions keep the sum, and
+    the chain's bit check reports them."""
+    dev = _dev()
+    w = workloads.normal_matrix(512, 512, 0.02, seed=10)
+    d = df11.encode(w).to(dev)
+    cnt = d.arrays["counts"]
+    cnt[thread] += 1
+    with pytest.raises(df11.CorruptStreamError):
+        df11.decode(d)
+    cnt[thread + 1] -= 1  # same block: the block's sum is right again
+    with pytest.raises(df11.CorruptStreamError):
+        df11.decode(d)
+    cnt[thread] -= 1
+    cnt[thread + 1] += 1  # restored
+    np.testing.assert_array_equal(_bits(df11.decode(d)), w.reshape(-1))
 
 
 def test_sign_mantissa_flip_changes_only_that_weight():
@@ -173,35 +200,37 @@ def test_bad_arguments_rejected():
 @pytest.mark.parametrize("cap", [12, 32])
 def test_config3_llama8b_block_full_size(cap):
     """The benchmark's workload, in the benchmark's launch configuration
-    (cap 12, the default), and with uncapped codes (cap 32, long-code path):
-    every element compared with the oracle's decode of the same stream."""
+    (cap 12, the default, stored counts), with uncapped codes (cap 32,
+    long-code path), and without the stored counts (count pass): every
+    element compared with the oracle's decode of the same stream."""
     dev = _dev()
     mats = workloads.llama8b_block(seed=0)
     blk = df11.encode_multi(mats, df11.Params(max_code_len=cap))
     assert blk.n_elems == 218_112_000
     d = blk.to(dev)
-    scratch = torch.empty(blk.n_elems, dtype=torch.bfloat16, device=dev)
-    df11.decode_block(d, scratch)
-    got = _bits(scratch)
     ref = _oracle_decode(blk)
-    np.testing.assert_array_equal(got, ref)
     np.testing.assert_array_equal(ref, np.concatenate([m.reshape(-1) for m in mats]))
+    scratch = torch.empty(blk.n_elems, dtype=torch.bfloat16, device=dev)
+    for dd in (d, d.without_counts()):
+        scratch.fill_(float("nan"))
+        df11.decode_block(dd, scratch)
+        np.testing.assert_array_equal(_bits(scratch), ref)
 
 
 @pytest.mark.slow
 @pytest.mark.parametrize("cap", [32, 12])
 def test_config4_heavy_tail_full_size(cap):
     """Long codes (cap 32: up to 27 bits, through the long-code path) and the
-    default 12-bit cap."""
+    default 12-bit cap; with and without the stored counts."""
     dev = _dev()
     w = workloads.heavy_tail_matrix(seed=4)
     t = df11.encode(w, df11.Params(max_code_len=cap))
     assert t.code_len.max() >= (20 if cap == 32 else 12)
     d = t.to(dev)
-    got = _bits(df11.decode(d))
     ref = _oracle_decode(t)
-    np.testing.assert_array_equal(got, ref)
     np.testing.assert_array_equal(ref, w.reshape(-1))
+    for dd in (d, d.without_counts()):
+        np.testing.assert_array_equal(_bits(df11.decode(dd)), ref)
 
 
 @pytest.mark.parametrize("offset_elems", [8, 16])
@@ -269,7 +298,7 @@ def test_maximum_size_tensor():
         assert bool(torch.all((got - ref).abs() <= (4096 + 32) * 2.0 ** -24 * mag + 1e-30)), off
     # the device encoder on the same weights: arrays identical to the host encoder's
     e = df11.encode_device(torch.from_numpy(w.view(np.int16)).to(dev).view(torch.bfloat16))
-    for k in ("enc", "sm", "gaps", "block_start", "lut"):
+    for k in ("enc", "sm", "gaps", "block_start", "lut", "counts"):
         nb = d.nbytes(k)
         assert e.nbytes(k) == nb and torch.equal(e.arrays[k][:nb], d.arrays[k][:nb]), k
 

@@ -75,12 +75,13 @@ def test_fused_block_all_matrices(T):
     d = df11.encode_multi(mats).to(dev)
     idx = [j for j, m in enumerate(mats) if m.ndim == 2]
     xs_np = {j: _x(T, mats[j].shape[1], 100 + j) for j in idx}
-    ys = df11.decode_gemv(d, {j: _bf16(xs_np[j]).to(dev) for j in idx})
-    torch.cuda.synchronize()
-    assert sorted(ys) == idx
-    for j in idx:
-        assert ys[j].shape == (T, mats[j].shape[0]) and ys[j].dtype == torch.float32
-        _check(ys[j], mats[j], xs_np[j])
+    for dd in (d, d.without_counts()):  # stored counts, and the count pass
+        ys = df11.decode_gemv(dd, {j: _bf16(xs_np[j]).to(dev) for j in idx})
+        torch.cuda.synchronize()
+        assert sorted(ys) == idx
+        for j in idx:
+            assert ys[j].shape == (T, mats[j].shape[0]) and ys[j].dtype == torch.float32
+            _check(ys[j], mats[j], xs_np[j])
 
 
 def test_fused_subset_accumulates_into_y():
@@ -148,10 +149,11 @@ def test_fused_other_instances(kind):
     need = t.desc.max_block_codes + 15
     assert (need > 8192) if kind == "dense" else (7152 < need <= 8192)
     d = t.to(dev)
-    for T in (1, 4):
-        xb = _x(T, 96, 40 + T)
-        y = df11.decode_gemv(d, {0: _bf16(xb).to(dev)})[0]
-        _check(y, w, xb)
+    for dd in (d, d.without_counts()):  # stored counts, and the count pass
+        for T in (1, 4):
+            xb = _x(T, 96, 40 + T)
+            y = df11.decode_gemv(dd, {0: _bf16(xb).to(dev)})[0]
+            _check(y, w, xb)
 
 
 def test_fused_argument_checks():

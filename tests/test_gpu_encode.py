@@ -13,7 +13,7 @@ pytestmark = pytest.mark.gpu
 import huffman_decode_02_b200 as df11  # noqa: E402
 
 FIELDS = ["n_elems", "total_bits", "n_threads", "n_blocks", "max_block_codes", "enc_bytes", "sm_bytes",
-          "gaps_bytes", "block_start_bytes", "lut_bytes"]
+          "gaps_bytes", "block_start_bytes", "lut_bytes", "counts_bytes"]
 
 
 def _dev():
@@ -30,7 +30,7 @@ def _same(host: df11.DF11Tensor, d: df11.DF11Tensor):
     for f in FIELDS:
         assert getattr(host.desc, f) == getattr(d.desc, f), f
     assert bytes(host.desc.code_len) == bytes(d.desc.code_len)
-    for k in ("enc", "sm", "gaps", "block_start", "lut"):
+    for k in ("enc", "sm", "gaps", "block_start", "lut", "counts"):
         a = host.host_array(k).view(np.uint8)[: host.nbytes(k)]
         b = d.host_array(k).view(np.uint8)[: d.nbytes(k)]
         np.testing.assert_array_equal(a, b, err_msg=k)

@@ -30,9 +30,10 @@ def test_rows_bit_exact(shape):
     rng = np.random.default_rng(shape[1])
     rows = np.concatenate([[0, shape[0] - 1, shape[0] // 2, shape[0] // 2],
                            rng.integers(0, shape[0], 200)]).astype(np.int32)
-    out = df11.decode_rows(d, shape[1], torch.from_numpy(rows).to(dev))
-    torch.cuda.synchronize()
-    np.testing.assert_array_equal(_rows_bits(out), w[rows])
+    for dd in (d, d.without_counts()):  # stored counts, and the count pass
+        out = df11.decode_rows(dd, shape[1], torch.from_numpy(rows).to(dev))
+        torch.cuda.synchronize()
+        np.testing.assert_array_equal(_rows_bits(out), w[rows])
 
 
 def test_rows_heavy_tail_long_codes():
@@ -46,8 +47,9 @@ def test_rows_heavy_tail_long_codes():
     assert t.code_len.max() > 12  # the long-code instance
     d = t.to(dev)
     rows = torch.from_numpy(rng.integers(0, 600, 100).astype(np.int32)).to(dev)
-    out = df11.decode_rows(d, w.shape[1], rows)
-    np.testing.assert_array_equal(_rows_bits(out), w[rows.cpu().numpy()])
+    for dd in (d, d.without_counts()):  # stored counts, and the count pass
+        out = df11.decode_rows(dd, w.shape[1], rows)
+        np.testing.assert_array_equal(_rows_bits(out), w[rows.cpu().numpy()])
 
 
 def test_bad_row_index_reported_other_rows_written():
@@ -115,6 +117,7 @@ def test_rows_other_instances(kind):
     assert (need > 8192) if kind == "dense" else (7152 < need <= 8192)
     d = t.to(dev)
     rows = torch.from_numpy(rng.integers(0, 4000, 300).astype(np.int32)).to(dev)
-    out = df11.decode_rows(d, 96, rows)
-    np.testing.assert_array_equal(_rows_bits(out), w[rows.cpu().numpy()])
-    np.testing.assert_array_equal(_rows_bits(df11.decode(d)).reshape(w.shape), w)
+    for dd in (d, d.without_counts()):  # stored counts, and the count pass
+        out = df11.decode_rows(dd, 96, rows)
+        np.testing.assert_array_equal(_rows_bits(out), w[rows.cpu().numpy()])
+        np.testing.assert_array_equal(_rows_bits(df11.decode(dd)).reshape(w.shape), w)

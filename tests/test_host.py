@@ -30,7 +30,7 @@ def test_library_exports_every_declared_symbol():
     assert len(names) >= 14
     for name in names:
         assert hasattr(lib, name), name
-    assert df11._lib().df11_abi_version() == 2
+    assert df11._lib().df11_abi_version() == 3
 
 
 def test_status_strings():
@@ -85,6 +85,13 @@ def check_against_oracle(w, t, cap=12):
     n_fields = t.n_blocks * 256
     assert np.array_equal(_unpack_gaps(packed, n_fields), a["gaps"])
     assert np.array_equal(packed[: (5 * n_fields + 7) // 8], oracle.pack_gaps(a["gaps"]))
+    # the optional per-thread code counts: the oracle's counts of code starts
+    if t.has_counts:
+        cnt = t.host_array("counts")
+        assert t.nbytes("counts") == n_fields + 16
+        assert np.array_equal(cnt[:n_fields], a["counts"].astype(np.uint8))
+        assert a["counts"].max(initial=0) <= 64
+        assert not cnt[n_fields:].any()
     # and the oracle decodes the product's stream back to the input
     out = oracle.decode(enc_o, bits_o, sm_o, w.size, lengths)
     assert np.array_equal(out, w)
@@ -129,7 +136,7 @@ def test_encode_multi_equals_concatenation():
             enumerate([(64, 96, 0.02), (3, 5, 0.05), (128, 64, 0.01), (1, 1, 1.0)])]
     blk = df11.encode_multi(mats)
     cat = df11.encode(np.concatenate([m.reshape(-1) for m in mats]))
-    for name in ("enc", "sm", "gaps", "block_start", "lut"):
+    for name in ("enc", "sm", "gaps", "block_start", "lut", "counts"):
         assert np.array_equal(blk.host_array(name), cat.host_array(name)), name
     assert blk.offsets == [0, 64 * 96, 64 * 96 + 15, 64 * 96 + 15 + 128 * 64, 64 * 96 + 15 + 128 * 64 + 1]
 
@@ -268,7 +275,8 @@ def test_save_load_round_trip(tmp_path):
     u = df11.load(path)
     assert bytes(u.desc)[:8] == bytes(t.desc)[:8] and u.n_elems == t.n_elems and u.total_bits == t.total_bits
     assert u.shapes == [(64, 48), (5, 7)] and u.offsets == t.offsets
-    for k in ("enc", "sm", "gaps", "block_start", "lut"):
+    assert u.has_counts
+    for k in ("enc", "sm", "gaps", "block_start", "lut", "counts"):
         np.testing.assert_array_equal(u.host_array(k).view(np.uint8)[: u.nbytes(k)],
                                       t.host_array(k).view(np.uint8)[: t.nbytes(k)])
     out = oracle.decode(u.host_array("enc"), u.total_bits, u.host_array("sm"), u.n_elems, u.code_len)
@@ -298,7 +306,7 @@ def test_concurrent_host_encodes_match_sequential():
         th.join()
     for a, b in zip(seq, got):
         assert a.total_bits == b.total_bits and a.n_blocks == b.n_blocks
-        for k in ("enc", "sm", "gaps", "block_start", "lut"):
+        for k in ("enc", "sm", "gaps", "block_start", "lut", "counts"):
             np.testing.assert_array_equal(a.host_array(k)[: a.nbytes(k)], b.host_array(k)[: b.nbytes(k)])
 
 

@@ -383,3 +383,31 @@ def test_llm_like_statistics_near_the_pages():
     assert 2.2 < h < 3.0
     assert 15 <= k <= 45
     assert 10.0 < 8 + mean < 12.0
+
+
+def test_decode_range_pieces_at_block_starts():
+    """The stream cut at thread-block starts (bit 16384*b plus the gap of the
+    block's first thread; element block_start[b]) decodes piece by piece to
+    the same weights as the whole stream; a cut one bit off does not."""
+    w = workloads.normal_matrix(300, 256, 0.02, seed=13).reshape(-1)
+    c = oracle.compress(w, 12)
+    a = oracle.aux(c["enc"], c["total_bits"], w.size, c["lengths"], 8, 256)
+    bs, gaps, nb = a["block_start"], a["gaps"], a["n_blocks"]
+    assert nb >= 5
+
+    def first_bit(b):
+        return c["total_bits"] if b >= nb else 16384 * b + int(gaps[256 * b])
+
+    cuts = [0, 1, 3, nb - 1, nb]
+    got = np.concatenate([
+        oracle.decode_range(c["enc"], first_bit(b0), first_bit(b1), c["sm"][bs[b0]:bs[b1]], int(bs[b1] - bs[b0]),
+                            c["lengths"]) for b0, b1 in zip(cuts[:-1], cuts[1:])])
+    np.testing.assert_array_equal(got, w)
+    b = 2
+    n = int(bs[b + 1] - bs[b])
+    try:
+        bad = oracle.decode_range(c["enc"], first_bit(b) + 1, first_bit(b + 1), c["sm"][bs[b]:bs[b + 1]], n,
+                                  c["lengths"])
+        assert not np.array_equal(bad, w[bs[b]:bs[b + 1]])
+    except oracle.OracleError:
+        pass  # the shifted piece does not even end on its last code

@@ -17,7 +17,7 @@ pytestmark = pytest.mark.gpu
 import huffman_decode_02_b200 as df11  # noqa: E402
 
 FIELDS = ["n_elems", "total_bits", "n_threads", "n_blocks", "max_block_codes", "enc_bytes", "sm_bytes",
-          "gaps_bytes", "block_start_bytes", "lut_bytes"]
+          "gaps_bytes", "block_start_bytes", "lut_bytes", "counts_bytes"]
 
 
 def _dev():
@@ -30,7 +30,7 @@ def _same(a: df11.DF11Tensor, b: df11.DF11Tensor):
     for f in FIELDS:
         assert getattr(a.desc, f) == getattr(b.desc, f), f
     assert bytes(a.desc.code_len) == bytes(b.desc.code_len)
-    for k in ("enc", "sm", "gaps", "block_start", "lut"):
+    for k in ("enc", "sm", "gaps", "block_start", "lut", "counts"):
         np.testing.assert_array_equal(a.host_array(k).view(np.uint8)[: a.nbytes(k)],
                                       b.host_array(k).view(np.uint8)[: b.nbytes(k)], err_msg=k)
 
