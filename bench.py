@@ -50,11 +50,16 @@ WORKLOADS = {
                 "also a 256-row gather (embedding lookup) timed", lambda r: [workloads.normal_matrix(128256, 4096, 0.02,
                                                                                               seed=5 + r)]),
     "decode-gemm": ("32 llama3.1-8b blocks (seeds 32*rank + 0..31), each decoded into one reused BF16 scratch, "
-                    "then every matrix multiplied by N(0,1) BF16 activations [T, in], T in {1,16,64,256} "
-                    "(seed 1000 + T), FP32-accumulate GEMM on tcgen05", None),
+                    "then every matrix multiplied by N(0,1) BF16 activations [T, in], T in {1,4,16,64,256} "
+                    "(seed 1000 + T), FP32-accumulate GEMM on tcgen05; beside it the fused decode -> tcgen05 GEMM "
+                    "on the first 8 blocks encoded in tile order (one launch per block)", None),
     "decode-gemv": ("llama3.1-8b transformer block (218,112,000 BF16 weights, seed = rank), all seven matrices "
                     "multiplied by N(0,1) BF16 activations [T, in] (seed 1000 + T) in ONE fused decode -> "
                     "matrix-vector launch (weights never written to memory); T from --T (1..4)", None),
+    "fused-gemm": ("llama3.1-8b transformer block (218,112,000 BF16 weights, seed = rank) stored in tile order, "
+                   "all seven matrices multiplied by N(0,1) BF16 activations [T, in] (seed 1000 + T) in ONE fused "
+                   "decode -> tcgen05 GEMM launch (weights decoded into shared-memory operand tiles, never "
+                   "written to memory); T from --T (1..256)", None),
     "gemm": ("consumer GEMM Y = X W^T on one weight shape (default 14336x4096, the gate/up projection), "
              "W N(0, 0.02^2) BF16 in three copies used in turn (351 MB, larger than L2), X N(0,1) BF16 [T, in]",
              None),
@@ -299,16 +304,18 @@ def _encode_block_raw_worker(seed: int, cap: int):
     return out + (workloads.llama8b_block(seed=seed),)
 
 
-def _encode_block_worker(seed: int, cap: int):
-    """Generates and encodes one block in a worker process; returns the
-    compressed arrays and a checksum of the original bits."""
+def _encode_block_worker(seed: int, cap: int, tile_order: bool = False):
+    """Generates and encodes one block in a worker process (its matrices in
+    tile order if asked); returns the compressed arrays and a checksum of the
+    original bits."""
     import huffman_decode_02_b200 as df11
     mats = workloads.llama8b_block(seed=seed)
-    blk = df11.encode_multi(mats, df11.Params(max_code_len=cap))
+    blk = df11.encode_multi(mats, df11.Params(max_code_len=cap), tile_order=tile_order)
     flat = np.concatenate([m.reshape(-1) for m in mats]).astype(np.int64)
     idx = np.arange(flat.size, dtype=np.int64) & 0xFFFF
     chk = (int(flat.sum()), int((flat * idx).sum()))
-    return bytes(blk.desc), {k: np.asarray(v) for k, v in blk.arrays.items()}, blk.shapes, blk.offsets, chk
+    return (bytes(blk.desc), {k: np.asarray(v) for k, v in blk.arrays.items()}, blk.shapes, blk.offsets, chk,
+            blk.tiled)
 
 
 def run_decode_gemm(args, rank: int, world: int):
@@ -319,8 +326,10 @@ def run_decode_gemm(args, rank: int, world: int):
     seeds = [args.blocks * rank + b for b in range(args.blocks)]
     workers = max(1, min(len(seeds), (os.cpu_count() or 1) // 2, 16))
     t0 = time.time()
+    n_tiled = min(8, len(seeds))  # blocks also encoded in tile order, for the fused tensor-core product
     with mp.get_context("spawn").Pool(workers) as pool:  # before any CUDA call
         enc = pool.starmap(_encode_block_worker, [(sd, args.max_code_len) for sd in seeds])
+        enc_t = pool.starmap(_encode_block_worker, [(sd, args.max_code_len, True) for sd in seeds[:n_tiled]])
     encode_s = time.time() - t0
 
     import torch
@@ -333,11 +342,14 @@ def run_decode_gemm(args, rank: int, world: int):
     if world > 1:
         from datetime import timedelta
         dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=dev)
-    blocks = []
-    for desc, arrays, shapes, offsets, chk in enc:
-        t = df11.DF11Tensor(df11._Tensor.from_buffer_copy(desc), arrays, "cpu", shapes, offsets)
+    blocks, tblocks = [], []
+    for desc, arrays, shapes, offsets, chk, tiled in enc:
+        t = df11.DF11Tensor(df11._Tensor.from_buffer_copy(desc), arrays, "cpu", shapes, offsets, tiled)
         blocks.append((t.to(dev), chk))
-    del enc
+    for desc, arrays, shapes, offsets, chk, tiled in enc_t:
+        t = df11.DF11Tensor(df11._Tensor.from_buffer_copy(desc), arrays, "cpu", shapes, offsets, tiled)
+        tblocks.append(t.to(dev))
+    del enc, enc_t
     n = blocks[0][0].n_elems
     scratch = torch.empty(n, dtype=torch.bfloat16, device=dev)
     err = torch.zeros(1, dtype=torch.int32, device=dev)
@@ -445,6 +457,40 @@ def run_decode_gemm(args, rank: int, world: int):
             per_T[str(T)].update({"fused_us": t_fused * 1e3, "fused_vs_bf16": t_fused / t_bf16,
                                   "fused_speedup_vs_unfused": t_both / t_fused, "fused_rel_fro": frel,
                                   "fused_launches_per_block": 2})
+        if T >= 4:
+            # fused decode -> tensor-core GEMM (blocks in tile order): per block
+            # one zeroing of the seven outputs and one launch for all seven
+            # products; the decoded weights never reach memory
+            rows_tot = sum(int(w.shape[0]) for w in gemm_mats)
+            ybuf = torch.empty(T * rows_tot, dtype=torch.float32, device=dev)
+            mat_idx = [j for j, til in enumerate(tblocks[0].tiled) if til]
+            xs_f, ys_f, off = {}, {}, 0
+            for j, w in zip(mat_idx, gemm_mats):
+                xs_f[j] = xs[w.shape[1]]
+                ys_f[j] = ybuf[off: off + T * w.shape[0]].view(T, w.shape[0])
+                off += T * w.shape[0]
+            # numerics: block 0, decoded in row order for the reference weights
+            df11.decode_block(blocks[0][0], scratch, err, stream)
+            ybuf.zero_()
+            df11.decode_gemm(tblocks[0], xs_f, ys_f, err, stream)
+            trel = 0.0
+            for j, w in zip(mat_idx, gemm_mats):
+                cols = torch.arange(0, w.shape[0], max(1, w.shape[0] // 256), device=dev)
+                ref = xs[w.shape[1]].double() @ w[cols].double().T
+                trel = max(trel, float((ys_f[j][:, cols].double() - ref).norm() / ref.norm()))
+
+            def fused_tc_all():
+                for d in tblocks:
+                    ybuf.zero_()
+                    df11.decode_gemm(d, xs_f, ys_f, err, stream)
+
+            t_ftc = timed(fused_tc_all, args.steps) / len(tblocks)
+            per_T[str(T)].update({"fused_tc_us": t_ftc * 1e3, "fused_tc_vs_bf16": t_ftc / t_bf16,
+                                  "fused_tc_speedup_vs_unfused": t_both / t_ftc, "fused_tc_rel_fro": trel,
+                                  "fused_tc_blocks": len(tblocks), "fused_tc_launches_per_block": 2})
+            # the last decode left block 0 in the scratch: put back the last
+            # block's weights for the views of the next T
+            df11.decode_block(blocks[-1][0], scratch, err, stream)
     assert df11.read_error(err, stream) == 0
     pipe.check(stream)
     if rank == 0:
@@ -487,7 +533,7 @@ def run_offload(args, rank: int, world: int):
         from datetime import timedelta
         dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=dev)
     blocks, raws, chks = [], [], []
-    for desc, arrays, shapes, offsets, chk, mats in enc:
+    for desc, arrays, shapes, offsets, chk, _tiled, mats in enc:
         pinned = {k: torch.empty(max(a.size, 16), dtype=torch.uint8, pin_memory=True) for k, a in arrays.items()}
         for k, a in arrays.items():
             pinned[k][: a.size].copy_(torch.from_numpy(a.view(np.uint8)))
@@ -554,11 +600,13 @@ def run_offload(args, rank: int, world: int):
         dist.destroy_process_group()
 
 
-def run_decode_gemv(args, rank: int, world: int):
-    """Fused decode -> matrix-vector products on one block: per step the seven
+def run_decode_gemv(args, rank: int, world: int, tc: bool = False):
+    """Fused decode -> matrix products on one block: per step the seven
     outputs are zeroed and one launch decodes the block and multiplies every
-    matrix by its activations.  Timed next to the unfused path (block decode
-    into the scratch, then the seven T <= 4 GEMMs)."""
+    matrix by its activations -- on the CUDA cores for T <= 4
+    (decode_gemv), or (tc, the fused-gemm workload) on the tensor cores for
+    any T with the block stored in tile order (decode_gemm).  Timed next to the
+    unfused path (block decode into the scratch, then the seven GEMMs)."""
     import torch
     import torch.distributed as dist
 
@@ -571,8 +619,11 @@ def run_decode_gemv(args, rank: int, world: int):
         dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=dev)
     T = args.T
     mats = workloads.llama8b_block(seed=rank_seed(rank))
-    blk = df11.encode_multi(mats, df11.Params(max_code_len=args.max_code_len))
+    params = df11.Params(max_code_len=args.max_code_len)
+    blk = df11.encode_multi(mats, params, tile_order=tc)
     d = blk.to(dev)
+    du = df11.encode_multi(mats, params).to(dev) if tc else d  # row order, for the unfused path
+    product = df11.decode_gemm if tc else df11.decode_gemv
     idx = [j for j, m in enumerate(mats) if m.ndim == 2]
     g = torch.Generator().manual_seed(1000 + T)
     xs_in = {k: torch.randn(T, k, generator=g).to(torch.bfloat16) for k in sorted({mats[j].shape[1] for j in idx})}
@@ -588,7 +639,7 @@ def run_decode_gemv(args, rank: int, world: int):
 
     def fused():
         ybuf.zero_()
-        df11.decode_gemv(d, xs, ys, err, stream)
+        product(d, xs, ys, err, stream)
 
     # numerics: 256 sampled rows of every matrix against FP64
     fused()
@@ -602,11 +653,11 @@ def run_decode_gemv(args, rank: int, world: int):
         rel = max(rel, float((got - ref).norm() / ref.norm()))
     assert df11.read_error(err, stream) == 0
     scratch = torch.empty(d.n_elems, dtype=torch.bfloat16, device=dev)
-    views = d.views(scratch)
+    views = du.views(scratch)
     yu = {j: torch.empty(T, mats[j].shape[0], dtype=torch.float32, device=dev) for j in idx}
 
     def unfused():
-        df11.decode_block(d, scratch, err, stream)
+        df11.decode_block(du, scratch, err, stream)
         for j in idx:
             df11.gemm(xs[j], views[j], yu[j], err, stream)
 
@@ -640,7 +691,7 @@ def run_decode_gemv(args, rank: int, world: int):
     def forward_order():
         ybuf.zero_()
         for grp in groups:
-            df11.decode_gemv(d, {j: xs[j] for j in grp}, {j: ys[j] for j in grp}, err, stream)
+            product(d, {j: xs[j] for j in grp}, {j: ys[j] for j in grp}, err, stream)
 
     ms_forward = timed(forward_order, max(1, args.steps // 4))
     assert df11.read_error(err, stream) == 0
@@ -650,11 +701,13 @@ def run_decode_gemv(args, rank: int, world: int):
         io = sum(T * mats[j].shape[1] * 2 + T * mats[j].shape[0] * 4 for j in idx)
         alg = comp + io
         achieved = alg / (ms_fused * 1e-3) / 1e9
-        line = {"metric": "fused decode -> matrix-vector time per llama3.1-8b block", "value": ms_fused * 1e3,
+        what = "tensor-core GEMM" if tc else "matrix-vector"
+        line = {"metric": f"fused decode -> {what} time per llama3.1-8b block", "value": ms_fused * 1e3,
                 "unit": "us", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
                 "ms_per_step": ms_fused, "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
                 "dtype": "bf16 x bf16 -> f32 (decode u32)", "data": "synthetic",
-                "config": {"workload": WORKLOADS["decode-gemv"][0], "T": T, "n_elems_per_rank": d.n_elems,
+                "config": {"workload": WORKLOADS["fused-gemm" if tc else "decode-gemv"][0], "T": T,
+                           "n_elems_per_rank": d.n_elems,
                            "l2": f"inputs larger than L2 ({comp / 1e6:.0f} MB compressed per step), no flush",
                            "timing": "K steps (zeroing of y + one fused launch) between CUDA events"},
                 "rel_fro_sampled_rows": rel,
@@ -665,10 +718,25 @@ def run_decode_gemv(args, rank: int, world: int):
                              "peak_kind": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs, copy burst)",
                              "algorithmic_bytes_per_launch": alg},
                 "gpu_launches": args.steps, "clocks": clocks}
+        if tc:  # the tensor cores' side of the roofline (bf16 dense burst peak, measured)
+            flops = 2.0 * T * sum(mats[j].size for j in idx)
+            tpk = _tensor_peak()
+            line["tensor"] = {"achieved_tflops": flops / (ms_fused * 1e-3) / 1e12, "peak_tflops": tpk,
+                              "frac": flops / (ms_fused * 1e-3) / 1e12 / tpk}
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
+
+
+def _tensor_peak() -> float:
+    """Measured dense BF16 burst TFLOP/s (MEASURED_PEAKS.json), else the
+    fallback 1590."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["bf16_tflops"])
+    except Exception:
+        return 1590.0
 
 
 def run_gemm(args, rank: int, world: int):
@@ -831,6 +899,9 @@ def main():
         return
     if args.workload == "decode-gemv":
         run_decode_gemv(args, rank, world)
+        return
+    if args.workload == "fused-gemm":
+        run_decode_gemv(args, rank, world, tc=True)
         return
     if args.workload == "gemm":
         run_gemm(args, rank, world)

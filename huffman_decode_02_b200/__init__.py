@@ -30,7 +30,9 @@ from . import build as _build
 
 __all__ = [
     "DF11Error", "CorruptStreamError", "Params", "DF11Tensor", "encode", "encode_multi",
-    "encode_device", "encode_device_noalloc", "save", "load", "decode", "decode_block", "decode_rows", "decode_gemv", "gemm", "read_error", "exponent_histogram", "lib_path", "sm_count",
+    "encode_device", "encode_device_noalloc", "save", "load", "decode", "decode_block", "decode_rows", "decode_gemv",
+    "decode_gemm", "gemm", "read_error", "exponent_histogram", "lib_path", "sm_count", "to_tile_order",
+    "from_tile_order",
     "KERR_COUNT_MISMATCH", "KERR_BAD_CODE", "KERR_BAD_BLOCK", "KERR_OVERRUN", "KERR_TIMEOUT", "KERR_BAD_ROW",
 ]
 
@@ -116,6 +118,9 @@ def _lib():
     lib.df11_gemm_bf16.argtypes = [vp, vp, vp, u32, u32, u32, vp, vp]
     lib.df11_decode_rows.argtypes = [P(_Tensor), ctypes.c_uint64, vp, u32, vp, vp, vp]
     lib.df11_decode_gemv.argtypes = [P(_Tensor), P(_GemvMat), u32, u32, vp, vp]
+    lib.df11_decode_gemm.argtypes = [P(_Tensor), P(_GemvMat), u32, u32, vp, vp]
+    lib.df11_to_tile_order.argtypes = [vp, u32, u32, vp]
+    lib.df11_from_tile_order.argtypes = [vp, u32, u32, vp]
     lib.df11_encode_device_scratch_bytes.argtypes = [u64]
     lib.df11_encode_device_scratch_bytes.restype = u64
     lib.df11_encode_device_size.argtypes = [vp, u64, P(_Params), P(T), vp, u64, vp]
@@ -198,12 +203,14 @@ class DF11Tensor:
     or on a CUDA device (torch tensors).  ``shapes`` records the original
     matrix shapes for block tensors (element offsets in ``offsets``)."""
 
-    def __init__(self, desc: _Tensor, arrays: dict, device: str, shapes, offsets):
+    def __init__(self, desc: _Tensor, arrays: dict, device: str, shapes, offsets, tiled=None):
         self.desc = desc
         self.arrays = arrays
         self.device = device
         self.shapes = list(shapes)
         self.offsets = list(offsets)
+        # per matrix: stored in tile order (128 x 64 tiles, for decode_gemm)
+        self.tiled = list(tiled) if tiled is not None else [False] * len(self.shapes)
 
     # scalar fields
     n_elems = property(lambda self: int(self.desc.n_elems))
@@ -242,7 +249,7 @@ class DF11Tensor:
         arrays = {k: v for k, v in self.arrays.items() if k != "counts"}
         desc = _Tensor.from_buffer_copy(self.desc)
         desc.counts_bytes = 0
-        return DF11Tensor(desc, arrays, self.device, self.shapes, self.offsets)
+        return DF11Tensor(desc, arrays, self.device, self.shapes, self.offsets, self.tiled)
 
     def host_array(self, which: str) -> np.ndarray:
         a = self.arrays[which]
@@ -272,10 +279,12 @@ class DF11Tensor:
             b = torch.empty(a.numel() * a.element_size(), dtype=torch.uint8, device=dev)
             b.copy_(a.view(torch.uint8).reshape(-1), non_blocking=non_blocking)
             arrays[name] = b
-        return DF11Tensor(_Tensor.from_buffer_copy(self.desc), arrays, str(dev), self.shapes, self.offsets)
+        return DF11Tensor(_Tensor.from_buffer_copy(self.desc), arrays, str(dev), self.shapes, self.offsets,
+                          self.tiled)
 
     def views(self, decoded):
-        """Splits a decoded block buffer into the original matrices."""
+        """Splits a decoded block buffer into the original matrices (a matrix
+        stored in tile order comes back in tile order: see from_tile_order)."""
         out = []
         for shape, lo, hi in zip(self.shapes, self.offsets[:-1], self.offsets[1:]):
             out.append(decoded[lo:hi].view(*shape) if shape else decoded[lo:hi])
@@ -292,8 +301,34 @@ def _alloc_host(nbytes: int, pinned: bool):
     return raw[off: off + max(nbytes, 16)]
 
 
+def to_tile_order(w) -> np.ndarray:
+    """A [rows, cols] BF16 matrix (numpy uint16 bits or a CPU torch tensor;
+    rows a multiple of 128, cols of 64) in tile order: its 128 x 64 tiles, row
+    tiles in order, the 64-column tiles of a row tile in order, each tile
+    row-major (the element order df11_decode_gemm reads).  Flat uint16."""
+    a = _as_u16(w)
+    shape = tuple(getattr(w, "shape", ()))
+    if len(shape) != 2:
+        raise ValueError("to_tile_order expects a 2-D matrix")
+    out = np.empty(a.size, dtype=np.uint16)
+    _check(_lib().df11_to_tile_order(ctypes.c_void_p(a.ctypes.data), int(shape[0]), int(shape[1]),
+                                     ctypes.c_void_p(out.ctypes.data)), "to_tile_order")
+    return out
+
+
+def from_tile_order(tiled, rows: int, cols: int) -> np.ndarray:
+    """Inverse of to_tile_order: the [rows, cols] row-major matrix (uint16)."""
+    a = _as_u16(tiled)
+    if a.size != rows * cols:
+        raise ValueError("size does not match rows x cols")
+    out = np.empty((rows, cols), dtype=np.uint16)
+    _check(_lib().df11_from_tile_order(ctypes.c_void_p(a.ctypes.data), int(rows), int(cols),
+                                       ctypes.c_void_p(out.ctypes.data)), "from_tile_order")
+    return out
+
+
 def _encode_impl(mats: list[np.ndarray], shapes, params: Params | None, pinned: bool,
-                 counts: bool = True) -> DF11Tensor:
+                 counts: bool = True, tiled=None) -> DF11Tensor:
     lib = _lib()
     k = len(mats)
     ptrs = (ctypes.POINTER(ctypes.c_uint16) * max(1, k))(*[_u16_ptr(m) for m in mats])
@@ -314,7 +349,7 @@ def _encode_impl(mats: list[np.ndarray], shapes, params: Params | None, pinned: 
     offsets = [0]
     for m in mats:
         offsets.append(offsets[-1] + m.size)
-    return DF11Tensor(desc, arrays, "cpu", shapes, offsets)
+    return DF11Tensor(desc, arrays, "cpu", shapes, offsets, tiled)
 
 
 def encode(w, params: Params | None = None, pinned: bool = False, counts: bool = True) -> DF11Tensor:
@@ -326,12 +361,16 @@ def encode(w, params: Params | None = None, pinned: bool = False, counts: bool =
 
 
 def encode_multi(mats: Sequence, params: Params | None = None, pinned: bool = False,
-                 counts: bool = True) -> DF11Tensor:
+                 counts: bool = True, tile_order: bool = False) -> DF11Tensor:
     """Encodes several matrices (a transformer block) as one stream with one
-    shared table; ``DF11Tensor.offsets`` gives each matrix's element offset."""
-    arrs = [_as_u16(m) for m in mats]
+    shared table; ``DF11Tensor.offsets`` gives each matrix's element offset.
+    ``tile_order``: every 2-D matrix whose rows are a multiple of 128 and
+    columns of 64 is stored in tile order (to_tile_order), as decode_gemm
+    needs; ``DF11Tensor.tiled`` records which ones."""
     shapes = [tuple(getattr(m, "shape", ())) for m in mats]
-    return _encode_impl(arrs, shapes, params, pinned, counts)
+    tiled = [bool(tile_order and len(sh) == 2 and sh[0] % 128 == 0 and sh[1] % 64 == 0) for sh in shapes]
+    arrs = [to_tile_order(m) if t else _as_u16(m) for m, t in zip(mats, tiled)]
+    return _encode_impl(arrs, shapes, params, pinned, counts, tiled)
 
 
 def encode_device(mats, params: Params | None = None, stream=None) -> DF11Tensor:
@@ -423,7 +462,8 @@ def save(t: DF11Tensor, path: str) -> None:
     arrays = {name: t.host_array(name).view(np.uint8).reshape(-1)[: t.nbytes(name)] for name in t.arrays}
     shapes = np.array([len(s) for s in t.shapes] + [d for s in t.shapes for d in s], dtype=np.int64)
     np.savez(path, magic=np.frombuffer(_FILE_MAGIC, dtype=np.uint8), desc=np.frombuffer(bytes(desc), dtype=np.uint8),
-             offsets=np.asarray(t.offsets, dtype=np.int64), shapes=shapes, **arrays)
+             offsets=np.asarray(t.offsets, dtype=np.int64), shapes=shapes,
+             tiled=np.asarray(t.tiled, dtype=np.uint8), **arrays)
 
 
 def load(path: str, pinned: bool = False) -> DF11Tensor:
@@ -453,6 +493,7 @@ def load(path: str, pinned: bool = False) -> DF11Tensor:
             arrays[name] = buf
         offsets = [int(v) for v in z["offsets"]]
         sh = [int(v) for v in z["shapes"]]
+        tiled = [bool(v) for v in z["tiled"]] if "tiled" in z.files else None
     k = len(offsets) - 1
     ndims, dims = sh[:k], sh[k:]
     shapes, pos = [], 0
@@ -460,7 +501,7 @@ def load(path: str, pinned: bool = False) -> DF11Tensor:
         shapes.append(tuple(dims[pos: pos + nd]))
         pos += nd
     _check(_lib().df11_validate(ctypes.byref(desc)), "load")
-    return DF11Tensor(desc, arrays, "cpu", shapes, offsets)
+    return DF11Tensor(desc, arrays, "cpu", shapes, offsets, tiled)
 
 
 def exponent_histogram(mats: Iterable) -> np.ndarray:
@@ -595,6 +636,53 @@ def decode_gemv(t: DF11Tensor, xs: dict, ys: dict | None = None, err=None, strea
         _check(_lib().df11_decode_gemv(ctypes.byref(t._bind()), mats, len(order), T,
                                        ctypes.c_void_p(err.data_ptr()), _stream_handle(stream, t.device)),
                "decode_gemv")
+    if own_err:
+        read_error(err, stream)
+    return {j: ys[j] for j in order}
+
+
+def decode_gemm(t: DF11Tensor, xs: dict, ys: dict | None = None, err=None, stream=None) -> dict:
+    """Fused decode and tensor-core matrix products for any batch 1..256 (one
+    launch): for each matrix index j in ``xs`` (a 2-D [out, in] matrix stored
+    in tile order: ``encode_multi(..., tile_order=True)``), y_j = x_j @ W_j^T
+    with W_j decoded into shared-memory operand tiles and never written to
+    memory.  ``xs[j]``: [T, in] bfloat16 CUDA tensors, one T for all;
+    ``ys[j]`` ([T, out] float32), when given, are added into, otherwise
+    zero-filled outputs are allocated.  Returns {j: y_j}."""
+    import torch
+    _check_device(t)
+    if not xs:
+        return {}
+    order = sorted(xs)
+    T = None
+    if ys is None:
+        ys = {}
+    mats = (_GemvMat * len(order))()
+    for i, j in enumerate(order):
+        shape = t.shapes[j]
+        if len(shape) != 2 or not t.tiled[j]:
+            raise ValueError(f"matrix {j} is not a 2-D matrix stored in tile order")
+        rows, cols = int(shape[0]), int(shape[1])
+        x = xs[j]
+        if x.dtype != torch.bfloat16 or x.dim() != 2 or x.shape[1] != cols or not x.is_contiguous():
+            raise TypeError(f"x for matrix {j} must be a contiguous [T, {cols}] bfloat16 tensor")
+        if T is None:
+            T = int(x.shape[0])
+        elif int(x.shape[0]) != T:
+            raise ValueError("every x must have the same batch T")
+        if j not in ys:
+            ys[j] = torch.zeros(T, rows, dtype=torch.float32, device=t.device)
+        y = ys[j]
+        if y.dtype != torch.float32 or tuple(y.shape) != (T, rows) or not y.is_contiguous():
+            raise TypeError(f"y for matrix {j} must be a contiguous [{T}, {rows}] float32 tensor")
+        mats[i] = _GemvMat(int(t.offsets[j]), rows, cols, x.data_ptr(), y.data_ptr())
+    own_err = err is None
+    if own_err:
+        err = _new_err(t.device)
+    with _on(t.device):
+        _check(_lib().df11_decode_gemm(ctypes.byref(t._bind()), mats, len(order), T,
+                                       ctypes.c_void_p(err.data_ptr()), _stream_handle(stream, t.device)),
+               "decode_gemm")
     if own_err:
         read_error(err, stream)
     return {j: ys[j] for j in order}

@@ -63,6 +63,7 @@
 
 #include "df11.h"
 #include "df11_internal.h"
+#include "df11_tc.cuh"
 
 namespace {
 
@@ -118,9 +119,10 @@ static_assert(kLutBytes % 16 == 0, "bulk copy size");
 // table (tensors without stored per-thread counts); without it, the counts
 // come from the tensor's `counts` array, staged per block, and the 32 KB of
 // the count table are free for buffers and table copies.
-template <int G, int S, int SC, bool CT = true>
+template <int G, int S, int SC, bool CT = true, bool SMS = true>
 struct Cfg {
     static constexpr bool kCountTable = CT;
+    static constexpr bool kStageSm = SMS;  // the block's sign/mantissa bytes are staged in shared memory
     static constexpr uint32_t kSymCopies = SC;  // symbol-table copies (lane l reads copy l mod SC)
     static constexpr uint32_t kOffSymRep = CT ? kOffCountRep + 4u * kCountCopies * (1u << kW1Max) : kOffCountRep;
     static constexpr uint32_t kOffGroups = kOffSymRep + 8u * SC * (1u << kW2Max);
@@ -135,7 +137,7 @@ struct Cfg {
     static constexpr uint32_t kGrpCnt = kGrpBs + 32u;  // the block's stored counts (instances without CT)
     static constexpr uint32_t kCntStage = CT ? 0u : (uint32_t)kThreadsPerBlockFmt;
     static constexpr uint32_t kGrpSm = kGrpCnt + kCntStage;  // the block's sign/mantissa bytes
-    static constexpr uint32_t kSmBytes = S + 16u;
+    static constexpr uint32_t kSmBytes = SMS ? S + 16u : 0u;
     static constexpr uint32_t kGrpMbar = kGrpSm + kSmBytes;
     static constexpr uint32_t kGrpAux = kGrpMbar + 16u;  // row gather: the row's block range
     static constexpr uint32_t kGroupBytes = kGrpAux + 16u;
@@ -146,9 +148,16 @@ struct Cfg {
     static_assert(kGroupBytes % 16 == 0 && kGrpEnc % 16 == 0 && kGrpGap % 16 == 0 && kGrpBs % 16 == 0 &&
                       kGrpCnt % 16 == 0 && kGrpSm % 16 == 0,
                   "bulk copy destinations are 16-byte aligned");
-    static_assert(kLutBytes <= G * kGroupBytes, "tables stage in the group area");
+    // where the staged symbol LUT lands (right after the header when the count
+    // LUT is not staged) and how many bytes the staging takes
+    static constexpr uint32_t kStageSym = CT ? kOffSymLut : kOffCountLut;
+    static constexpr uint32_t kStageBytes = kStageSym + (kLutBytes - kOffSymLut);
+    static_assert(kStageBytes <= G * kGroupBytes, "tables stage in the group area");
     static_assert(kSmemBytes <= 227u * 1024u, "fits one CTA's shared memory");
 };
+// (SMS = false: the merge reads the sign/mantissa bytes from global memory;
+// only the fused decode -> GEMM kernel, which needs the room for its operand
+// tiles, does so)
 // (S = 7152 is the largest buffer with which 8 groups and two symbol-table
 // copies fit beside the count table: 232,336 of the 232,448 bytes a CTA may
 // use)
@@ -165,6 +174,12 @@ using CfgDense = Cfg<4, 16400, 1>;   // any block (1-bit codes: 16384 per block)
 using CfgTypicalC = Cfg<8, DF11_TYPICAL_C_SYMS, DF11_TYPICAL_C_COPIES, false>;
 using CfgWideC = Cfg<8, 8192, 2, false>;
 using CfgDenseC = Cfg<4, 16400, 2, false>;
+// The fused decode -> GEMM kernel's decoder: stored counts, one symbol-table
+// copy, 6 or 4 groups (the rest of the shared memory holds the operand tiles;
+// the largest X tiles leave no room to stage the sign/mantissa bytes).
+using CfgFused6 = Cfg<6, 7152, 1, false>;          // T <= 64
+using CfgFused4 = Cfg<4, 7152, 1, false>;          // T <= 128
+using CfgFused4U = Cfg<4, 7152, 1, false, false>;  // T <= 256: no sign/mantissa staging
 
 struct DecodeArgs {
     const uint8_t *enc;
@@ -588,9 +603,9 @@ __device__ __forceinline__ bool load_tables(const uint8_t *lut, uint32_t *err_ou
             mbar_expect(s_tmbar, kLutBytes);
             bulk_g2s(s_stage, lut, kLutBytes, s_tmbar);
         } else {  // header, limits and symbols; then the symbol LUT (the count LUT is not used)
-            mbar_expect(s_tmbar, kOffCountLut + (kLutBytes - kOffSymLut));
+            mbar_expect(s_tmbar, C::kStageBytes);
             bulk_g2s(s_stage, lut, kOffCountLut, s_tmbar);
-            bulk_g2s(s_stage + kOffSymLut, lut + kOffSymLut, kLutBytes - kOffSymLut, s_tmbar);
+            bulk_g2s(s_stage + C::kStageSym, lut + kOffSymLut, kLutBytes - kOffSymLut, s_tmbar);
         }
     }
     const bool staged = wait_phase(s_tmbar, 0u);
@@ -610,7 +625,7 @@ __device__ __forceinline__ bool load_tables(const uint8_t *lut, uint32_t *err_ou
         bool bad = !(hdr->magic == kMagic && w1 >= 1u && w1 <= (uint32_t)kW1Max && w2 >= 1u &&
                      w2 <= (uint32_t)kW2Max && max_len <= 32u);
         // header, limits and symbol list go to the front
-        for (uint32_t i = tid; i < kOffCountLut / 16u; i += C::kCtaThreads) {
+        for (uint32_t i = tid; i < kOffCountLut / 16u; i += blockDim.x) {
             const uint4 v = lds_u4(s_stage + 16u * i);
             sts_u4(s_base + 16u * i, v.x, v.y, v.z, v.w);
         }
@@ -620,7 +635,7 @@ __device__ __forceinline__ bool load_tables(const uint8_t *lut, uint32_t *err_ou
         constexpr uint32_t kCW = kCountCopies < 4u ? kCountCopies : 4u;
         constexpr uint32_t kSW = kSymCopies % 2u == 0u ? 2u : 1u;
         static_assert(kCountCopies % kCW == 0u && kSymCopies % kSW == 0u, "copies fill whole stores");
-        for (uint32_t i = tid; C::kCountTable && i < (1u << kW1Max) * (kCountCopies / kCW); i += C::kCtaThreads) {
+        for (uint32_t i = tid; C::kCountTable && i < (1u << kW1Max) * (kCountCopies / kCW); i += blockDim.x) {
             const uint32_t ent = lds_u32(s_stage + kOffCountLut + 4u * (i / (kCountCopies / kCW)));
             const uint32_t nb = count_entry_bits(ent), nc = count_entry_codes(ent);
             bad |= ent != kEscape && (ent != count_entry(nb, nc) || nb == 0u || nb > w1 || nc == 0u || nc > nb);
@@ -629,8 +644,8 @@ __device__ __forceinline__ bool load_tables(const uint8_t *lut, uint32_t *err_ou
             else if (kCW == 2u) asm volatile("st.shared.v2.u32 [%0], {%1, %1};" ::"r"(dst), "r"(ent) : "memory");
             else sts_u32(dst, ent);
         }
-        for (uint32_t i = tid; i < (1u << kW2Max) * (kSymCopies / kSW); i += C::kCtaThreads) {
-            const uint2 ent = lds_u2(s_stage + kOffSymLut + 8u * (i / (kSymCopies / kSW)));
+        for (uint32_t i = tid; i < (1u << kW2Max) * (kSymCopies / kSW); i += blockDim.x) {
+            const uint2 ent = lds_u2(s_stage + C::kStageSym + 8u * (i / (kSymCopies / kSW)));
             const uint32_t nb = sym_entry_bits(ent.y), nc = sym_entry_codes(ent.y);
             bad |= ent.y != kEscape && (ent.y != sym_entry_meta(nb, nc) || nb == 0u || nb > w2 || nc == 0u ||
                                         nc > (uint32_t)kSymsPerEntry || nc > nb);
@@ -651,11 +666,24 @@ __device__ __forceinline__ bool load_tables(const uint8_t *lut, uint32_t *err_ou
 }
 
 // Where a decoded block goes: StoreSink writes it as BF16 (the decoder);
-// the fused matrix-vector product below multiplies it into y instead.  A
-// sink takes the whole chunks of a block (`chunks`, every thread of the
-// group) and its two edge chunks (`edges`, warp 0), and clears every buffer
-// chunk it reads.
-struct StoreSink {
+// the fused matrix-vector product below multiplies it into y instead, and
+// the fused GEMM writes it into tensor-core operand tiles.  A sink takes the
+// whole chunks of a block (`chunks`, every thread of the group) and its two
+// edge chunks (`edges`, warp 0), and clears every buffer chunk it reads.
+// Hooks let a sink publish what it wrote: `begin_block(s, e)` before a
+// block's merge and `block_done(s, e, ok, range_ok)` after it (every thread;
+// the block's element range, whether it decoded and whether its range was
+// even plausible), `published(lt)`
+// right after the next group barrier (every thread of the group has then
+// finished that merge), and `finish(group, lt)` after the group's last block.
+struct NoHooks {
+    __device__ __forceinline__ void begin_block(uint32_t, uint32_t) {}
+    __device__ __forceinline__ void block_done(uint32_t, uint32_t, bool, bool) {}
+    __device__ __forceinline__ void published(uint32_t) {}
+    __device__ __forceinline__ void finish(uint32_t, uint32_t) {}
+};
+
+struct StoreSink : NoHooks {
     uint16_t *out;
     const uint8_t *sm;
     uint64_t n_elems;
@@ -671,13 +699,14 @@ struct StoreSink {
     }
 };
 
-// The persistent decode loop of one CTA: loads the tables, then each group
-// decodes format blocks blk_first + (CTA * groups + group) + k * stride,
-// below blk_end, and hands every decoded block to the sink.
+// The persistent decode loop of one group (the tables are loaded): the group
+// decodes format blocks blk, blk + stride, ... below blk_end and hands every
+// decoded block to the sink.
 // kLong: compiled with the long-code path (codes longer than the table
 // windows); without it the loops carry no escape handling at all.
 template <class C, bool kLong, class Sink>
-__device__ __forceinline__ void decode_blocks(const DecodeArgs &a, Sink &sink, uint64_t blk_first, uint64_t blk_end) {
+__device__ __forceinline__ void decode_loop(const DecodeArgs &a, Sink &sink, uint64_t blk, uint64_t stride,
+                                            uint64_t blk_end) {
     extern __shared__ __align__(128) uint8_t smem[];
     const uint32_t s_base = smem_addr(smem);
     const uint32_t s_lim = s_base + kOffLim;
@@ -697,10 +726,6 @@ __device__ __forceinline__ void decode_blocks(const DecodeArgs &a, Sink &sink, u
     uint32_t *buf = reinterpret_cast<uint32_t *>(smem + C::kOffGroups + group * C::kGroupBytes);
     uint32_t my_err = 0;
 
-    const uint64_t stride = (uint64_t)gridDim.x * C::kGroups;
-    uint64_t blk = blk_first + (uint64_t)blockIdx.x * C::kGroups + group;
-
-    if (!load_tables<C>(a.lut, a.err, smem, s_base, tid)) return;
     const LutHeader *hdr = reinterpret_cast<const LutHeader *>(smem + kOffHeader);
     const uint32_t w1 = hdr->w1, w2 = hdr->w2, max_len = hdr->max_len;
     const uint32_t sh1 = 32u - w1, sh2 = 32u - w2;
@@ -770,10 +795,11 @@ __device__ __forceinline__ void decode_blocks(const DecodeArgs &a, Sink &sink, u
         // every thread has read this block's staged inputs: fetch the next
         const uint64_t nxt = blk + stride;
         if (lt == 0 && nxt < blk_end) issue_inputs<C>(a, nxt, grp, mb_in);
+        sink.published(lt);  // the previous block's merge is done by the whole group
         // and this block's sign/mantissa bytes (chunks c_lo .. the block's
         // last chunk; always at least 16 bytes).  Every thread of the group
         // has passed its previous merge, so the staging area is free.
-        if (lt == 0) {
+        if (C::kStageSm && lt == 0) {
             // (64-bit: the end of the last chunk passes 2^32 when the tensor
             // holds nearly 2^32 elements)
             const uint64_t from = range_ok ? (uint64_t)base + 16u * c_lo : 0u;
@@ -806,22 +832,39 @@ __device__ __forceinline__ void decode_blocks(const DecodeArgs &a, Sink &sink, u
         group_barrier(group);
 
         // ---- merge with sign/mantissa and store, 16 weights per step
-        if (!wait_phase(mb_sm, ph_sm)) my_err |= kKernErrTimeout;
-        ph_sm ^= 1u;
+        if (C::kStageSm) {
+            if (!wait_phase(mb_sm, ph_sm)) my_err |= kKernErrTimeout;
+            ph_sm ^= 1u;
+        }
+        sink.begin_block(s, e);
         if (ok) {
             sink.template chunks<C::kSbufBytes>(sb, base, c0, c_full, grp + C::kGrpSm, c_lo);
             if (warp == 0) sink.edges(sb, base, c_full, span, s, e, lane);
         }
+        sink.block_done(s, e, ok, range_ok);
         // No barrier here: the next block's buffer writes and staging copies
         // come after its scan barrier, which every thread reaches only after
         // this merge.
     }
+    sink.finish(group, lt);
     if (my_err && a.err) atomicOr(a.err, my_err);
+}
+
+// Loads the tables (whole CTA), then runs the decode loop of this thread's
+// group over blocks blk_first + (CTA * groups + group) + k * (grid * groups)
+// below blk_end.
+template <class C, bool kLong, class Sink>
+__device__ __forceinline__ void decode_blocks(const DecodeArgs &a, Sink &sink, uint64_t blk_first, uint64_t blk_end) {
+    extern __shared__ __align__(128) uint8_t smem[];
+    if (!load_tables<C>(a.lut, a.err, smem, smem_addr(smem), threadIdx.x)) return;
+    const uint32_t group = threadIdx.x / kGroupThreads;
+    decode_loop<C, kLong>(a, sink, blk_first + (uint64_t)blockIdx.x * C::kGroups + group,
+                          (uint64_t)gridDim.x * C::kGroups, blk_end);
 }
 
 template <class C, bool kLong>
 __global__ void __launch_bounds__(C::kCtaThreads, 1) df11_decode_kernel(const DecodeArgs a) {
-    StoreSink sink{a.out, a.sm, a.n_elems, a.out_al32};
+    StoreSink sink{{}, a.out, a.sm, a.n_elems, a.out_al32};
     decode_blocks<C, kLong>(a, sink, 0u, a.n_blocks);
 }
 
@@ -1092,7 +1135,7 @@ __device__ __forceinline__ void flush_runs(const float (&lo)[TM], const float (&
 // warp's elements (they only grow: chunks within a block, then blocks by
 // stride).
 template <uint32_t TM>
-struct GemvSink {
+struct GemvSink : NoHooks {
     const GemvArgs &g;
     uint32_t m;
 
@@ -1286,8 +1329,421 @@ __global__ void __launch_bounds__(C::kCtaThreads, 1) df11_decode_gemv_kernel(con
     const uint32_t lane = threadIdx.x & 31u;
     const uint64_t b0 = find_block(g.d.bstart, g.d.n_blocks, g.e_first, lane);
     const uint64_t b1 = find_block(g.d.bstart, g.d.n_blocks, g.e_last, lane) + 1u;
-    GemvSink<TM> sink{g, 0u};
+    GemvSink<TM> sink{{}, g, 0u};
     decode_blocks<C, kLong>(g.d, sink, b0, b1);
+}
+
+// ------------------------------------------------- fused decode -> tcgen05 GEMM
+// Decompressing each matrix right before its multiplication ("Decompression
+// adaptee a l'inference GPU") taken to the tensor cores for batches T > 4:
+// the decoder's merge writes the BF16 weights straight into shared-memory
+// operand tiles of tcgen05.mma instead of global memory, so a block's weights
+// never reach HBM (only the compressed arrays are read).
+//
+// The matrices must be encoded in tile order: a [rows, cols] matrix (rows a
+// multiple of 128, cols of 64) as its 128 x 64 tiles, row tiles in order and
+// the 64-column k-tiles of a row tile in order, each tile row-major (the
+// format itself is unchanged; only the order of the elements is).  Then every
+// k-tile is 8192 consecutive elements of the stream, and a range of k-tiles is
+// a range of the stream.
+//
+// Work: the listed matrices' k-tiles, numbered in stream order, are split
+// evenly over the CTAs.  A CTA decodes the format blocks covering its range
+// (groups take them in turn, as in the decode kernel) and its decoder groups
+// merge each block into a ring of 128 x 64 BF16 tiles in the UMMA layout
+// (128-byte swizzle): element (r, c) of a tile at byte r * 128 + ((c / 8) XOR
+// (r mod 8)) * 16 + (c mod 8) * 2.  Each group makes its stores visible to the
+// async proxy, and after its next group barrier one thread counts the bytes
+// into the tile's mbarrier (complete_tx; a tile completes at 16384 bytes).  One
+// more warp consumes the tiles in order: one thread loads each k-tile's
+// activations X [n_pad x 64] by TMA (no multicast) and issues four UMMAs
+// (M = 128 rows of W, N = n_pad, K = 16) into an FP32 accumulator in tensor
+// memory, then releases the tile slot with tcgen05.commit; at the end of a
+// run of k-tiles of one row tile (a segment) four epilogue warps read the
+// accumulator (two buffers, so the next segment's MMAs need not wait) and add
+// it into Y with FP32 atomics.  Every wait is bounded; a timeout sets the
+// error bit 0x20 and lets the CTA finish without further waits.
+constexpr uint32_t kFusedMaxMats = 16;
+constexpr uint32_t kTileElems = 8192;   // 128 rows x 64 columns
+constexpr uint32_t kTileBytes = 16384;  // as BF16
+constexpr uint32_t kFusedErrTimeout = 0x20u;
+
+struct FusedMat {
+    uint32_t off;    // first element in the tensor (a multiple of 16)
+    uint32_t end;    // off + rows * cols
+    uint32_t kt;     // k-tiles per row tile: cols / 64
+    uint32_t rows;   // out features (a multiple of 128)
+    uint32_t tbase;  // number of k-tiles of the matrices before this one
+    float *y;        // [T][rows] FP32, accumulated into
+};
+
+struct FusedArgs {
+    DecodeArgs d;
+    FusedMat m[kFusedMaxMats];  // ordered by offset, not overlapping
+    uint32_t n_mats, T, n_pad;  // n_pad: T rounded up to 16 (UMMA N)
+    uint32_t n_tiles;           // k-tiles of all listed matrices
+    uint32_t ring, xring;       // W-tile and X-tile slots
+    uint32_t tmem_cols;         // power of two >= 2 * n_pad
+};
+
+struct FusedMaps {
+    CUtensorMap x[kFusedMaxMats];  // X_j [T, cols_j], box [n_pad, 64], 128-byte swizzle
+};
+
+// The shared-memory area after the decoder's: ring slots, barriers, flags.
+struct FusedSmem {
+    uint32_t wring, xring;  // 1024-aligned slot arrays
+    uint32_t xbytes;        // bytes of one X slot
+    uint32_t full0, empty0, xfull0, xempty0, accfull0, accempty0, final_bar;
+    uint32_t tmem_slot, abort_flag;
+};
+
+__device__ __forceinline__ FusedSmem fused_layout(const FusedArgs &f, uint32_t dec_end) {
+    FusedSmem L;
+    L.wring = (dec_end + 1023u) & ~1023u;
+    L.xbytes = f.n_pad * 128u;
+    L.xring = L.wring + f.ring * kTileBytes;
+    uint32_t b = L.xring + f.xring * L.xbytes;
+    L.full0 = b;
+    L.empty0 = b + 8u * f.ring;
+    L.xfull0 = b + 16u * f.ring;
+    L.xempty0 = L.xfull0 + 8u * f.xring;
+    L.accfull0 = L.xempty0 + 8u * f.xring;
+    L.accempty0 = L.accfull0 + 16u;
+    L.final_bar = L.accempty0 + 16u;
+    L.tmem_slot = L.final_bar + 8u;
+    L.abort_flag = L.tmem_slot + 4u;
+    return L;
+}
+
+// Bounded wait that gives up, for good, once any wait of the CTA timed out or
+// a block could not be placed (the CTA's abort flag, polled while waiting).
+// Between rounds of probes the thread sleeps `sleep_ns`, so that waiters that
+// are not on the critical path (the epilogue, a full ring) leave the issue
+// slots to the decoder warps.
+__device__ __forceinline__ bool fused_wait(uint32_t bar, uint32_t parity, uint32_t abort_flag, uint32_t &err,
+                                           uint32_t sleep_ns) {
+    for (uint32_t round = 0; round < (1u << 20); ++round) {
+        if (df11::tc::mbar_wait(bar, parity, 8u)) return true;
+        if (lds_u32(abort_flag)) return false;
+        if (sleep_ns) __nanosleep(sleep_ns);
+    }
+    err |= kFusedErrTimeout;
+    sts_u32(abort_flag, 1u);
+    return false;
+}
+
+// The k-tile at a global k-tile index: matrix, row tile and k-tile column.
+struct TileAt {
+    uint32_t j, rt, kt;
+};
+__device__ __forceinline__ TileAt tile_at(const FusedArgs &f, uint32_t K) {
+    uint32_t j = 0;
+    while (j + 1u < f.n_mats && K >= f.m[j + 1u].tbase) ++j;
+    const uint32_t lk = K - f.m[j].tbase;
+    return TileAt{j, lk / f.m[j].kt, lk % f.m[j].kt};
+}
+
+// The decoder side: the merge of a decoded block writes into the tile ring.
+// kStaged: the block's sign/mantissa bytes are staged in shared memory (else
+// read from global memory).
+template <bool kStaged>
+struct TileSink {
+    static constexpr uint32_t kNoTile = 0xFFFFFFFFu;
+    const FusedArgs &f;
+    FusedSmem L;
+    uint32_t K0, NT;     // this CTA's k-tiles [K0, K0 + NT)
+    uint32_t avail;      // local tiles [0, avail) are known to have a free slot
+    uint32_t m;          // matrix hint for the chunk search
+    uint32_t ta, tb;     // the local tiles of the block's first and last elements (a block meets at most two)
+    uint32_t ba, bb;     // bytes this thread wrote into them
+    uint32_t err;
+
+    // Local tile index of element g and its position in the tile; false if
+    // g is in no listed matrix or in another CTA's tiles.
+    __device__ __forceinline__ bool locate(uint32_t g, uint32_t &mm, uint32_t &i, uint32_t &p) const {
+        while (mm < f.n_mats && g >= f.m[mm].end) ++mm;
+        if (mm >= f.n_mats || g < f.m[mm].off) return false;
+        const uint32_t q = g - f.m[mm].off;
+        const uint32_t K = f.m[mm].tbase + q / kTileElems;
+        if (K < K0 || K - K0 >= NT) return false;
+        i = K - K0;
+        p = q % kTileElems;
+        return true;
+    }
+    // Waits until local tile i's slot no longer holds an unconsumed tile;
+    // false once the CTA has aborted (then nothing more is written or counted:
+    // a count that lands in a phase that never completes would push the tile
+    // mbarrier's transaction count out of its range).
+    __device__ __forceinline__ bool ensure(uint32_t i) {
+        if (i < avail) return true;
+        const uint32_t r = i / f.ring;
+        if (r > 0u && !fused_wait(L.empty0 + 8u * (i % f.ring), (r - 1u) & 1u, L.abort_flag, err, 64u))
+            return false;
+        avail = i + 1u;
+        return true;
+    }
+    __device__ __forceinline__ uint32_t slot_addr(uint32_t i, uint32_t p) const {
+        const uint32_t r = p >> 6, c = p & 63u;
+        return L.wring + (i % f.ring) * kTileBytes + r * 128u + ((((c >> 3) ^ (r & 7u))) << 4) + (c & 7u) * 2u;
+    }
+    __device__ __forceinline__ void tally(uint32_t i, uint32_t bytes) {
+        if (i == ta) ba += bytes;
+        else bb += bytes;
+    }
+
+    // Every thread of the group, before the block's merge.
+    __device__ __forceinline__ void begin_block(uint32_t s, uint32_t e) {
+        ta = tb = kNoTile;
+        ba = bb = 0u;
+        uint32_t mm = 0, i, p;
+        if (e <= s) return;
+        if (locate(s, mm, i, p)) ta = i;
+        mm = 0;
+        if (locate(e - 1u, mm, i, p) && i != ta) tb = i;
+    }
+
+    template <uint32_t kBufBytes>
+    __device__ __forceinline__ void chunks(uint32_t sb, uint32_t base, uint32_t c_first, uint32_t c_end,
+                                           uint32_t sm_s, uint32_t c_lo) {
+        for (uint32_t c = c_first; c < c_end; c += kGroupThreads) {
+            if (!DF11_BOUNDS_OK(16u * (c + 1u) <= kBufBytes && c >= c_lo &&
+                                (uint64_t)base + 16u * (c + 1u) <= f.d.n_elems &&
+                                (!kStaged || 16u * (c - c_lo + 1u) <= kBufBytes)))
+                continue;
+            // (unstaged: 16-byte loads from global memory, coalesced over the warp)
+            const uint4 smv = kStaged ? lds_u4(sm_s + 16u * (c - c_lo))
+                                      : __ldg(reinterpret_cast<const uint4 *>(f.d.sm + base + 16u * c));
+            const uint4 ex = lds_u4(sb + 16u * c);
+            sts_zero16(sb + 16u * c);
+            uint32_t i, p;
+            if (!locate(base + 16u * c, m, i, p) || !ensure(i)) continue;
+            uint32_t o[8];
+            merge16(smv, ex, o);
+            // 16 weights = two 16-byte pieces of one tile row (p is a multiple of 16)
+            const uint32_t r = p >> 6, j = (p & 63u) >> 3;
+            const uint32_t row = L.wring + (i % f.ring) * kTileBytes + r * 128u;
+            if (DF11_BOUNDS_OK(i < NT)) {
+                sts_u4(row + (((j) ^ (r & 7u)) << 4), o[0], o[1], o[2], o[3]);
+                sts_u4(row + (((j + 1u) ^ (r & 7u)) << 4), o[4], o[5], o[6], o[7]);
+            }
+            tally(i, 32u);
+        }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
+    __device__ __forceinline__ void edges(uint32_t sb, uint32_t base, uint32_t c_full, uint32_t span, uint32_t s,
+                                          uint32_t e, uint32_t lane) {
+        const bool head = s != base;
+        const bool tail = (span & 15u) != 0u && !(head && c_full == 0u);
+        const uint32_t c = (lane < 16u) ? 0u : c_full;
+        const bool mine = (lane < 16u) ? head : tail;
+        const uint32_t g = base + 16u * c + (lane & 15u);
+        uint32_t mm = 0, i, p;
+        if (mine && g >= s && g < e && DF11_BOUNDS_OK(g - base < kMaxCodesPerBlock + 16u) && locate(g, mm, i, p) &&
+            ensure(i)) {
+            const uint32_t sm8 = __ldg(f.d.sm + g);
+            const uint32_t rr = lds_u8(sb + (g - base));
+            const uint32_t hi8 = (sm8 & 0x80u) | (rr & 0x7Fu);
+            const uint32_t lo8 = (rr & 0x80u) | (sm8 & 0x7Fu);
+            asm volatile("st.shared.u16 [%0], %1;" ::"r"(slot_addr(i, p)), "h"((uint16_t)(lo8 | (hi8 << 8)))
+                         : "memory");
+            tally(i, 2u);
+        }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        __syncwarp();
+        if ((lane == 0u && head) || (lane == 16u && tail)) sts_zero16(sb + 16u * (lane == 0u ? 0u : c_full));
+    }
+    // After the block's merge (every thread of the group): each warp counts
+    // the bytes it wrote into the tiles' mbarriers right away (lane 0; the
+    // writers' stores were made visible to the async proxy, the warp sync
+    // gathers them, and the fence orders them before the relaxed count).  A
+    // block that failed its checks wrote nothing but still counts its range,
+    // so its tiles complete and the CTA finishes (the error word says the
+    // product is garbage); a block whose range cannot even be placed aborts the
+    // CTA's waits instead.
+    __device__ __forceinline__ void block_done(uint32_t s, uint32_t e, bool ok, bool range_ok) {
+        const uint32_t lane = threadIdx.x & 31u;
+        if (!range_ok) {
+            if ((threadIdx.x % kGroupThreads) == 0u) sts_u32(L.abort_flag, 1u);
+            return;
+        }
+        if (ok) {
+            __syncwarp();
+            const uint32_t a = __reduce_add_sync(0xFFFFFFFFu, ba), b = __reduce_add_sync(0xFFFFFFFFu, bb);
+            if (lane == 0u && (a | b) != 0u && !lds_u32(L.abort_flag)) {
+                asm volatile("fence.acq_rel.cta;" ::: "memory");
+                if (a) df11::tc::mbar_complete_tx(L.full0 + 8u * (ta % f.ring), a);
+                if (b) df11::tc::mbar_complete_tx(L.full0 + 8u * (tb % f.ring), b);
+            }
+        } else if ((threadIdx.x % kGroupThreads) == 0u && e > s) {
+            for (uint32_t q = 0; q < 2u; ++q) {
+                const uint32_t i = q == 0u ? ta : tb;
+                if (i == kNoTile || !ensure(i)) continue;  // the count must land in this round of the slot
+                uint32_t mm = 0, ii, p;
+                const uint32_t x = q == 0u ? s : e - 1u;
+                if (!locate(x, mm, ii, p)) continue;
+                const uint32_t ts = x - p, te = ts + kTileElems;
+                const uint32_t lo = s > ts ? s : ts, hi = e < te ? e : te;
+                if (lds_u32(L.abort_flag)) break;
+                asm volatile("fence.acq_rel.cta;" ::: "memory");
+                df11::tc::mbar_complete_tx(L.full0 + 8u * (i % f.ring), 2u * (hi - lo));
+            }
+        }
+    }
+    __device__ __forceinline__ void published(uint32_t) {}
+    __device__ __forceinline__ void finish(uint32_t, uint32_t) {}
+};
+
+constexpr uint32_t kFusedExtraThreads = 160;  // four epilogue warps and the MMA warp
+
+template <class C, bool kLong>
+__global__ void __launch_bounds__(C::kCtaThreads + kFusedExtraThreads, 1)
+    df11_decode_gemm_kernel(const __grid_constant__ FusedArgs f, const __grid_constant__ FusedMaps maps) {
+    extern __shared__ __align__(128) uint8_t smem[];  // the tile rings are aligned to 1024 by hand
+    const uint32_t s_base = smem_addr(smem);
+    const uint32_t tid = threadIdx.x;
+    constexpr uint32_t kDec = C::kCtaThreads;  // decoder threads; then 4 epilogue warps and the MMA warp
+    const FusedSmem L = fused_layout(f, s_base + C::kSmemBytes);
+    const uint32_t K0 = (uint32_t)((uint64_t)f.n_tiles * blockIdx.x / gridDim.x);
+    const uint32_t K1 = (uint32_t)((uint64_t)f.n_tiles * (blockIdx.x + 1u) / gridDim.x);
+    const uint32_t NT = K1 - K0;
+    uint32_t err = 0;
+
+    if (!load_tables<C>(f.d.lut, f.d.err, smem, s_base, tid)) return;  // uniform over the CTA
+    if (tid == 0) {
+        for (uint32_t s = 0; s < f.ring; ++s) {
+            df11::tc::mbar_init(L.full0 + 8u * s, 1);
+            df11::tc::mbar_init(L.empty0 + 8u * s, 1);
+        }
+        for (uint32_t s = 0; s < f.xring; ++s) {
+            df11::tc::mbar_init(L.xfull0 + 8u * s, 1);
+            df11::tc::mbar_init(L.xempty0 + 8u * s, 1);
+        }
+        for (uint32_t a = 0; a < 2u; ++a) {
+            df11::tc::mbar_init(L.accfull0 + 8u * a, 1);
+            df11::tc::mbar_init(L.accempty0 + 8u * a, 4);  // one arrival per epilogue warp
+        }
+        df11::tc::mbar_init(L.final_bar, 1);
+        sts_u32(L.abort_flag, 0u);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (tid >= kDec && tid < kDec + 32u) {  // the first epilogue warp allocates the accumulators
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(L.tmem_slot),
+                     "r"(f.tmem_cols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    __syncthreads();
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    const uint32_t tmem = lds_u32(L.tmem_slot);
+
+    if (tid < kDec) {
+        // ---- decoders: the format blocks covering elements of k-tiles [K0, K1)
+        const uint32_t lane = tid & 31u;
+        const TileAt a0 = tile_at(f, K0), a1 = tile_at(f, K1 - 1u);
+        const FusedMat &m0 = f.m[a0.j], &m1 = f.m[a1.j];
+        const uint64_t e_first = m0.off + (uint64_t)(K0 - m0.tbase) * kTileElems;
+        const uint64_t e_last = m1.off + (uint64_t)(K1 - m1.tbase) * kTileElems - 1u;
+        const uint64_t b0 = find_block(f.d.bstart, f.d.n_blocks, e_first, lane);
+        const uint64_t b1 = find_block(f.d.bstart, f.d.n_blocks, e_last, lane) + 1u;
+        TileSink<C::kStageSm> sink{f, L, K0, NT, 0u, 0u, 0u, 0u, 0u, 0u, 0u};  // (tiles set per block)
+        const uint32_t group = tid / kGroupThreads;
+        decode_loop<C, kLong>(f.d, sink, b0 + group, C::kGroups, b1);
+        err |= sink.err;
+    } else if (tid >= kDec + 128u) {
+        // ---- the MMA warp: one thread issues the MMAs and loads X
+        if (tid == kDec + 128u) {
+            const uint32_t idesc = df11::tc::instr_desc_bf16(f.n_pad, 128u);
+            // X tile of local k-tile i into slot i % xring
+            auto load_x = [&](uint32_t i) {
+                const uint32_t xs = i % f.xring, xr = i / f.xring;
+                if (xr > 0u && !fused_wait(L.xempty0 + 8u * xs, (xr - 1u) & 1u, L.abort_flag, err, 0u)) return;
+                const TileAt t = tile_at(f, K0 + i);
+                df11::tc::mbar_arrive_expect_tx(L.xfull0 + 8u * xs, L.xbytes);
+                df11::tc::tma_load_2d(L.xring + xs * L.xbytes, &maps.x[t.j], L.xfull0 + 8u * xs,
+                                      (int32_t)(t.kt * 64u), 0);
+            };
+            // X tiles are loaded `look` tiles ahead, each into the slot of the
+            // tile two before the current one, whose MMA has long finished
+            const uint32_t look = f.xring - 2u;
+            for (uint32_t i = 0; i < look && i < NT; ++i) load_x(i);
+            uint32_t seg = 0;  // segments started
+            for (uint32_t i = 0; i < NT; ++i) {
+                // once aborted, arm no more phases (a second arrival on a phase
+                // that never completed is not allowed)
+                if (lds_u32(L.abort_flag)) break;
+                if (i + look < NT) load_x(i + look);
+                const TileAt t = tile_at(f, K0 + i);
+                const bool first = (i == 0u) || t.kt == 0u;
+                const bool last = (i + 1u == NT) || t.kt + 1u == f.m[t.j].kt;
+                const uint32_t abuf = seg & 1u;
+                // the accumulator buffer's previous segment has been drained
+                if (first && seg >= 2u)
+                    fused_wait(L.accempty0 + 8u * abuf, ((seg >> 1) - 1u) & 1u, L.abort_flag, err, 64u);
+                const uint32_t s = i % f.ring, r = i / f.ring;
+                df11::tc::mbar_arrive_expect_tx(L.full0 + 8u * s, kTileBytes);  // this round's tile
+                const uint32_t xs = i % f.xring, xr = i / f.xring;
+                const bool ok = fused_wait(L.full0 + 8u * s, r & 1u, L.abort_flag, err, 32u) &&
+                                fused_wait(L.xfull0 + 8u * xs, xr & 1u, L.abort_flag, err, 0u);
+                if (ok) {
+                    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+                    const uint32_t wa = L.wring + s * kTileBytes, xa = L.xring + xs * L.xbytes;
+#pragma unroll
+                    for (uint32_t kk = 0; kk < 4u; ++kk)  // K = 16 per UMMA: 32 bytes along the swizzled row
+                        df11::tc::umma_bf16(tmem + abuf * f.n_pad, df11::tc::smem_desc_sw128(wa + kk * 32u),
+                                            df11::tc::smem_desc_sw128(xa + kk * 32u), idesc,
+                                            (first && kk == 0u) ? 0u : 1u);
+                }
+                df11::tc::umma_commit(L.empty0 + 8u * s);
+                df11::tc::umma_commit(L.xempty0 + 8u * xs);
+                if (last) {
+                    df11::tc::umma_commit(L.accfull0 + 8u * abuf);
+                    ++seg;
+                }
+            }
+            // every issued MMA has completed before the accumulators are freed
+            // (not skipped on abort: issued MMAs finish on their own)
+            df11::tc::umma_commit(L.final_bar);
+            if (!df11::tc::mbar_wait(L.final_bar, 0u)) err |= kFusedErrTimeout;
+        }
+        __syncwarp();
+    } else {
+        // ---- epilogue: warp ew (0..3) reads TMEM lanes 32 ew .. 32 ew + 31 (rows
+        // of the row tile) of each segment's accumulator and adds them into Y
+        const uint32_t ew = (tid - kDec) >> 5, lane = tid & 31u;
+        uint32_t seg = 0;
+        for (uint32_t i = 0; i < NT; ++i) {
+            const TileAt t = tile_at(f, K0 + i);
+            if (!((i + 1u == NT) || t.kt + 1u == f.m[t.j].kt)) continue;  // not the end of a segment
+            const uint32_t abuf = seg & 1u;
+            const bool have = fused_wait(L.accfull0 + 8u * abuf, (seg >> 1) & 1u, L.abort_flag, err, 256u);
+            asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+            const FusedMat &M = f.m[t.j];
+            const uint32_t row = t.rt * 128u + ew * 32u + lane;
+            for (uint32_t c0 = 0; c0 < f.n_pad; c0 += 16u) {
+                uint32_t v[16];
+                df11::tc::tmem_ld16(tmem + ((ew * 32u) << 16) + abuf * f.n_pad + c0, v);
+                if (have) {
+#pragma unroll
+                    for (uint32_t q = 0; q < 16u; ++q)
+                        if (c0 + q < f.T) atomicAdd(M.y + (uint64_t)(c0 + q) * M.rows + row, __uint_as_float(v[q]));
+                }
+            }
+            asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+            __syncwarp();
+            if (lane == 0u) df11::tc::mbar_arrive(L.accempty0 + 8u * abuf);
+            ++seg;
+        }
+    }
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    __syncthreads();
+    if (tid >= kDec && tid < kDec + 32u) {
+        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(f.tmem_cols)
+                     : "memory");
+    }
+    if (err && f.d.err) atomicOr(f.d.err, err);
 }
 
 // ----------------------------------------------------------------- host
@@ -1560,9 +2016,116 @@ df11_status launch_gemv(const df11_tensor *t, const df11_gemv_mat *mats, uint32_
     return DF11_OK;
 }
 
+// ---- fused decode -> GEMM launcher
+constexpr uint32_t kSmemLimit = 227u * 1024u;
+constexpr uint32_t kFusedTail = 1024u + 256u;  // alignment slack of the rings, barriers and flags
+
+template <class C>
+bool fused_fit(uint32_t n_pad, uint32_t &ring, uint32_t &xring, uint32_t &smem) {
+    const uint32_t xbytes = 128u * n_pad;
+    // X slots: loads run xring - 2 = 1 tile ahead of the MMAs (the decoders,
+    // not the X loads, set the pace: a tile every few microseconds per CTA)
+    xring = 3u;
+    if (C::kSmemBytes + kFusedTail + xring * xbytes + 2u * kTileBytes > kSmemLimit) return false;
+    ring = (kSmemLimit - C::kSmemBytes - kFusedTail - xring * xbytes) / kTileBytes;
+    if (ring > 8u) ring = 8u;
+    smem = C::kSmemBytes + kFusedTail + xring * xbytes + ring * kTileBytes;
+    return true;
+}
+
+template <class C, bool kLong>
+cudaError_t fused_launch(const FusedArgs &f, const FusedMaps &maps, uint32_t smem, unsigned grid, cudaStream_t s) {
+    cudaError_t e = cudaFuncSetAttribute(df11_decode_gemm_kernel<C, kLong>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemLimit);
+    if (e != cudaSuccess) return e;
+    df11_decode_gemm_kernel<C, kLong><<<grid, C::kCtaThreads + kFusedExtraThreads, smem, s>>>(f, maps);
+    return cudaGetLastError();
+}
+
+df11_status launch_fused(const df11_tensor *t, const df11_gemv_mat *mats, uint32_t n_mats, uint32_t T,
+                         uint32_t *err_word, void *stream) {
+    if (!t) return DF11_ERR_INVALID_ARG;
+    df11_status st = df11_validate(t);
+    if (st != DF11_OK) return st;
+    if (n_mats == 0) return DF11_OK;
+    if (!mats) return DF11_ERR_INVALID_ARG;
+    if (n_mats > kFusedMaxMats || T < 1u || T > 256u || !t->counts) return DF11_ERR_UNSUPPORTED;
+    FusedArgs f;
+    st = prepare_args(t, f.d);
+    if (st != DF11_OK) return st;
+    Inst inst;
+    bool lng;
+    pick_instance(t, inst, lng);
+    if (inst != Inst::kTypicalC) return DF11_ERR_UNSUPPORTED;  // blocks larger than the fused kernel's buffers
+    uint64_t prev_end = 0, tiles = 0;
+    for (uint32_t j = 0; j < n_mats; ++j) {
+        const df11_gemv_mat &mj = mats[j];
+        if (mj.rows == 0 || mj.cols == 0 || !mj.x || !mj.y || !aligned16(mj.x) || ((uintptr_t)mj.y & 3u) ||
+            (mj.elem_offset & 15u))
+            return DF11_ERR_INVALID_ARG;
+        if (mj.rows % 128u || mj.cols % 64u) return DF11_ERR_UNSUPPORTED;
+        const uint64_t size = (uint64_t)mj.rows * mj.cols;
+        if (mj.elem_offset < prev_end || mj.elem_offset > t->n_elems || size > t->n_elems - mj.elem_offset)
+            return DF11_ERR_INVALID_ARG;
+        FusedMat &M = f.m[j];
+        M.off = (uint32_t)mj.elem_offset;  // n_elems < 2^32 (df11_validate)
+        M.end = (uint32_t)(mj.elem_offset + size);
+        M.kt = mj.cols / 64u;
+        M.rows = mj.rows;
+        M.tbase = (uint32_t)tiles;
+        M.y = mj.y;
+        tiles += size / kTileElems;
+        prev_end = mj.elem_offset + size;
+    }
+    for (uint32_t j = n_mats; j < kFusedMaxMats; ++j) f.m[j] = FusedMat{};
+    f.n_mats = n_mats;
+    f.T = T;
+    f.n_pad = (T + 15u) & ~15u;
+    f.n_tiles = (uint32_t)tiles;
+    f.tmem_cols = 32u;
+    while (f.tmem_cols < 2u * f.n_pad) f.tmem_cols <<= 1;
+    f.d.err = err_word;
+    FusedMaps maps;
+    for (uint32_t j = 0; j < n_mats; ++j)
+        if (!df11::tc::make_bf16_tile_map(&maps.x[j], mats[j].x, T, mats[j].cols, f.n_pad)) return DF11_ERR_CUDA;
+    for (uint32_t j = n_mats; j < kFusedMaxMats; ++j) maps.x[j] = maps.x[0];
+    int sms = 0;
+    st = prepare_device(&sms);
+    if (st != DF11_OK) return st;
+    const unsigned grid = (unsigned)(f.n_tiles < (uint32_t)sms ? f.n_tiles : (uint32_t)sms);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    // six decode groups when the rings leave room for 4 operand tiles, else four
+#ifndef DF11_FUSED_GROUPS
+#define DF11_FUSED_GROUPS 0  // 0: by the rule above; 4 or 6: forced
+#endif
+    uint32_t smem = 0;
+    cudaError_t e;
+    // the most decode groups whose rings still hold 4 operand tiles (3 with
+    // the largest X tiles, which also leave no room to stage sign/mantissa)
+    if (DF11_FUSED_GROUPS != 4 && fused_fit<CfgFused6>(f.n_pad, f.ring, f.xring, smem) &&
+        (f.ring >= 4u || DF11_FUSED_GROUPS == 6)) {
+        e = lng ? fused_launch<CfgFused6, true>(f, maps, smem, grid, s)
+                : fused_launch<CfgFused6, false>(f, maps, smem, grid, s);
+    } else if (fused_fit<CfgFused4>(f.n_pad, f.ring, f.xring, smem) && f.ring >= 4u) {
+        e = lng ? fused_launch<CfgFused4, true>(f, maps, smem, grid, s)
+                : fused_launch<CfgFused4, false>(f, maps, smem, grid, s);
+    } else if (fused_fit<CfgFused4U>(f.n_pad, f.ring, f.xring, smem)) {
+        e = lng ? fused_launch<CfgFused4U, true>(f, maps, smem, grid, s)
+                : fused_launch<CfgFused4U, false>(f, maps, smem, grid, s);
+    } else {
+        return DF11_ERR_UNSUPPORTED;
+    }
+    return e == cudaSuccess ? DF11_OK : DF11_ERR_CUDA;
+}
+
 }  // namespace
 
 extern "C" {
+
+df11_status df11_decode_gemm(const df11_tensor *t, const df11_gemv_mat *mats, uint32_t n_mats, uint32_t T,
+                             uint32_t *err_word, void *stream) {
+    return launch_fused(t, mats, n_mats, T, err_word, stream);
+}
 
 df11_status df11_decode(const df11_tensor *t, uint16_t *out, uint32_t *err_word, void *stream) {
     return launch_decode(t, out, err_word, stream);

@@ -33,6 +33,7 @@
 #include <mutex>
 
 #include "df11.h"
+#include "df11_tc.cuh"
 
 namespace {
 
@@ -43,7 +44,6 @@ constexpr uint32_t kThreads = 128;
 constexpr uint32_t kMaxStages = 8;
 constexpr uint32_t kSmemBudget = 200u * 1024u;
 constexpr uint32_t kGemmErrTimeout = 0x20u;
-constexpr uint32_t kSpin = 1u << 24;   // bounded waits
 
 struct GemmArgs {
     float *y;
@@ -58,66 +58,7 @@ struct GemmArgs {
     uint32_t atomic_out; // 1: add into Y (split-K), 0: store
 };
 
-__device__ __forceinline__ uint32_t smem_u32(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
-
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
-    uint32_t done = 0;
-    for (uint32_t it = 0; it < kSpin && !done; ++it) {
-        asm volatile(
-            "{\n\t.reg .pred p;\n\t"
-            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-            "selp.u32 %0, 1, 0, p;\n\t}"
-            : "=r"(done)
-            : "r"(bar), "r"(parity)
-            : "memory");
-    }
-    return done != 0;
-}
-
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, uint32_t bar, int32_t x,
-                                            int32_t y) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];" ::"r"(
-            dst),
-        "l"(map), "r"(bar), "r"(x), "r"(y)
-        : "memory");
-}
-
-// Shared-memory matrix descriptor for a K-major tile written by TMA with the
-// 128-byte swizzle: rows of 128 bytes, 8-row groups 1024 bytes apart.
-__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr) {
-    uint64_t d = 0;
-    d |= (uint64_t)((addr >> 4) & 0x3FFFu);        // start address
-    d |= (uint64_t)1u << 16;                       // leading byte offset (unused with swizzle)
-    d |= (uint64_t)(1024u >> 4) << 32;             // stride byte offset: 8 rows x 128 B
-    d |= (uint64_t)1u << 46;                       // descriptor version (sm_100)
-    d |= (uint64_t)2u << 61;                       // layout: 128-byte swizzle
-    return d;
-}
-
-// Instruction descriptor: BF16 x BF16 -> FP32, both operands K-major.
-__device__ __forceinline__ uint32_t instr_desc_bf16(uint32_t n, uint32_t m) {
-    return (1u << 4)            // D format F32
-           | (1u << 7)          // A format BF16
-           | (1u << 10)         // B format BF16
-           | ((n >> 3) << 17)   // N / 8
-           | ((m >> 4) << 24);  // M / 16
-}
-
-__device__ __forceinline__ void umma_bf16(uint32_t tmem_d, uint64_t da, uint64_t db, uint32_t idesc,
-                                          uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
-        "l"(da), "l"(db), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-
-__device__ __forceinline__ void umma_commit(uint32_t bar) {
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
-                 : "memory");
-}
+using namespace df11::tc;
 
 __global__ void __launch_bounds__(kThreads, 1)
     df11_gemm_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUtensorMap map_x,
@@ -205,13 +146,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t row = m_tile * kBlockM + warp * 32u + lane;
     for (uint32_t c0 = 0; c0 < g.n_pad; c0 += 16u) {
         uint32_t v[16];
-        asm volatile(
-            "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
-            "%14, %15}, [%16];"
-            : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
-              "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
-            : "r"(tmem_d + ((warp * 32u) << 16) + c0));
-        asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+        tmem_ld16(tmem_d + ((warp * 32u) << 16) + c0, v);
         if (have) {
 #pragma unroll
             for (uint32_t j = 0; j < 16; ++j) {
@@ -364,9 +299,16 @@ bool get_encoder() {
     return g_encode != nullptr;
 }
 
+bool make_map(CUtensorMap *m, const void *ptr, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+    return df11::tc::make_bf16_tile_map(m, ptr, rows, cols, box_rows);
+}
+
+}  // namespace
+
 // 2-D BF16 tensor map over a row-major [rows, cols] matrix, box [box_rows, 64]
 // with the 128-byte swizzle; rows past the end read as zero.
-bool make_map(CUtensorMap *m, const void *ptr, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+bool df11::tc::make_bf16_tile_map(CUtensorMap *m, const void *ptr, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+    if (!get_encoder()) return false;
     const cuuint64_t dims[2] = {cols, rows};
     const cuuint64_t strides[1] = {cols * 2u};
     const cuuint32_t box[2] = {kBlockK, box_rows};
@@ -375,8 +317,6 @@ bool make_map(CUtensorMap *m, const void *ptr, uint64_t rows, uint64_t cols, uin
                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
-
-}  // namespace
 
 extern "C" df11_status df11_gemm_bf16(const uint16_t *x, const uint16_t *w, float *y, uint32_t T, uint32_t out,
                                       uint32_t in, uint32_t *err_word, void *stream) {

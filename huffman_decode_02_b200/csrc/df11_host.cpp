@@ -609,6 +609,36 @@ df11_status df11_encode(const uint16_t *bf16, uint64_t n, df11_tensor *t) {
     return df11_encode_multi(mats, sizes, 1, t);
 }
 
+// Tile order (the fused decode -> GEMM's element order): 128 x 64 tiles, row
+// tiles in order, the k-tiles of a row tile in order, each tile row-major.
+df11_status df11_to_tile_order(const uint16_t *w, uint32_t rows, uint32_t cols, uint16_t *out) {
+    if (!w || !out) return DF11_ERR_INVALID_ARG;
+    if (rows == 0 || cols == 0 || rows % 128u || cols % 64u) return DF11_ERR_UNSUPPORTED;
+    const uint32_t kt = cols / 64u;
+    parallel_tasks(rows / 128u, [&](size_t rt) {
+        for (uint32_t k = 0; k < kt; ++k) {
+            uint16_t *dst = out + ((uint64_t)rt * kt + k) * 8192u;
+            for (uint32_t r = 0; r < 128u; ++r)
+                std::memcpy(dst + 64u * r, w + ((uint64_t)rt * 128u + r) * cols + 64u * k, 128);
+        }
+    });
+    return DF11_OK;
+}
+
+df11_status df11_from_tile_order(const uint16_t *tiled, uint32_t rows, uint32_t cols, uint16_t *out) {
+    if (!tiled || !out) return DF11_ERR_INVALID_ARG;
+    if (rows == 0 || cols == 0 || rows % 128u || cols % 64u) return DF11_ERR_UNSUPPORTED;
+    const uint32_t kt = cols / 64u;
+    parallel_tasks(rows / 128u, [&](size_t rt) {
+        for (uint32_t k = 0; k < kt; ++k) {
+            const uint16_t *src = tiled + ((uint64_t)rt * kt + k) * 8192u;
+            for (uint32_t r = 0; r < 128u; ++r)
+                std::memcpy(out + ((uint64_t)rt * 128u + r) * cols + 64u * k, src + 64u * r, 128);
+        }
+    });
+    return DF11_OK;
+}
+
 df11_status df11_validate(const df11_tensor *t) {
     if (!t) return DF11_ERR_INVALID_ARG;
     const df11_params &p = t->params;

@@ -73,7 +73,7 @@ class BlockStreamer:
         desc = _Tensor.from_buffer_copy(b.desc)
         if "counts" not in self.keys:
             desc.counts_bytes = 0
-        return DF11Tensor(desc, arrays, str(self.device), b.shapes, b.offsets)
+        return DF11Tensor(desc, arrays, str(self.device), b.shapes, b.offsets, b.tiled)
 
     def _copy(self, b: DF11Tensor, slot: int):
         for k in self.keys:

@@ -321,6 +321,43 @@ typedef struct df11_gemv_mat {
 df11_status df11_decode_gemv(const df11_tensor *t, const df11_gemv_mat *mats, uint32_t n_mats, uint32_t T,
                              uint32_t *err_word, void *stream);
 
+/* Fused decode and matrix multiplication on the tensor cores (any batch
+ * 1 <= T <= 256; meant for T > 4, where df11_decode_gemv's CUDA-core product
+ * stops paying): for each listed matrix, y += x * W^T with W decoded on the
+ * fly into shared-memory operand tiles of tcgen05.mma and never written to
+ * memory.  The pages decompress each matrix right before its multiplication
+ * and discard it after ("Decompression adaptee a l'inference GPU"); here the
+ * decoded tiles go straight from the decoder to the tensor cores, so only the
+ * compressed arrays are read from HBM.
+ *  The listed matrices must be encoded in TILE ORDER (df11_to_tile_order):
+ *  the same DF11 format, with each matrix's elements ordered as its 128 x 64
+ *  tiles (row tiles in order, the 64-column tiles of a row tile in order, each
+ *  tile row-major), so that every tile is a contiguous piece of the stream.
+ *  mats: as for df11_decode_gemv (HOST array, <= 16 descriptors ordered by
+ *        elem_offset, not overlapping; x [T, cols] BF16 16-byte aligned; y
+ *        [T, rows] FP32 4-byte aligned, ADDED INTO: zero it first for a plain
+ *        product), with rows a multiple of 128 and cols a multiple of 64.
+ *  The tensor must carry its per-thread counts (t->counts), and its blocks
+ *  must be LLM-like (at most 7137 codes per thread block, df11_tensor's
+ *  max_block_codes); otherwise DF11_ERR_UNSUPPORTED.  So are T outside
+ *  1..256, more than 16 matrices, and rows / cols off those multiples.
+ *  FP32 accumulation in tensor memory; the partial sums of a row tile that two
+ *  CTAs share are added with FP32 atomics, so the last bits of y may differ
+ *  run to run.  A wait that timed out sets bit 0x20 of err_word.  One launch,
+ *  asynchronous on `stream`; n_mats == 0 is a no-op. */
+df11_status df11_decode_gemm(const df11_tensor *t, const df11_gemv_mat *mats, uint32_t n_mats, uint32_t T,
+                             uint32_t *err_word, void *stream);
+
+/* Tile order for df11_decode_gemm (host, plain copies): df11_to_tile_order
+ * writes the row-major [rows, cols] BF16 matrix w (rows a multiple of 128,
+ * cols of 64) into out as its 128 x 64 tiles (row tiles in order, the
+ * 64-column tiles of a row tile in order, each tile row-major);
+ * df11_from_tile_order is the inverse.  w and out must not overlap;
+ * DF11_ERR_INVALID_ARG for NULL pointers, DF11_ERR_UNSUPPORTED for other
+ * shapes. */
+df11_status df11_to_tile_order(const uint16_t *w, uint32_t rows, uint32_t cols, uint16_t *out);
+df11_status df11_from_tile_order(const uint16_t *tiled, uint32_t rows, uint32_t cols, uint16_t *out);
+
 /* Consumer of a decoded weight matrix: Y = X * W^T with BF16 inputs and FP32
  * accumulation, the matrix multiplication the decompressed weights feed
  * ("Decompression adaptee a l'inference GPU": a matrix is decompressed right

@@ -90,3 +90,27 @@ def test_decode_paths_without_bounds_errors(debug_lib):
             ref = xs[j].cpu().double() @ w64.T
             assert float((ys[j].cpu().double() - ref).norm() / ref.norm()) < 1e-5
     assert debug_lib.df11_debug_bounds_errors(1) == 0
+
+
+def test_fused_gemm_without_bounds_errors(debug_lib):
+    """The fused decode -> tensor-core GEMM through the bounds-checked build
+    (every data-dependent shared-memory index of its decoder, the tile-ring
+    stores included): no failed check, the product within 2e-3."""
+    dev = _dev()
+    mats = [workloads.normal_matrix(256, 128, 0.02, seed=1), workloads.normal_matrix(1, 64, 0.02, seed=2)[0],
+            workloads.normal_matrix(512, 320, 0.03, seed=3)]
+    rng = np.random.default_rng(5)
+    x = (rng.standard_t(3, (256, 512)) * 0.015).astype(np.float32)
+    x[rng.random(x.shape) < 0.001] *= 1000.0
+    for blk_mats, p in ((mats, df11.Params()), ([workloads.round_to_bf16(x)], df11.Params(max_code_len=32))):
+        blk = df11.encode_multi(blk_mats, p, tile_order=True).to(dev)
+        idx = [j for j in range(len(blk_mats)) if blk.tiled[j]]
+        for T in (16, 96):
+            xs = {j: torch.randn(T, blk_mats[j].shape[1], generator=torch.Generator().manual_seed(j))
+                  .to(torch.bfloat16).to(dev) for j in idx}
+            ys = df11.decode_gemm(blk, xs)
+            for j in idx:
+                w64 = torch.from_numpy(np.ascontiguousarray(blk_mats[j]).view(np.int16)).view(torch.bfloat16).double()
+                ref = xs[j].cpu().double() @ w64.T
+                assert float((ys[j].cpu().double() - ref).norm() / ref.norm()) < 2e-3
+    assert debug_lib.df11_debug_bounds_errors(1) == 0

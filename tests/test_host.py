@@ -379,3 +379,68 @@ def test_header_compiles_as_plain_c(tmp_path):
                         os.path.join(ROOT, "include"), "-c", str(src), "-o", str(tmp_path / "use_df11.o")],
                        capture_output=True, text=True)
     assert r.returncode == 0, r.stderr
+
+
+def test_tile_order_round_trip_and_layout():
+    """Tile order against an independent numpy route: the [rows, cols] matrix
+    as [rows/128, 128, cols/64, 64], axes (0, 2, 1, 3), flattened; and the
+    inverse restores the matrix."""
+    w = workloads.normal_matrix(384, 192, 0.02, seed=31)
+    t = df11.to_tile_order(w)
+    ref = w.reshape(3, 128, 3, 64).transpose(0, 2, 1, 3).reshape(-1)
+    np.testing.assert_array_equal(t, ref)
+    np.testing.assert_array_equal(df11.from_tile_order(t, 384, 192), w)
+    lib = df11._lib()
+    buf = np.zeros(64 * 64, dtype=np.uint16)
+    assert lib.df11_to_tile_order(ctypes.c_void_p(buf.ctypes.data), 64, 64, ctypes.c_void_p(buf.ctypes.data)) == 2
+    assert lib.df11_to_tile_order(None, 128, 64, ctypes.c_void_p(buf.ctypes.data)) == 1
+
+
+def test_encode_multi_tile_order_flags():
+    mats = [workloads.normal_matrix(256, 128, 0.02, seed=1), workloads.normal_matrix(1, 128, 0.02, seed=2)[0],
+            workloads.normal_matrix(100, 64, 0.02, seed=3)]
+    blk = df11.encode_multi(mats, tile_order=True)
+    assert blk.tiled == [True, False, False]
+    flat = np.concatenate([df11.to_tile_order(mats[0]), mats[1].reshape(-1), mats[2].reshape(-1)])
+    np.testing.assert_array_equal(blk.host_array("enc"), df11.encode(flat).host_array("enc"))
+
+
+def test_decode_gemm_argument_checks():
+    """df11_decode_gemm refuses bad calls before any GPU work: a tensor
+    without per-thread counts, T outside 1..256, rows not a multiple of 128 or
+    cols of 64 are unsupported; misaligned, overlapping or out-of-range
+    matrices and NULL vectors are invalid; no matrices is a no-op."""
+    lib = df11._lib()
+    mats = [workloads.normal_matrix(128, 64, 0.02, seed=1), workloads.normal_matrix(256, 128, 0.02, seed=2)]
+    t = df11.encode_multi(mats, tile_order=True)
+    keep = []
+
+    def bind(tt):
+        d = tt._bind()
+        for name in tt.arrays:
+            v, owner = _aligned_copy(tt.host_array(name))
+            keep.append(owner)
+            setattr(d, name, v.ctypes.data)
+        return d
+
+    d, dn = bind(t), bind(t.without_counts())
+    xbuf, xown = _aligned_copy(np.zeros(256 * 128 + 8, dtype=np.uint16))
+    ybuf = np.zeros(256 * 256 + 4, dtype=np.float32)
+    X, Y = xbuf.ctypes.data, ybuf.ctypes.data
+
+    def call(descs, T=16, n=None, dd=None):
+        arr = (df11._GemvMat * max(1, len(descs)))(*[df11._GemvMat(*m) for m in descs])
+        return lib.df11_decode_gemm(ctypes.byref(dd or d), arr, len(descs) if n is None else n, T, None, None)
+
+    good = [(0, 128, 64, X, Y), (8192, 256, 128, X, Y)]
+    assert call(good, n=0) == 0
+    assert call(good, dd=dn) == 2                              # no stored counts
+    assert call(good, T=0) == 2 and call(good, T=257) == 2
+    assert call([(0, 64, 128, X, Y)]) == 2                     # rows not a multiple of 128
+    assert call([(0, 128, 32, X, Y)]) == 2                     # cols not a multiple of 64
+    assert call([(8, 128, 64, X, Y)]) == 1                     # offset not a multiple of 16
+    assert call([(0, 128, 64, X + 2, Y)]) == 1                 # x not 16-byte aligned
+    assert call([(0, 128, 64, None, Y)]) == 1                  # NULL x
+    assert call([(8192, 256, 128, X, Y), (0, 128, 64, X, Y)]) == 1   # out of order
+    assert call([(16384, 256, 128, X, Y)]) == 1                # runs past the tensor's end
+    assert call(good * 9) == 2                                 # more than 16 matrices
