@@ -180,6 +180,7 @@ using CfgDenseC = Cfg<4, 16400, 2, false>;
 using CfgFused6 = Cfg<6, 7152, 1, false>;          // T <= 64
 using CfgFused4 = Cfg<4, 7152, 1, false>;          // T <= 128
 using CfgFused4U = Cfg<4, 7152, 1, false, false>;  // T <= 256: no sign/mantissa staging
+using CfgFused6U = Cfg<6, 7152, 1, false, false>;
 
 struct DecodeArgs {
     const uint8_t *enc;
@@ -701,12 +702,16 @@ struct StoreSink : NoHooks {
 
 // The persistent decode loop of one group (the tables are loaded): the group
 // decodes format blocks blk, blk + stride, ... below blk_end and hands every
-// decoded block to the sink.
+// decoded block to the sink.  With `counter` (the shared-memory address of a
+// u32 holding the CTA's next block; 0: the fixed stride) the groups instead
+// take the CTA's blocks in order from that counter, whichever group is free
+// first (the group's leader takes one at each first barrier and passes it on
+// through the group's aux word, which the others read after the second).
 // kLong: compiled with the long-code path (codes longer than the table
 // windows); without it the loops carry no escape handling at all.
 template <class C, bool kLong, class Sink>
 __device__ __forceinline__ void decode_loop(const DecodeArgs &a, Sink &sink, uint64_t blk, uint64_t stride,
-                                            uint64_t blk_end) {
+                                            uint64_t blk_end, uint32_t counter = 0u) {
     extern __shared__ __align__(128) uint8_t smem[];
     const uint32_t s_base = smem_addr(smem);
     const uint32_t s_lim = s_base + kOffLim;
@@ -735,16 +740,22 @@ __device__ __forceinline__ void decode_loop(const DecodeArgs &a, Sink &sink, uin
 
     // ---- the group's mbarriers (inputs of the next block; first
     // sign/mantissa vectors of this one) and its first block's inputs
+    const uint32_t aux = grp + C::kGrpAux;
     if (lt == 0) {
         mbar_init(mb_in);
         mbar_init(mb_sm);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        if (counter) {
+            blk = atomicAdd(reinterpret_cast<uint32_t *>(smem + (counter - s_base)), 1u);
+            sts_u32(aux, (uint32_t)blk);
+        }
         if (blk < blk_end) issue_inputs<C>(a, blk, grp, mb_in);
     }
     group_barrier(group);
+    if (counter) blk = lds_u32(aux);
     uint32_t ph_in = 0, ph_sm = 0;
 
-    for (; blk < blk_end; blk += stride) {
+    while (blk < blk_end) {
         if (!wait_phase(mb_in, ph_in)) my_err |= kKernErrTimeout;
         ph_in ^= 1u;
         const uint64_t tA = blk * (uint64_t)kThreadsPerBlockFmt + 2u * lt;
@@ -793,8 +804,14 @@ __device__ __forceinline__ void decode_loop(const DecodeArgs &a, Sink &sink, uin
         if (lane == 31u) sts_u32(wtot + 4u * warp, incl);
         group_barrier(group);
         // every thread has read this block's staged inputs: fetch the next
-        const uint64_t nxt = blk + stride;
-        if (lt == 0 && nxt < blk_end) issue_inputs<C>(a, nxt, grp, mb_in);
+        uint64_t nxt = blk + stride;
+        if (lt == 0) {
+            if (counter) {
+                nxt = atomicAdd(reinterpret_cast<uint32_t *>(smem + (counter - s_base)), 1u);
+                sts_u32(aux, (uint32_t)nxt);  // read by the group after the next barrier
+            }
+            if (nxt < blk_end) issue_inputs<C>(a, nxt, grp, mb_in);
+        }
         sink.published(lt);  // the previous block's merge is done by the whole group
         // and this block's sign/mantissa bytes (chunks c_lo .. the block's
         // last chunk; always at least 16 bytes).  Every thread of the group
@@ -845,6 +862,7 @@ __device__ __forceinline__ void decode_loop(const DecodeArgs &a, Sink &sink, uin
         // No barrier here: the next block's buffer writes and staging copies
         // come after its scan barrier, which every thread reaches only after
         // this merge.
+        blk = counter ? (uint64_t)lds_u32(aux) : blk + stride;
     }
     sink.finish(group, lt);
     if (my_err && a.err) atomicOr(a.err, my_err);
@@ -1383,6 +1401,7 @@ struct FusedArgs {
     uint32_t n_mats, T, n_pad;  // n_pad: T rounded up to 16 (UMMA N)
     uint32_t n_tiles;           // k-tiles of all listed matrices
     uint32_t ring, xring;       // W-tile and X-tile slots
+    uint32_t look;              // X tiles are loaded `look` tiles ahead (xring - look >= 2 tiles back are reused)
     uint32_t tmem_cols;         // power of two >= 2 * n_pad
 };
 
@@ -1395,7 +1414,7 @@ struct FusedSmem {
     uint32_t wring, xring;  // 1024-aligned slot arrays
     uint32_t xbytes;        // bytes of one X slot
     uint32_t full0, empty0, xfull0, xempty0, accfull0, accempty0, final_bar;
-    uint32_t tmem_slot, abort_flag;
+    uint32_t tmem_slot, abort_flag, next_block;
 };
 
 __device__ __forceinline__ FusedSmem fused_layout(const FusedArgs &f, uint32_t dec_end) {
@@ -1413,6 +1432,7 @@ __device__ __forceinline__ FusedSmem fused_layout(const FusedArgs &f, uint32_t d
     L.final_bar = L.accempty0 + 16u;
     L.tmem_slot = L.final_bar + 8u;
     L.abort_flag = L.tmem_slot + 4u;
+    L.next_block = L.abort_flag + 4u;  // the decoder groups' block counter
     return L;
 }
 
@@ -1610,6 +1630,18 @@ __global__ void __launch_bounds__(C::kCtaThreads + kFusedExtraThreads, 1)
     uint32_t err = 0;
 
     if (!load_tables<C>(f.d.lut, f.d.err, smem, s_base, tid)) return;  // uniform over the CTA
+    // the format blocks covering elements of k-tiles [K0, K1) (every warp
+    // finds them: the search is warp-collective)
+    uint64_t b0, b1;
+    {
+        const uint32_t lane = tid & 31u;
+        const TileAt a0 = tile_at(f, K0), a1 = tile_at(f, K1 - 1u);
+        const FusedMat &m0 = f.m[a0.j], &m1 = f.m[a1.j];
+        const uint64_t e_first = m0.off + (uint64_t)(K0 - m0.tbase) * kTileElems;
+        const uint64_t e_last = m1.off + (uint64_t)(K1 - m1.tbase) * kTileElems - 1u;
+        b0 = find_block(f.d.bstart, f.d.n_blocks, e_first, lane);
+        b1 = find_block(f.d.bstart, f.d.n_blocks, e_last, lane) + 1u;
+    }
     if (tid == 0) {
         for (uint32_t s = 0; s < f.ring; ++s) {
             df11::tc::mbar_init(L.full0 + 8u * s, 1);
@@ -1625,6 +1657,7 @@ __global__ void __launch_bounds__(C::kCtaThreads + kFusedExtraThreads, 1)
         }
         df11::tc::mbar_init(L.final_bar, 1);
         sts_u32(L.abort_flag, 0u);
+        sts_u32(L.next_block, (uint32_t)b0);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if (tid >= kDec && tid < kDec + 32u) {  // the first epilogue warp allocates the accumulators
@@ -1639,17 +1672,11 @@ __global__ void __launch_bounds__(C::kCtaThreads + kFusedExtraThreads, 1)
     const uint32_t tmem = lds_u32(L.tmem_slot);
 
     if (tid < kDec) {
-        // ---- decoders: the format blocks covering elements of k-tiles [K0, K1)
-        const uint32_t lane = tid & 31u;
-        const TileAt a0 = tile_at(f, K0), a1 = tile_at(f, K1 - 1u);
-        const FusedMat &m0 = f.m[a0.j], &m1 = f.m[a1.j];
-        const uint64_t e_first = m0.off + (uint64_t)(K0 - m0.tbase) * kTileElems;
-        const uint64_t e_last = m1.off + (uint64_t)(K1 - m1.tbase) * kTileElems - 1u;
-        const uint64_t b0 = find_block(f.d.bstart, f.d.n_blocks, e_first, lane);
-        const uint64_t b1 = find_block(f.d.bstart, f.d.n_blocks, e_last, lane) + 1u;
+        // ---- decoders: the CTA's blocks, taken in order from the counter
+        // (tiles are consumed in order, so a group that ran ahead would only
+        // wait for a slot; a free group takes the next block instead)
         TileSink<C::kStageSm> sink{f, L, K0, NT, 0u, 0u, 0u, 0u, 0u, 0u, 0u};  // (tiles set per block)
-        const uint32_t group = tid / kGroupThreads;
-        decode_loop<C, kLong>(f.d, sink, b0 + group, C::kGroups, b1);
+        decode_loop<C, kLong>(f.d, sink, b0, 1u, b1, L.next_block);
         err |= sink.err;
     } else if (tid >= kDec + 128u) {
         // ---- the MMA warp: one thread issues the MMAs and loads X
@@ -1665,8 +1692,10 @@ __global__ void __launch_bounds__(C::kCtaThreads + kFusedExtraThreads, 1)
                                       (int32_t)(t.kt * 64u), 0);
             };
             // X tiles are loaded `look` tiles ahead, each into the slot of the
-            // tile two before the current one, whose MMA has long finished
-            const uint32_t look = f.xring - 2u;
+            // tile xring - look before the current one: its MMA has had that
+            // many tiles' time to finish (waiting on the MMA of the tile just
+            // before would tie the loop to the MMAs' latency)
+            const uint32_t look = f.look;
             for (uint32_t i = 0; i < look && i < NT; ++i) load_x(i);
             uint32_t seg = 0;  // segments started
             for (uint32_t i = 0; i < NT; ++i) {
@@ -2020,13 +2049,12 @@ df11_status launch_gemv(const df11_tensor *t, const df11_gemv_mat *mats, uint32_
 constexpr uint32_t kSmemLimit = 227u * 1024u;
 constexpr uint32_t kFusedTail = 1024u + 256u;  // alignment slack of the rings, barriers and flags
 
+// Shared memory of an instance with `xring` X slots: true if at least
+// `min_ring` operand-tile slots fit (then as many as fit, at most 8).
 template <class C>
-bool fused_fit(uint32_t n_pad, uint32_t &ring, uint32_t &xring, uint32_t &smem) {
+bool fused_fit(uint32_t n_pad, uint32_t xring, uint32_t min_ring, uint32_t &ring, uint32_t &smem) {
     const uint32_t xbytes = 128u * n_pad;
-    // X slots: loads run xring - 2 = 1 tile ahead of the MMAs (the decoders,
-    // not the X loads, set the pace: a tile every few microseconds per CTA)
-    xring = 3u;
-    if (C::kSmemBytes + kFusedTail + xring * xbytes + 2u * kTileBytes > kSmemLimit) return false;
+    if (C::kSmemBytes + kFusedTail + xring * xbytes + min_ring * kTileBytes > kSmemLimit) return false;
     ring = (kSmemLimit - C::kSmemBytes - kFusedTail - xring * xbytes) / kTileBytes;
     if (ring > 8u) ring = 8u;
     smem = C::kSmemBytes + kFusedTail + xring * xbytes + ring * kTileBytes;
@@ -2094,26 +2122,39 @@ df11_status launch_fused(const df11_tensor *t, const df11_gemv_mat *mats, uint32
     if (st != DF11_OK) return st;
     const unsigned grid = (unsigned)(f.n_tiles < (uint32_t)sms ? f.n_tiles : (uint32_t)sms);
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    // six decode groups when the rings leave room for 4 operand tiles, else four
-#ifndef DF11_FUSED_GROUPS
-#define DF11_FUSED_GROUPS 0  // 0: by the rule above; 4 or 6: forced
-#endif
     uint32_t smem = 0;
     cudaError_t e;
-    // the most decode groups whose rings still hold 4 operand tiles (3 with
-    // the largest X tiles, which also leave no room to stage sign/mantissa)
-    if (DF11_FUSED_GROUPS != 4 && fused_fit<CfgFused6>(f.n_pad, f.ring, f.xring, smem) &&
-        (f.ring >= 4u || DF11_FUSED_GROUPS == 6)) {
+    // Prefer six X slots (loads 3 tiles ahead, slots reused 3 tiles later),
+    // then the most decode groups (staging the sign/mantissa bytes if there is
+    // room) whose ring still holds 4 operand tiles; with the largest X tiles,
+    // four unstaged groups and fewer X slots.
+#ifndef DF11_FUSED_CFG
+#define DF11_FUSED_CFG 0  // 0: by the rule above; 1..4: 6 staged, 6 unstaged, 4 staged, 4 unstaged groups
+#endif
+    const int forced = DF11_FUSED_CFG;
+    f.xring = 6u;
+    f.look = 3u;
+    if ((forced == 0 || forced == 1) && fused_fit<CfgFused6>(f.n_pad, f.xring, forced ? 2u : 4u, f.ring, smem)) {
         e = lng ? fused_launch<CfgFused6, true>(f, maps, smem, grid, s)
                 : fused_launch<CfgFused6, false>(f, maps, smem, grid, s);
-    } else if (fused_fit<CfgFused4>(f.n_pad, f.ring, f.xring, smem) && f.ring >= 4u) {
+    } else if ((forced == 0 || forced == 2) &&
+               fused_fit<CfgFused6U>(f.n_pad, f.xring, forced ? 2u : 4u, f.ring, smem)) {
+        e = lng ? fused_launch<CfgFused6U, true>(f, maps, smem, grid, s)
+                : fused_launch<CfgFused6U, false>(f, maps, smem, grid, s);
+    } else if ((forced == 0 || forced == 3) &&
+               fused_fit<CfgFused4>(f.n_pad, f.xring, forced ? 2u : 4u, f.ring, smem)) {
         e = lng ? fused_launch<CfgFused4, true>(f, maps, smem, grid, s)
                 : fused_launch<CfgFused4, false>(f, maps, smem, grid, s);
-    } else if (fused_fit<CfgFused4U>(f.n_pad, f.ring, f.xring, smem)) {
+    } else {
+        // four unstaged groups; fewer X slots until a ring of 3 fits
+        bool fit = false;
+        for (f.xring = 6u; f.xring >= 3u && !fit; --f.xring)
+            fit = fused_fit<CfgFused4U>(f.n_pad, f.xring, 3u, f.ring, smem);
+        if (!fit) return DF11_ERR_UNSUPPORTED;
+        ++f.xring;  // (the loop stepped past the one that fit)
+        f.look = f.xring / 2u;
         e = lng ? fused_launch<CfgFused4U, true>(f, maps, smem, grid, s)
                 : fused_launch<CfgFused4U, false>(f, maps, smem, grid, s);
-    } else {
-        return DF11_ERR_UNSUPPORTED;
     }
     return e == cudaSuccess ? DF11_OK : DF11_ERR_CUDA;
 }
