@@ -283,6 +283,12 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t
                  : "memory");
 }
 
+// Bulk prefetch of [src, src + bytes) into L2 (16-byte aligned, a multiple of
+// 16 bytes); no completion to wait for.
+__device__ __forceinline__ void bulk_prefetch_l2(const void *src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
 // Length of a code longer than the table window, from the canonical limits
 // in shared memory (non-decreasing in l): the smallest l in [from, max_len]
 // with window < lim[l], by binary search.  0 if none.
@@ -318,18 +324,26 @@ __device__ __forceinline__ void merge16(const uint4 smv, const uint4 ex, uint32_
     }
 }
 
+// Sign/mantissa byte of element g of a block whose output starts at element
+// `base`: from the block's staged bytes at shared address sm_s0 (chunk 0 on),
+// or from global memory when they are not staged (sm_s0 = 0).
+__device__ __forceinline__ uint32_t sm_byte(const uint8_t *sm, uint32_t sm_s0, uint32_t g, uint32_t base) {
+    return sm_s0 ? lds_u8(sm_s0 + (g - base)) : (uint32_t)__ldg(sm + g);
+}
+
 // The chunks holding the block's first and last elements, by one warp:
 // lanes 0..15 take the first chunk, lanes 16..31 the last one, one element
 // each (only elements inside [s, e) are written).
-__device__ __forceinline__ void merge_edges(const uint8_t *sm, uint16_t *out, uint32_t sb, uint32_t base,
-                                            uint32_t c_full, uint32_t span, uint32_t s, uint32_t e, uint32_t lane) {
+__device__ __forceinline__ void merge_edges(const uint8_t *sm, uint32_t sm_s0, uint16_t *out, uint32_t sb,
+                                            uint32_t base, uint32_t c_full, uint32_t span, uint32_t s, uint32_t e,
+                                            uint32_t lane) {
     const bool head = s != base;
     const bool tail = (span & 15u) != 0u && !(head && c_full == 0u);
     const uint32_t c = (lane < 16u) ? 0u : c_full;
     const bool mine = (lane < 16u) ? head : tail;
     const uint32_t g = base + 16u * c + (lane & 15u);
     if (mine && g >= s && g < e && DF11_BOUNDS_OK(g - base < kMaxCodesPerBlock + 16u)) {
-        const uint32_t sm8 = __ldg(sm + g);
+        const uint32_t sm8 = sm_byte(sm, sm_s0, g, base);
         const uint32_t r = lds_u8(sb + (g - base));
         // r = rotated exponent: high byte (s & 0x80) | (r & 0x7F), low byte (r & 0x80) | (s & 0x7F)
         const uint32_t hi8 = (sm8 & 0x80u) | (r & 0x7Fu);
@@ -338,10 +352,10 @@ __device__ __forceinline__ void merge_edges(const uint8_t *sm, uint16_t *out, ui
     }
 }
 // merge_edges, then clears the two edge chunks (whole warp, converged).
-__device__ __forceinline__ void merge_edges_clear(const uint8_t *sm, uint16_t *out, uint32_t sb, uint32_t base,
-                                                  uint32_t c_full, uint32_t span, uint32_t s, uint32_t e,
-                                                  uint32_t lane) {
-    merge_edges(sm, out, sb, base, c_full, span, s, e, lane);
+__device__ __forceinline__ void merge_edges_clear(const uint8_t *sm, uint32_t sm_s0, uint16_t *out, uint32_t sb,
+                                                  uint32_t base, uint32_t c_full, uint32_t span, uint32_t s,
+                                                  uint32_t e, uint32_t lane) {
+    merge_edges(sm, sm_s0, out, sb, base, c_full, span, s, e, lane);
     __syncwarp();
     const bool head = s != base;
     const bool tail = (span & 15u) != 0u && !(head && c_full == 0u);
@@ -676,8 +690,11 @@ __device__ __forceinline__ bool load_tables(const uint8_t *lut, uint32_t *err_ou
 // the block's element range, whether it decoded and whether its range was
 // even plausible), `published(lt)`
 // right after the next group barrier (every thread of the group has then
-// finished that merge), and `finish(group, lt)` after the group's last block.
+// finished that merge), `plan(s, e, lt)` right after it too (the block about
+// to be decoded: a sink may prepare its merge there), and `finish(group, lt)`
+// after the group's last block.
 struct NoHooks {
+    __device__ __forceinline__ void plan(uint32_t, uint32_t, uint32_t) {}
     __device__ __forceinline__ void begin_block(uint32_t, uint32_t) {}
     __device__ __forceinline__ void block_done(uint32_t, uint32_t, bool, bool) {}
     __device__ __forceinline__ void published(uint32_t) {}
@@ -695,8 +712,8 @@ struct StoreSink : NoHooks {
         merge_chunks<kBufBytes>(out, sb, base, c_first, c_end, sm_s, c_lo, al32, n_elems);
     }
     __device__ __forceinline__ void edges(uint32_t sb, uint32_t base, uint32_t c_full, uint32_t span, uint32_t s,
-                                          uint32_t e, uint32_t lane) {
-        merge_edges_clear(sm, out, sb, base, c_full, span, s, e, lane);
+                                          uint32_t e, uint32_t lane, uint32_t sm_s0) {
+        merge_edges_clear(sm, sm_s0, out, sb, base, c_full, span, s, e, lane);
     }
 };
 
@@ -813,19 +830,28 @@ __device__ __forceinline__ void decode_loop(const DecodeArgs &a, Sink &sink, uin
             if (nxt < blk_end) issue_inputs<C>(a, nxt, grp, mb_in);
         }
         sink.published(lt);  // the previous block's merge is done by the whole group
-        // and this block's sign/mantissa bytes (chunks c_lo .. the block's
-        // last chunk; always at least 16 bytes).  Every thread of the group
-        // has passed its previous merge, so the staging area is free.
-        if (C::kStageSm && lt == 0) {
+        sink.plan(s, e, lt);
+        // and this block's sign/mantissa bytes (chunks 0 .. the block's last
+        // chunk, at most kBufSyms bytes: the edge chunks are read from there
+        // too; always at least 16 bytes).  Every thread of the group has
+        // passed its previous merge, so the staging area is free.
+        if (lt == 0) {
             // (64-bit: the end of the last chunk passes 2^32 when the tensor
             // holds nearly 2^32 elements)
-            const uint64_t from = range_ok ? (uint64_t)base + 16u * c_lo : 0u;
+            const uint64_t from = range_ok ? (uint64_t)base : 0u;
             const uint64_t upto = range_ok ? (((uint64_t)e + 15u) & ~15ull) : 16u;
-            const uint32_t bytes = upto > from ? (uint32_t)min((uint64_t)C::kSmBytes, upto - from) : 16u;
+            const uint32_t bytes =
+                upto > from ? (uint32_t)min((uint64_t)(C::kStageSm ? C::kSmBytes : C::kSbufBytes), upto - from) : 16u;
             const uint64_t src = upto > from ? from : (range_ok ? base : 0u);
-            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-            mbar_expect(mb_sm, bytes);
-            bulk_g2s(grp + C::kGrpSm, a.sm + src, bytes, mb_sm);
+            if (C::kStageSm) {
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                mbar_expect(mb_sm, bytes);
+                bulk_g2s(grp + C::kGrpSm, a.sm + src, bytes, mb_sm);
+            } else {
+                // unstaged (the merge reads them from global memory): bring
+                // them into L2 while the block decodes
+                bulk_prefetch_l2(a.sm + src, bytes);
+            }
         }
 
         uint32_t wsum = (lane < kWarps) ? lds_u32(wtot + 4u * lane) : 0u;
@@ -855,8 +881,9 @@ __device__ __forceinline__ void decode_loop(const DecodeArgs &a, Sink &sink, uin
         }
         sink.begin_block(s, e);
         if (ok) {
-            sink.template chunks<C::kSbufBytes>(sb, base, c0, c_full, grp + C::kGrpSm, c_lo);
-            if (warp == 0) sink.edges(sb, base, c_full, span, s, e, lane);
+            // (the staged bytes start at chunk 0; the chunk merges index them from c_lo)
+            sink.template chunks<C::kSbufBytes>(sb, base, c0, c_full, grp + C::kGrpSm + 16u * c_lo, c_lo);
+            if (warp == 0) sink.edges(sb, base, c_full, span, s, e, lane, C::kStageSm ? grp + C::kGrpSm : 0u);
         }
         sink.block_done(s, e, ok, range_ok);
         // No barrier here: the next block's buffer writes and staging copies
@@ -1299,7 +1326,7 @@ struct GemvSink : NoHooks {
     // 16..31 the last, one element each; each half-warp's sum is added once
     // (a chunk lies in one row of one matrix or in none).
     __device__ __forceinline__ void edges(uint32_t sb, uint32_t base, uint32_t c_full, uint32_t span, uint32_t s,
-                                          uint32_t e, uint32_t lane) {
+                                          uint32_t e, uint32_t lane, uint32_t sm_s0) {
         const bool head = s != base;
         const bool tail = (span & 15u) != 0u && !(head && c_full == 0u);
         const uint32_t c = (lane < 16u) ? 0u : c_full;
@@ -1317,7 +1344,7 @@ struct GemvSink : NoHooks {
             row = gemv_row(gc - M.off, M.magic, M.shift);
             const uint32_t gel = gc + (lane & 15u);
             if (gel >= s && gel < e && DF11_BOUNDS_OK(gel - base < kMaxCodesPerBlock + 16u)) {
-                const uint32_t sm8 = __ldg(g.d.sm + gel);
+                const uint32_t sm8 = sm_byte(g.d.sm, sm_s0, gel, base);
                 const uint32_t r = lds_u8(sb + (gel - base));
                 const uint32_t hi8 = (sm8 & 0x80u) | (r & 0x7Fu);
                 const uint32_t lo8 = (r & 0x80u) | (sm8 & 0x7Fu);
@@ -1384,6 +1411,7 @@ __global__ void __launch_bounds__(C::kCtaThreads, 1) df11_decode_gemv_kernel(con
 constexpr uint32_t kFusedMaxMats = 16;
 constexpr uint32_t kTileElems = 8192;   // 128 rows x 64 columns
 constexpr uint32_t kTileBytes = 16384;  // as BF16
+static_assert(kTileBytes == 1u << 14, "slot offset >> 11 = slot index x 8 (mbarrier bytes)");
 constexpr uint32_t kFusedErrTimeout = 0x20u;
 
 struct FusedMat {
@@ -1415,6 +1443,7 @@ struct FusedSmem {
     uint32_t xbytes;        // bytes of one X slot
     uint32_t full0, empty0, xfull0, xempty0, accfull0, accempty0, final_bar;
     uint32_t tmem_slot, abort_flag, next_block;
+    uint32_t plan0;  // per decoder group 32 bytes: the tiles of its current block (TileSink::plan)
 };
 
 __device__ __forceinline__ FusedSmem fused_layout(const FusedArgs &f, uint32_t dec_end) {
@@ -1433,6 +1462,7 @@ __device__ __forceinline__ FusedSmem fused_layout(const FusedArgs &f, uint32_t d
     L.tmem_slot = L.final_bar + 8u;
     L.abort_flag = L.tmem_slot + 4u;
     L.next_block = L.abort_flag + 4u;  // the decoder groups' block counter
+    L.plan0 = L.next_block + 4u;
     return L;
 }
 
@@ -1464,9 +1494,37 @@ __device__ __forceinline__ TileAt tile_at(const FusedArgs &f, uint32_t K) {
     return TileAt{j, lk / f.m[j].kt, lk % f.m[j].kt};
 }
 
+// Walks the k-tiles in stream order: matrix j, row tile rt, k-tile column kt
+// (KT k-tiles per row tile, RT row tiles in matrix j).
+struct TileCursor {
+    uint32_t j, rt, kt, KT, RT;
+    __device__ __forceinline__ void start(const FusedArgs &f, uint32_t K) {
+        const TileAt a = tile_at(f, K);
+        j = a.j;
+        rt = a.rt;
+        kt = a.kt;
+        KT = f.m[j].kt;
+        RT = f.m[j].rows / 128u;
+    }
+    __device__ __forceinline__ void next(const FusedArgs &f) {
+        if (++kt < KT) return;
+        kt = 0;
+        if (++rt < RT) return;
+        rt = 0;
+        if (++j < f.n_mats) {
+            KT = f.m[j].kt;
+            RT = f.m[j].rows / 128u;
+        }
+    }
+};
+
 // The decoder side: the merge of a decoded block writes into the tile ring.
 // kStaged: the block's sign/mantissa bytes are staged in shared memory (else
-// read from global memory).
+// read from global memory, prefetched into L2 while the block decodes).
+// A block (at most 7152 elements) meets at most two k-tiles (8192 elements
+// each, consecutive in the stream, 16-aligned) and each of them holds the
+// block's first or last element; they are located once per block, so the
+// per-chunk work is two range tests and two swizzled stores.
 template <bool kStaged>
 struct TileSink {
     static constexpr uint32_t kNoTile = 0xFFFFFFFFu;
@@ -1474,14 +1532,16 @@ struct TileSink {
     FusedSmem L;
     uint32_t K0, NT;     // this CTA's k-tiles [K0, K0 + NT)
     uint32_t avail;      // local tiles [0, avail) are known to have a free slot
-    uint32_t m;          // matrix hint for the chunk search
-    uint32_t ta, tb;     // the local tiles of the block's first and last elements (a block meets at most two)
+    uint32_t ta, tb;     // the local tiles of the block's first and last elements (kNoTile: none)
+    uint32_t ga, gb;     // the stream index of their first elements
+    uint32_t sa, sb_;    // their slots' shared-memory addresses
     uint32_t ba, bb;     // bytes this thread wrote into them
     uint32_t err;
 
     // Local tile index of element g and its position in the tile; false if
     // g is in no listed matrix or in another CTA's tiles.
-    __device__ __forceinline__ bool locate(uint32_t g, uint32_t &mm, uint32_t &i, uint32_t &p) const {
+    __device__ __forceinline__ bool locate(uint32_t g, uint32_t &i, uint32_t &p) const {
+        uint32_t mm = 0;
         while (mm < f.n_mats && g >= f.m[mm].end) ++mm;
         if (mm >= f.n_mats || g < f.m[mm].off) return false;
         const uint32_t q = g - f.m[mm].off;
@@ -1503,75 +1563,141 @@ struct TileSink {
         avail = i + 1u;
         return true;
     }
-    __device__ __forceinline__ uint32_t slot_addr(uint32_t i, uint32_t p) const {
-        const uint32_t r = p >> 6, c = p & 63u;
-        return L.wring + (i % f.ring) * kTileBytes + r * 128u + ((((c >> 3) ^ (r & 7u))) << 4) + (c & 7u) * 2u;
+    // The tile-complete mbarrier of the slot at shared-memory address `slot`.
+    __device__ __forceinline__ uint32_t full_bar(uint32_t slot) const { return L.full0 + ((slot - L.wring) >> 11); }
+    // Shared-memory address of position p (a multiple of 8: a 16-byte piece)
+    // of the tile whose slot starts at `slot` (UMMA 128-byte swizzle).
+    __device__ __forceinline__ static uint32_t piece(uint32_t slot, uint32_t p) {
+        const uint32_t r = p >> 6, j = (p & 63u) >> 3;
+        return slot + r * 128u + ((j ^ (r & 7u)) << 4);
     }
-    __device__ __forceinline__ void tally(uint32_t i, uint32_t bytes) {
-        if (i == ta) ba += bytes;
-        else bb += bytes;
+    // The tile holding element g (a chunk's first element): slot address and
+    // position; false if g is in neither of the block's tiles.
+    __device__ __forceinline__ bool which(uint32_t g, bool &in_a, uint32_t &slot, uint32_t &p) {
+        in_a = ta != kNoTile && g - ga < kTileElems;
+        if (in_a) {
+            p = g - ga;
+            slot = sa;
+        } else if (tb != kNoTile && g - gb < kTileElems) {
+            p = g - gb;
+            slot = sb_;
+        } else {
+            return false;
+        }
+        return ensure(in_a ? ta : tb);
     }
 
+    // Two threads of the group, after the scan barrier: the tiles of the
+    // block's first element (thread 64) and last element (thread 96) into the
+    // group's plan words (tile, first element, slot address), read by the
+    // whole group after the next barrier.  (The previous block's plan was read
+    // before its merge, which every thread finished before the scan barrier.)
+    __device__ __forceinline__ void plan(uint32_t s, uint32_t e, uint32_t lt) {
+        if (lt != 64u && lt != 96u) return;
+        const uint32_t at = L.plan0 + 32u * (threadIdx.x / kGroupThreads) + (lt == 64u ? 0u : 12u);
+        const uint32_t g = lt == 64u ? s : e - 1u;
+        uint32_t i, p;
+        if (e > s && locate(g, i, p)) {
+            sts_u32(at, i);
+            sts_u32(at + 4u, g - p);
+            sts_u32(at + 8u, L.wring + (i % f.ring) * kTileBytes);
+        } else {
+            sts_u32(at, kNoTile);
+        }
+    }
     // Every thread of the group, before the block's merge.
-    __device__ __forceinline__ void begin_block(uint32_t s, uint32_t e) {
-        ta = tb = kNoTile;
+    __device__ __forceinline__ void begin_block(uint32_t, uint32_t) {
+        const uint32_t at = L.plan0 + 32u * (threadIdx.x / kGroupThreads);
         ba = bb = 0u;
-        uint32_t mm = 0, i, p;
-        if (e <= s) return;
-        if (locate(s, mm, i, p)) ta = i;
-        mm = 0;
-        if (locate(e - 1u, mm, i, p) && i != ta) tb = i;
+        ta = lds_u32(at);
+        ga = lds_u32(at + 4u);
+        sa = lds_u32(at + 8u);
+        tb = lds_u32(at + 12u);
+        gb = lds_u32(at + 16u);
+        sb_ = lds_u32(at + 20u);
+        if (tb == ta) tb = kNoTile;
+    }
+
+    __device__ __forceinline__ void put16(const uint4 smv, const uint4 ex, uint32_t g) {
+        bool in_a;
+        uint32_t slot, p;
+        if (!which(g, in_a, slot, p)) return;
+        uint32_t o[8];
+        merge16(smv, ex, o);
+        // 16 weights = two 16-byte pieces of one tile row (p is a multiple of 16)
+        sts_u4(piece(slot, p), o[0], o[1], o[2], o[3]);
+        sts_u4(piece(slot, p + 8u), o[4], o[5], o[6], o[7]);
+        if (in_a) ba += 32u;
+        else bb += 32u;
     }
 
     template <uint32_t kBufBytes>
-    __device__ __forceinline__ void chunks(uint32_t sb, uint32_t base, uint32_t c_first, uint32_t c_end,
+    __device__ __forceinline__ void chunks(uint32_t sbuf, uint32_t base, uint32_t c_first, uint32_t c_end,
                                            uint32_t sm_s, uint32_t c_lo) {
-        for (uint32_t c = c_first; c < c_end; c += kGroupThreads) {
-            if (!DF11_BOUNDS_OK(16u * (c + 1u) <= kBufBytes && c >= c_lo &&
-                                (uint64_t)base + 16u * (c + 1u) <= f.d.n_elems &&
-                                (!kStaged || 16u * (c - c_lo + 1u) <= kBufBytes)))
-                continue;
-            // (unstaged: 16-byte loads from global memory, coalesced over the warp)
-            const uint4 smv = kStaged ? lds_u4(sm_s + 16u * (c - c_lo))
-                                      : __ldg(reinterpret_cast<const uint4 *>(f.d.sm + base + 16u * c));
-            const uint4 ex = lds_u4(sb + 16u * c);
-            sts_zero16(sb + 16u * c);
-            uint32_t i, p;
-            if (!locate(base + 16u * c, m, i, p) || !ensure(i)) continue;
-            uint32_t o[8];
-            merge16(smv, ex, o);
-            // 16 weights = two 16-byte pieces of one tile row (p is a multiple of 16)
-            const uint32_t r = p >> 6, j = (p & 63u) >> 3;
-            const uint32_t row = L.wring + (i % f.ring) * kTileBytes + r * 128u;
-            if (DF11_BOUNDS_OK(i < NT)) {
-                sts_u4(row + (((j) ^ (r & 7u)) << 4), o[0], o[1], o[2], o[3]);
-                sts_u4(row + (((j + 1u) ^ (r & 7u)) << 4), o[4], o[5], o[6], o[7]);
+        if (kStaged) {
+            for (uint32_t c = c_first; c < c_end; c += kGroupThreads) {
+                if (!DF11_BOUNDS_OK(16u * (c + 1u) <= kBufBytes && c >= c_lo &&
+                                    (uint64_t)base + 16u * (c + 1u) <= f.d.n_elems &&
+                                    16u * (c - c_lo + 1u) <= kBufBytes))
+                    continue;
+                const uint4 smv = lds_u4(sm_s + 16u * (c - c_lo));
+                const uint4 ex = lds_u4(sbuf + 16u * c);
+                sts_zero16(sbuf + 16u * c);
+                put16(smv, ex, base + 16u * c);
             }
-            tally(i, 32u);
+        } else {
+            // the thread's (at most four per round) 16-byte loads from global
+            // memory are all issued before the first is used
+            constexpr uint32_t kRound = 4;
+            for (uint32_t c1 = c_first; c1 < c_end; c1 += kRound * kGroupThreads) {
+                uint4 v[kRound];
+#pragma unroll
+                for (uint32_t q = 0; q < kRound; ++q) {
+                    const uint32_t c = c1 + q * kGroupThreads;
+                    if (c < c_end && DF11_BOUNDS_OK((uint64_t)base + 16u * (c + 1u) <= f.d.n_elems))
+                        v[q] = __ldg(reinterpret_cast<const uint4 *>(f.d.sm + base + 16u * c));
+                }
+#pragma unroll
+                for (uint32_t q = 0; q < kRound; ++q) {
+                    const uint32_t c = c1 + q * kGroupThreads;
+                    if (!(c < c_end) || !DF11_BOUNDS_OK(16u * (c + 1u) <= kBufBytes && c >= c_lo &&
+                                                       (uint64_t)base + 16u * (c + 1u) <= f.d.n_elems))
+                        continue;
+                    const uint4 ex = lds_u4(sbuf + 16u * c);
+                    sts_zero16(sbuf + 16u * c);
+                    put16(v[q], ex, base + 16u * c);
+                }
+            }
         }
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     }
-    __device__ __forceinline__ void edges(uint32_t sb, uint32_t base, uint32_t c_full, uint32_t span, uint32_t s,
-                                          uint32_t e, uint32_t lane) {
+    __device__ __forceinline__ void edges(uint32_t sbuf, uint32_t base, uint32_t c_full, uint32_t span, uint32_t s,
+                                          uint32_t e, uint32_t lane, uint32_t sm_s0) {
         const bool head = s != base;
         const bool tail = (span & 15u) != 0u && !(head && c_full == 0u);
         const uint32_t c = (lane < 16u) ? 0u : c_full;
         const bool mine = (lane < 16u) ? head : tail;
         const uint32_t g = base + 16u * c + (lane & 15u);
-        uint32_t mm = 0, i, p;
-        if (mine && g >= s && g < e && DF11_BOUNDS_OK(g - base < kMaxCodesPerBlock + 16u) && locate(g, mm, i, p) &&
-            ensure(i)) {
-            const uint32_t sm8 = __ldg(f.d.sm + g);
-            const uint32_t rr = lds_u8(sb + (g - base));
+        bool in_a;
+        uint32_t slot, p;
+        if (mine && g >= s && g < e && DF11_BOUNDS_OK(g - base < kMaxCodesPerBlock + 16u) &&
+            which(g & ~15u, in_a, slot, p)) {
+            const uint32_t sm8 = sm_byte(f.d.sm, sm_s0, g, base);
+            const uint32_t rr = lds_u8(sbuf + (g - base));
             const uint32_t hi8 = (sm8 & 0x80u) | (rr & 0x7Fu);
             const uint32_t lo8 = (rr & 0x80u) | (sm8 & 0x7Fu);
-            asm volatile("st.shared.u16 [%0], %1;" ::"r"(slot_addr(i, p)), "h"((uint16_t)(lo8 | (hi8 << 8)))
+            const uint32_t pe = p + (g & 15u);  // the element's own position (same row as the chunk's)
+            const uint32_t r = pe >> 6, cc = pe & 63u;
+            asm volatile("st.shared.u16 [%0], %1;" ::"r"(slot + r * 128u + (((cc >> 3) ^ (r & 7u)) << 4) +
+                                                         (cc & 7u) * 2u),
+                         "h"((uint16_t)(lo8 | (hi8 << 8)))
                          : "memory");
-            tally(i, 2u);
+            if (in_a) ba += 2u;
+            else bb += 2u;
         }
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         __syncwarp();
-        if ((lane == 0u && head) || (lane == 16u && tail)) sts_zero16(sb + 16u * (lane == 0u ? 0u : c_full));
+        if ((lane == 0u && head) || (lane == 16u && tail)) sts_zero16(sbuf + 16u * (lane == 0u ? 0u : c_full));
     }
     // After the block's merge (every thread of the group): each warp counts
     // the bytes it wrote into the tiles' mbarriers right away (lane 0; the
@@ -1592,21 +1718,18 @@ struct TileSink {
             const uint32_t a = __reduce_add_sync(0xFFFFFFFFu, ba), b = __reduce_add_sync(0xFFFFFFFFu, bb);
             if (lane == 0u && (a | b) != 0u && !lds_u32(L.abort_flag)) {
                 asm volatile("fence.acq_rel.cta;" ::: "memory");
-                if (a) df11::tc::mbar_complete_tx(L.full0 + 8u * (ta % f.ring), a);
-                if (b) df11::tc::mbar_complete_tx(L.full0 + 8u * (tb % f.ring), b);
+                if (a) df11::tc::mbar_complete_tx(full_bar(sa), a);
+                if (b) df11::tc::mbar_complete_tx(full_bar(sb_), b);
             }
         } else if ((threadIdx.x % kGroupThreads) == 0u && e > s) {
             for (uint32_t q = 0; q < 2u; ++q) {
                 const uint32_t i = q == 0u ? ta : tb;
                 if (i == kNoTile || !ensure(i)) continue;  // the count must land in this round of the slot
-                uint32_t mm = 0, ii, p;
-                const uint32_t x = q == 0u ? s : e - 1u;
-                if (!locate(x, mm, ii, p)) continue;
-                const uint32_t ts = x - p, te = ts + kTileElems;
+                const uint32_t ts = q == 0u ? ga : gb, te = ts + kTileElems;
                 const uint32_t lo = s > ts ? s : ts, hi = e < te ? e : te;
                 if (lds_u32(L.abort_flag)) break;
                 asm volatile("fence.acq_rel.cta;" ::: "memory");
-                df11::tc::mbar_complete_tx(L.full0 + 8u * (i % f.ring), 2u * (hi - lo));
+                df11::tc::mbar_complete_tx(full_bar(q == 0u ? sa : sb_), 2u * (hi - lo));
             }
         }
     }
@@ -1623,6 +1746,7 @@ __global__ void __launch_bounds__(C::kCtaThreads + kFusedExtraThreads, 1)
     const uint32_t s_base = smem_addr(smem);
     const uint32_t tid = threadIdx.x;
     constexpr uint32_t kDec = C::kCtaThreads;  // decoder threads; then 4 epilogue warps and the MMA warp
+    static_assert(C::kGroups <= 6u, "the shared-memory tail holds six groups' tile plans");
     const FusedSmem L = fused_layout(f, s_base + C::kSmemBytes);
     const uint32_t K0 = (uint32_t)((uint64_t)f.n_tiles * blockIdx.x / gridDim.x);
     const uint32_t K1 = (uint32_t)((uint64_t)f.n_tiles * (blockIdx.x + 1u) / gridDim.x);
@@ -1675,53 +1799,65 @@ __global__ void __launch_bounds__(C::kCtaThreads + kFusedExtraThreads, 1)
         // ---- decoders: the CTA's blocks, taken in order from the counter
         // (tiles are consumed in order, so a group that ran ahead would only
         // wait for a slot; a free group takes the next block instead)
-        TileSink<C::kStageSm> sink{f, L, K0, NT, 0u, 0u, 0u, 0u, 0u, 0u, 0u};  // (tiles set per block)
+        TileSink<C::kStageSm> sink{f, L, K0, NT, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};  // (tiles set per block)
         decode_loop<C, kLong>(f.d, sink, b0, 1u, b1, L.next_block);
         err |= sink.err;
     } else if (tid >= kDec + 128u) {
         // ---- the MMA warp: one thread issues the MMAs and loads X
         if (tid == kDec + 128u) {
             const uint32_t idesc = df11::tc::instr_desc_bf16(f.n_pad, 128u);
-            // X tile of local k-tile i into slot i % xring
-            auto load_x = [&](uint32_t i) {
-                const uint32_t xs = i % f.xring, xr = i / f.xring;
-                if (xr > 0u && !fused_wait(L.xempty0 + 8u * xs, (xr - 1u) & 1u, L.abort_flag, err, 0u)) return;
-                const TileAt t = tile_at(f, K0 + i);
-                df11::tc::mbar_arrive_expect_tx(L.xfull0 + 8u * xs, L.xbytes);
-                df11::tc::tma_load_2d(L.xring + xs * L.xbytes, &maps.x[t.j], L.xfull0 + 8u * xs,
-                                      (int32_t)(t.kt * 64u), 0);
+            // descriptors of slot 0; a slot (and a K = 16 step, 32 bytes along
+            // the swizzled row) adds its byte offset / 16 to the address field
+            const uint64_t dw0 = df11::tc::smem_desc_sw128(L.wring), dx0 = df11::tc::smem_desc_sw128(L.xring);
+            // X tile of the next local k-tile to load (index xl, its slot and
+            // the slot's round), walked by its own cursor
+            TileCursor cx;
+            cx.start(f, K0);
+            uint32_t xl_slot = 0, xl_round = 0;
+            auto load_x = [&]() {
+                if (xl_round == 0u ||
+                    fused_wait(L.xempty0 + 8u * xl_slot, (xl_round - 1u) & 1u, L.abort_flag, err, 0u)) {
+                    df11::tc::mbar_arrive_expect_tx(L.xfull0 + 8u * xl_slot, L.xbytes);
+                    df11::tc::tma_load_2d(L.xring + xl_slot * L.xbytes, &maps.x[cx.j], L.xfull0 + 8u * xl_slot,
+                                          (int32_t)(cx.kt * 64u), 0);
+                }
+                cx.next(f);
+                if (++xl_slot == f.xring) {
+                    xl_slot = 0;
+                    ++xl_round;
+                }
             };
             // X tiles are loaded `look` tiles ahead, each into the slot of the
             // tile xring - look before the current one: its MMA has had that
             // many tiles' time to finish (waiting on the MMA of the tile just
             // before would tie the loop to the MMAs' latency)
             const uint32_t look = f.look;
-            for (uint32_t i = 0; i < look && i < NT; ++i) load_x(i);
-            uint32_t seg = 0;  // segments started
+            for (uint32_t i = 0; i < look && i < NT; ++i) load_x();
+            TileCursor ct;
+            ct.start(f, K0);
+            uint32_t seg = 0;             // segments started
+            uint32_t s = 0, sph = 0;      // W slot of tile i and the parity of its round
+            uint32_t xs = 0, xph = 0;     // X slot of tile i and the parity of its round
             for (uint32_t i = 0; i < NT; ++i) {
                 // once aborted, arm no more phases (a second arrival on a phase
                 // that never completed is not allowed)
                 if (lds_u32(L.abort_flag)) break;
-                if (i + look < NT) load_x(i + look);
-                const TileAt t = tile_at(f, K0 + i);
-                const bool first = (i == 0u) || t.kt == 0u;
-                const bool last = (i + 1u == NT) || t.kt + 1u == f.m[t.j].kt;
+                if (i + look < NT) load_x();
+                const bool first = (i == 0u) || ct.kt == 0u;
+                const bool last = (i + 1u == NT) || ct.kt + 1u == ct.KT;
                 const uint32_t abuf = seg & 1u;
                 // the accumulator buffer's previous segment has been drained
                 if (first && seg >= 2u)
                     fused_wait(L.accempty0 + 8u * abuf, ((seg >> 1) - 1u) & 1u, L.abort_flag, err, 64u);
-                const uint32_t s = i % f.ring, r = i / f.ring;
                 df11::tc::mbar_arrive_expect_tx(L.full0 + 8u * s, kTileBytes);  // this round's tile
-                const uint32_t xs = i % f.xring, xr = i / f.xring;
-                const bool ok = fused_wait(L.full0 + 8u * s, r & 1u, L.abort_flag, err, 32u) &&
-                                fused_wait(L.xfull0 + 8u * xs, xr & 1u, L.abort_flag, err, 0u);
+                const bool ok = fused_wait(L.full0 + 8u * s, sph, L.abort_flag, err, 32u) &&
+                                fused_wait(L.xfull0 + 8u * xs, xph, L.abort_flag, err, 0u);
                 if (ok) {
                     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-                    const uint32_t wa = L.wring + s * kTileBytes, xa = L.xring + xs * L.xbytes;
+                    const uint64_t dw = dw0 + ((s * kTileBytes) >> 4), dx = dx0 + ((xs * L.xbytes) >> 4);
 #pragma unroll
-                    for (uint32_t kk = 0; kk < 4u; ++kk)  // K = 16 per UMMA: 32 bytes along the swizzled row
-                        df11::tc::umma_bf16(tmem + abuf * f.n_pad, df11::tc::smem_desc_sw128(wa + kk * 32u),
-                                            df11::tc::smem_desc_sw128(xa + kk * 32u), idesc,
+                    for (uint32_t kk = 0; kk < 4u; ++kk)
+                        df11::tc::umma_bf16(tmem + abuf * f.n_pad, dw + 2u * kk, dx + 2u * kk, idesc,
                                             (first && kk == 0u) ? 0u : 1u);
                 }
                 df11::tc::umma_commit(L.empty0 + 8u * s);
@@ -1729,6 +1865,15 @@ __global__ void __launch_bounds__(C::kCtaThreads + kFusedExtraThreads, 1)
                 if (last) {
                     df11::tc::umma_commit(L.accfull0 + 8u * abuf);
                     ++seg;
+                }
+                ct.next(f);
+                if (++s == f.ring) {
+                    s = 0;
+                    sph ^= 1u;
+                }
+                if (++xs == f.xring) {
+                    xs = 0;
+                    xph ^= 1u;
                 }
             }
             // every issued MMA has completed before the accumulators are freed
@@ -1742,9 +1887,14 @@ __global__ void __launch_bounds__(C::kCtaThreads + kFusedExtraThreads, 1)
         // of the row tile) of each segment's accumulator and adds them into Y
         const uint32_t ew = (tid - kDec) >> 5, lane = tid & 31u;
         uint32_t seg = 0;
-        for (uint32_t i = 0; i < NT; ++i) {
-            const TileAt t = tile_at(f, K0 + i);
-            if (!((i + 1u == NT) || t.kt + 1u == f.m[t.j].kt)) continue;  // not the end of a segment
+        TileCursor ce;  // the first k-tile of each segment
+        ce.start(f, K0);
+        for (uint32_t i = 0; i < NT;) {
+            const uint32_t n = min(ce.KT - ce.kt, NT - i);  // the segment's k-tiles
+            const TileAt t{ce.j, ce.rt, 0u};
+            i += n;
+            ce.kt += n - 1u;
+            ce.next(f);
             const uint32_t abuf = seg & 1u;
             const bool have = fused_wait(L.accfull0 + 8u * abuf, (seg >> 1) & 1u, L.abort_flag, err, 256u);
             asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
@@ -2047,7 +2197,10 @@ df11_status launch_gemv(const df11_tensor *t, const df11_gemv_mat *mats, uint32_
 
 // ---- fused decode -> GEMM launcher
 constexpr uint32_t kSmemLimit = 227u * 1024u;
-constexpr uint32_t kFusedTail = 1024u + 256u;  // alignment slack of the rings, barriers and flags
+// alignment slack of the rings (1024), barriers and flags (at most 276 bytes)
+// and the decoder groups' tile plans (32 bytes per group)
+constexpr uint32_t kFusedTail = 1024u + 512u;
+static_assert(16u * 8u + 16u * 6u + 48u + 6u * 32u <= 512u, "ring <= 8, xring <= 6, <= 6 groups");
 
 // Shared memory of an instance with `xring` X slots: true if at least
 // `min_ring` operand-tile slots fit (then as many as fit, at most 8).
