@@ -924,12 +924,12 @@ struct GatherArgs {
     uint32_t n_rows;
 };
 
-// Largest b in [0, n_blocks) with bs[b] <= x, by one warp (32-way search,
-// ceil(log32 n_blocks) rounds of one load per lane).  bs[0] is 0 for valid
-// data; with corrupt starts the result is still some block in range (the
-// per-block range checks then catch the inconsistency).
-__device__ __forceinline__ uint64_t find_block(const uint32_t *bs, uint64_t n_blocks, uint64_t x, uint32_t lane) {
-    uint64_t lo = 0, hi = n_blocks;  // the answer lies in [lo, hi)
+// Largest b in [lo, hi) with bs[b] <= x (lo if none), by one warp (32-way
+// search, ceil(log32 (hi - lo)) rounds of one load per lane).  bs[0] is 0 for
+// valid data; with corrupt starts the result is still some block in range
+// (the per-block range checks then catch the inconsistency).
+__device__ __forceinline__ uint64_t find_block_in(const uint32_t *bs, uint64_t lo, uint64_t hi, uint64_t x,
+                                                 uint32_t lane) {
     while (hi - lo > 1u) {
         const uint64_t step = (hi - lo + 31u) / 32u;
         const uint64_t p = lo + (uint64_t)lane * step;
@@ -940,6 +940,21 @@ __device__ __forceinline__ uint64_t find_block(const uint32_t *bs, uint64_t n_bl
         hi = min(hi, lo + step);
     }
     return lo;
+}
+__device__ __forceinline__ uint64_t find_block(const uint32_t *bs, uint64_t n_blocks, uint64_t x, uint32_t lane) {
+    return find_block_in(bs, 0u, n_blocks, x, lane);
+}
+// The same answer, probing the 32 blocks from `hint` first (one load per
+// lane): the 32-way search runs only when the answer lies outside them.
+__device__ __forceinline__ uint64_t find_block_near(const uint32_t *bs, uint64_t n_blocks, uint64_t hint, uint64_t x,
+                                                    uint32_t lane) {
+    hint = min(hint, n_blocks - 1u);
+    const uint64_t p = hint + lane;
+    const uint32_t m = __ballot_sync(kFull, p < n_blocks && (uint64_t)__ldg(bs + p) <= x);
+    if (m == 0u) return find_block_in(bs, 0u, hint, x, lane);  // (hint = 0: block 0)
+    const uint32_t j = 31u - __clz(m);
+    if (j < 31u || hint + 32u >= n_blocks) return hint + j;
+    return find_block_in(bs, hint + 31u, n_blocks, x, lane);
 }
 
 // One group per requested row (grid-stride over rows): the format blocks
@@ -1442,7 +1457,7 @@ struct FusedSmem {
     uint32_t wring, xring;  // 1024-aligned slot arrays
     uint32_t xbytes;        // bytes of one X slot
     uint32_t full0, empty0, xfull0, xempty0, accfull0, accempty0, final_bar;
-    uint32_t tmem_slot, abort_flag, next_block;
+    uint32_t tmem_slot, abort_flag, next_block, block_end;
     uint32_t plan0;  // per decoder group 32 bytes: the tiles of its current block (TileSink::plan)
 };
 
@@ -1462,7 +1477,8 @@ __device__ __forceinline__ FusedSmem fused_layout(const FusedArgs &f, uint32_t d
     L.tmem_slot = L.final_bar + 8u;
     L.abort_flag = L.tmem_slot + 4u;
     L.next_block = L.abort_flag + 4u;  // the decoder groups' block counter
-    L.plan0 = L.next_block + 4u;
+    L.block_end = L.next_block + 4u;   // and the end of the CTA's blocks
+    L.plan0 = L.block_end + 4u;
     return L;
 }
 
@@ -1481,6 +1497,17 @@ __device__ __forceinline__ bool fused_wait(uint32_t bar, uint32_t parity, uint32
     err |= kFusedErrTimeout;
     sts_u32(abort_flag, 1u);
     return false;
+}
+
+// The number of listed k-tiles that start before stream element E (k-tiles
+// are numbered in stream order; a matrix's tiles start at off + 8192 k).
+__device__ __forceinline__ uint32_t tiles_before(const FusedArgs &f, uint64_t E) {
+    for (uint32_t j = 0; j < f.n_mats; ++j) {
+        const FusedMat &M = f.m[j];
+        if (E <= M.off) return M.tbase;
+        if (E < M.end) return M.tbase + (uint32_t)((E - M.off + kTileElems - 1u) / kTileElems);
+    }
+    return f.n_tiles;
 }
 
 // The k-tile at a global k-tile index: matrix, row tile and k-tile column.
@@ -1737,7 +1764,42 @@ struct TileSink {
     __device__ __forceinline__ void finish(uint32_t, uint32_t) {}
 };
 
-constexpr uint32_t kFusedExtraThreads = 160;  // four epilogue warps and the MMA warp
+// four epilogue warps (a warp reads the TMEM lanes of its rank in its
+// warpgroup; the decoder threads are a multiple of 128, so the four are one
+// warpgroup) and the MMA warp, which never reads TMEM itself (a variant whose
+// MMA warp also drained a quarter of the accumulators stopped completing
+// MMAs on B200: every wait then ran into its limit)
+constexpr uint32_t kFusedExtraThreads = 160;
+
+// One warp's share of a finished segment (the k-tiles of row tile rt of
+// matrix j, accumulated in buffer seg & 1): TMEM lanes 32 q .. 32 q + 31 are
+// rows rt * 128 + 32 q + lane, added into Y with FP32 atomics; then the warp
+// arrives on the buffer's accempty barrier.  The wait for the segment is
+// bounded; after an abort the accumulators are read but nothing is added.
+__device__ __forceinline__ void drain_segment(const FusedArgs &f, const FusedSmem &L, uint32_t tmem, uint32_t j,
+                                              uint32_t rt, uint32_t seg, uint32_t q, uint32_t &err) {
+    const uint32_t lane = threadIdx.x & 31u;
+    const uint32_t abuf = seg & 1u;
+    // (every lane waits; the warp is converged again before the
+    // .sync.aligned loads)
+    const bool have = fused_wait(L.accfull0 + 8u * abuf, (seg >> 1) & 1u, L.abort_flag, err, 256u);
+    __syncwarp();
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    const FusedMat &M = f.m[j];
+    const uint32_t row = rt * 128u + q * 32u + lane;
+    for (uint32_t c0 = 0; c0 < f.n_pad; c0 += 16u) {
+        uint32_t v[16];
+        df11::tc::tmem_ld16(tmem + ((q * 32u) << 16) + abuf * f.n_pad + c0, v);
+        if (have) {
+#pragma unroll
+            for (uint32_t k = 0; k < 16u; ++k)
+                if (c0 + k < f.T) atomicAdd(M.y + (uint64_t)(c0 + k) * M.rows + row, __uint_as_float(v[k]));
+        }
+    }
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    __syncwarp();
+    if (lane == 0u) df11::tc::mbar_arrive(L.accempty0 + 8u * abuf);
+}
 
 template <class C, bool kLong>
 __global__ void __launch_bounds__(C::kCtaThreads + kFusedExtraThreads, 1)
@@ -1748,24 +1810,40 @@ __global__ void __launch_bounds__(C::kCtaThreads + kFusedExtraThreads, 1)
     constexpr uint32_t kDec = C::kCtaThreads;  // decoder threads; then 4 epilogue warps and the MMA warp
     static_assert(C::kGroups <= 6u, "the shared-memory tail holds six groups' tile plans");
     const FusedSmem L = fused_layout(f, s_base + C::kSmemBytes);
-    const uint32_t K0 = (uint32_t)((uint64_t)f.n_tiles * blockIdx.x / gridDim.x);
-    const uint32_t K1 = (uint32_t)((uint64_t)f.n_tiles * (blockIdx.x + 1u) / gridDim.x);
+    // The work split follows the decoding, the larger share of the work: CTA
+    // c takes the format blocks [Bc, Bn) = the c-th of gridDim.x equal shares
+    // and owns the k-tiles that start inside their elements [Ec, En) (the
+    // elements per block vary with the matrices' statistics, so equal tile
+    // shares would not be equal decode work).  Valid block starts increase,
+    // so the shares partition the tiles; a CTA whose boundaries are out of
+    // order reports it (the product is then incomplete).
+    const uint64_t nbk = f.d.n_blocks;
+    const uint64_t Bc = nbk * blockIdx.x / gridDim.x, Bn = nbk * (blockIdx.x + 1u) / gridDim.x;
+    const uint64_t Ec = blockIdx.x == 0u ? 0u : (uint64_t)__ldg(f.d.bstart + Bc);
+    const uint64_t En = blockIdx.x + 1u == gridDim.x ? ~0ull : (uint64_t)__ldg(f.d.bstart + Bn);
+    const uint32_t K0 = tiles_before(f, Ec), K1 = tiles_before(f, En);
+    if (K1 <= K0) {  // uniform over the CTA
+        if (K1 < K0 && tid == 0u && f.d.err) atomicOr(f.d.err, (uint32_t)DF11_KERR_BAD_BLOCK);
+        return;
+    }
     const uint32_t NT = K1 - K0;
     uint32_t err = 0;
 
-    if (!load_tables<C>(f.d.lut, f.d.err, smem, s_base, tid)) return;  // uniform over the CTA
-    // the format blocks covering elements of k-tiles [K0, K1) (every warp
-    // finds them: the search is warp-collective)
-    uint64_t b0, b1;
-    {
-        const uint32_t lane = tid & 31u;
+    // warp 0: the format blocks covering the elements of k-tiles [K0, K1),
+    // searched near the share's ends
+    if (tid < 32u) {
         const TileAt a0 = tile_at(f, K0), a1 = tile_at(f, K1 - 1u);
         const FusedMat &m0 = f.m[a0.j], &m1 = f.m[a1.j];
         const uint64_t e_first = m0.off + (uint64_t)(K0 - m0.tbase) * kTileElems;
         const uint64_t e_last = m1.off + (uint64_t)(K1 - m1.tbase) * kTileElems - 1u;
-        b0 = find_block(f.d.bstart, f.d.n_blocks, e_first, lane);
-        b1 = find_block(f.d.bstart, f.d.n_blocks, e_last, lane) + 1u;
+        const uint64_t b0 = find_block_near(f.d.bstart, nbk, Bc, e_first, tid);
+        const uint64_t b1 = find_block_near(f.d.bstart, nbk, Bn > 0u ? Bn - 1u : 0u, e_last, tid) + 1u;
+        if (tid == 0u) {
+            sts_u32(L.next_block, (uint32_t)b0);  // n_blocks < 2^32 (n_elems < 2^32)
+            sts_u32(L.block_end, (uint32_t)b1);
+        }
     }
+    if (!load_tables<C>(f.d.lut, f.d.err, smem, s_base, tid)) return;  // uniform over the CTA
     if (tid == 0) {
         for (uint32_t s = 0; s < f.ring; ++s) {
             df11::tc::mbar_init(L.full0 + 8u * s, 1);
@@ -1777,11 +1855,10 @@ __global__ void __launch_bounds__(C::kCtaThreads + kFusedExtraThreads, 1)
         }
         for (uint32_t a = 0; a < 2u; ++a) {
             df11::tc::mbar_init(L.accfull0 + 8u * a, 1);
-            df11::tc::mbar_init(L.accempty0 + 8u * a, 4);  // one arrival per epilogue warp
+            df11::tc::mbar_init(L.accempty0 + 8u * a, 4);  // one arrival per draining warp
         }
         df11::tc::mbar_init(L.final_bar, 1);
         sts_u32(L.abort_flag, 0u);
-        sts_u32(L.next_block, (uint32_t)b0);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if (tid >= kDec && tid < kDec + 32u) {  // the first epilogue warp allocates the accumulators
@@ -1800,17 +1877,34 @@ __global__ void __launch_bounds__(C::kCtaThreads + kFusedExtraThreads, 1)
         // (tiles are consumed in order, so a group that ran ahead would only
         // wait for a slot; a free group takes the next block instead)
         TileSink<C::kStageSm> sink{f, L, K0, NT, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};  // (tiles set per block)
-        decode_loop<C, kLong>(f.d, sink, b0, 1u, b1, L.next_block);
+        decode_loop<C, kLong>(f.d, sink, 0u, 1u, lds_u32(L.block_end), L.next_block);
         err |= sink.err;
-    } else if (tid >= kDec + 128u) {
-        // ---- the MMA warp: one thread issues the MMAs and loads X
-        if (tid == kDec + 128u) {
+    } else if (tid < kDec + 128u) {
+        // ---- epilogue warps 0..3: TMEM lanes 32 q .. 32 q + 31 of each segment
+        const uint32_t q = (tid - kDec) >> 5;
+        uint32_t seg = 0;
+        TileCursor ce;  // the first k-tile of each segment
+        ce.start(f, K0);
+        for (uint32_t i = 0; i < NT;) {
+            const uint32_t n = min(ce.KT - ce.kt, NT - i);  // the segment's k-tiles
+            const uint32_t j = ce.j, rt = ce.rt;
+            i += n;
+            ce.kt += n - 1u;
+            ce.next(f);
+            drain_segment(f, L, tmem, j, rt, seg, q, err);
+            ++seg;
+        }
+    } else {
+        // ---- the MMA warp: one thread loads X and issues the MMAs (the
+        // others wait at the end; a loop run by the whole warp with one lane
+        // doing the work measured slower)
+        if ((tid & 31u) == 0u) {
             const uint32_t idesc = df11::tc::instr_desc_bf16(f.n_pad, 128u);
             // descriptors of slot 0; a slot (and a K = 16 step, 32 bytes along
             // the swizzled row) adds its byte offset / 16 to the address field
             const uint64_t dw0 = df11::tc::smem_desc_sw128(L.wring), dx0 = df11::tc::smem_desc_sw128(L.xring);
-            // X tile of the next local k-tile to load (index xl, its slot and
-            // the slot's round), walked by its own cursor
+            // X tile of the next local k-tile to load (its slot and the slot's
+            // round), walked by its own cursor
             TileCursor cx;
             cx.start(f, K0);
             uint32_t xl_slot = 0, xl_round = 0;
@@ -1835,9 +1929,9 @@ __global__ void __launch_bounds__(C::kCtaThreads + kFusedExtraThreads, 1)
             for (uint32_t i = 0; i < look && i < NT; ++i) load_x();
             TileCursor ct;
             ct.start(f, K0);
-            uint32_t seg = 0;             // segments started
-            uint32_t s = 0, sph = 0;      // W slot of tile i and the parity of its round
-            uint32_t xs = 0, xph = 0;     // X slot of tile i and the parity of its round
+            uint32_t seg = 0;          // segments started
+            uint32_t s = 0, sph = 0;   // W slot of tile i and the parity of its round
+            uint32_t xs = 0, xph = 0;  // X slot of tile i and the parity of its round
             for (uint32_t i = 0; i < NT; ++i) {
                 // once aborted, arm no more phases (a second arrival on a phase
                 // that never completed is not allowed)
@@ -1882,38 +1976,6 @@ __global__ void __launch_bounds__(C::kCtaThreads + kFusedExtraThreads, 1)
             if (!df11::tc::mbar_wait(L.final_bar, 0u)) err |= kFusedErrTimeout;
         }
         __syncwarp();
-    } else {
-        // ---- epilogue: warp ew (0..3) reads TMEM lanes 32 ew .. 32 ew + 31 (rows
-        // of the row tile) of each segment's accumulator and adds them into Y
-        const uint32_t ew = (tid - kDec) >> 5, lane = tid & 31u;
-        uint32_t seg = 0;
-        TileCursor ce;  // the first k-tile of each segment
-        ce.start(f, K0);
-        for (uint32_t i = 0; i < NT;) {
-            const uint32_t n = min(ce.KT - ce.kt, NT - i);  // the segment's k-tiles
-            const TileAt t{ce.j, ce.rt, 0u};
-            i += n;
-            ce.kt += n - 1u;
-            ce.next(f);
-            const uint32_t abuf = seg & 1u;
-            const bool have = fused_wait(L.accfull0 + 8u * abuf, (seg >> 1) & 1u, L.abort_flag, err, 256u);
-            asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-            const FusedMat &M = f.m[t.j];
-            const uint32_t row = t.rt * 128u + ew * 32u + lane;
-            for (uint32_t c0 = 0; c0 < f.n_pad; c0 += 16u) {
-                uint32_t v[16];
-                df11::tc::tmem_ld16(tmem + ((ew * 32u) << 16) + abuf * f.n_pad + c0, v);
-                if (have) {
-#pragma unroll
-                    for (uint32_t q = 0; q < 16u; ++q)
-                        if (c0 + q < f.T) atomicAdd(M.y + (uint64_t)(c0 + q) * M.rows + row, __uint_as_float(v[q]));
-                }
-            }
-            asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-            __syncwarp();
-            if (lane == 0u) df11::tc::mbar_arrive(L.accempty0 + 8u * abuf);
-            ++seg;
-        }
     }
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
     __syncthreads();
@@ -2200,7 +2262,7 @@ constexpr uint32_t kSmemLimit = 227u * 1024u;
 // alignment slack of the rings (1024), barriers and flags (at most 276 bytes)
 // and the decoder groups' tile plans (32 bytes per group)
 constexpr uint32_t kFusedTail = 1024u + 512u;
-static_assert(16u * 8u + 16u * 6u + 48u + 6u * 32u <= 512u, "ring <= 8, xring <= 6, <= 6 groups");
+static_assert(16u * 8u + 16u * 6u + 56u + 6u * 32u <= 512u, "ring <= 8, xring <= 6, <= 6 groups");
 
 // Shared memory of an instance with `xring` X slots: true if at least
 // `min_ring` operand-tile slots fit (then as many as fit, at most 8).
@@ -2280,7 +2342,8 @@ df11_status launch_fused(const df11_tensor *t, const df11_gemv_mat *mats, uint32
     // Prefer six X slots (loads 3 tiles ahead, slots reused 3 tiles later),
     // then the most decode groups (staging the sign/mantissa bytes if there is
     // room) whose ring still holds 4 operand tiles; with the largest X tiles,
-    // four unstaged groups and fewer X slots.
+    // four unstaged groups and fewer X slots.  (Seven groups do not fit: with
+    // the five warps of the MMA side they pass 1024 threads.)
 #ifndef DF11_FUSED_CFG
 #define DF11_FUSED_CFG 0  // 0: by the rule above; 1..4: 6 staged, 6 unstaged, 4 staged, 4 unstaged groups
 #endif
