@@ -1483,16 +1483,17 @@ __device__ __forceinline__ FusedSmem fused_layout(const FusedArgs &f, uint32_t d
 }
 
 // Bounded wait that gives up, for good, once any wait of the CTA timed out or
-// a block could not be placed (the CTA's abort flag, polled while waiting).
-// Between rounds of probes the thread sleeps `sleep_ns`, so that waiters that
-// are not on the critical path (the epilogue, a full ring) leave the issue
-// slots to the decoder warps.
+// a block could not be placed (the CTA's abort flag, checked between probes).
+// Each probe suspends the thread for up to `hint_ns` while the phase is
+// incomplete (it resumes when the phase completes), so waiters leave the
+// issue slots to the decoder warps instead of spinning; the number of probes
+// bounds the wait at about two seconds even if no probe suspends for long.
 __device__ __forceinline__ bool fused_wait(uint32_t bar, uint32_t parity, uint32_t abort_flag, uint32_t &err,
-                                           uint32_t sleep_ns) {
-    for (uint32_t round = 0; round < (1u << 20); ++round) {
-        if (df11::tc::mbar_wait(bar, parity, 8u)) return true;
+                                           uint32_t hint_ns) {
+    const uint32_t rounds = 2000000000u / (hint_ns + 100u);
+    for (uint32_t round = 0; round < rounds; ++round) {
+        if (df11::tc::mbar_try_wait_hint(bar, parity, hint_ns)) return true;
         if (lds_u32(abort_flag)) return false;
-        if (sleep_ns) __nanosleep(sleep_ns);
     }
     err |= kFusedErrTimeout;
     sts_u32(abort_flag, 1u);
@@ -1585,7 +1586,7 @@ struct TileSink {
     __device__ __forceinline__ bool ensure(uint32_t i) {
         if (i < avail) return true;
         const uint32_t r = i / f.ring;
-        if (r > 0u && !fused_wait(L.empty0 + 8u * (i % f.ring), (r - 1u) & 1u, L.abort_flag, err, 64u))
+        if (r > 0u && !fused_wait(L.empty0 + 8u * (i % f.ring), (r - 1u) & 1u, L.abort_flag, err, 2000u))
             return false;
         avail = i + 1u;
         return true;
@@ -1782,7 +1783,7 @@ __device__ __forceinline__ void drain_segment(const FusedArgs &f, const FusedSme
     const uint32_t abuf = seg & 1u;
     // (every lane waits; the warp is converged again before the
     // .sync.aligned loads)
-    const bool have = fused_wait(L.accfull0 + 8u * abuf, (seg >> 1) & 1u, L.abort_flag, err, 256u);
+    const bool have = fused_wait(L.accfull0 + 8u * abuf, (seg >> 1) & 1u, L.abort_flag, err, 20000u);
     __syncwarp();
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
     const FusedMat &M = f.m[j];
@@ -1910,7 +1911,7 @@ __global__ void __launch_bounds__(C::kCtaThreads + kFusedExtraThreads, 1)
             uint32_t xl_slot = 0, xl_round = 0;
             auto load_x = [&]() {
                 if (xl_round == 0u ||
-                    fused_wait(L.xempty0 + 8u * xl_slot, (xl_round - 1u) & 1u, L.abort_flag, err, 0u)) {
+                    fused_wait(L.xempty0 + 8u * xl_slot, (xl_round - 1u) & 1u, L.abort_flag, err, 2000u)) {
                     df11::tc::mbar_arrive_expect_tx(L.xfull0 + 8u * xl_slot, L.xbytes);
                     df11::tc::tma_load_2d(L.xring + xl_slot * L.xbytes, &maps.x[cx.j], L.xfull0 + 8u * xl_slot,
                                           (int32_t)(cx.kt * 64u), 0);
@@ -1942,10 +1943,10 @@ __global__ void __launch_bounds__(C::kCtaThreads + kFusedExtraThreads, 1)
                 const uint32_t abuf = seg & 1u;
                 // the accumulator buffer's previous segment has been drained
                 if (first && seg >= 2u)
-                    fused_wait(L.accempty0 + 8u * abuf, ((seg >> 1) - 1u) & 1u, L.abort_flag, err, 64u);
+                    fused_wait(L.accempty0 + 8u * abuf, ((seg >> 1) - 1u) & 1u, L.abort_flag, err, 2000u);
                 df11::tc::mbar_arrive_expect_tx(L.full0 + 8u * s, kTileBytes);  // this round's tile
-                const bool ok = fused_wait(L.full0 + 8u * s, sph, L.abort_flag, err, 32u) &&
-                                fused_wait(L.xfull0 + 8u * xs, xph, L.abort_flag, err, 0u);
+                const bool ok = fused_wait(L.full0 + 8u * s, sph, L.abort_flag, err, 2000u) &&
+                                fused_wait(L.xfull0 + 8u * xs, xph, L.abort_flag, err, 2000u);
                 if (ok) {
                     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
                     const uint64_t dw = dw0 + ((s * kTileBytes) >> 4), dx = dx0 + ((xs * L.xbytes) >> 4);
