@@ -418,17 +418,38 @@ def run_decode_gemm(args, rank: int, world: int):
                 for w in gemm_mats:
                     torch.matmul(xs[w.shape[1]], w.T)
 
+        pairs = [(xs[w.shape[1]], w) for w in gemm_mats]
+
+        def multi_all():  # the seven products in one grouped launch per block
+            for _ in range(nb):
+                df11.gemm_multi(pairs, ys, err, stream)
+
+        def both_multi():
+            for d, _ in blocks:
+                df11.decode_block(d, scratch, err, stream)
+                df11.gemm_multi(pairs, ys, err, stream)
+
         def piped():  # decode of block b+1 on a side stream overlaps the GEMMs of block b
             pipe.run(range(nb), lambda bi, views: [df11.gemm(xs[w.shape[1]], v, y, err, stream)
                                                    for w, v, y in zip(gemm_mats, views[:7], ys)], stream)
 
-        t_dec, t_gemm, t_both, t_bf16, t_pipe = (timed(f, args.steps) / nb
-                                                 for f in (dec_all, gemm_all, both, bf16_all, piped))
+        t_dec, t_gemm, t_both, t_bf16, t_pipe, t_multi, t_both_multi = (
+            timed(f, args.steps) / nb for f in (dec_all, gemm_all, both, bf16_all, piped, multi_all, both_multi))
+        # numerics of the grouped launch: sampled columns vs FP64
+        df11.gemm_multi(pairs, ys, err, stream)
+        rel_multi = 0.0
+        for w, y in zip(gemm_mats, ys):
+            cols = torch.arange(0, w.shape[0], max(1, w.shape[0] // 256), device=dev)
+            ref = xs[w.shape[1]].double() @ w[cols].double().T
+            rel_multi = max(rel_multi, float((y[:, cols].double() - ref).norm() / ref.norm()))
         x_bytes = sum(T * w.shape[1] * 2 + T * w.shape[0] * 4 for w in gemm_mats)
         per_T[str(T)] = {"decode_us": t_dec * 1e3, "gemm_us": t_gemm * 1e3, "total_us": t_both * 1e3,
                          "bf16_gemm_us": t_bf16 * 1e3, "slowdown_vs_bf16": t_both / t_bf16,
                          "pipelined_total_us": t_pipe * 1e3,
-                         "gemm_gbs": (w_bytes + x_bytes) / (t_gemm * 1e-3) / 1e9, "gemm_rel_fro": rel}
+                         "gemm_gbs": (w_bytes + x_bytes) / (t_gemm * 1e-3) / 1e9, "gemm_rel_fro": rel,
+                         "gemm_multi_us": t_multi * 1e3, "total_multi_us": t_both_multi * 1e3,
+                         "gemm_multi_gbs": (w_bytes + x_bytes) / (t_multi * 1e-3) / 1e9,
+                         "gemm_multi_rel_fro": rel_multi}
         if T <= 4:
             # fused decode -> matrix-vector products: per block, one zeroing of
             # the seven outputs and one launch for all seven matrices; the
@@ -777,8 +798,22 @@ def run_gemm(args, rank: int, world: int):
     b.record(stream)
     torch.cuda.synchronize(dev)
     ms = a.elapsed_time(b) / args.steps
+
+    def other(fn):  # the same protocol for another implementation
+        for i in range(args.warmup):
+            fn(i)
+        torch.cuda.synchronize(dev)
+        a.record(stream)
+        for i in range(args.steps):
+            fn(i)
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        return a.elapsed_time(b) / args.steps
+
+    ms_cublas = other(lambda i: torch.matmul(x, ws[i % 3].T))
+    ms_multi = other(lambda i: df11.gemm_multi([(x, ws[i % 3])], [y], err, stream))
     if world > 1:
-        ms = max_over_ranks(ms, dist, dev)
+        ms, ms_cublas, ms_multi = (max_over_ranks(v, dist, dev) for v in (ms, ms_cublas, ms_multi))
     assert df11.read_error(err, stream) == 0
     if rank == 0:
         hbm, hbm_kind = _peaks()
@@ -802,7 +837,8 @@ def run_gemm(args, rank: int, world: int):
                 "config": {"workload": WORKLOADS["gemm"][0], "shape": [out, inn], "T": T,
                            "kernel": "CUDA-core matrix-vector stream" if T <= 4 else "tcgen05",
                            "l2": "W in three copies used in turn (3 x 2 out in bytes > L2), no flush"},
-                "rel_fro_sampled_rows": rel, "roofline": roof, "gpu_launches": args.steps}
+                "rel_fro_sampled_rows": rel, "roofline": roof, "gpu_launches": args.steps,
+                "cublas_us": ms_cublas * 1e3, "grouped_kernel_us": ms_multi * 1e3}
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()

@@ -31,7 +31,7 @@ from . import build as _build
 __all__ = [
     "DF11Error", "CorruptStreamError", "Params", "DF11Tensor", "encode", "encode_multi",
     "encode_device", "encode_device_noalloc", "save", "load", "decode", "decode_block", "decode_rows", "decode_gemv",
-    "decode_gemm", "gemm", "read_error", "exponent_histogram", "lib_path", "sm_count", "to_tile_order",
+    "decode_gemm", "gemm", "gemm_multi", "read_error", "exponent_histogram", "lib_path", "sm_count", "to_tile_order",
     "from_tile_order",
     "KERR_COUNT_MISMATCH", "KERR_BAD_CODE", "KERR_BAD_BLOCK", "KERR_OVERRUN", "KERR_TIMEOUT", "KERR_BAD_ROW",
 ]
@@ -75,6 +75,11 @@ class _Tensor(ctypes.Structure):
                 ("block_start", ctypes.c_void_p), ("lut", ctypes.c_void_p), ("counts", ctypes.c_void_p)]
 
 
+class _GemmMat(ctypes.Structure):
+    _fields_ = [("x", ctypes.c_void_p), ("w", ctypes.c_void_p), ("y", ctypes.c_void_p),
+                ("out", ctypes.c_uint32), ("in_", ctypes.c_uint32)]
+
+
 class _GemvMat(ctypes.Structure):
     _fields_ = [("elem_offset", ctypes.c_uint64), ("rows", ctypes.c_uint32), ("cols", ctypes.c_uint32),
                 ("x", ctypes.c_void_p), ("y", ctypes.c_void_p)]
@@ -116,6 +121,7 @@ def _lib():
     lib.df11_read_error.argtypes = [vp, vp, P(u32)]
     lib.df11_device_sm_count.argtypes = [P(ctypes.c_int)]
     lib.df11_gemm_bf16.argtypes = [vp, vp, vp, u32, u32, u32, vp, vp]
+    lib.df11_gemm_bf16_multi.argtypes = [P(_GemmMat), u32, u32, vp, vp]
     lib.df11_decode_rows.argtypes = [P(_Tensor), ctypes.c_uint64, vp, u32, vp, vp, vp]
     lib.df11_decode_gemv.argtypes = [P(_Tensor), P(_GemvMat), u32, u32, vp, vp]
     lib.df11_decode_gemm.argtypes = [P(_Tensor), P(_GemvMat), u32, u32, vp, vp]
@@ -714,6 +720,42 @@ def gemm(x, w, out=None, err=None, stream=None):
     if own_err:
         read_error(err, stream)
     return out
+
+
+def gemm_multi(pairs, outs=None, err=None, stream=None):
+    """Several products Y_j = X_j @ W_j^T in one call (one persistent
+    tensor-core launch for T > 4): ``pairs`` is a list of (x [T, in_j],
+    w [out_j, in_j]) BF16 CUDA tensors with one T; returns the FP32 results
+    [T, out_j] (written into ``outs`` when given)."""
+    import torch
+    if not pairs:
+        return []
+    dev = pairs[0][0].device
+    T = int(pairs[0][0].shape[0])
+    if outs is None:
+        outs = [torch.empty(T, w.shape[0], dtype=torch.float32, device=dev) for _, w in pairs]
+    if len(outs) != len(pairs):
+        raise ValueError("one output per product")
+    mats = (_GemmMat * len(pairs))()
+    for k, ((x, w), y) in enumerate(zip(pairs, outs)):
+        if x.dtype != torch.bfloat16 or w.dtype != torch.bfloat16 or x.dim() != 2 or w.dim() != 2:
+            raise TypeError("gemm_multi expects 2-D bfloat16 tensors")
+        if not x.is_contiguous() or not w.is_contiguous() or not y.is_contiguous():
+            raise ValueError("gemm_multi expects contiguous tensors")
+        if x.shape[0] != T or x.shape[1] != w.shape[1] or tuple(y.shape) != (T, w.shape[0]):
+            raise ValueError("shapes do not match")
+        if y.dtype != torch.float32 or x.device != dev or w.device != dev or y.device != dev:
+            raise ValueError("gemm_multi expects FP32 outputs and one device")
+        mats[k] = _GemmMat(x.data_ptr(), w.data_ptr(), y.data_ptr(), int(w.shape[0]), int(w.shape[1]))
+    own_err = err is None
+    if own_err:
+        err = _new_err(dev)
+    with _on(dev):
+        _check(_lib().df11_gemm_bf16_multi(mats, len(pairs), T, ctypes.c_void_p(err.data_ptr()),
+                                           _stream_handle(stream, dev)), "gemm_multi")
+    if own_err:
+        read_error(err, stream)
+    return outs
 
 
 def read_error(err, stream=None) -> int:

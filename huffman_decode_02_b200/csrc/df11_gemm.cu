@@ -169,6 +169,247 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (err && g.err) atomicOr(g.err, err);
 }
 
+// ---------------------------------------------------------------- grouped
+// Several products Y_j = X_j W_j^T in one persistent launch (e.g. the seven
+// matrices of a decoded transformer block).  The 128 x 64 k-tiles of all the
+// matrices, numbered matrix by matrix, row tile by row tile and along K,
+// are split evenly over the CTAs: no launch leaves a tail and every SM
+// streams the same number of weight bytes.  Warp 0 loads the W and X tiles
+// of each k-tile by TMA (128-byte swizzle, no multicast) into a ring of
+// stages; warp 1 issues four tcgen05.mma (K = 16 each) per k-tile into one
+// of two FP32 accumulators in tensor memory, which alternate between
+// segments (a segment = the k-tiles of one row tile in this CTA); warps 2..5
+// read each finished segment (tcgen05.ld, TMEM lanes of their rank in the
+// warpgroup) and add it into Y with FP32 atomics (a row tile split between
+// two CTAs gets two partial sums; the launcher zeroes Y).  Every wait is
+// bounded and suspends on the mbarrier instead of spinning.
+constexpr uint32_t kMultiMax = 16;
+constexpr uint32_t kMultiThreads = 192;
+constexpr uint32_t kMultiStagesMax = 16;
+constexpr uint32_t kTileW = kBlockM * kBlockK * 2u;  // one W k-tile: 16 KB
+
+struct MultiMat {
+    float *y;
+    uint32_t rows;   // out
+    uint32_t kt;     // k-tiles per row tile: in / 64
+    uint32_t rt;     // row tiles: out / 128
+    uint32_t tbase;  // first k-tile of this matrix in the numbering
+};
+struct MultiArgs {
+    MultiMat m[kMultiMax];
+    uint32_t *err;
+    uint32_t n_mats, T, n_pad, n_tiles, stages, xbytes, tmem_cols;
+    uint32_t sub;  // k-tiles per stage (1 or 2; every matrix's k-tiles per row tile are a multiple)
+};
+struct MultiMaps {
+    CUtensorMap w[kMultiMax];  // W_j [out, in], box [128, 64]
+    CUtensorMap x[kMultiMax];  // X_j [T, in], box [n_pad, 64]
+};
+
+// k-tile cursor: matrix j, row tile r, k-tile column k
+struct MultiCursor {
+    uint32_t j, r, k;
+    __device__ __forceinline__ void start(const MultiArgs &g, uint32_t K) {
+        j = 0;
+        while (j + 1u < g.n_mats && K >= g.m[j + 1u].tbase) ++j;
+        const uint32_t l = K - g.m[j].tbase;
+        r = l / g.m[j].kt;
+        k = l % g.m[j].kt;
+    }
+    __device__ __forceinline__ void next(const MultiArgs &g) {
+        if (++k < g.m[j].kt) return;
+        k = 0;
+        if (++r < g.m[j].rt) return;
+        r = 0;
+        ++j;
+    }
+};
+
+// Bounded wait (about two seconds at most) that gives up once the CTA's
+// abort flag is set.  hint_ns > 0: each probe suspends up to hint_ns while
+// the phase is incomplete (for waiters off the critical path); 0: plain
+// probes (the producer and the MMA issuer, whose wake-up latency sets the
+// pipeline's pace).
+__device__ __forceinline__ bool multi_wait(uint32_t bar, uint32_t parity, uint32_t abort_flag, uint32_t &err,
+                                           uint32_t hint_ns) {
+    const uint32_t rounds = 2000000000u / (hint_ns + 100u);
+    for (uint32_t i = 0; i < rounds; ++i) {
+        if (hint_ns ? mbar_try_wait_hint(bar, parity, hint_ns) : mbar_wait(bar, parity, 1u)) return true;
+        uint32_t a;
+        asm volatile("ld.shared.u32 %0, [%1];" : "=r"(a) : "r"(abort_flag) : "memory");
+        if (a) return false;
+    }
+    err |= kGemmErrTimeout;
+    asm volatile("st.shared.u32 [%0], %1;" ::"r"(abort_flag), "r"(1u) : "memory");
+    return false;
+}
+
+// Zeroes every product's Y [T, out] (one launch for all of them; 16-byte
+// stores where the buffer allows, else 4-byte ones).
+__global__ void zero_y_kernel(const __grid_constant__ MultiArgs g) {
+    const uint64_t stride = (uint64_t)gridDim.x * blockDim.x;
+    for (uint32_t j = 0; j < g.n_mats; ++j) {
+        float *y = g.m[j].y;
+        const uint64_t n = (uint64_t)g.T * g.m[j].rows;
+        const uint64_t i0 = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x;
+        if (((uintptr_t)y & 15u) == 0u) {
+            for (uint64_t i = i0; i < n / 4u; i += stride) reinterpret_cast<float4 *>(y)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (uint64_t i = (n / 4u) * 4u + i0; i < n; i += stride) y[i] = 0.f;
+        } else {
+            for (uint64_t i = i0; i < n; i += stride) y[i] = 0.f;
+        }
+    }
+}
+
+__global__ void __launch_bounds__(kMultiThreads, 1)
+    df11_gemm_multi_kernel(const __grid_constant__ MultiArgs g, const __grid_constant__ MultiMaps maps) {
+    extern __shared__ __align__(1024) uint8_t smem[];
+    const uint32_t tid = threadIdx.x, warp = tid >> 5, lane = tid & 31u;
+    const uint32_t stage_bytes = g.sub * (kTileW + g.xbytes);  // multiples of 1024 (n_pad is a multiple of 16)
+    const uint32_t base = (smem_u32(smem) + 1023u) & ~1023u;
+    const uint32_t full0 = base + g.stages * stage_bytes, empty0 = full0 + 8u * kMultiStagesMax;
+    const uint32_t accfull0 = empty0 + 8u * kMultiStagesMax, accempty0 = accfull0 + 16u;
+    const uint32_t final_bar = accempty0 + 16u, tmem_slot = final_bar + 8u, abort_flag = tmem_slot + 4u;
+    // whole stages per CTA (n_tiles is a multiple of sub)
+    const uint32_t n_st = g.n_tiles / g.sub;
+    const uint32_t K0 = g.sub * (uint32_t)((uint64_t)n_st * blockIdx.x / gridDim.x);
+    const uint32_t NT = g.sub * (uint32_t)((uint64_t)n_st * (blockIdx.x + 1u) / gridDim.x) - K0;
+    uint32_t err = 0;
+
+    if (tid == 0) {
+        for (uint32_t s = 0; s < g.stages; ++s) {
+            mbar_init(full0 + 8u * s, 1);
+            mbar_init(empty0 + 8u * s, 1);
+        }
+        for (uint32_t a = 0; a < 2u; ++a) {
+            mbar_init(accfull0 + 8u * a, 1);
+            mbar_init(accempty0 + 8u * a, 4);  // one arrival per epilogue warp
+        }
+        mbar_init(final_bar, 1);
+        asm volatile("st.shared.u32 [%0], %1;" ::"r"(abort_flag), "r"(0u) : "memory");
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 2) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(tmem_slot),
+                     "r"(g.tmem_cols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    __syncthreads();
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    uint32_t tmem;
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(tmem) : "r"(tmem_slot) : "memory");
+
+    if (warp == 0) {
+        if (lane == 0) {  // ---- producer
+            MultiCursor c;
+            c.start(g, K0);
+            uint32_t s = 0, use = 0;
+            for (uint32_t i = 0; i < NT; i += g.sub) {
+                if (use > 0u && !multi_wait(empty0 + 8u * s, (use - 1u) & 1u, abort_flag, err, 0u)) break;
+                const uint32_t a = base + s * stage_bytes;
+                mbar_arrive_expect_tx(full0 + 8u * s, stage_bytes);
+                for (uint32_t u = 0; u < g.sub; ++u) {
+                    tma_load_2d(a + u * kTileW, &maps.w[c.j], full0 + 8u * s, (int32_t)(c.k * kBlockK),
+                                (int32_t)(c.r * kBlockM));
+                    tma_load_2d(a + g.sub * kTileW + u * g.xbytes, &maps.x[c.j], full0 + 8u * s,
+                                (int32_t)(c.k * kBlockK), 0);
+                    c.next(g);
+                }
+                if (++s == g.stages) {
+                    s = 0;
+                    ++use;
+                }
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        if (lane == 0) {  // ---- MMA issuer
+            const uint32_t idesc = instr_desc_bf16(g.n_pad, kBlockM);
+            const uint64_t d0 = smem_desc_sw128(base);
+            MultiCursor c;
+            c.start(g, K0);
+            uint32_t s = 0, use = 0, seg = 0;
+            bool stop = false;
+            for (uint32_t i = 0; i < NT && !stop; i += g.sub) {
+                if (!multi_wait(full0 + 8u * s, use & 1u, abort_flag, err, 0u)) break;
+                const uint64_t da0 = d0 + ((s * stage_bytes) >> 4), db0 = da0 + ((g.sub * kTileW) >> 4);
+                for (uint32_t u = 0; u < g.sub; ++u) {  // (segments start and end on stage boundaries)
+                    const bool first = i + u == 0u || c.k == 0u;
+                    const bool last = i + u + 1u == NT || c.k + 1u == g.m[c.j].kt;
+                    const uint32_t abuf = seg & 1u;
+                    if (first && seg >= 2u &&
+                        !multi_wait(accempty0 + 8u * abuf, ((seg >> 1) - 1u) & 1u, abort_flag, err, 0u)) {
+                        stop = true;
+                        break;
+                    }
+                    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+                    const uint64_t da = da0 + ((u * kTileW) >> 4), db = db0 + ((u * g.xbytes) >> 4);
+#pragma unroll
+                    for (uint32_t kk = 0; kk < kBlockK / kUmmaK; ++kk)  // K = 16: 32 bytes along the swizzled row
+                        umma_bf16(tmem + abuf * g.n_pad, da + 2u * kk, db + 2u * kk, idesc,
+                                  (first && kk == 0u) ? 0u : 1u);
+                    if (last) {
+                        umma_commit(accfull0 + 8u * abuf);
+                        ++seg;
+                    }
+                    c.next(g);
+                }
+                umma_commit(empty0 + 8u * s);
+                if (++s == g.stages) {
+                    s = 0;
+                    ++use;
+                }
+            }
+            // every issued MMA has completed before the accumulators are freed
+            umma_commit(final_bar);
+            if (!mbar_wait(final_bar, 0u)) err |= kGemmErrTimeout;
+        }
+        __syncwarp();
+    } else {
+        // ---- epilogue: warp rank q in its warpgroup reads TMEM lanes 32q..32q+31
+        const uint32_t q = warp & 3u;
+        MultiCursor c;
+        c.start(g, K0);
+        uint32_t seg = 0;
+        for (uint32_t i = 0; i < NT;) {
+            const uint32_t n = min(g.m[c.j].kt - c.k, NT - i);  // the segment's k-tiles
+            const uint32_t j = c.j, rtile = c.r;
+            i += n;
+            c.k += n - 1u;
+            c.next(g);
+            const uint32_t abuf = seg & 1u;
+            const bool have = multi_wait(accfull0 + 8u * abuf, (seg >> 1) & 1u, abort_flag, err, 2000u);
+            __syncwarp();
+            asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+            const MultiMat &M = g.m[j];
+            const uint32_t row = rtile * kBlockM + q * 32u + lane;
+            for (uint32_t c0 = 0; c0 < g.n_pad; c0 += 16u) {
+                uint32_t v[16];
+                tmem_ld16(tmem + ((q * 32u) << 16) + abuf * g.n_pad + c0, v);
+                if (have) {
+#pragma unroll
+                    for (uint32_t t = 0; t < 16u; ++t)
+                        if (c0 + t < g.T) atomicAdd(M.y + (uint64_t)(c0 + t) * M.rows + row, __uint_as_float(v[t]));
+                }
+            }
+            asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+            __syncwarp();
+            if (lane == 0u) mbar_arrive(accempty0 + 8u * abuf);
+            ++seg;
+        }
+    }
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    __syncthreads();
+    if (warp == 2) {
+        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(g.tmem_cols)
+                     : "memory");
+    }
+    if (err && g.err) atomicOr(g.err, err);
+}
+
 // ---------------------------------------------------------------- T <= 4
 // With T <= 4 tokens every weight feeds at most 8 flops: the product is a
 // matrix-vector stream bound by reading W, and the tensor-core tiling (128
@@ -377,6 +618,82 @@ extern "C" df11_status df11_gemm_bf16(const uint16_t *x, const uint16_t *w, floa
     if (g.atomic_out && cudaMemsetAsync(y, 0, (size_t)T * out * sizeof(float), s) != cudaSuccess)
         return DF11_ERR_CUDA;
     df11_gemm_kernel<<<m_tiles * splits, kThreads, smem, s>>>(mw, mx, g);
+    if (cudaGetLastError() != cudaSuccess) return DF11_ERR_CUDA;
+    return DF11_OK;
+}
+
+extern "C" df11_status df11_gemm_bf16_multi(const df11_gemm_mat *mats, uint32_t n_mats, uint32_t T,
+                                            uint32_t *err_word, void *stream) {
+    if (n_mats == 0) return DF11_OK;
+    if (!mats) return DF11_ERR_INVALID_ARG;
+    if (n_mats > kMultiMax || T == 0 || T > 256) return DF11_ERR_UNSUPPORTED;
+    for (uint32_t j = 0; j < n_mats; ++j) {
+        const df11_gemm_mat &m = mats[j];
+        if (!m.x || !m.w || !m.y) return DF11_ERR_INVALID_ARG;
+        if (m.out == 0 || m.out % kBlockM != 0 || m.in == 0 || m.in % kBlockK != 0) return DF11_ERR_UNSUPPORTED;
+        if (((uintptr_t)m.x & 15u) || ((uintptr_t)m.w & 15u) || ((uintptr_t)m.y & 3u)) return DF11_ERR_INVALID_ARG;
+    }
+    if (T <= 4u) {  // matrix-vector streams (one launch per matrix)
+        for (uint32_t j = 0; j < n_mats; ++j) {
+            const df11_status st = df11_gemm_bf16(mats[j].x, mats[j].w, mats[j].y, T, mats[j].out, mats[j].in,
+                                                  err_word, stream);
+            if (st != DF11_OK) return st;
+        }
+        return DF11_OK;
+    }
+    if (!get_encoder()) return DF11_ERR_CUDA;
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return DF11_ERR_CUDA;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return DF11_ERR_CUDA;
+    MultiArgs g;
+    MultiMaps maps;
+    g.err = err_word;
+    g.n_mats = n_mats;
+    g.T = T;
+    g.n_pad = (T + 15u) & ~15u;
+    g.xbytes = g.n_pad * kBlockK * 2u;
+    g.tmem_cols = 32u;
+    while (g.tmem_cols < 2u * g.n_pad) g.tmem_cols <<= 1;
+    // two k-tiles per stage (each W row read 256 contiguous bytes at a time)
+    // when the X tiles are small and every row tile has an even k-tile count
+    g.sub = g.n_pad <= 128u ? 2u : 1u;
+    for (uint32_t j = 0; j < n_mats; ++j)
+        if ((mats[j].in / kBlockK) % 2u) g.sub = 1u;
+    uint64_t tiles = 0;
+    for (uint32_t j = 0; j < n_mats; ++j) {
+        const df11_gemm_mat &m = mats[j];
+        g.m[j] = MultiMat{m.y, m.out, m.in / kBlockK, m.out / kBlockM, (uint32_t)tiles};
+        tiles += (uint64_t)(m.out / kBlockM) * (m.in / kBlockK);
+        if (!make_map(&maps.w[j], m.w, m.out, m.in, kBlockM) || !make_map(&maps.x[j], m.x, T, m.in, g.n_pad))
+            return DF11_ERR_CUDA;
+    }
+    if (tiles >= (1ull << 32)) return DF11_ERR_UNSUPPORTED;
+    for (uint32_t j = n_mats; j < kMultiMax; ++j) {
+        g.m[j] = MultiMat{nullptr, 0u, 1u, 1u, (uint32_t)tiles};
+        maps.w[j] = maps.w[0];
+        maps.x[j] = maps.x[0];
+    }
+    g.n_tiles = (uint32_t)tiles;
+    // the deepest ring that fits: stages of one W k-tile and one X k-tile
+    constexpr uint32_t kMultiSmem = 227u * 1024u;
+    constexpr uint32_t kTail = 1024u + 8u * (2u * kMultiStagesMax + 5u) + 16u;  // alignment, barriers, flags
+    const uint32_t stage_bytes = g.sub * (kTileW + g.xbytes);
+    g.stages = (kMultiSmem - kTail) / stage_bytes;
+    if (g.stages > kMultiStagesMax) g.stages = kMultiStagesMax;
+    if (g.stages < 2u) return DF11_ERR_UNSUPPORTED;
+    const uint32_t smem = kTail + g.stages * stage_bytes;
+    static std::atomic<int> attr_set[64];
+    if (!attr_set[dev].load(std::memory_order_acquire)) {
+        if (cudaFuncSetAttribute(df11_gemm_multi_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)kMultiSmem) != cudaSuccess)
+            return DF11_ERR_CUDA;
+        attr_set[dev].store(1, std::memory_order_release);
+    }
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    zero_y_kernel<<<2u * (unsigned)sms, 256, 0, s>>>(g);  // partial sums are added into Y
+    const uint32_t n_st = g.n_tiles / g.sub;  // every CTA gets at least one stage
+    const unsigned grid = (unsigned)(n_st < (uint32_t)sms ? n_st : (uint32_t)sms);
+    df11_gemm_multi_kernel<<<grid, kMultiThreads, smem, s>>>(g, maps);
     if (cudaGetLastError() != cudaSuccess) return DF11_ERR_CUDA;
     return DF11_OK;
 }

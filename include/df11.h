@@ -375,6 +375,32 @@ df11_status df11_from_tile_order(const uint16_t *tiled, uint32_t rows, uint32_t 
 df11_status df11_gemm_bf16(const uint16_t *x, const uint16_t *w, float *y, uint32_t T, uint32_t out,
                            uint32_t in, uint32_t *err_word, void *stream);
 
+/* One product of df11_gemm_bf16_multi: Y = X * W^T with
+ *  x: DEVICE [T, in] BF16 (uint16 bits), row-major, 16-byte aligned
+ *  w: DEVICE [out, in] BF16, row-major, 16-byte aligned
+ *  y: DEVICE [T, out] FP32, row-major, 4-byte aligned; fully overwritten
+ *  out a multiple of 128, in a multiple of 64. */
+typedef struct df11_gemm_mat {
+    const uint16_t *x;
+    const uint16_t *w;
+    float *y;
+    uint32_t out, in;
+} df11_gemm_mat;
+
+/* Several consumer products of decoded weights, e.g. the seven matrices of a
+ * decoded transformer block ("Decompression adaptee a l'inference GPU": each
+ * matrix is multiplied right after its decompression), in ONE persistent
+ * tensor-core launch for T > 4: the 128 x 64 weight tiles of all products
+ * are split evenly over the SMs (no per-matrix launch tail), partial sums
+ * are added into Y with FP32 atomics after the Y buffers are zeroed on the
+ * stream (the last bits may differ run to run).  T <= 4: one matrix-vector
+ * launch per product, as df11_gemm_bf16.  1 <= n_mats <= 16, 1 <= T <= 256
+ * (else DF11_ERR_UNSUPPORTED; shape and alignment faults as for
+ * df11_gemm_bf16).  err_word: bit 0x20 when a wait timed out; may be NULL.
+ * Asynchronous on `stream`; `mats` is read before the call returns. */
+df11_status df11_gemm_bf16_multi(const df11_gemm_mat *mats, uint32_t n_mats, uint32_t T, uint32_t *err_word,
+                                 void *stream);
+
 /* Copies *err_word to the host after the stream's work so far completes
  * (synchronises the stream) and returns DF11_ERR_CORRUPT if any bit is set. */
 df11_status df11_read_error(const uint32_t *err_word, void *stream, uint32_t *host_value);

@@ -128,3 +128,85 @@ def test_gemm_lm_head_shape(T):
     cols = torch.from_numpy(np.random.default_rng(T).choice(128256, 1024, replace=False)).to(dev)
     ref = (x.double() @ w[cols].double().T).cpu().numpy()
     assert _rel_fro(y[:, cols].double().cpu().numpy(), ref) <= TOL
+
+
+def _mats(shapes, T, seed):
+    rng = np.random.default_rng(seed)
+    out = []
+    for o, i in shapes:
+        x = workloads.round_to_bf16(rng.standard_normal((T, i), dtype=np.float32))
+        w = workloads.round_to_bf16(rng.standard_normal((o, i), dtype=np.float32) * np.float32(0.02))
+        out.append((x, w))
+    return out
+
+
+def _check_multi(shapes, T, seed, rows=None):
+    """gemm_multi against FP64 per product: every output within the FP32
+    accumulation bound (K + 64) * 2^-23 * sum |w x| and the relative
+    Frobenius error within 2e-3.  `rows`: sampled output rows per product."""
+    dev = _dev()
+    data = _mats(shapes, T, seed)
+    pairs = [(_bf16(x).to(dev), _bf16(w).to(dev)) for x, w in data]
+    ys = df11.gemm_multi(pairs)
+    torch.cuda.synchronize()
+    for (x, w), y in zip(data, ys):
+        X, W = _bf16(x).double(), _bf16(w).double()
+        got = y.cpu().double()
+        if rows is not None:
+            r = np.unique(np.concatenate([[0, w.shape[0] - 1], np.random.default_rng(seed).integers(0, w.shape[0], rows)]))
+            W, got = W[torch.as_tensor(r)], got[:, torch.as_tensor(r)]
+        ref, mag = X @ W.T, X.abs() @ W.abs().T
+        assert bool(torch.all((got - ref).abs() <= (w.shape[1] + 64) * 2.0 ** -23 * mag + 1e-30))
+        assert float((got - ref).norm() / ref.norm()) <= TOL
+
+
+@pytest.mark.parametrize("T", [5, 16, 17, 64, 200, 256])
+def test_gemm_multi_mixed_shapes(T):
+    """Products of several shapes in one launch: row tiles split between
+    CTAs (partial sums added), matrices smaller than a CTA's share, a
+    single-tile matrix, T not a multiple of 16."""
+    _check_multi([(256, 128), (128, 64), (1024, 4096), (384, 192), (128, 1024)], T, seed=T)
+
+
+@pytest.mark.parametrize("T", [5, 16, 33, 64, 128])
+def test_gemm_multi_two_tiles_per_stage(T):
+    """Every product with an even number of k-tiles per row tile: stages of
+    two k-tiles (a stage may end one row tile and start the next)."""
+    _check_multi([(256, 128), (1024, 4096), (128, 1024), (512, 256), (128, 128)], T, seed=50 + T)
+
+
+@pytest.mark.parametrize("T", [1, 4])
+def test_gemm_multi_matrix_vector(T):
+    _check_multi([(256, 128), (1024, 4096)], T, seed=10 + T)
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("T", [16, 64, 256])
+def test_gemm_multi_llama_block(T):
+    """The seven Llama-3.1-8B block shapes in one launch; 256 sampled rows
+    of each output (first and last among them) against FP64."""
+    shapes = [(4096, 4096), (1024, 4096), (1024, 4096), (4096, 4096), (14336, 4096), (14336, 4096), (4096, 14336)]
+    _check_multi(shapes, T, seed=100 + T, rows=254)
+
+
+def test_gemm_multi_overwrites_y():
+    """Y is overwritten (zeroed, then the partial sums added), not added into."""
+    dev = _dev()
+    data = _mats([(512, 2048)], 32, 7)
+    x, w = (_bf16(a).to(dev) for a in data[0])
+    y = torch.full((32, 512), 3.0, dtype=torch.float32, device=dev)
+    df11.gemm_multi([(x, w)], outs=[y])
+    ref = _bf16(data[0][0]).double() @ _bf16(data[0][1]).double().T
+    assert float((y.cpu().double() - ref).norm() / ref.norm()) <= TOL
+
+
+def test_gemm_multi_rejects_unsupported():
+    dev = _dev()
+    x = torch.zeros(16, 64, dtype=torch.bfloat16, device=dev)
+    w = torch.zeros(100, 64, dtype=torch.bfloat16, device=dev)
+    with pytest.raises(df11.DF11Error):
+        df11.gemm_multi([(x, w)])
+    x2 = torch.zeros(300, 64, dtype=torch.bfloat16, device=dev)
+    w2 = torch.zeros(128, 64, dtype=torch.bfloat16, device=dev)
+    with pytest.raises(df11.DF11Error):
+        df11.gemm_multi([(x2, w2)])

@@ -444,3 +444,29 @@ def test_decode_gemm_argument_checks():
     assert call([(8192, 256, 128, X, Y), (0, 128, 64, X, Y)]) == 1   # out of order
     assert call([(16384, 256, 128, X, Y)]) == 1                # runs past the tensor's end
     assert call(good * 9) == 2                                 # more than 16 matrices
+
+
+def test_gemm_multi_argument_checks():
+    """df11_gemm_bf16_multi refuses bad calls before any GPU work: no
+    products is a no-op; more than 16 products, T outside 1..256, out not a
+    multiple of 128 or in of 64 are unsupported; NULL or misaligned pointers
+    are invalid."""
+    lib = df11._lib()
+    buf, own = _aligned_copy(np.zeros(4096, dtype=np.uint16))
+    A = buf.ctypes.data
+
+    def call(descs, T=16, n=None):
+        arr = (df11._GemmMat * max(1, len(descs)))(*[df11._GemmMat(*m) for m in descs])
+        return lib.df11_gemm_bf16_multi(arr, len(descs) if n is None else n, T, None, None)
+
+    good = (A, A, A, 128, 64)
+    assert call([good], n=0) == 0
+    assert call([good] * 17) == 2
+    assert call([good], T=0) == 2 and call([good], T=257) == 2
+    assert call([(A, A, A, 100, 64)]) == 2                     # out not a multiple of 128
+    assert call([(A, A, A, 128, 32)]) == 2                     # in not a multiple of 64
+    assert call([(0, A, A, 128, 64)]) == 1                     # NULL x
+    assert call([(A + 2, A, A, 128, 64)]) == 1                 # x not 16-byte aligned
+    assert call([(A, A + 8, A, 128, 64)]) == 1                 # w not 16-byte aligned
+    assert call([(A, A, A + 2, 128, 64)]) == 1                 # y not 4-byte aligned
+    assert lib.df11_gemm_bf16_multi(None, 1, 16, None, None) == 1
