@@ -60,8 +60,9 @@ WORKLOADS = {
                    "all seven matrices multiplied by N(0,1) BF16 activations [T, in] (seed 1000 + T) in ONE fused "
                    "decode -> tcgen05 GEMM launch (weights decoded into shared-memory operand tiles, never "
                    "written to memory); T from --T (1..256)", None),
-    "gemm": ("consumer GEMM Y = X W^T on one weight shape (default 14336x4096, the gate/up projection), "
-             "W N(0, 0.02^2) BF16 in three copies used in turn (351 MB, larger than L2), X N(0,1) BF16 [T, in]",
+    "gemm": ("consumer GEMM Y = X W^T on one weight shape (default 14336x4096, the gate/up projection) or, with "
+             "--shape llama8b-block, on the seven matrices of a llama3.1-8b block; W N(0, 0.02^2) BF16 in three "
+             "copies used in turn (larger than L2), X N(0,1) BF16 [T, in]",
              None),
     "encode-device": ("llama3.1-8b transformer block (218,112,000 BF16 weights, seed = rank) already in device memory, "
                       "encoded on the GPU (histogram + packing; code lengths on the host)", None),
@@ -761,59 +762,76 @@ def _tensor_peak() -> float:
 
 
 def run_gemm(args, rank: int, world: int):
-    """The consumer GEMM alone on one shape: CUDA-core matrix-vector stream for
-    T <= 4, tcgen05 kernel above; three copies of W are used in turn so every
-    launch reads W from HBM."""
+    """The consumer GEMM alone: on one weight shape (CUDA-core matrix-vector
+    stream for T <= 4, the tcgen05 kernel above), or with --shape
+    llama8b-block on the seven matrices of a Llama block (the grouped kernel:
+    one launch for the seven products).  cuBLAS (torch.matmul, one call per
+    matrix) runs the same protocol beside it.  Three copies of the weights are
+    used in turn so every launch reads them from HBM."""
     import torch
     import torch.distributed as dist
 
     import huffman_decode_02_b200 as df11
+    import workloads
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     if world > 1:
         from datetime import timedelta
         dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=dev)
-    out, inn = (int(v) for v in args.shape.lower().split("x"))
+    block = args.shape.lower() == "llama8b-block"
+    shapes = list(workloads.LLAMA8B_BLOCK_SHAPES[:7]) if block else \
+        [tuple(int(v) for v in args.shape.lower().split("x"))]
     T = args.T
     g = torch.Generator(device=dev).manual_seed(rank)
-    ws = [(torch.randn(out, inn, device=dev, generator=g) * 0.02).to(torch.bfloat16) for _ in range(3)]
-    x = torch.randn(T, inn, device=dev, generator=g).to(torch.bfloat16)
-    y = torch.empty(T, out, dtype=torch.float32, device=dev)
+    ws = [[(torch.randn(o, i, device=dev, generator=g) * 0.02).to(torch.bfloat16) for o, i in shapes]
+          for _ in range(3)]
+    xs = {i: torch.randn(T, i, device=dev, generator=g).to(torch.bfloat16) for _, i in shapes}
+    ys = [torch.empty(T, o, dtype=torch.float32, device=dev) for o, _ in shapes]
     err = torch.zeros(1, dtype=torch.int32, device=dev)
     stream = torch.cuda.current_stream(dev)
-    df11.gemm(x, ws[0], y, err, stream)
-    rows = torch.arange(0, out, max(1, out // 256), device=dev)
-    ref = x.double().cpu() @ ws[0][rows].double().cpu().T
-    rel = float((y[:, rows].double().cpu() - ref).norm() / ref.norm())
-    for i in range(args.warmup):
-        df11.gemm(x, ws[i % 3], y, err, stream)
-    torch.cuda.synchronize(dev)
-    if world > 1:
-        dist.barrier()
-    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record(stream)
-    for i in range(args.steps):
-        df11.gemm(x, ws[i % 3], y, err, stream)
-    b.record(stream)
-    torch.cuda.synchronize(dev)
-    ms = a.elapsed_time(b) / args.steps
 
-    def other(fn):  # the same protocol for another implementation
+    def ours(c):
+        if block:
+            df11.gemm_multi([(xs[w.shape[1]], w) for w in ws[c]], ys, err, stream)
+        else:
+            df11.gemm(xs[shapes[0][1]], ws[c][0], ys[0], err, stream)
+
+    ours(0)
+    rel = 0.0
+    for w, y in zip(ws[0], ys):
+        rows = torch.arange(0, w.shape[0], max(1, w.shape[0] // 256), device=dev)
+        ref = xs[w.shape[1]].double().cpu() @ w[rows].double().cpu().T
+        rel = max(rel, float((y[:, rows].double().cpu() - ref).norm() / ref.norm()))
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+    def timed(fn):
         for i in range(args.warmup):
-            fn(i)
+            fn(i % 3)
         torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
         a.record(stream)
         for i in range(args.steps):
-            fn(i)
+            fn(i % 3)
         b.record(stream)
         torch.cuda.synchronize(dev)
-        return a.elapsed_time(b) / args.steps
+        ms = a.elapsed_time(b) / args.steps
+        return max_over_ranks(ms, dist, dev) if world > 1 else ms
 
-    ms_cublas = other(lambda i: torch.matmul(x, ws[i % 3].T))
-    ms_multi = other(lambda i: df11.gemm_multi([(x, ws[i % 3])], [y], err, stream))
-    if world > 1:
-        ms, ms_cublas, ms_multi = (max_over_ranks(v, dist, dev) for v in (ms, ms_cublas, ms_multi))
+    ms = timed(ours)
+
+    def cublas(c):
+        for w in ws[c]:
+            torch.matmul(xs[w.shape[1]], w.T)
+
+    ms_cublas = timed(cublas)
+    ms_other = None
+    if T > 4:  # the other tensor-core kernel on the same work
+        if block:
+            ms_other = timed(lambda c: [df11.gemm(xs[w.shape[1]], w, y, err, stream) for w, y in zip(ws[c], ys)])
+        else:
+            ms_other = timed(lambda c: df11.gemm_multi([(xs[shapes[0][1]], ws[c][0])], ys, err, stream))
     assert df11.read_error(err, stream) == 0
     if rank == 0:
         hbm, hbm_kind = _peaks()
@@ -822,8 +840,8 @@ def run_gemm(args, rank: int, world: int):
                 tf_peak, tf_kind = float(json.load(f)["bf16_tflops"]), "measured"
         except Exception:
             tf_peak, tf_kind = 1590.0, "fallback"
-        nbytes = 2 * out * inn + 2 * T * inn + 4 * T * out
-        flops = 2.0 * T * out * inn
+        nbytes = sum(2 * o * i + 2 * T * i + 4 * T * o for o, i in shapes)
+        flops = sum(2.0 * T * o * i for o, i in shapes)
         gbs, tfs = nbytes / (ms * 1e-3) / 1e9, flops / (ms * 1e-3) / 1e12
         hbm_bound = nbytes / hbm >= flops / (tf_peak * 1e3)  # both in us per unit
         roof = ({"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
@@ -831,14 +849,21 @@ def run_gemm(args, rank: int, world: int):
                 {"bound": "tensor", "achieved": tfs, "peak": tf_peak, "unit": "TFLOP/s", "frac": tfs / tf_peak,
                  "peak_kind": f"{tf_kind} (MEASURED_PEAKS.json bf16_tflops, cuBLAS burst)"})
         roof.update({"traffic": None, "algorithmic_bytes_per_launch": nbytes, "flops_per_launch": flops})
+        if T <= 4:
+            kernel = "CUDA-core matrix-vector stream" + (" (one launch per matrix)" if block else "")
+        else:
+            kernel = "grouped tcgen05 kernel (one launch for the seven products)" if block else "tcgen05"
         line = {"metric": "consumer GEMM time", "value": ms * 1e3, "unit": "us", "n_gpus": world,
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": False,
                 "scaling": "weak", "vs_baseline": None, "dtype": "bf16 x bf16 -> f32", "data": "synthetic",
-                "config": {"workload": WORKLOADS["gemm"][0], "shape": [out, inn], "T": T,
-                           "kernel": "CUDA-core matrix-vector stream" if T <= 4 else "tcgen05",
-                           "l2": "W in three copies used in turn (3 x 2 out in bytes > L2), no flush"},
-                "rel_fro_sampled_rows": rel, "roofline": roof, "gpu_launches": args.steps,
-                "cublas_us": ms_cublas * 1e3, "grouped_kernel_us": ms_multi * 1e3}
+                "config": {"workload": WORKLOADS["gemm"][0], "shape": "llama8b-block" if block else list(shapes[0]),
+                           "T": T, "kernel": kernel,
+                           "l2": "weights in three copies used in turn (each larger than L2 or 3 x > L2), no flush"},
+                "rel_fro_sampled_rows": rel, "roofline": roof,
+                "gpu_launches": args.steps * (len(shapes) if (T <= 4 and block) else 1) * (2 if block and T > 4 else 1),
+                "cublas_us": ms_cublas * 1e3, "vs_cublas": ms_cublas / ms}
+        if ms_other is not None:
+            line["per_matrix_launches_us" if block else "grouped_kernel_us"] = ms_other * 1e3
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
@@ -912,7 +937,7 @@ def main():
     ap.add_argument("--blocks", type=int, default=None, help="blocks of the decode-gemm (32) / offload (4) workloads")
     ap.add_argument("--repeat", type=int, default=4, help="passes over the blocks in the offload workload")
     ap.add_argument("--T", type=int, default=1, help="batch of the decode-gemv (1..4) and gemm (1..256) workloads")
-    ap.add_argument("--shape", default="14336x4096", help="OUTxIN of the gemm workload")
+    ap.add_argument("--shape", default="14336x4096", help="OUTxIN of the gemm workload, or llama8b-block")
     ap.add_argument("--no-counts", action="store_true",
                     help="decode without the stored per-thread counts (count pass + decoding pass)")
     args = ap.parse_args()
