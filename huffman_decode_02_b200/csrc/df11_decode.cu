@@ -896,14 +896,16 @@ __device__ __forceinline__ void decode_loop(const DecodeArgs &a, Sink &sink, uin
 }
 
 // Loads the tables (whole CTA), then runs the decode loop of this thread's
-// group over blocks blk_first + (CTA * groups + group) + k * (grid * groups)
-// below blk_end.
+// group over blocks blk_first + (CTA + group * grid) + k * (grid * groups)
+// below blk_end: the first blocks go to every CTA's group 0 before any
+// CTA's group 1, so a tensor of few blocks is spread over all the SMs (one
+// block per SM decodes faster than eight on one).
 template <class C, bool kLong, class Sink>
 __device__ __forceinline__ void decode_blocks(const DecodeArgs &a, Sink &sink, uint64_t blk_first, uint64_t blk_end) {
     extern __shared__ __align__(128) uint8_t smem[];
     if (!load_tables<C>(a.lut, a.err, smem, smem_addr(smem), threadIdx.x)) return;
     const uint32_t group = threadIdx.x / kGroupThreads;
-    decode_loop<C, kLong>(a, sink, blk_first + (uint64_t)blockIdx.x * C::kGroups + group,
+    decode_loop<C, kLong>(a, sink, blk_first + blockIdx.x + (uint64_t)group * gridDim.x,
                           (uint64_t)gridDim.x * C::kGroups, blk_end);
 }
 
@@ -948,6 +950,7 @@ __device__ __forceinline__ uint64_t find_block(const uint32_t *bs, uint64_t n_bl
 // lane): the 32-way search runs only when the answer lies outside them.
 __device__ __forceinline__ uint64_t find_block_near(const uint32_t *bs, uint64_t n_blocks, uint64_t hint, uint64_t x,
                                                     uint32_t lane) {
+    if (n_blocks == 0u) return 0u;
     hint = min(hint, n_blocks - 1u);
     const uint64_t p = hint + lane;
     const uint32_t m = __ballot_sync(kFull, p < n_blocks && (uint64_t)__ldg(bs + p) <= x);
@@ -1386,9 +1389,13 @@ struct GemvSink : NoHooks {
 template <class C, bool kLong, uint32_t TM>
 __global__ void __launch_bounds__(C::kCtaThreads, 1) df11_decode_gemv_kernel(const __grid_constant__ GemvArgs g) {
     // the format blocks that hold the matrices' elements (each warp finds them)
+    // (probed first near the blocks the elements' positions suggest: blocks
+    // hold about n_elems / n_blocks elements each)
     const uint32_t lane = threadIdx.x & 31u;
-    const uint64_t b0 = find_block(g.d.bstart, g.d.n_blocks, g.e_first, lane);
-    const uint64_t b1 = find_block(g.d.bstart, g.d.n_blocks, g.e_last, lane) + 1u;
+    const uint64_t nb = g.d.n_blocks, ne = g.d.n_elems ? g.d.n_elems : 1u;
+    const uint64_t h0 = (uint64_t)((double)g.e_first / (double)ne * (double)nb), h1 = (uint64_t)((double)g.e_last / (double)ne * (double)nb);
+    const uint64_t b0 = find_block_near(g.d.bstart, nb, h0 > 16u ? h0 - 16u : 0u, g.e_first, lane);
+    const uint64_t b1 = find_block_near(g.d.bstart, nb, h1 > 16u ? h1 - 16u : 0u, g.e_last, lane) + 1u;
     GemvSink<TM> sink{{}, g, 0u};
     decode_blocks<C, kLong>(g.d, sink, b0, b1);
 }
@@ -2031,8 +2038,8 @@ bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
 
 template <class C, bool kLong>
 void launch(const DecodeArgs &a, uint64_t n_blocks, int sms, cudaStream_t stream) {
-    const uint64_t ctas_needed = (n_blocks + C::kGroups - 1) / C::kGroups;
-    const unsigned grid = (unsigned)(ctas_needed < (uint64_t)sms ? ctas_needed : (uint64_t)sms);
+    // one CTA per SM, or one per block when there are fewer blocks
+    const unsigned grid = (unsigned)(n_blocks < (uint64_t)sms ? (n_blocks ? n_blocks : 1u) : (uint64_t)sms);
     df11_decode_kernel<C, kLong><<<grid, C::kCtaThreads, C::kSmemBytes, stream>>>(a);
 }
 
@@ -2171,8 +2178,7 @@ df11_status launch_rows(const df11_tensor *t, uint64_t row_len, const uint32_t *
 
 template <class C, bool kLong, uint32_t TM>
 void launch_gemv_inst(const GemvArgs &g, uint64_t blocks_est, int sms, cudaStream_t stream) {
-    const uint64_t ctas_needed = (blocks_est + C::kGroups - 1) / C::kGroups;
-    const unsigned grid = (unsigned)(ctas_needed < (uint64_t)sms ? ctas_needed : (uint64_t)sms);
+    const unsigned grid = (unsigned)(blocks_est < (uint64_t)sms ? (blocks_est ? blocks_est : 1u) : (uint64_t)sms);
     df11_decode_gemv_kernel<C, kLong, TM><<<grid, C::kCtaThreads, C::kSmemBytes, stream>>>(g);
 }
 
