@@ -198,9 +198,15 @@ def _on(device):
     """Makes `device` the current CUDA device for the duration of a library
     call: the C entry points launch on the current device, so the data's own
     device must be current (another device's memory would be read without
-    peer access)."""
+    peer access).  No switch when it already is (the common case; the switch
+    costs two driver calls per library call)."""
+    import contextlib
+
     import torch
-    return torch.cuda.device(torch.device(device))
+    dev = torch.device(device)
+    if dev.type == "cuda" and (dev.index is None or dev.index == torch.cuda.current_device()):
+        return contextlib.nullcontext()
+    return torch.cuda.device(dev)
 
 
 class DF11Tensor:
@@ -266,12 +272,38 @@ class DF11Tensor:
         return a.view(np.uint32) if which == "block_start" else a.view(np.uint8)
 
     def _bind(self) -> _Tensor:
+        """A new descriptor with the arrays' current addresses."""
         d = _Tensor.from_buffer_copy(self.desc)
         for name in _ARRAYS:
             a = self.arrays.get(name)
             ptr = None if a is None else (a.ctypes.data if isinstance(a, np.ndarray) else a.data_ptr())
             setattr(d, name, ptr)
         return d
+
+    def _desc_for_call(self) -> _Tensor:
+        """The descriptor for a library call (the entry points only read it):
+        rebuilt only when an array's address or the descriptor changed since
+        the last call, so repeated calls on small tensors skip the marshalling."""
+        ptrs = tuple(None if a is None else (a.ctypes.data if isinstance(a, np.ndarray) else a.data_ptr())
+                     for a in (self.arrays.get(name) for name in _ARRAYS))
+        key = (ptrs, bytes(self.desc))
+        cached = getattr(self, "_bound", None)
+        if cached is None or cached[0] != key:
+            d = _Tensor.from_buffer_copy(self.desc)
+            for name, ptr in zip(_ARRAYS, ptrs):
+                setattr(d, name, ptr)
+            cached = (key, d)
+            self._bound = cached
+        return cached[1]
+
+    def _offsets_c(self):
+        """The matrix offsets as a ctypes uint64 array (built once)."""
+        key = tuple(self.offsets)
+        cached = getattr(self, "_offs_c", None)
+        if cached is None or cached[0] != key:
+            cached = (key, (ctypes.c_uint64 * len(key))(*key))
+            self._offs_c = cached
+        return cached[1]
 
     def to(self, device, non_blocking: bool = False) -> "DF11Tensor":
         """Copies the five arrays to a device (torch tensors, 16-byte aligned)."""
@@ -543,7 +575,7 @@ def decode(t: DF11Tensor, out=None, err=None, stream=None):
     own_err = err is None
     if own_err:
         err = _new_err(t.device)
-    d = t._bind()
+    d = t._desc_for_call()
     with _on(t.device):
         _check(_lib().df11_decode(ctypes.byref(d), ctypes.c_void_p(out.data_ptr()),
                                   ctypes.c_void_p(err.data_ptr()), _stream_handle(stream, t.device)), "decode")
@@ -565,8 +597,8 @@ def decode_block(t: DF11Tensor, scratch=None, err=None, stream=None):
     own_err = err is None
     if own_err:
         err = _new_err(t.device)
-    offs = (ctypes.c_uint64 * len(t.offsets))(*t.offsets)
-    d = t._bind()
+    offs = t._offsets_c()
+    d = t._desc_for_call()
     with _on(t.device):
         _check(_lib().df11_decode_block(ctypes.byref(d), offs, len(t.offsets) - 1,
                                         ctypes.c_void_p(scratch.data_ptr()),
@@ -593,7 +625,7 @@ def decode_rows(t: DF11Tensor, row_len: int, rows, out=None, err=None, stream=No
     if own_err:
         err = _new_err(t.device)
     with _on(t.device):
-        _check(_lib().df11_decode_rows(ctypes.byref(t._bind()), int(row_len), ctypes.c_void_p(rows.data_ptr()), n,
+        _check(_lib().df11_decode_rows(ctypes.byref(t._desc_for_call()), int(row_len), ctypes.c_void_p(rows.data_ptr()), n,
                                        ctypes.c_void_p(out.data_ptr()), ctypes.c_void_p(err.data_ptr()),
                                        _stream_handle(stream, t.device)), "decode_rows")
     if own_err:
@@ -639,7 +671,7 @@ def decode_gemv(t: DF11Tensor, xs: dict, ys: dict | None = None, err=None, strea
     if own_err:
         err = _new_err(t.device)
     with _on(t.device):
-        _check(_lib().df11_decode_gemv(ctypes.byref(t._bind()), mats, len(order), T,
+        _check(_lib().df11_decode_gemv(ctypes.byref(t._desc_for_call()), mats, len(order), T,
                                        ctypes.c_void_p(err.data_ptr()), _stream_handle(stream, t.device)),
                "decode_gemv")
     if own_err:
@@ -686,7 +718,7 @@ def decode_gemm(t: DF11Tensor, xs: dict, ys: dict | None = None, err=None, strea
     if own_err:
         err = _new_err(t.device)
     with _on(t.device):
-        _check(_lib().df11_decode_gemm(ctypes.byref(t._bind()), mats, len(order), T,
+        _check(_lib().df11_decode_gemm(ctypes.byref(t._desc_for_call()), mats, len(order), T,
                                        ctypes.c_void_p(err.data_ptr()), _stream_handle(stream, t.device)),
                "decode_gemm")
     if own_err:
