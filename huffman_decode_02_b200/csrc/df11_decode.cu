@@ -1704,7 +1704,8 @@ struct TileSink {
                 }
             }
         }
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        // (the stores are made visible to the async proxy in block_done,
+        // one fence per thread for the chunks and the edges together)
     }
     __device__ __forceinline__ void edges(uint32_t sbuf, uint32_t base, uint32_t c_full, uint32_t span, uint32_t s,
                                           uint32_t e, uint32_t lane, uint32_t sm_s0) {
@@ -1730,8 +1731,7 @@ struct TileSink {
             if (in_a) ba += 2u;
             else bb += 2u;
         }
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        __syncwarp();
+        __syncwarp();  // every lane has read the edge chunks before they are cleared
         if ((lane == 0u && head) || (lane == 16u && tail)) sts_zero16(sbuf + 16u * (lane == 0u ? 0u : c_full));
     }
     // After the block's merge (every thread of the group): each warp counts
@@ -1749,6 +1749,9 @@ struct TileSink {
             return;
         }
         if (ok) {
+            // this thread's tile stores (chunks and edges) become visible to
+            // the tensor cores' async proxy; the warp sync gathers them
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             __syncwarp();
             const uint32_t a = __reduce_add_sync(0xFFFFFFFFu, ba), b = __reduce_add_sync(0xFFFFFFFFu, bb);
             if (lane == 0u && (a | b) != 0u && !lds_u32(L.abort_flag)) {
