@@ -600,20 +600,16 @@ __device__ __forceinline__ void chain_counts(const Chain &A, const Chain &B, uin
 // replicates them (whole CTA).  Returns false, uniformly over the CTA and with
 // the error reported, when they did not arrive in time or are malformed;
 // nothing has been written to global memory then.
+// Issues the bulk copy of the compact tables (thread 0; nothing else of the
+// CTA may write the group area until finish_tables): the CTA can do other
+// work (a block search) while they travel.
 template <class C>
-__device__ __forceinline__ bool load_tables(const uint8_t *lut, uint32_t *err_out, uint8_t *smem, uint32_t s_base,
-                                            uint32_t tid) {
-    constexpr uint32_t kOffGroups = C::kOffGroups;
-    constexpr uint32_t kSymCopies = C::kSymCopies;
-    const uint32_t s_tmbar = s_base + kOffGroups + C::kGroups * C::kGroupBytes;
-    const uint32_t s_stage = s_base + kOffGroups;  // compact tables land here first
-    // ---- decode tables: one bulk copy, then validate and replicate
+__device__ __forceinline__ void issue_tables(const uint8_t *lut, uint32_t s_base, uint32_t tid) {
+    const uint32_t s_tmbar = s_base + C::kOffGroups + C::kGroups * C::kGroupBytes;
+    const uint32_t s_stage = s_base + C::kOffGroups;  // compact tables land here first
     if (tid == 0) {
         mbar_init(s_tmbar);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    }
-    __syncthreads();
-    if (tid == 0) {
         if (C::kCountTable) {
             mbar_expect(s_tmbar, kLutBytes);
             bulk_g2s(s_stage, lut, kLutBytes, s_tmbar);
@@ -623,6 +619,18 @@ __device__ __forceinline__ bool load_tables(const uint8_t *lut, uint32_t *err_ou
             bulk_g2s(s_stage + C::kStageSym, lut + kOffSymLut, kLutBytes - kOffSymLut, s_tmbar);
         }
     }
+}
+
+// Waits for the tables issue_tables requested, validates every entry and
+// replicates them (whole CTA; the same contract as load_tables).
+template <class C>
+__device__ __forceinline__ bool finish_tables(const uint8_t *lut, uint32_t *err_out, uint8_t *smem, uint32_t s_base,
+                                              uint32_t tid) {
+    constexpr uint32_t kOffGroups = C::kOffGroups;
+    constexpr uint32_t kSymCopies = C::kSymCopies;
+    const uint32_t s_tmbar = s_base + kOffGroups + C::kGroups * C::kGroupBytes;
+    const uint32_t s_stage = s_base + kOffGroups;
+    __syncthreads();  // the barrier's initialisation is visible to every waiter
     const bool staged = wait_phase(s_tmbar, 0u);
     if (__syncthreads_or(!staged)) {
         // Uniform over the CTA.  One more bounded wait so no copy is left in
@@ -678,6 +686,13 @@ __device__ __forceinline__ bool load_tables(const uint8_t *lut, uint32_t *err_ou
     }
     __syncthreads();  // the replicated tables are complete before any lookup
     return true;
+}
+
+template <class C>
+__device__ __forceinline__ bool load_tables(const uint8_t *lut, uint32_t *err_out, uint8_t *smem, uint32_t s_base,
+                                            uint32_t tid) {
+    issue_tables<C>(lut, s_base, tid);
+    return finish_tables<C>(lut, err_out, smem, s_base, tid);
 }
 
 // Where a decoded block goes: StoreSink writes it as BF16 (the decoder);
@@ -901,9 +916,12 @@ __device__ __forceinline__ void decode_loop(const DecodeArgs &a, Sink &sink, uin
 // CTA's group 1, so a tensor of few blocks is spread over all the SMs (one
 // block per SM decodes faster than eight on one).
 template <class C, bool kLong, class Sink>
-__device__ __forceinline__ void decode_blocks(const DecodeArgs &a, Sink &sink, uint64_t blk_first, uint64_t blk_end) {
+__device__ __forceinline__ void decode_blocks(const DecodeArgs &a, Sink &sink, uint64_t blk_first, uint64_t blk_end,
+                                              bool tables_issued = false) {
     extern __shared__ __align__(128) uint8_t smem[];
-    if (!load_tables<C>(a.lut, a.err, smem, smem_addr(smem), threadIdx.x)) return;
+    if (tables_issued ? !finish_tables<C>(a.lut, a.err, smem, smem_addr(smem), threadIdx.x)
+                      : !load_tables<C>(a.lut, a.err, smem, smem_addr(smem), threadIdx.x))
+        return;
     const uint32_t group = threadIdx.x / kGroupThreads;
     decode_loop<C, kLong>(a, sink, blk_first + blockIdx.x + (uint64_t)group * gridDim.x,
                           (uint64_t)gridDim.x * C::kGroups, blk_end);
@@ -1391,13 +1409,15 @@ __global__ void __launch_bounds__(C::kCtaThreads, 1) df11_decode_gemv_kernel(con
     // the format blocks that hold the matrices' elements (each warp finds them)
     // (probed first near the blocks the elements' positions suggest: blocks
     // hold about n_elems / n_blocks elements each)
+    extern __shared__ __align__(128) uint8_t smem[];
+    issue_tables<C>(g.d.lut, smem_addr(smem), threadIdx.x);  // in flight during the search
     const uint32_t lane = threadIdx.x & 31u;
     const uint64_t nb = g.d.n_blocks, ne = g.d.n_elems ? g.d.n_elems : 1u;
     const uint64_t h0 = (uint64_t)((double)g.e_first / (double)ne * (double)nb), h1 = (uint64_t)((double)g.e_last / (double)ne * (double)nb);
     const uint64_t b0 = find_block_near(g.d.bstart, nb, h0 > 16u ? h0 - 16u : 0u, g.e_first, lane);
     const uint64_t b1 = find_block_near(g.d.bstart, nb, h1 > 16u ? h1 - 16u : 0u, g.e_last, lane) + 1u;
     GemvSink<TM> sink{{}, g, 0u};
-    decode_blocks<C, kLong>(g.d, sink, b0, b1);
+    decode_blocks<C, kLong>(g.d, sink, b0, b1, true);
 }
 
 // ------------------------------------------------- fused decode -> tcgen05 GEMM
@@ -1840,6 +1860,7 @@ __global__ void __launch_bounds__(C::kCtaThreads + kFusedExtraThreads, 1)
     const uint32_t NT = K1 - K0;
     uint32_t err = 0;
 
+    issue_tables<C>(f.d.lut, s_base, tid);  // in flight during the search
     // warp 0: the format blocks covering the elements of k-tiles [K0, K1),
     // searched near the share's ends
     if (tid < 32u) {
@@ -1854,7 +1875,7 @@ __global__ void __launch_bounds__(C::kCtaThreads + kFusedExtraThreads, 1)
             sts_u32(L.block_end, (uint32_t)b1);
         }
     }
-    if (!load_tables<C>(f.d.lut, f.d.err, smem, s_base, tid)) return;  // uniform over the CTA
+    if (!finish_tables<C>(f.d.lut, f.d.err, smem, s_base, tid)) return;  // uniform over the CTA
     if (tid == 0) {
         for (uint32_t s = 0; s < f.ring; ++s) {
             df11::tc::mbar_init(L.full0 + 8u * s, 1);
