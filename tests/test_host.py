@@ -470,3 +470,20 @@ def test_gemm_multi_argument_checks():
     assert call([(A, A + 8, A, 128, 64)]) == 1                 # w not 16-byte aligned
     assert call([(A, A, A + 2, 128, 64)]) == 1                 # y not 4-byte aligned
     assert lib.df11_gemm_bf16_multi(None, 1, 16, None, None) == 1
+
+
+def test_call_descriptor_follows_the_arrays():
+    """The descriptor the binding passes to the library is reused while the
+    arrays stay where they are and rebuilt as soon as one moves; _bind()
+    always returns a fresh copy (callers may edit it)."""
+    t = df11.encode(workloads.normal_matrix(64, 64, 0.02, seed=3))
+    d1 = t._desc_for_call()
+    assert t._desc_for_call() is d1
+    assert d1.enc == t.host_array("enc").ctypes.data
+    b = t._bind()
+    assert b is not d1 and b.enc == d1.enc
+    b.enc = 0  # editing a fresh copy leaves the call descriptor alone
+    assert t._desc_for_call().enc == d1.enc
+    t.arrays["enc"] = np.array(t.host_array("enc"), copy=True)  # the array moves
+    d2 = t._desc_for_call()
+    assert d2 is not d1 and d2.enc == t.arrays["enc"].ctypes.data
